@@ -1,0 +1,387 @@
+"""Benchmark of the SSD layer forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full SSD forward (every stage kernel) over one batch of the
+workload's synthetic inputs, resident in HBM.  Each step is timed on the
+launching stream by events the library records around its own kernels
+(``ssd_fwd_timed``); L2 is flushed (a 256 MiB write) between steps, outside
+the timed spans.  ``value`` is tokens/s over all ranks: sum of tokens ÷ the
+max over ranks of the K-step time.  ``e2e`` repeats the measurement through
+the same public call with the inputs copied in from pinned host memory and y
+plus final_state copied back inside the timed region.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch of
+the workload (independent sequences, no collective on the data path), so
+scaling is weak.  The only collectives are the barriers and the max-reduction
+of the timings.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), on a
+bounded sample of (batch, head) sequences per step, and prints the same line
+with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD fwd tokens/s and TFLOP/s (% of roofline) at Mamba-2-2.7B layer shape"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+N_SM = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (block-decomposition count of the pages' cost analysis)
+# ---------------------------------------------------------------------------
+def algorithmic(w):
+    """Per-call algorithmic bytes and FLOPs of the whole pass and of each stage.
+
+    Bytes: x, B, C (input dtype), dt, A, D, init (fp32) read; y (input dtype)
+    and final_state (fp32) written; intermediates excluded.  FLOPs per
+    (batch, chunk): 2Q^2 N G (C B^T, once per group) + 2Q^2 P H (masked X
+    product over the full QxQ block) + 2QNP H (chunk states) + 2QNP H
+    (inter-chunk output) + 2NP H (state passing).
+    """
+    es = 2 if w.dtype == "bf16" else 4
+    b, T, H, P, N, G, Q, nc = w.batch, w.T, w.H, w.P, w.N, w.G, w.Q, w.nc
+    state = 4 * b * H * P * N
+    bytes_ = (es * b * T * H * P * 2 + es * b * T * G * N * 2 + 4 * b * T * H + 8 * H
+              + state * (2 if w.with_init else 1))
+    per_chunk = 2 * Q * Q * N * G + 2 * Q * Q * P * H + 4 * Q * N * P * H + 2 * N * P * H
+    flops = b * nc * per_chunk
+    stages = {
+        "ssd_chunk_cumsum": ("hbm", 4 * b * T * H + 4 * H + 4 * b * H * nc * Q),
+        "ssd_chunk_state": ("flop", b * nc * 2 * Q * N * P * H),
+        "ssd_state_passing": ("hbm", 2 * 4 * b * nc * H * P * N + state * (2 if w.with_init else 1)),
+        "ssd_chunk_scan": ("flop", b * nc * (2 * Q * Q * N * G + 2 * Q * Q * P * H + 2 * Q * N * P * H)),
+    }
+    return bytes_, flops, stages
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the baseline, and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_time(inp, w, pairs):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.ssd_ref_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       init_state=inp["init_state"], pairs=pairs)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp, w, budget_pairs=None):
+    """Time the oracle on a bounded set of (batch, head) sequences; tokens/s equivalent."""
+    import oracle
+    allpairs = [(b, h) for b in range(w.batch) for h in range(w.H)]
+    cost = w.T * w.P * w.N  # per sequence
+    if budget_pairs is None:
+        # about 40 core-seconds at the oracle's ~0.5 GFLOP/s per core
+        budget_pairs = max(1, int(40 * 0.5e9 / (4 * cost)))
+    step = max(1, len(allpairs) // budget_pairs)
+    pairs = allpairs[::step][:budget_pairs]
+    secs = oracle_sample_time(inp, w, pairs)
+    tokens = len(pairs) * w.T / w.H  # a sequence is one head's share of T tokens
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": f"{len(pairs)} of {len(allpairs)} (batch, head) sequences of {w.name}, all {w.T} tokens, "
+                      f"fp64, {secs:.2f} s wall"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from structured_state_space_ssd_b200.inputs import workload_inputs
+    import oracle
+    inp = workload_inputs(w)
+    cores = oracle.default_threads()
+    allpairs = [(b, h) for b in range(w.batch) for h in range(w.H)]
+    per_step = max(1, min(len(allpairs), 2 * cores))
+    times = []
+    for k in range(args.warmup + args.steps):
+        pairs = [allpairs[(k * per_step + i) % len(allpairs)] for i in range(per_step)]
+        t = oracle_sample_time(inp, w, pairs)
+        if k >= args.warmup:
+            times.append(t)
+    tok = per_step * w.T / w.H
+    value = tok * len(times) / sum(times)
+    sample = (f"{per_step} (batch, head) sequences of {w.name} per step (all {w.T} tokens each), fp64, "
+              f"{cores} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, n):
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.T, "heads": w.H, "head_dim": w.P,
+            "state_dim": w.N, "groups": w.G, "chunk": w.Q, "init_state": w.with_init,
+            "parallelism": f"replicas{n}" if n > 1 else "single", "l2": "flushed (256 MiB write) between steps"}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    from structured_state_space_ssd_b200.inputs import HEADLINE, WORKLOADS, workload_inputs
+    w = WORKLOADS[args.workload or HEADLINE]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from structured_state_space_ssd_b200 import ssd as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    S.load()
+    host = workload_inputs(w) if world == 1 else _rank_inputs(w, rank)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((w.batch, w.H, w.P, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(S.ssd_fwd_workspace_bytes(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = S.ssd_fwd_stage_names(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
+
+    def step(stage_ms=None):
+        S.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], w.Q, d["init_state"], y=y, final_state=fin,
+                  workspace=ws, stream=stream, stage_ms=stage_ms)
+
+    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local)
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.2)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    per_step = []
+    per_stage = [[] for _ in names]
+    for _ in range(args.steps):
+        flush.zero_()
+        ms = []
+        step(ms)
+        for i in range(len(names)):
+            per_stage[i].append(ms[i])
+        per_step.append(ms[-1])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = sum(per_step)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.tokens * world
+    value = tokens / (ms_per_step * 1e-3)
+
+    # --- end to end: pinned host inputs in, y and final_state out, every step
+    e2e_steps = args.e2e_steps or args.steps
+    pinned = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    fin_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size() + fin_host.numel() * fin_host.element_size()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            if v is not None:
+                d[k].copy_(v, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        fin_host.copy_(fin, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        alg_bytes, alg_flops, stages = algorithmic(w)
+        stage_avg = {n: sum(v) / len(v) for n, v in zip(names, per_stage)}
+        dom = max(stage_avg, key=stage_avg.get)
+        kind, amount = stages[dom]
+        dom_ms = stage_avg[dom]
+        if kind == "hbm":
+            roof = {"bound": "hbm", "achieved": amount / (dom_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+        else:
+            tc = _stage_uses_tensor_cores(dom, w)
+            if tc:
+                roof = {"bound": "tensor", "achieved": amount / (dom_ms * 1e-3) / 1e12,
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+            else:
+                fp32_peak = N_SM * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+                roof = {"bound": "alu", "achieved": amount / (dom_ms * 1e-3) / 1e12, "peak": fp32_peak,
+                        "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = _traffic_from_profiles(dom, w)
+        roof["kernel"] = dom
+        roof["peak_source"] = f"{peak_src} (burst)" if roof["bound"] != "alu" else \
+            "derived: 148 SMs x 128 fp32 FMA/clk x 2 x max SM clock"
+        t_roof = max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flops / (peaks["bf16_tflops"] * 1e12))
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1)/softplus inputs, see inputs.py)",
+            "config": config_of(w, world),
+            "tflops": alg_flops * world / (ms_per_step * 1e-3) / 1e12,
+            "pass_roofline": {"alg_bytes": alg_bytes, "alg_flops": alg_flops, "roofline_ms": t_roof * 1e3,
+                              "frac": t_roof * 1e3 / ms_per_step, "peaks": peak_src},
+            "roofline": roof,
+            "kernels_ms": stage_avg,
+            "clocks": clocks,
+            "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": S.ssd_fwd_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
+            * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(host, w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _stage_uses_tensor_cores(name, w):
+    return False
+
+
+def _traffic_from_profiles(kernel, w):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one matches."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    return t.get(w.name, {}).get(kernel)
+
+
+def _rank_inputs(w, rank):
+    from structured_state_space_ssd_b200.inputs import make_inputs
+    return make_inputs(w.batch, w.T, w.H, w.P, w.N, w.G, w.dtype, w.seed + 7919 * rank, w.with_init)
+
+
+if __name__ == "__main__":
+    main()

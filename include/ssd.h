@@ -1,0 +1,144 @@
+/*
+ * ssd.h -- C ABI of libssd.so, the B200 (sm_100a) SSD layer forward.
+ *
+ * The operation is the SSD layer Y = SSD(A, B, C)(X) of "Transformers are
+ * SSMs: Generalized Models and Efficient Algorithms Through Structured State
+ * Space Duality" (arXiv 2405.21060; analysis page, section "The SSD Layer:
+ * Formal Definition"), i.e. the scalar-identity selective SSM of section "The
+ * Scalar-Identity SSM":
+ *
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + B_t x_t^T        (state [P x N] per head)
+ *     y_t = C_t^T h_t + D_h * x_t
+ *
+ * with h_{-1} = init_state (zero when NULL), computed by the block
+ * decomposition of section "The Block-Decomposition SSD Algorithm": chunks of
+ * Q tokens (stage 0, ceil(T/Q) chunks, the last one may be short), the
+ * quadratic masked form inside each chunk (stage 1), chunk-final states
+ * (stage 2), the scalar recurrence between chunks (stage 3), the inter-chunk
+ * output (stage 4) and their sum (stage 5).  The exponential discretisation,
+ * the D_h skip and the place of init_state are not written on the pages; they
+ * are the readings stated above.  Head h reads B/C group g = h / (H / G)
+ * (grouped heads: analysis page, "The Mamba-2 Architecture", G divides H).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *    and densely packed in the layouts given below.  The library never
+ *    allocates device memory; scratch lives in the caller's workspace.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream and never synchronise the
+ *    host, except ssd_fwd_check which waits for the stream.
+ *  - Return values are ssd status codes (SSD_OK = 0).  Argument errors are
+ *    detected on the host before anything is launched.
+ *  - Stateless and thread-safe; concurrent calls must use distinct
+ *    workspaces.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+
+/* Every declared entry point is exported; everything else in libssd.so is hidden. */
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of x, B, C and y.  dt, A, D and both states are always fp32. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
+
+enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1, /* NULL required pointer, bad dimension, H % G != 0,
+                                misaligned pointer, workspace too small */
+    SSD_ERR_UNSUPPORTED = 2, /* valid shape outside the kernels' limits
+                                (P > 128, N > 256, Q > 256) */
+    SSD_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+    SSD_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see ssd_fwd_check) */
+};
+
+/*
+ * Bytes of device workspace ssd_fwd needs for this problem (256-byte
+ * multiple).  Returns 0 for invalid dimensions.  The workspace holds the
+ * per-chunk log-decay prefix sums (stage 0 / 1), the chunk states (stages 2-3)
+ * and a status word.
+ */
+SSD_API size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
+
+/*
+ * SSD layer forward.
+ *
+ *   x           [batch][T][H][P]   dtype      input sequence X
+ *   dt          [batch][T][H]      fp32       step sizes, already positive (no softplus inside)
+ *   A           [H]                fp32       per-head log-decay rate, a_t = exp(dt_t * A_h)
+ *   B, C        [batch][T][G][N]   dtype      expansion / contraction vectors
+ *   D           [H]                fp32       skip weight
+ *   Q                                         chunk length (1 <= Q <= 256)
+ *   init_state  [batch][H][P][N]   fp32       h_{-1}; NULL = zero
+ *   y           [batch][T][H][P]   dtype      output (written)
+ *   final_state [batch][H][P][N]   fp32       h_{T-1} (written); NULL = not written
+ *   workspace   >= ssd_fwd_workspace_bytes(...) bytes of device memory, 256-byte aligned
+ *
+ * Limits: batch, H, G, P, N, Q >= 1, T >= 0, H % G == 0, P <= 128, N <= 256,
+ * Q <= 256.  Pointers must be aligned to their element size (16 bytes for
+ * the bf16 tensor-core path).  y must not alias any input.  T == 0 writes
+ * final_state = init_state (or zero) and nothing else.
+ *
+ * Returns SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
+ * Device-side failures of bounded waits are reported by ssd_fwd_check.
+ */
+SSD_API int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C,
+            const float *D, int Q, const float *init_state, void *y, float *final_state,
+            int batch, int T, int H, int P, int G, int N, int dtype, void *workspace,
+            size_t workspace_bytes, void *stream);
+
+/*
+ * Number of kernel launches ssd_fwd issues for these arguments (0 when the
+ * arguments are invalid).  Lets callers account for launches without a
+ * profiler.
+ */
+SSD_API int ssd_fwd_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
+
+/*
+ * ssd_fwd, instrumented for measurement: records a CUDA event on `stream`
+ * before the first kernel and after each kernel, waits for the stream, and
+ * writes each kernel's duration in milliseconds to stage_ms[0 .. k-1]
+ * (k = min(ssd_fwd_launch_count(...), max_stages)) and the span of the whole
+ * call to *total_ms (either pointer may be NULL).  The events are created on
+ * the first call in each host thread and kept until the process exits.  Same
+ * arguments and results as ssd_fwd otherwise.
+ */
+SSD_API int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                  const float *D, int Q, const float *init_state, void *y, float *final_state,
+                  int batch, int T, int H, int P, int G, int N, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream, float *stage_ms, int max_stages,
+                  float *total_ms);
+
+/*
+ * Name of kernel `i` (0-based, launch order) of the sequence ssd_fwd issues
+ * for these arguments, or NULL when i is out of range.
+ */
+SSD_API const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int Q, int dtype, int i);
+
+/*
+ * Waits for `stream`, then reads the status word the kernels of the last
+ * ssd_fwd on this workspace left (SSD_OK or SSD_ERR_TIMEOUT).  Returns
+ * SSD_ERR_CUDA if the wait or the copy fails.
+ */
+SSD_API int ssd_fwd_check(const void *workspace, void *stream);
+
+/* Static, NUL-terminated description of a status code. */
+SSD_API const char *ssd_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SSD_API int ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

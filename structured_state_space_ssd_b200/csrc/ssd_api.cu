@@ -1,0 +1,214 @@
+// ssd_api.cu -- the extern "C" boundary of libssd.so (declared in include/ssd.h):
+// argument validation, workspace carving and the launch sequence of the
+// block-decomposition stages on the caller's stream.
+#include <stdint.h>
+
+#include "ssd_common.cuh"
+
+namespace ssd {
+cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const Shape &sh, cudaStream_t st);
+template <typename T>
+cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st);
+cudaError_t launch_state_passing(float *S, const float *s, const float *init, float *fin, const Shape &sh,
+                                 cudaStream_t st);
+template <typename T>
+cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D, const float *s,
+                              const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
+}  // namespace ssd
+
+using ssd::Shape;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxP = 128, kMaxN = 256, kMaxQ = 256;
+constexpr int64_t kMaxElems = int64_t(1) << 46;
+
+// Validates the dimensions; fills `sh` on success.
+int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, Shape *sh) {
+    if (batch < 1 || T < 0 || H < 1 || P < 1 || G < 1 || N < 1 || Q < 1) return SSD_ERR_INVALID_ARG;
+    if (H % G != 0) return SSD_ERR_INVALID_ARG;
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    const int64_t bt = int64_t(batch) * T;
+    if (bt * H * P > kMaxElems || bt * G * N > kMaxElems || int64_t(batch) * H * P * N > kMaxElems)
+        return SSD_ERR_INVALID_ARG;
+    if (P > kMaxP || N > kMaxN || Q > kMaxQ) return SSD_ERR_UNSUPPORTED;
+    sh->batch = batch;
+    sh->T = T;
+    sh->H = H;
+    sh->P = P;
+    sh->G = G;
+    sh->N = N;
+    sh->Q = Q;
+    sh->nc = (T + Q - 1) / Q;
+    sh->heads_per_group = H / G;
+    return SSD_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+const char *const kStageNames[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
+                                   "ssd_chunk_scan"};
+constexpr int kMaxStages = 8;
+
+// Optional per-kernel event marks: ev[0] before the first kernel, ev[k+1] after kernel k.
+struct Marks {
+    cudaEvent_t *ev = nullptr;
+    int n = 0;
+    cudaError_t mark(int i, cudaStream_t st) const {
+        return (ev && i < n) ? cudaEventRecord(ev[i], st) : cudaSuccess;
+    }
+};
+
+template <typename T>
+int run_path(const Shape &sh, const T *x, const float *dt, const float *A, const T *B, const T *C,
+             const float *D, const float *init, T *y, float *fin, char *ws, cudaStream_t st, const Marks &mk) {
+    const ssd::Workspace w = ssd::workspace_layout(sh);
+    float *s = reinterpret_cast<float *>(ws + w.s_off);
+    float *S = reinterpret_cast<float *>(ws + w.state_off);
+    if (mk.mark(0, st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || mk.mark(1, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st) != cudaSuccess || mk.mark(2, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || mk.mark(3, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || mk.mark(4, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+int launch_count(const Shape &sh) { return sh.T == 0 ? 0 : 4; }
+
+int fwd_impl(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
+             const float *init_state, void *y, float *final_state, int batch, int T, int H, int P, int G, int N,
+             int dtype, void *workspace, size_t workspace_bytes, void *stream, const Marks &mk) {
+    Shape sh;
+    int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
+    if (rc != SSD_OK) return rc;
+    if (!x || !dt || !A || !B || !C || !D || !y || !workspace) return SSD_ERR_INVALID_ARG;
+    const size_t es = (dtype == SSD_BF16) ? 2 : 4;
+    if (!aligned(x, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es) || !aligned(dt, 4) ||
+        !aligned(A, 4) || !aligned(D, 4) || !aligned(workspace, 256) || (init_state && !aligned(init_state, 4)) ||
+        (final_state && !aligned(final_state, 4)))
+        return SSD_ERR_INVALID_ARG;
+    const ssd::Workspace w = ssd::workspace_layout(sh);
+    if (workspace_bytes < w.total) return SSD_ERR_INVALID_ARG;
+    const size_t ybytes = es * (size_t)batch * T * H * P;
+    const size_t bcbytes = es * (size_t)batch * T * G * N;
+    if (ybytes && (overlaps(y, ybytes, x, ybytes) || overlaps(y, ybytes, B, bcbytes) ||
+                   overlaps(y, ybytes, C, bcbytes)))
+        return SSD_ERR_INVALID_ARG;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    if (cudaMemsetAsync(ws + w.status_off, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (T == 0) {
+        if (mk.mark(0, st) != cudaSuccess) return SSD_ERR_CUDA;
+        if (!final_state) return SSD_OK;
+        const size_t fb = sizeof(float) * (size_t)batch * H * P * N;
+        cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, fb, cudaMemcpyDeviceToDevice, st)
+                                   : cudaMemsetAsync(final_state, 0, fb, st);
+        return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    }
+    if (dtype == SSD_BF16)
+        return run_path<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
+                                       static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C),
+                                       D, init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, st, mk);
+    return run_path<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
+                           static_cast<const float *>(C), D, init_state, static_cast<float *>(y), final_state, ws,
+                           st, mk);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
+    Shape sh;
+    if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
+    return ssd::workspace_layout(sh).total;
+}
+
+int ssd_fwd_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
+    Shape sh;
+    if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
+    return launch_count(sh);
+}
+
+const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int Q, int dtype, int i) {
+    Shape sh;
+    if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return nullptr;
+    if (i < 0 || i >= launch_count(sh)) return nullptr;
+    return kStageNames[i];
+}
+
+int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
+            const float *init_state, void *y, float *final_state, int batch, int T, int H, int P, int G, int N,
+            int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return fwd_impl(x, dt, A, B, C, D, Q, init_state, y, final_state, batch, T, H, P, G, N, dtype, workspace,
+                    workspace_bytes, stream, Marks{});
+}
+
+int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
+                  int Q, const float *init_state, void *y, float *final_state, int batch, int T, int H, int P,
+                  int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream, float *stage_ms,
+                  int max_stages, float *total_ms) {
+    thread_local cudaEvent_t events[kMaxStages + 1];
+    thread_local int events_device = -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
+    if (events_device != dev) {
+        for (int i = 0; i <= kMaxStages; ++i)
+            if (cudaEventCreate(&events[i]) != cudaSuccess) return SSD_ERR_CUDA;
+        events_device = dev;
+    }
+    Shape sh;
+    int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
+    if (rc != SSD_OK) return rc;
+    const int k = launch_count(sh);
+    Marks mk;
+    mk.ev = events;
+    mk.n = k + 1;
+    rc = fwd_impl(x, dt, A, B, C, D, Q, init_state, y, final_state, batch, T, H, P, G, N, dtype, workspace,
+                  workspace_bytes, stream, mk);
+    if (rc != SSD_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    for (int i = 0; i < k && i < max_stages && stage_ms; ++i)
+        if (cudaEventElapsedTime(&stage_ms[i], events[i], events[i + 1]) != cudaSuccess) return SSD_ERR_CUDA;
+    if (total_ms) {
+        *total_ms = 0.f;
+        if (k > 0 && cudaEventElapsedTime(total_ms, events[0], events[k]) != cudaSuccess) return SSD_ERR_CUDA;
+    }
+    return SSD_OK;
+}
+
+int ssd_fwd_check(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    int status = 0;
+    if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    return status;
+}
+
+const char *ssd_status_string(int status) {
+    switch (status) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "unsupported shape (P <= 128, N <= 256, Q <= 256)";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int ssd_version(void) { return kVersion; }
+
+}  // extern "C"

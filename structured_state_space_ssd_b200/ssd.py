@@ -1,0 +1,185 @@
+"""Thin ctypes binding of ``libssd.so`` (argument marshalling only).
+
+Every step of the SSD forward runs in the library's CUDA kernels; this module
+checks tensor devices, dtypes and contiguity, allocates outputs and the
+workspace with torch (device memory is the only thing torch provides here),
+and passes raw device pointers plus the current CUDA stream to the C ABI of
+``include/ssd.h``.  There is no fallback: a missing library or a non-zero
+status raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
+_lib = None
+
+SSD_F32, SSD_BF16 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "SSD_ERR_CUDA",
+          4: "SSD_ERR_TIMEOUT"}
+
+# Every symbol include/ssd.h declares.
+EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
+           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version")
+
+
+class SSDError(RuntimeError):
+    """A non-zero status returned by libssd.so."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Open libssd.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m structured_state_space_ssd_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ssd_fwd.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.ssd_fwd.restype = i
+    lib.ssd_fwd_workspace_bytes.argtypes = [i] * 8
+    lib.ssd_fwd_workspace_bytes.restype = sz
+    lib.ssd_fwd_launch_count.argtypes = [i] * 8
+    lib.ssd_fwd_launch_count.restype = i
+    lib.ssd_fwd_timed.argtypes = lib.ssd_fwd.argtypes + [fp, i, fp]
+    lib.ssd_fwd_timed.restype = i
+    lib.ssd_fwd_stage_name.argtypes = [i] * 9
+    lib.ssd_fwd_stage_name.restype = ctypes.c_char_p
+    lib.ssd_fwd_check.argtypes = [vp, vp]
+    lib.ssd_fwd_check.restype = i
+    lib.ssd_status_string.argtypes = [i]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_version.argtypes = []
+    lib.ssd_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().ssd_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return SSD_F32
+    if t == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"x/B/C must be float32 or bfloat16, got {t}")
+
+
+def ssd_fwd_workspace_bytes(batch, T, H, P, G, N, Q, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load().ssd_fwd_workspace_bytes(batch, T, H, P, G, N, Q, code))
+
+
+def ssd_fwd_launch_count(batch, T, H, P, G, N, Q, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load().ssd_fwd_launch_count(batch, T, H, P, G, N, Q, code))
+
+
+def ssd_fwd_stage_names(batch, T, H, P, G, N, Q, dtype) -> list:
+    """Names of the kernels ssd_fwd launches for this problem, in launch order."""
+    code = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    lib = load()
+    names = []
+    while True:
+        n = lib.ssd_fwd_stage_name(batch, T, H, P, G, N, Q, code, len(names))
+        if n is None:
+            return names
+        names.append(n.decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def ssd_fwd(x, dt, A, B, C, D, Q: int, init_state=None, *, y=None, final_state=None,
+            return_final_state: bool = True, workspace=None, stream=None, stage_ms=None):
+    """SSD layer forward on the GPU.
+
+    x [b,T,H,P], B/C [b,T,G,N] (fp32 or bf16, same dtype), dt [b,T,H], A [H],
+    D [H], init_state [b,H,P,N] (fp32 or None) -- contiguous CUDA tensors on
+    one device.  Returns ``(y, final_state)``; y has x's dtype, final_state is
+    fp32 (None when ``return_final_state`` is False and no buffer is given).
+    Runs on ``stream`` (default: the current torch stream) without host sync.
+    With ``stage_ms`` (a list) the call goes through ``ssd_fwd_timed`` instead:
+    it waits for the stream and appends each kernel's milliseconds, then the
+    whole call's span, to the list.
+    """
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_fwd needs CUDA tensors (there is no CPU path)")
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code = _dtype_code(x.dtype)
+    named = dict(x=x, dt=dt, A=A, B=B, C=C, D=D)
+    if init_state is not None:
+        named["init_state"] = init_state
+    for k, t in named.items():
+        if t.device != dev:
+            raise ValueError(f"{k} is on {t.device}, x on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{k} must be contiguous")
+    if B.dtype != x.dtype or C.dtype != x.dtype:
+        raise TypeError("x, B and C must share one dtype")
+    for k in ("dt", "A", "D") + (("init_state",) if init_state is not None else ()):
+        if named[k].dtype != torch.float32:
+            raise TypeError(f"{k} must be float32")
+    if tuple(dt.shape) != (b, T, H) or tuple(A.shape) != (H,) or tuple(D.shape) != (H,):
+        raise ValueError("dt must be [b,T,H]; A and D must be [H]")
+    if tuple(B.shape) != (b, T, G, N) or tuple(C.shape) != (b, T, G, N):
+        raise ValueError("B and C must be [b,T,G,N]")
+    if init_state is not None and tuple(init_state.shape) != (b, H, P, N):
+        raise ValueError("init_state must be [b,H,P,N]")
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    lib = load()
+    need = int(lib.ssd_fwd_workspace_bytes(b, T, H, P, G, N, int(Q), code))
+    if need == 0:
+        raise SSDError(1, "ssd_fwd_workspace_bytes")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    args = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(Q), _ptr(init_state),
+            _ptr(y), _ptr(final_state), b, T, H, P, G, N, code, _ptr(workspace),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size()), ctypes.c_void_p(handle))
+    if stage_ms is None:
+        rc = lib.ssd_fwd(*args)
+        if rc != 0:
+            raise SSDError(rc, "ssd_fwd")
+    else:
+        ms = (ctypes.c_float * 8)()
+        total = ctypes.c_float(0)
+        rc = lib.ssd_fwd_timed(*args, ctypes.cast(ms, ctypes.c_void_p), 8,
+                               ctypes.cast(ctypes.pointer(total), ctypes.c_void_p))
+        if rc != 0:
+            raise SSDError(rc, "ssd_fwd_timed")
+        k = int(lib.ssd_fwd_launch_count(b, T, H, P, G, N, int(Q), code))
+        stage_ms.extend(float(ms[i]) for i in range(min(k, 8)))
+        stage_ms.append(float(total.value))
+    return y, final_state
+
+
+def ssd_fwd_check(workspace, stream=None) -> int:
+    """Wait for the stream and return the device-side status word of the last call."""
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return int(load().ssd_fwd_check(_ptr(workspace), ctypes.c_void_p(handle)))

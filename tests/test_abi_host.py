@@ -1,0 +1,97 @@
+"""Host-side checks of libssd.so: it loads, exports what include/ssd.h declares,
+and rejects bad arguments before touching the GPU.
+
+No test here launches anything: every ssd_fwd call below fails argument
+validation, which runs on the host before the first CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from structured_state_space_ssd_b200 import ssd
+from structured_state_space_ssd_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return ssd.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SSD_API\s+[\w\s\*]*?\b(ssd_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(ssd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.lib_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(ssd_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    # nothing but the declared API leaks out
+    assert exported == set(_declared())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ssd_version() >= 100
+    for code in range(5):
+        assert ssd.status_string(code)
+    assert ssd.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    f = lib.ssd_fwd_workspace_bytes
+    w = f(4, 2048, 80, 64, 1, 128, 256, 1)
+    assert w % 256 == 0
+    nc = 8
+    assert w >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
+    assert f(0, 2048, 80, 64, 1, 128, 256, 1) == 0      # batch < 1
+    assert f(4, 2048, 80, 64, 3, 128, 256, 1) == 0      # H % G != 0
+    assert f(4, 2048, 80, 64, 1, 128, 256, 7) == 0      # bad dtype
+    assert f(4, 2048, 80, 256, 1, 128, 256, 1) == 0     # P above the limit
+    assert f(1, 0, 2, 16, 1, 16, 64, 0) > 0             # empty sequence is valid
+
+
+def test_launch_count(lib):
+    assert lib.ssd_fwd_launch_count(4, 2048, 80, 64, 1, 128, 256, 1) >= 1
+    assert lib.ssd_fwd_launch_count(1, 0, 2, 16, 1, 16, 64, 0) == 0
+    assert lib.ssd_fwd_launch_count(1, 10, 3, 16, 2, 16, 64, 0) == 0
+
+
+def _call(lib, **over):
+    """ssd_fwd with fake (never dereferenced) pointers; only validation runs."""
+    args = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, Q=64, init=None,
+                y=0x70000, fin=None, batch=1, T=256, H=2, P=16, G=1, N=16, dtype=0, ws=0x80000, wsb=0,
+                stream=None)
+    args.update(over)
+    v = lambda a: None if a is None else ctypes.c_void_p(a)  # noqa: E731
+    return lib.ssd_fwd(v(args["x"]), v(args["dt"]), v(args["A"]), v(args["B"]), v(args["C"]), v(args["D"]),
+                       args["Q"], v(args["init"]), v(args["y"]), v(args["fin"]), args["batch"], args["T"],
+                       args["H"], args["P"], args["G"], args["N"], args["dtype"], v(args["ws"]),
+                       ctypes.c_size_t(args["wsb"]), v(args["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(x=None), 1), (dict(dt=None), 1), (dict(A=None), 1), (dict(B=None), 1), (dict(C=None), 1),
+    (dict(D=None), 1), (dict(y=None), 1), (dict(ws=None), 1),
+    (dict(batch=0), 1), (dict(T=-1), 1), (dict(H=0), 1), (dict(P=0), 1), (dict(N=0), 1), (dict(Q=0), 1),
+    (dict(G=0), 1), (dict(H=3, G=2), 1), (dict(dtype=5), 1),
+    (dict(P=129), 2), (dict(N=257), 2), (dict(Q=257), 2),
+    (dict(x=0x10002), 1),                 # fp32 tensor not 4-byte aligned
+    (dict(ws=0x80010), 1),                # workspace not 256-byte aligned
+    (dict(wsb=16), 1),                    # workspace too small
+    (dict(y=0x10000, wsb=1 << 30), 1),    # y aliases x
+])
+def test_invalid_arguments_are_rejected_on_the_host(lib, over, code):
+    assert _call(lib, **over) == code

@@ -1,0 +1,171 @@
+"""GPU parity: libssd.so (through its C ABI) against the fp64 CPU oracle.
+
+Small shapes are compared element by element on every output; the full
+workloads are compared on sampled (batch, head) sequences, which the oracle
+computes one by one (every token and channel of those sequences, plus their
+final states).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close, metrics
+from structured_state_space_ssd_b200 import WORKLOADS, make_inputs, workload_inputs
+from structured_state_space_ssd_b200.ssd import ssd_fwd, ssd_fwd_check
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(inp, Q, dev):
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    y, fin = ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], Q, d["init_state"])
+    torch.cuda.synchronize(dev)
+    return y.float().cpu().numpy(), fin.cpu().numpy()
+
+
+def _oracle(inp, pairs=None):
+    return oracle.ssd_ref_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                              init_state=inp["init_state"], pairs=pairs)
+
+
+SMALL = [
+    # batch, T, H, P, N, G, Q, dtype, init
+    (1, 256, 2, 16, 16, 1, 64, "f32", False),     # the tiny fp32 workload's shape
+    (2, 100, 4, 16, 16, 2, 64, "f32", True),      # ragged last chunk, grouped heads, initial state
+    (1, 37, 2, 8, 8, 1, 1, "f32", True),          # Q = 1: the pure recurrence
+    (1, 96, 3, 5, 7, 1, 96, "f32", False),        # one chunk, odd P and N
+    (1, 1, 2, 4, 4, 2, 16, "f32", True),          # a single token
+    (1, 1000, 2, 16, 16, 1, 16, "f32", True),     # 63 chunks for the state recurrence
+    (1, 300, 2, 128, 256, 1, 256, "f32", True),   # largest P, N and Q, ragged
+    (2, 200, 4, 1, 1, 4, 32, "f32", False),       # P = N = 1, G = H
+    (2, 333, 4, 64, 128, 2, 128, "bf16", True),   # bf16, ragged, grouped
+    (1, 512, 8, 64, 64, 1, 256, "bf16", False),
+    (1, 700, 6, 64, 16, 3, 256, "bf16", True),    # small N, ragged
+    (1, 256, 2, 64, 256, 1, 64, "bf16", False),   # largest N in bf16
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "b{}_T{}_H{}_P{}_N{}_G{}_Q{}_{}_{}".format(*c))
+def test_small_shapes_match_oracle(case, cuda_device):
+    batch, T, H, P, N, G, Q, dtype, init = case
+    inp = make_inputs(batch, T, H, P, N, G, dtype, seed=100 + SMALL.index(case), with_init=init)
+    y, fin = _gpu(inp, Q, cuda_device)
+    y_ref, fin_ref = _oracle(inp)
+    assert_close(y, y_ref, dtype, "y")
+    assert_close(fin, fin_ref, dtype, "final_state")
+
+
+@pytest.mark.parametrize("mode", ["A_zero", "zero_decay", "steep_decay"])
+def test_special_decays_match_oracle(mode, cuda_device):
+    inp = make_inputs(2, 300, 4, 32, 32, 2, "f32", seed=5, with_init=True)
+    if mode == "A_zero":           # no decay: causal linear attention
+        inp["A"] = torch.zeros_like(inp["A"])
+    elif mode == "zero_decay":     # exp underflows to 0: only the diagonal term is left
+        inp["A"] = torch.full_like(inp["A"], -1e8)
+    else:                          # log-decays far below the fp32 exp range inside one chunk
+        inp["dt"] = inp["dt"] * 300
+    y, fin = _gpu(inp, 64, cuda_device)
+    y_ref, fin_ref = _oracle(inp)
+    assert_close(y, y_ref, "f32", "y")
+    assert_close(fin, fin_ref, "f32", "final_state")
+
+
+def test_empty_sequence_copies_initial_state(cuda_device):
+    inp = make_inputs(2, 0, 2, 8, 8, 1, "f32", seed=1, with_init=True)
+    y, fin = _gpu(inp, 64, cuda_device)
+    assert y.shape == (2, 0, 2, 8)
+    np.testing.assert_array_equal(fin, inp["init_state"].numpy())
+    inp["init_state"] = None
+    _, fin = _gpu(inp, 64, cuda_device)
+    assert (fin == 0).all()
+
+
+@pytest.mark.parametrize("dtype,split", [("f32", 128), ("f32", 77), ("bf16", 256), ("bf16", 301)])
+def test_sequence_continuation_on_gpu(dtype, split, cuda_device):
+    """[0, s) then [s, T) seeded with the first final state equals one run."""
+    inp = make_inputs(1, 600, 4, 64, 64, 1, dtype, seed=9, with_init=True)
+    y, fin = _gpu(inp, 128, cuda_device)
+    first = {k: (v[:, :split].contiguous() if k in ("x", "dt", "B", "C") else v) for k, v in inp.items()}
+    second = {k: (v[:, split:].contiguous() if k in ("x", "dt", "B", "C") else v) for k, v in inp.items()}
+    ya, fa = _gpu(first, 128, cuda_device)
+    second["init_state"] = torch.from_numpy(fa)
+    yb, fb = _gpu(second, 128, cuda_device)
+    assert_close(np.concatenate([ya, yb], axis=1), y, dtype, "y")
+    assert_close(fb, fin, dtype, "final_state")
+
+
+@pytest.mark.parametrize("Q", [16, 64, 128, 256])
+def test_chunk_size_does_not_change_the_function(Q, cuda_device):
+    inp = make_inputs(1, 512, 4, 64, 128, 1, "bf16", seed=13, with_init=True)
+    y, fin = _gpu(inp, Q, cuda_device)
+    y_ref, fin_ref = _oracle(inp)
+    assert_close(y, y_ref, "bf16", f"y Q={Q}")
+    assert_close(fin, fin_ref, "bf16", f"final_state Q={Q}")
+
+
+def test_repeated_runs_are_bitwise_identical(cuda_device):
+    w = WORKLOADS["mamba2_2p7b_layer"]
+    inp = workload_inputs(w)
+    y1, f1 = _gpu(inp, w.Q, cuda_device)
+    y2, f2 = _gpu(inp, w.Q, cuda_device)
+    assert np.array_equal(y1, y2) and np.array_equal(f1, f2)
+
+
+def _sample_pairs(w, k):
+    rng = np.random.default_rng(w.seed)
+    pairs = {(0, 0), (w.batch - 1, w.H - 1)}
+    while len(pairs) < min(k, w.batch * w.H):
+        pairs.add((int(rng.integers(w.batch)), int(rng.integers(w.H))))
+    return sorted(pairs)
+
+
+def _fold_pairs(inp, w, pairs):
+    """The sampled (batch, head) sequences as one oracle problem: batch 1, one head and one group each.
+
+    Head i of the folded problem is sequence (b_i, h_i) with its own A, D, dt,
+    initial state and its group's B/C, so the oracle's result for it is exactly
+    that sequence's result in the full problem.
+    """
+    hpg = w.H // w.G
+    bs = [p[0] for p in pairs]
+    hs = [p[1] for p in pairs]
+    gs = [h // hpg for h in hs]
+    fold = {
+        "x": torch.stack([inp["x"][b, :, h] for b, h in pairs], dim=1)[None],
+        "dt": torch.stack([inp["dt"][b, :, h] for b, h in pairs], dim=1)[None],
+        "A": inp["A"][hs], "D": inp["D"][hs],
+        "B": torch.stack([inp["B"][b, :, g] for b, g in zip(bs, gs)], dim=1)[None],
+        "C": torch.stack([inp["C"][b, :, g] for b, g in zip(bs, gs)], dim=1)[None],
+        "init_state": None if inp["init_state"] is None else
+        torch.stack([inp["init_state"][b, h] for b, h in pairs])[None],
+    }
+    return fold
+
+
+@pytest.mark.parametrize("name", [n for n in WORKLOADS])
+def test_workload_matches_oracle_on_sampled_heads(name, cuda_device):
+    w = WORKLOADS[name]
+    inp = workload_inputs(w)
+    d = {k: (v.to(cuda_device) if v is not None else None) for k, v in inp.items()}
+    y, fin = ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], w.Q, d["init_state"])
+    torch.cuda.synchronize(cuda_device)
+    # every output is finite, not only the sampled ones
+    assert bool(torch.isfinite(y).all()) and bool(torch.isfinite(fin).all())
+    pairs = _sample_pairs(w, 6 if w.T > 8192 else 8)
+    got_y = torch.stack([y[b, :, h] for b, h in pairs], dim=1).float().cpu().numpy()
+    got_f = torch.stack([fin[b, h] for b, h in pairs]).cpu().numpy()
+    del y, fin, d
+    y_ref, fin_ref = _oracle(_fold_pairs(inp, w, pairs))
+    assert_close(got_y, y_ref[0], w.dtype, f"{name} y")
+    assert_close(got_f, fin_ref[0], w.dtype, f"{name} final_state")
+
+
+def test_status_word_is_clear_after_a_run(cuda_device):
+    inp = make_inputs(1, 256, 2, 16, 16, 1, "f32", seed=3)
+    d = {k: (v.to(cuda_device) if v is not None else None) for k, v in inp.items()}
+    from structured_state_space_ssd_b200.ssd import ssd_fwd_workspace_bytes
+    ws = torch.zeros(ssd_fwd_workspace_bytes(1, 256, 2, 16, 1, 16, 64, torch.float32), dtype=torch.uint8,
+                     device=cuda_device)
+    ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], 64, None, workspace=ws)
+    assert ssd_fwd_check(ws) == 0
