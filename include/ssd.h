@@ -86,7 +86,8 @@ SSD_API size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, in
  * Limits: batch, H, G, P, N, Q >= 1, T >= 0, H % G == 0, P <= 128, N <= 256,
  * Q <= 256.  Pointers must be aligned to their element size (16 bytes for
  * the bf16 tensor-core path).  y must not alias any input.  T == 0 writes
- * final_state = init_state (or zero) and nothing else.
+ * final_state = init_state (or zero) and nothing else; x, dt, B, C and y are
+ * not read then and may be NULL.
  *
  * Returns SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
  * Device-side failures of bounded waits are reported by ssd_fwd_check.

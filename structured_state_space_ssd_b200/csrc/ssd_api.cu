@@ -91,7 +91,8 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     Shape sh;
     int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
     if (rc != SSD_OK) return rc;
-    if (!x || !dt || !A || !B || !C || !D || !y || !workspace) return SSD_ERR_INVALID_ARG;
+    // Per-token tensors are empty when T == 0 and may then be NULL.
+    if ((T > 0 && (!x || !dt || !B || !C || !y)) || !A || !D || !workspace) return SSD_ERR_INVALID_ARG;
     const size_t es = (dtype == SSD_BF16) ? 2 : 4;
     if (!aligned(x, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es) || !aligned(dt, 4) ||
         !aligned(A, 4) || !aligned(D, 4) || !aligned(workspace, 256) || (init_state && !aligned(init_state, 4)) ||

@@ -19,7 +19,7 @@ namespace ssd {
 // of the 1-semiseparable mask).  grid (nc, batch), 256 threads; each warp
 // scans one head's chunk: a sequential run over <= 8 elements per lane, then a
 // shuffle scan of the lane totals.  Rows past the end of a short last chunk
-// contribute 0, so s[Q-1] is always the chunk total.
+// copy the last valid row, so s[Q-1] is always the chunk total.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restrict__ dt,
                                                            const float *__restrict__ A,
@@ -59,8 +59,16 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restri
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int i = lane * E + e;
-                if (e < E && i < sh.Q) tile[i * 33 + hh] = loc[e] + excl;
+                if (e < E && i < len) tile[i * 33 + hh] = loc[e] + excl;
             }
+        }
+        __syncthreads();
+        // Rows past a short last chunk repeat the last valid row bit for bit, so
+        // s[Q-1] is exactly s[len-1] and exp(s_end - s_last) is exactly 1 (a
+        // reassociated sum could differ by one ulp, which is 8 at |s| ~ 1e8).
+        for (int idx = threadIdx.x; idx < (sh.Q - len) * 32; idx += blockDim.x) {
+            const int i = len + (idx >> 5), hh = idx & 31;
+            tile[i * 33 + hh] = tile[(len - 1) * 33 + hh];
         }
         __syncthreads();
         for (int idx = threadIdx.x; idx < hn * sh.Q; idx += blockDim.x) {
