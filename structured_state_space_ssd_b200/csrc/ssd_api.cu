@@ -3,6 +3,8 @@
 // block-decomposition stages on the caller's stream.
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "ssd_common.cuh"
 
 namespace ssd {
@@ -14,6 +16,10 @@ cudaError_t launch_state_passing(float *S, const float *s, const float *init, fl
 template <typename T>
 cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D, const float *s,
                               const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
+bool tc_scan_supported(const Shape &sh, int dtype, const void *x, const void *B, const void *C, const void *y);
+cudaError_t launch_chunk_scan_tc(const __nv_bfloat16 *x, const __nv_bfloat16 *B, const __nv_bfloat16 *C,
+                                 const float *D, const float *s, const float *Sprev, __nv_bfloat16 *y, int *status,
+                                 const Shape &sh, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -54,6 +60,17 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 const char *const kStageNames[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
                                    "ssd_chunk_scan"};
+const char *const kStageNamesTc[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
+                                     "ssd_chunk_scan_tc"};
+
+// Which chunk-scan kernel a call uses: the tensor-core one for bf16 with P = 64,
+// N in {64, 128}, Q in {128, 256} and 16-byte aligned x/B/C/y; the CUDA-core one
+// otherwise.  Pointers may be null when only the shape is known (then the
+// alignment test is assumed to pass).
+bool use_tc(const Shape &sh, int dtype, const void *x, const void *B, const void *C, const void *y) {
+    const void *a = reinterpret_cast<const void *>(uintptr_t(256));
+    return ssd::tc_scan_supported(sh, dtype, x ? x : a, B ? B : a, C ? C : a, y ? y : a);
+}
 constexpr int kMaxStages = 8;
 
 // Optional per-kernel event marks: ev[0] before the first kernel, ev[k+1] after kernel k.
@@ -78,8 +95,16 @@ int run_path(const Shape &sh, const T *x, const float *dt, const float *A, const
         return SSD_ERR_CUDA;
     if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || mk.mark(3, st) != cudaSuccess)
         return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || mk.mark(4, st) != cudaSuccess)
-        return SSD_ERR_CUDA;
+    cudaError_t e;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (use_tc(sh, SSD_BF16, x, B, C, y))
+            e = ssd::launch_chunk_scan_tc(x, B, C, D, s, S, y, reinterpret_cast<int *>(ws + w.status_off), sh, st);
+        else
+            e = ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st);
+    } else {
+        e = ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st);
+    }
+    if (e != cudaSuccess || mk.mark(4, st) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
 
@@ -146,7 +171,7 @@ const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int
     Shape sh;
     if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return nullptr;
     if (i < 0 || i >= launch_count(sh)) return nullptr;
-    return kStageNames[i];
+    return use_tc(sh, dtype, nullptr, nullptr, nullptr, nullptr) ? kStageNamesTc[i] : kStageNames[i];
 }
 
 int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
