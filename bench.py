@@ -81,7 +81,10 @@ def algorithmic(w):
               + state * (2 if w.with_init else 1))
     per_chunk = 2 * Q * Q * N * G + 2 * Q * Q * P * H + 4 * Q * N * P * H + 2 * N * P * H
     flops = b * nc * per_chunk
+    # the fused kernel reads the prefix sums s in place of dt: same size per token
+    fused_bytes = bytes_ - 4 * b * T * H + 4 * b * H * nc * Q
     stages = {
+        "ssd_fused": ("pass", (fused_bytes, flops)),
         "ssd_chunk_cumsum": ("hbm", 4 * b * T * H + 4 * H + 4 * b * H * nc * Q),
         "ssd_chunk_state": ("flop", b * nc * 2 * Q * N * P * H),
         "ssd_state_passing": ("hbm", 2 * 4 * b * nc * H * P * N + state * (2 if w.with_init else 1)),
@@ -323,11 +326,21 @@ def main():
         dom = max(stage_avg, key=stage_avg.get)
         kind, amount = stages[dom]
         dom_ms = stage_avg[dom]
+        both = None
+        if kind == "pass":
+            # bytes and FLOPs both matter: the bound is the slower of the two at peak
+            fb, ff = amount
+            t_mem, t_tc = fb / (peaks["hbm_gbs"] * 1e9), ff / (peaks["bf16_tflops"] * 1e12)
+            both = {"hbm_GBps": fb / (dom_ms * 1e-3) / 1e9, "hbm_frac": fb / (dom_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "tensor_TFLOPs": ff / (dom_ms * 1e-3) / 1e12,
+                    "tensor_frac": ff / (dom_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                    "alg_bytes": fb, "alg_flops": ff}
+            kind, amount = ("hbm", fb) if t_mem >= t_tc else ("tensor", ff)
         if kind == "hbm":
             roof = {"bound": "hbm", "achieved": amount / (dom_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s"}
         else:
-            tc = _stage_uses_tensor_cores(dom, w)
+            tc = _stage_uses_tensor_cores(dom, w) or both is not None
             if tc:
                 roof = {"bound": "tensor", "achieved": amount / (dom_ms * 1e-3) / 1e12,
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
@@ -338,6 +351,8 @@ def main():
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["traffic"] = _traffic_from_profiles(dom, w)
         roof["kernel"] = dom
+        if both is not None:
+            roof["both"] = both
         roof["peak_source"] = f"{peak_src} (burst)" if roof["bound"] != "alu" else \
             "derived: 148 SMs x 128 fp32 FMA/clk x 2 x max SM clock"
         t_roof = max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flops / (peaks["bf16_tflops"] * 1e12))

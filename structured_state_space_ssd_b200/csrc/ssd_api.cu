@@ -1,9 +1,7 @@
 // ssd_api.cu -- the extern "C" boundary of libssd.so (declared in include/ssd.h):
-// argument validation, workspace carving and the launch sequence of the
-// block-decomposition stages on the caller's stream.
+// argument validation, choice of launch sequence, workspace carving and the
+// launches on the caller's stream.
 #include <stdint.h>
-
-#include <type_traits>
 
 #include "ssd_common.cuh"
 
@@ -16,19 +14,21 @@ cudaError_t launch_state_passing(float *S, const float *s, const float *init, fl
 template <typename T>
 cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D, const float *s,
                               const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
-bool tc_scan_supported(const Shape &sh, int dtype, const void *x, const void *B, const void *C, const void *y);
-cudaError_t launch_chunk_scan_tc(const __nv_bfloat16 *x, const __nv_bfloat16 *B, const __nv_bfloat16 *C,
-                                 const float *D, const float *s, const float *Sprev, __nv_bfloat16 *y, int *status,
-                                 const Shape &sh, cudaStream_t st);
+bool fused_supported(const Shape &sh, int dtype);
+cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, const __nv_bfloat16 *C,
+                             const float *D, const float *s, const float *init, float *fin, float *ring, int *ready,
+                             int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
+                             cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
 constexpr int kMaxP = 128, kMaxN = 256, kMaxQ = 256;
 constexpr int64_t kMaxElems = int64_t(1) << 46;
+constexpr int kMaxStages = 8;
 
 // Validates the dimensions; fills `sh` on success.
 int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, Shape *sh) {
@@ -51,6 +51,10 @@ int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, S
     return SSD_OK;
 }
 
+ssd::Path choose_path(const Shape &sh, int dtype) {
+    return ssd::fused_supported(sh, dtype) ? ssd::kPathFused : ssd::kPathSimt;
+}
+
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -58,57 +62,50 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-const char *const kStageNames[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
-                                   "ssd_chunk_scan"};
-const char *const kStageNamesTc[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing",
-                                     "ssd_chunk_scan_tc"};
+const char *const kSimtStages[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan"};
+const char *const kFusedStages[] = {"ssd_chunk_cumsum", "ssd_fused"};
 
-// Which chunk-scan kernel a call uses: the tensor-core one for bf16 with P = 64,
-// N in {64, 128}, Q in {128, 256} and 16-byte aligned x/B/C/y; the CUDA-core one
-// otherwise.  Pointers may be null when only the shape is known (then the
-// alignment test is assumed to pass).
-bool use_tc(const Shape &sh, int dtype, const void *x, const void *B, const void *C, const void *y) {
-    const void *a = reinterpret_cast<const void *>(uintptr_t(256));
-    return ssd::tc_scan_supported(sh, dtype, x ? x : a, B ? B : a, C ? C : a, y ? y : a);
+int launch_count(const Shape &sh, ssd::Path path) {
+    if (sh.T == 0) return 0;
+    return path == ssd::kPathFused ? 2 : 4;
 }
-constexpr int kMaxStages = 8;
 
 // Optional per-kernel event marks: ev[0] before the first kernel, ev[k+1] after kernel k.
 struct Marks {
     cudaEvent_t *ev = nullptr;
     int n = 0;
-    cudaError_t mark(int i, cudaStream_t st) const {
-        return (ev && i < n) ? cudaEventRecord(ev[i], st) : cudaSuccess;
-    }
+    bool mark(int i, cudaStream_t st) const { return !(ev && i < n) || cudaEventRecord(ev[i], st) == cudaSuccess; }
 };
 
 template <typename T>
-int run_path(const Shape &sh, const T *x, const float *dt, const float *A, const T *B, const T *C,
-             const float *D, const float *init, T *y, float *fin, char *ws, cudaStream_t st, const Marks &mk) {
-    const ssd::Workspace w = ssd::workspace_layout(sh);
+int run_simt(const Shape &sh, const T *x, const float *dt, const float *A, const T *B, const T *C, const float *D,
+             const float *init, T *y, float *fin, char *ws, const ssd::Workspace &w, cudaStream_t st,
+             const Marks &mk) {
     float *s = reinterpret_cast<float *>(ws + w.s_off);
     float *S = reinterpret_cast<float *>(ws + w.state_off);
-    if (mk.mark(0, st) != cudaSuccess) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || mk.mark(1, st) != cudaSuccess)
+    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(1, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st) != cudaSuccess || !mk.mark(2, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || !mk.mark(3, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || !mk.mark(4, st))
         return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st) != cudaSuccess || mk.mark(2, st) != cudaSuccess)
-        return SSD_ERR_CUDA;
-    if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || mk.mark(3, st) != cudaSuccess)
-        return SSD_ERR_CUDA;
-    cudaError_t e;
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        if (use_tc(sh, SSD_BF16, x, B, C, y))
-            e = ssd::launch_chunk_scan_tc(x, B, C, D, s, S, y, reinterpret_cast<int *>(ws + w.status_off), sh, st);
-        else
-            e = ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st);
-    } else {
-        e = ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st);
-    }
-    if (e != cudaSuccess || mk.mark(4, st) != cudaSuccess) return SSD_ERR_CUDA;
     return SSD_OK;
 }
 
-int launch_count(const Shape &sh) { return sh.T == 0 ? 0 : 4; }
+int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
+              const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
+              const ssd::Workspace &w, cudaStream_t st, const Marks &mk) {
+    float *s = reinterpret_cast<float *>(ws + w.s_off);
+    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(1, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_ssd_fused(x, B, C, D, s, init, fin, reinterpret_cast<float *>(ws + w.ring_off),
+                              reinterpret_cast<int *>(ws + w.ready_off), reinterpret_cast<int *>(ws + w.cons_off),
+                              reinterpret_cast<int *>(ws + w.counter_off), reinterpret_cast<int *>(ws + w.status_off),
+                              y, sh, st) != cudaSuccess ||
+        !mk.mark(2, st))
+        return SSD_ERR_CUDA;
+    return SSD_OK;
+}
 
 int fwd_impl(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
              const float *init_state, void *y, float *final_state, int batch, int T, int H, int P, int G, int N,
@@ -118,12 +115,14 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     if (rc != SSD_OK) return rc;
     // Per-token tensors are empty when T == 0 and may then be NULL.
     if ((T > 0 && (!x || !dt || !B || !C || !y)) || !A || !D || !workspace) return SSD_ERR_INVALID_ARG;
+    const ssd::Path path = choose_path(sh, dtype);
     const size_t es = (dtype == SSD_BF16) ? 2 : 4;
-    if (!aligned(x, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es) || !aligned(dt, 4) ||
-        !aligned(A, 4) || !aligned(D, 4) || !aligned(workspace, 256) || (init_state && !aligned(init_state, 4)) ||
-        (final_state && !aligned(final_state, 4)))
+    const size_t ea = (path == ssd::kPathFused) ? 16 : es;  // TMA tiles need 16-byte aligned bases
+    if (!aligned(x, ea) || !aligned(B, ea) || !aligned(C, ea) || !aligned(y, ea) || !aligned(dt, 4) ||
+        !aligned(A, 4) || !aligned(D, 4) || !aligned(workspace, 256) || (init_state && !aligned(init_state, 16)) ||
+        (final_state && !aligned(final_state, 16)))
         return SSD_ERR_INVALID_ARG;
-    const ssd::Workspace w = ssd::workspace_layout(sh);
+    const ssd::Workspace w = ssd::workspace_layout(sh, path);
     if (workspace_bytes < w.total) return SSD_ERR_INVALID_ARG;
     const size_t ybytes = es * (size_t)batch * T * H * P;
     const size_t bcbytes = es * (size_t)batch * T * G * N;
@@ -133,22 +132,26 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
-    if (cudaMemsetAsync(ws + w.status_off, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, w.clear_bytes, st) != cudaSuccess) return SSD_ERR_CUDA;
     if (T == 0) {
-        if (mk.mark(0, st) != cudaSuccess) return SSD_ERR_CUDA;
+        if (!mk.mark(0, st)) return SSD_ERR_CUDA;
         if (!final_state) return SSD_OK;
         const size_t fb = sizeof(float) * (size_t)batch * H * P * N;
         cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, fb, cudaMemcpyDeviceToDevice, st)
                                    : cudaMemsetAsync(final_state, 0, fb, st);
         return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
     }
+    if (path == ssd::kPathFused)
+        return run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+                         static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
+                         final_state, ws, w, st, mk);
     if (dtype == SSD_BF16)
-        return run_path<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
+        return run_simt<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
                                        static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C),
-                                       D, init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, st, mk);
-    return run_path<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
+                                       D, init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, w, st, mk);
+    return run_simt<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
                            static_cast<const float *>(C), D, init_state, static_cast<float *>(y), final_state, ws,
-                           st, mk);
+                           w, st, mk);
 }
 
 }  // namespace
@@ -158,20 +161,21 @@ extern "C" {
 size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
     Shape sh;
     if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
-    return ssd::workspace_layout(sh).total;
+    return ssd::workspace_layout(sh, choose_path(sh, dtype)).total;
 }
 
 int ssd_fwd_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
     Shape sh;
     if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
-    return launch_count(sh);
+    return launch_count(sh, choose_path(sh, dtype));
 }
 
 const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int Q, int dtype, int i) {
     Shape sh;
     if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return nullptr;
-    if (i < 0 || i >= launch_count(sh)) return nullptr;
-    return use_tc(sh, dtype, nullptr, nullptr, nullptr, nullptr) ? kStageNamesTc[i] : kStageNames[i];
+    const ssd::Path path = choose_path(sh, dtype);
+    if (i < 0 || i >= launch_count(sh, path)) return nullptr;
+    return path == ssd::kPathFused ? kFusedStages[i] : kSimtStages[i];
 }
 
 int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
@@ -197,7 +201,7 @@ int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B,
     Shape sh;
     int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
     if (rc != SSD_OK) return rc;
-    const int k = launch_count(sh);
+    const int k = launch_count(sh, choose_path(sh, dtype));
     Marks mk;
     mk.ev = events;
     mk.n = k + 1;

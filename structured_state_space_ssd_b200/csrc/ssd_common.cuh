@@ -25,25 +25,47 @@ struct Shape {
     int heads_per_group;  // H / G
 };
 
+// The two launch sequences: stage-per-kernel on CUDA cores (any shape and
+// dtype within the limits) or the fused tensor-core kernel (bf16, P = 64,
+// N in {64, 128}, Q in {128, 256}).
+enum Path { kPathSimt = 0, kPathFused = 1 };
+
 // Workspace carve-up, computed identically by ssd_fwd_workspace_bytes and ssd_fwd.
+// The front 256-byte block holds the status word and the unit counter; it and
+// the per-(batch, head) flags after it are cleared by one memset per call.
 struct Workspace {
-    size_t status_off;  // int status word (+ padding)
+    size_t status_off;  // int status word
+    size_t counter_off; // int unit counter (fused path)
+    size_t ready_off;   // int ready[batch * H] (fused path)
+    size_t cons_off;    // int cons[batch * H] (fused path)
+    size_t clear_bytes; // bytes from offset 0 cleared per call
     size_t s_off;       // float s[batch][H][nc][Q]: inclusive log-decay prefix sums per chunk
-    size_t state_off;   // float S[batch][nc][H][P][N]: chunk states, then the state entering each chunk
+    size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
+    size_t ring_off;    // fused path: float ring[batch][H][2][P][N], outgoing states of the last two chunks
     size_t total;
 };
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline Workspace workspace_layout(const Shape &s) {
+inline Workspace workspace_layout(const Shape &s, Path path) {
     Workspace w;
-    size_t off = 0;
-    w.status_off = off;
-    off = align256(off + 256);
+    const size_t bh = (size_t)s.batch * s.H;
+    w.status_off = 0;
+    w.counter_off = 4;
+    size_t off = 256;
+    w.ready_off = off;
+    off += sizeof(int) * bh;
+    w.cons_off = off;
+    off += sizeof(int) * bh;
+    off = align256(off);
+    w.clear_bytes = (path == kPathFused) ? off : 256;
     w.s_off = off;
-    off = align256(off + sizeof(float) * (size_t)s.batch * s.H * s.nc * s.Q);
-    w.state_off = off;
-    off = align256(off + sizeof(float) * (size_t)s.batch * s.nc * s.H * s.P * s.N);
+    off = align256(off + sizeof(float) * bh * s.nc * s.Q);
+    w.state_off = w.ring_off = off;
+    if (path == kPathFused)
+        off = align256(off + sizeof(float) * bh * 2 * s.P * s.N);
+    else
+        off = align256(off + sizeof(float) * (size_t)s.batch * s.nc * s.H * s.P * s.N);
     w.total = off;
     return w;
 }

@@ -16,8 +16,9 @@ namespace ssd {
 
 // ---------------------------------------------------------------------------
 // Per-chunk inclusive prefix sums of dt*A (stage 0 partition + the exponents
-// of the 1-semiseparable mask).  grid (nc, batch), 256 threads; each warp
-// scans one head's chunk: a sequential run over <= 8 elements per lane, then a
+// of the 1-semiseparable mask).  grid (nc, batch, ceil(H/32)), 256 threads: a
+// block stages the [Q x 32] tile of dt for its heads with coalesced loads,
+// then each warp scans one head's chunk: a sequential run over <= 8 elements per lane, then a
 // shuffle scan of the lane totals.  Rows past the end of a short last chunk
 // copy the last valid row, so s[Q-1] is always the chunk total.
 // ---------------------------------------------------------------------------
@@ -30,7 +31,8 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restri
     const int len = min(sh.Q, sh.T - t0);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const int E = (sh.Q + 31) >> 5;
-    for (int h0 = 0; h0 < sh.H; h0 += 32) {
+    {
+        const int h0 = blockIdx.z * 32;
         const int hn = min(32, sh.H - h0);
         for (int idx = threadIdx.x; idx < sh.Q * 32; idx += blockDim.x) {
             const int i = idx >> 5, hh = idx & 31;
@@ -340,7 +342,7 @@ static int pow2_at_least(int v) {
 
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const Shape &sh, cudaStream_t st) {
     const size_t smem = sizeof(float) * (size_t)sh.Q * 33;
-    chunk_cumsum_kernel<<<dim3(sh.nc, sh.batch), 256, smem, st>>>(dt, A, s, sh);
+    chunk_cumsum_kernel<<<dim3(sh.nc, sh.batch, (sh.H + 31) / 32), 256, smem, st>>>(dt, A, s, sh);
     return cudaGetLastError();
 }
 

@@ -52,10 +52,12 @@ def test_version_and_status_strings(lib):
 
 def test_workspace_bytes(lib):
     f = lib.ssd_fwd_workspace_bytes
-    w = f(4, 2048, 80, 64, 1, 128, 256, 1)
+    w = f(4, 2048, 80, 64, 1, 128, 256, 1)      # fused tensor-core path: prefix sums + state ring
     assert w % 256 == 0
     nc = 8
-    assert w >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
+    assert w >= 4 * 80 * nc * 256 * 4 + 4 * 80 * 2 * 64 * 128 * 4
+    w32 = f(4, 2048, 80, 64, 1, 128, 256, 0)    # CUDA-core path: every chunk state
+    assert w32 >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
     assert f(0, 2048, 80, 64, 1, 128, 256, 1) == 0      # batch < 1
     assert f(4, 2048, 80, 64, 3, 128, 256, 1) == 0      # H % G != 0
     assert f(4, 2048, 80, 64, 1, 128, 256, 7) == 0      # bad dtype
