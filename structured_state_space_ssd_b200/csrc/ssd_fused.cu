@@ -28,15 +28,35 @@
 //    previous content are done.  Every wait is bounded: on expiry the status
 //    word is set to SSD_ERR_TIMEOUT and the CTA finishes without waiting.
 //
-// Warp roles: warps 0-7 (two warpgroups, each covering the 128 TMEM lanes) do
-// the CUDA-core work; one lane of warp 8 issues TMA loads and tcgen05.mma.
-// They hand buffers to each other through mbarriers: X tiles and chunk-state
-// accumulators are double-buffered per head, as are the output accumulators,
-// and the decay mask is split in two K-halves so that masking one half
-// overlaps the tensor-core product of the other.
+// Warp roles: each CTA runs two head pipelines side by side.  Pipeline pl
+// takes every other head of a unit; its CUDA-core warpgroup (warps 4pl..4pl+3,
+// covering the 128 TMEM lanes) and its issuer warp (8 + pl; one lane issues
+// TMA loads and tcgen05.mma) hand the pipeline's own X tile, state tile,
+// decay mask (one 128-token K-half at a time) and accumulators back and forth
+// through mbarriers, so that one pipeline's CUDA-core work overlaps the other's
+// tensor-core products.  C, B and G are shared by the unit's heads.
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
+
+// Optional phase timestamps for performance work: compiled in only with
+// -DSSD_TRACE, which also provides ssd_trace_buffer (one 16-slot record per
+// head and pipeline).  Production builds contain no trace code.
+#ifdef SSD_TRACE
+__device__ unsigned long long *ssd_trace_buffer = nullptr;
+#define SSD_TRACE_POINT(ev)                                                                                    \
+    do {                                                                                                       \
+        if (ssd_trace_buffer && wtid == 0 && trace_i < 60) {                                                   \
+            unsigned long long t_;                                                                             \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                           \
+            ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 16 + (ev)] = t_;               \
+        }                                                                                                      \
+    } while (0)
+#else
+#define SSD_TRACE_POINT(ev) \
+    do {                    \
+    } while (0)
+#endif
 
 namespace ssd {
 
@@ -44,29 +64,27 @@ using namespace tc;
 
 namespace fz {
 
-constexpr int kSimtThreads = 256;
-constexpr int kThreads = kSimtThreads + 32;
-constexpr int kIssuerWarp = 8;
-constexpr int kSimtBar = 1;  // named barrier of the CUDA-core warps
+constexpr int kWgThreads = 128;              // one warpgroup: the 128 TMEM lanes
+constexpr int kThreads = 2 * kWgThreads + 64; // warps 0-7: two warpgroups; warps 8-9: issuers
 constexpr int kRows = 128;
 constexpr int kP = 64;
 
-// TMEM columns (512 allocated)
+// TMEM columns (512 allocated).  Pipeline pl owns D[pl], M[pl] and Y[pl].
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColG = 0;    // G: 128 (first half) or 256 (second half) fp32 columns
-constexpr uint32_t kColD = 128;  // first half: chunk-state accumulators D[2], 64 columns each
-constexpr uint32_t kColM = 256;  // decay mask, bf16 pairs: K-half 0 at +0, K-half 1 at +64
-constexpr uint32_t kColY = 384;  // output accumulators Y[2], 64 columns each
+constexpr uint32_t kColD = 128;  // first half only: chunk-state accumulators, 64 columns per pipeline
+constexpr uint32_t kColM = 256;  // decay mask (one 128-token K-half, bf16 pairs), 64 columns per pipeline
+constexpr uint32_t kColY = 384;  // output accumulators, 64 columns per pipeline
 
 // Shared memory (bytes from a 1 KiB-aligned base)
-constexpr uint32_t kOffC = 0;                 // C rows of the half: 2 K-atoms x 128 rows x 128 B
-constexpr uint32_t kOffB = 32768;             // B rows 0..Q-1: 2 K-atoms x 256 rows x 128 B
-constexpr uint32_t kOffX = kOffB + 65536;     // X tiles: 2 buffers x 256 rows x 128 B
-constexpr uint32_t kOffX0 = kOffX + 65536;    // first half: X rows 0..127, undecayed
-constexpr uint32_t kOffS = kOffX0 + 16384;    // S~ as bf16 K-major: 2 buffers x 2 atoms x 64 rows x 128 B
-constexpr uint32_t kOffJ = kOffS + 32768;     // s values: 2 buffers x 256 floats
-constexpr uint32_t kOffF = kOffJ + 2048;      // column factors: 2 buffers x 256 floats
-constexpr uint32_t kSmemBytes = kOffF + 2048 + 1024;
+constexpr uint32_t kOffC = 0;                  // C rows of the half: 2 K-atoms x 128 rows x 128 B
+constexpr uint32_t kOffB = 32768;              // B rows 0..Q-1: 2 K-atoms x 256 rows x 128 B
+constexpr uint32_t kOffX = kOffB + 65536;      // per pipeline: X rows 0..Q-1, 256 rows x 128 B
+constexpr uint32_t kOffS = kOffX + 2 * 32768;  // per pipeline: S~ tile (2 atoms x 64 rows x 128 B), or
+                                               // the decayed X rows 0..127 before the chunk-state product
+constexpr uint32_t kOffJ = kOffS + 2 * 16384;  // per pipeline, 2 buffers: s values (256 floats)
+constexpr uint32_t kOffF = kOffJ + 4 * 1024;   // per pipeline, 2 buffers: column factors (256 floats)
+constexpr uint32_t kSmemBytes = kOffF + 4 * 1024 + 1024;
 
 constexpr uint32_t kBarPolls = 1u << 22;
 constexpr uint32_t kFlagPolls = 1u << 22;
@@ -90,22 +108,30 @@ struct Params {
     int n_units;
 };
 
+// One head pipeline: its issuer warp and its warpgroup.  Barriers signalled
+// once per head of the pipeline are waited with parity (use & 1), `use`
+// counting the pipeline's earlier heads; both sides keep identical counters.
+struct PipeBars {
+    uint64_t x_full;      // X tile landed (TMA)
+    uint64_t x_free;      // products reading the X tile done
+    uint64_t j_full[2];   // s values landed (bulk copy), double-buffered
+    uint64_t xd_full;     // first half: decayed X written (4 warp arrivals)
+    uint64_t d_done;      // first half: chunk-state product done
+    uint64_t s_full;      // S~ tile written (4 warp arrivals)
+    uint64_t inter_done;  // inter-chunk product done
+    uint64_t m_full;      // one mask K-half written (4 warp arrivals)
+    uint64_t m_free;      // product reading it done
+    uint64_t mx_done;     // every product of the head done
+    uint64_t y_free;      // output accumulator drained (4 warp arrivals)
+};
+
 struct Bars {
-    uint64_t cb;             // C and B tiles landed (TMA)
-    uint64_t x_full[2];      // X tile landed (TMA)
-    uint64_t x_free[2];      // last MMA reading an X tile done
-    uint64_t x0_full;        // undecayed X rows 0..127 landed (TMA)
-    uint64_t x0_free;        // MMA reading them done
-    uint64_t xd_full;        // decayed X written (8 warp arrivals); first-half heads only
-    uint64_t d_done;         // chunk-state product done; first-half heads only
-    uint64_t s_full[2];      // S~ tile written (8 warp arrivals)
-    uint64_t inter_done[2];  // inter-chunk product done
-    uint64_t m_full[2];      // mask K-half written (8 warp arrivals)
-    uint64_t m_free[2];      // MMA reading a mask K-half done
-    uint64_t mx_done[2];     // all products of a head done
-    uint64_t y_free[2];      // output accumulator drained (8 warp arrivals)
-    uint64_t unit_full;      // unit id posted (issuer)
-    uint64_t unit_empty;     // unit id read (8 warp arrivals)
+    uint64_t cb;          // C and B tiles landed (TMA)
+    uint64_t g_done;      // G = C B^T in TMEM
+    uint64_t unit_full;   // unit id posted (issuer 0)
+    uint64_t unit_empty;  // unit id read (8 CUDA-core warps + issuer 1)
+    uint64_t unit_done;   // both pipelines finished the unit (2 issuer arrivals)
+    PipeBars pb[2];
 };
 
 struct Unit {
@@ -154,7 +180,7 @@ __device__ __forceinline__ bool wait_flag(const int *flag, int target, volatile 
             *abort = 1;
             return false;
         }
-        __nanosleep(128);
+        __nanosleep(64);
     }
     atomicExch(status, SSD_ERR_TIMEOUT);
     *abort = 1;
@@ -169,16 +195,12 @@ using namespace fz;
 
 __global__ void __launch_bounds__(fz::kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
-                     const __grid_constant__ CUtensorMap mX, const fz::Params p) {
+                     const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY,
+                     const fz::Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint8_t *sC = smem + kOffC;
     uint8_t *sB = smem + kOffB;
-    uint8_t *sX = smem + kOffX;
-    uint8_t *sX0 = smem + kOffX0;
-    uint8_t *sS = smem + kOffS;
-    float *sJ = reinterpret_cast<float *>(smem + kOffJ);
-    float *sF = reinterpret_cast<float *>(smem + kOffF);
     __shared__ Bars bars;
     __shared__ uint32_t tslot;
     __shared__ int s_unit;
@@ -193,15 +215,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     if (tid == 0) {
         s_abort = 0;
-        // Phases: a barrier signalled once per head is waited with parity (use & 1),
-        // where `use` counts the heads that signalled it before; the two roles
-        // keep identical counters.
         uint64_t *all = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(Bars) / 8); ++i) mbar_init(&all[i], 1);
-        // CUDA-core arrivals: one per warp
-        uint64_t *eight[] = {&bars.xd_full,   &bars.s_full[0], &bars.s_full[1], &bars.m_full[0],
-                             &bars.m_full[1], &bars.y_free[0], &bars.y_free[1], &bars.unit_empty};
-        for (int i = 0; i < 8; ++i) mbar_init(eight[i], 8);
+        mbar_init(&bars.unit_empty, 9);
+        mbar_init(&bars.unit_done, 2);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&bars.pb[q].xd_full, 4);
+            mbar_init(&bars.pb[q].s_full, 4);
+            mbar_init(&bars.pb[q].m_full, 4);
+            mbar_init(&bars.pb[q].y_free, 4);
+        }
         mbar_fence_init();
     }
     fence_before_sync();
@@ -209,144 +232,172 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     fence_after_sync();
     const uint32_t tmem = tslot;
 
-    if (warp == kIssuerWarp) {
+    if (warp >= 8) {
         // ------------------------------------------------------------------
-        // TMA / MMA issue: the whole warp follows the control flow and waits;
-        // lane 0 alone issues loads, products and commits.
+        // Issuer warps: warp 8 drives pipeline 0 and also hands out units,
+        // loads C/B and forms G; warp 9 drives pipeline 1.  The whole warp
+        // follows the control flow and waits; lane 0 alone issues.
         // ------------------------------------------------------------------
+        const int pl = warp - 8;
         const bool leader = (lane == 0);
-        if (leader) {
+        PipeBars &pb = bars.pb[pl];
+        uint8_t *sXp = smem + kOffX + pl * 32768;
+        uint8_t *sSp = smem + kOffS + pl * 16384;
+        float *sJp = reinterpret_cast<float *>(smem + kOffJ) + pl * 512;
+        const uint32_t tY = tmem + kColY + pl * 64, tM = tmem + kColM + pl * 64, tD = tmem + kColD + pl * 64;
+        if (leader && pl == 0) {
             tma_prefetch_desc(&mC);
             tma_prefetch_desc(&mB);
             tma_prefetch_desc(&mX);
         }
-        uint32_t kh = 0, ucnt = 0, x0cnt = 0, cbcnt = 0;
-        uint32_t mcnt[2] = {0, 0};
+        uint32_t use = 0, r0use = 0, mcnt = 0, ucnt = 0, cbcnt = 0, units_done = 0;
         const uint32_t idG0 = idesc_bf16_f32(kRows, kRows, 0, 0);
         const uint32_t idG1 = idesc_bf16_f32(kRows, 2 * kRows, 0, 0);
         const uint32_t idInter = idesc_bf16_f32(kRows, kP, 0, 0);
         const uint32_t idState = idesc_bf16_f32(kRows, kP, 1, 1);
         const uint32_t idMX = idesc_bf16_f32(kRows, kP, 0, 1);
         for (;;) {
-            if (ucnt > 0) wait_bar(&bars.unit_empty, par_of(ucnt - 1), abort, p.status);
             int u = 0;
-            if (leader) {
-                u = atomicAdd(p.counter, 1);
-                s_unit = u;
-                mbar_arrive(&bars.unit_full);
+            if (pl == 0) {
+                if (ucnt > 0) wait_bar(&bars.unit_empty, par_of(ucnt - 1), abort, p.status);
+                if (leader) {
+                    u = atomicAdd(p.counter, 1);
+                    s_unit = u;
+                    mbar_arrive(&bars.unit_full);
+                }
+                u = __shfl_sync(0xffffffffu, u, 0);
+            } else {
+                wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
+                u = s_unit;
+                __syncwarp();
+                if (leader) mbar_arrive(&bars.unit_empty);
             }
-            u = __shfl_sync(0xffffffffu, u, 0);
             ++ucnt;
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
             if (un.row0 >= un.len) continue;
             const bool first = (un.r == 0);
-            // the previous unit's products must be done before its operands are replaced
-            if (kh > 0) wait_bar(&bars.mx_done[(kh - 1) & 1], par_of((kh - 1) >> 1), abort, p.status);
             const int qbox = Q / kRows;
-            if (leader) {
-                mbar_arrive_expect_tx(&bars.cb, (uint32_t)(NK + 2 * qbox) * 16384u);
-                for (int k = 0; k < NK; ++k)
-                    tma_load_4d(sC + k * 16384, &mC, &bars.cb, k * 64, un.g, un.t0 + un.row0, un.b);
-                for (int k = 0; k < 2; ++k)
-                    for (int q = 0; q < qbox; ++q)
-                        tma_load_4d(sB + k * 32768 + q * 16384, &mB, &bars.cb, k * 64, un.g, un.t0 + q * kRows,
-                                    un.b);
+            if (pl == 0) {
+                // both pipelines are done with the previous unit's C, B and G
+                if (units_done > 0) wait_bar(&bars.unit_done, par_of(units_done - 1), abort, p.status);
+                if (leader) {
+                    mbar_arrive_expect_tx(&bars.cb, (uint32_t)(NK + 2 * qbox) * 16384u);
+                    for (int k = 0; k < NK; ++k)
+                        tma_load_4d(sC + k * 16384, &mC, &bars.cb, k * 64, un.g, un.t0 + un.row0, un.b);
+                    for (int k = 0; k < 2; ++k)
+                        for (int q = 0; q < qbox; ++q)
+                            tma_load_4d(sB + k * 32768 + q * 16384, &mB, &bars.cb, k * 64, un.g,
+                                        un.t0 + q * kRows, un.b);
+                }
             }
+            ++units_done;
             wait_bar(&bars.cb, par_of(cbcnt++), abort, p.status);
             fence_after_sync();
-            // G = C_r B^T  (rows of this half x columns 0 .. end of this half)
-            if (leader)
-                for (int kk = 0; kk < NK * 4; ++kk) {
-                    const int atom = kk >> 2, kin = kk & 3;
-                    mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
-                           smem_desc_sw128(smem_u32(sB) + atom * 32768 + kin * 32, 16, 1024), first ? idG0 : idG1,
-                           kk > 0);
-                }
-            __syncwarp();
-            for (int h = un.h0; h < un.h1; ++h, ++kh) {
-                const int buf = kh & 1;
-                const uint32_t use = kh >> 1;
-                uint8_t *sXb = sX + buf * 32768;
-                uint8_t *sSb = sS + buf * 16384;
-                const uint32_t tY = tmem + kColY + buf * 64;
-                // X rows 0..Q-1 of head h
-                if (kh >= 2) wait_bar(&bars.x_free[buf], par_of(use - 1), abort, p.status);
+            if (pl == 0) {
+                // G = C_r B^T  (rows of this half x columns 0 .. end of this half)
                 if (leader) {
-                    mbar_arrive_expect_tx(&bars.x_full[buf], (uint32_t)qbox * 16384u);
-                    for (int q = 0; q < qbox; ++q)
-                        tma_load_4d(sXb + q * 16384, &mX, &bars.x_full[buf], 0, h, un.t0 + q * kRows, un.b);
-                }
-                if (first) {
-                    if (x0cnt > 0) wait_bar(&bars.x0_free, par_of(x0cnt - 1), abort, p.status);
-                    if (leader) {
-                        mbar_arrive_expect_tx(&bars.x0_full, 16384u);
-                        tma_load_4d(sX0, &mX, &bars.x0_full, 0, h, un.t0, un.b);
+                    for (int kk = 0; kk < NK * 4; ++kk) {
+                        const int atom = kk >> 2, kin = kk & 3;
+                        mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
+                               smem_desc_sw128(smem_u32(sB) + atom * 32768 + kin * 32, 16, 1024),
+                               first ? idG0 : idG1, kk > 0);
                     }
-                    // stage 2: D = B_c^T (decayed X), M = n (128), N = p, K = Q tokens
-                    wait_bar(&bars.xd_full, par_of(x0cnt), abort, p.status);
+                    mma_commit(&bars.g_done);
+                }
+                __syncwarp();
+            }
+            bool any = false;
+            for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
+                any = true;
+                const int jb = use & 1;
+                // this head's X rows 0..Q-1 and s values; warm L2 for the pipeline's next head
+                if (use > 0) wait_bar(&pb.x_free, par_of(use - 1), abort, p.status);
+                if (leader) {
+                    mbar_arrive_expect_tx(&pb.x_full, (uint32_t)qbox * 16384u);
+                    for (int q = 0; q < qbox; ++q)
+                        tma_load_4d(sXp + q * 16384, &mX, &pb.x_full, 0, h, un.t0 + q * kRows, un.b);
+                    mbar_arrive_expect_tx(&pb.j_full[jb], (uint32_t)Q * 4u);
+                    bulk_load(sJp + jb * 256, p.s + (((size_t)un.b * sh.H + h) * sh.nc + un.c) * Q,
+                              (uint32_t)Q * 4u, &pb.j_full[jb]);
+                    if (h + 2 < un.h1)
+                        for (int q = 0; q < qbox; ++q) tma_prefetch_4d(&mX, 0, h + 2, un.t0 + q * kRows, un.b);
+                }
+                __syncwarp();
+                if (first) {
+                    // stage 2: D = B_c^T (decayed X), M = n (128), N = p, K = Q tokens; the decayed
+                    // rows 0..127 sit in the S~ buffer, rows 128.. were decayed in place
+                    wait_bar(&pb.xd_full, par_of(r0use), abort, p.status);
                     fence_after_sync();
                     if (leader) {
-                        const uint32_t tD = tmem + kColD + buf * 64;
-                        for (int kk = 0; kk < Q / 16; ++kk)
+                        for (int kk = 0; kk < Q / 16; ++kk) {
+                            const uint32_t xb = (kk < 8) ? smem_u32(sSp) + kk * 2048 : smem_u32(sXp) + kk * 2048;
                             mma_ss(tD, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
-                                   smem_desc_sw128(smem_u32(sXb) + kk * 2048, 16, 1024), idState, kk > 0);
-                        mma_commit(&bars.d_done);
-                        mma_commit(&bars.x_free[buf]);
+                                   smem_desc_sw128(xb, 16, 1024), idState, kk > 0);
+                        }
+                        mma_commit(&pb.d_done);
                     }
                     __syncwarp();
+                    ++r0use;
                 }
                 // stage 4 product: Y = C_r S~^T
-                wait_bar(&bars.s_full[buf], par_of(use), abort, p.status);
-                if (kh >= 2) wait_bar(&bars.y_free[buf], par_of(use - 1), abort, p.status);
+                wait_bar(&pb.s_full, par_of(use), abort, p.status);
+                if (use > 0) wait_bar(&pb.y_free, par_of(use - 1), abort, p.status);
                 fence_after_sync();
                 if (leader) {
                     for (int kk = 0; kk < NK * 4; ++kk) {
                         const int atom = kk >> 2, kin = kk & 3;
                         mma_ss(tY, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
-                               smem_desc_sw128(smem_u32(sSb) + atom * 8192 + kin * 32, 16, 1024), idInter, kk > 0);
+                               smem_desc_sw128(smem_u32(sSp) + atom * 8192 + kin * 32, 16, 1024), idInter, kk > 0);
                     }
-                    mma_commit(&bars.inter_done[buf]);
+                    mma_commit(&pb.inter_done);
                 }
                 __syncwarp();
-                // stage 1 product: Y += M X, one K-half (128 tokens) at a time
+                // stage 1 product: Y += M X, one 128-token K-half at a time
                 const int nhalf = first ? 1 : 2;
                 for (int hf = 0; hf < nhalf; ++hf) {
-                    wait_bar(&bars.m_full[hf], par_of(mcnt[hf]), abort, p.status);
-                    if (hf == 0) {
-                        if (first)
-                            wait_bar(&bars.x0_full, par_of(x0cnt), abort, p.status);
-                        else
-                            wait_bar(&bars.x_full[buf], par_of(use), abort, p.status);
-                    }
+                    wait_bar(&pb.m_full, par_of(mcnt), abort, p.status);
+                    if (hf == 0 && !first) wait_bar(&pb.x_full, par_of(use), abort, p.status);
                     fence_after_sync();
                     if (leader) {
-                        const uint32_t xbase = first ? smem_u32(sX0) : smem_u32(sXb) + hf * 16384;
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tY, tmem + kColM + hf * 64 + kk * 8, smem_desc_sw128(xbase + kk * 2048, 16, 1024),
+                            mma_ts(tY, tM + kk * 8, smem_desc_sw128(smem_u32(sXp) + (hf * 8 + kk) * 2048, 16, 1024),
                                    idMX, 1);
-                        mma_commit(&bars.m_free[hf]);
+                        mma_commit(&pb.m_free);
                     }
                     __syncwarp();
-                    ++mcnt[hf];
+                    ++mcnt;
                 }
                 if (leader) {
-                    mma_commit(&bars.mx_done[buf]);
-                    mma_commit(first ? &bars.x0_free : &bars.x_free[buf]);
+                    mma_commit(&pb.mx_done);
+                    mma_commit(&pb.x_free);
                 }
                 __syncwarp();
-                if (first) ++x0cnt;
             }
+            // this pipeline is done with the unit once its last products completed
+            if (any) wait_bar(&pb.mx_done, par_of(use - 1), abort, p.status);
+            if (leader) mbar_arrive(&bars.unit_done);
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------------
-        // CUDA-core warps
+        // CUDA-core warpgroups: warpgroup pl serves pipeline pl
         // ------------------------------------------------------------------
-        const int wg = warp >> 2;                         // warpgroup: which 32 of the 64 columns
-        const int lrow = ((warp & 3) << 5) + lane;        // TMEM lane = row within the half
+        const int pl = warp >> 2;
+        const int wtid = tid & (kWgThreads - 1);
+        const int lrow = wtid;  // TMEM lane = row within the half
         const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
-        uint32_t kh = 0, ucnt = 0, r0cnt = 0;
-        uint32_t mcnt[2] = {0, 0};
+        const int wg_bar = 1 + pl;
+        PipeBars &pb = bars.pb[pl];
+        uint8_t *sXp = smem + kOffX + pl * 32768;
+        uint8_t *sSp = smem + kOffS + pl * 16384;
+        float *sJp = reinterpret_cast<float *>(smem + kOffJ) + pl * 512;
+        float *sFp = reinterpret_cast<float *>(smem + kOffF) + pl * 512;
+        const uint32_t tY = tmem + kColY + pl * 64, tM = tmem + kColM + pl * 64, tD = tmem + kColD + pl * 64;
+        uint32_t use = 0, r0use = 0, mcnt = 0, ucnt = 0, gcnt = 0;
+#ifdef SSD_TRACE
+        int trace_i = 0;
+#endif
         for (;;) {
             wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
             ++ucnt;
@@ -363,197 +414,278 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             }
             const bool first = (un.r == 0);
             const int j = un.row0 + lrow;  // this thread's row within the chunk
-            for (int h = un.h0; h < un.h1; ++h, ++kh) {
-                const int buf = kh & 1;
-                const uint32_t use = kh >> 1;
-                float *sJb = sJ + buf * 256;
-                float *sFb = sF + buf * 256;
-                uint8_t *sXb = sX + buf * 32768;
-                uint8_t *sSb = sS + buf * 16384;
-                const uint32_t tY = tmem + kColY + buf * 64;
+            const int kcols = un.row0 + kRows;
+            wait_bar(&bars.g_done, par_of(gcnt++), abort, p.status);
+            for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
+                const int jb = use & 1;
+                float *sJb = sJp + jb * 256;
+                float *sFb = sFp + jb * 256;
                 const size_t bh = (size_t)un.b * sh.H + h;
-                const float *sc = p.s + (bh * sh.nc + un.c) * Q;
-                for (int i = tid; i < Q; i += kSimtThreads) sJb[i] = sc[i];
-                named_bar_sync(kSimtBar, kSimtThreads);
-                const int kcols = un.row0 + kRows;
-                for (int i = tid; i < kcols; i += kSimtThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
+                SSD_TRACE_POINT(0);
+                // the previous head's y tile left the S~ buffer before it is overwritten (the
+                // stores are issued by the warpgroup's last thread, never by the thread that
+                // fences and publishes states, whose GPU-scope fence would wait for them)
+                if (wtid == kWgThreads - 1) bulk_wait_read();
+                SSD_TRACE_POINT(1);
+                wait_bar(&pb.j_full[jb], par_of(use >> 1), abort, p.status);
+                for (int i = wtid; i < kcols; i += kWgThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
+                named_bar_sync(wg_bar, kWgThreads);
+                SSD_TRACE_POINT(2);
 
                 if (first) {
-                    // decay X rows in place for the chunk state: x_i * exp(s_end - s_i)
-                    wait_bar(&bars.x_full[buf], par_of(use), abort, p.status);
+                    // x_i * exp(s_end - s_i) for the chunk state: rows 0..127 into the S~ buffer
+                    // (rows 0..127 of the X tile stay undecayed for the masked product), rows 128.. in place
+                    wait_bar(&pb.x_full, par_of(use), abort, p.status);
                     const float s_end = sJb[Q - 1];
-                    for (int idx = tid; idx < Q * 8; idx += kSimtThreads) {
-                        const int i = idx >> 3;
-                        const float w = expf(s_end - sJb[i]);
-                        uint4 *ptr = reinterpret_cast<uint4 *>(sXb + idx * 16);
-                        uint4 v = *ptr;
-                        v.x = pack_bf16x2(bf16lo(v.x) * w, bf16hi(v.x) * w);
-                        v.y = pack_bf16x2(bf16lo(v.y) * w, bf16hi(v.y) * w);
-                        v.z = pack_bf16x2(bf16lo(v.z) * w, bf16hi(v.z) * w);
-                        v.w = pack_bf16x2(bf16lo(v.w) * w, bf16hi(v.w) * w);
-                        *ptr = v;
+#pragma unroll 1
+                    for (int base = wtid; base < Q * 8; base += 4 * kWgThreads) {
+                        uint4 v[4];
+                        float w[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int idx = base + r * kWgThreads;
+                            v[r] = *reinterpret_cast<const uint4 *>(sXp + idx * 16);
+                            w[r] = expf(s_end - sJb[idx >> 3]);
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int idx = base + r * kWgThreads;
+                            uint4 o;
+                            o.x = pack_bf16x2(bf16lo(v[r].x) * w[r], bf16hi(v[r].x) * w[r]);
+                            o.y = pack_bf16x2(bf16lo(v[r].y) * w[r], bf16hi(v[r].y) * w[r]);
+                            o.z = pack_bf16x2(bf16lo(v[r].z) * w[r], bf16hi(v[r].z) * w[r]);
+                            o.w = pack_bf16x2(bf16lo(v[r].w) * w[r], bf16hi(v[r].w) * w[r]);
+                            *reinterpret_cast<uint4 *>(((idx >> 3) < kRows ? sSp : sXp) + idx * 16) = o;
+                        }
                     }
                     fence_view_async_shared();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars.xd_full);
+                    if (lane == 0) mbar_arrive(&pb.xd_full);
+                    SSD_TRACE_POINT(3);
                     // stage 3: S~_c = exp(s_end) S~_{c-1} + S_c
-                    if (tid == 0) {
+                    if (wtid == 0) {
                         if (un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
                         if (p.halves == 2 && un.c >= 2) wait_flag(p.cons + bh, un.c, abort, p.status);
                     }
-                    wait_bar(&bars.d_done, par_of(r0cnt), abort, p.status);
-                    ++r0cnt;
-                    named_bar_sync(kSimtBar, kSimtThreads);
+                    SSD_TRACE_POINT(4);
+                    wait_bar(&pb.d_done, par_of(r0use), abort, p.status);
+                    ++r0use;
+                    named_bar_sync(wg_bar, kWgThreads);
+                    SSD_TRACE_POINT(5);
                     fence_after_sync();
                     {
                         const float dchunk = expf(s_end);
                         const int n = lrow;
-                        const uint32_t tD = tmem + kColD + buf * 64 + wg * 32;
-                        uint32_t dv[32];
-                        tmem_ld16(tD + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[0]));
-                        tmem_ld16(tD + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[16]));
-                        tmem_wait_ld();
-                        if (n < N) {
-                            const size_t PN = (size_t)kP * N;
-                            const float *src = (un.c == 0) ? p.init : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
-                            float *dst = (un.c == sh.nc - 1) ? p.fin : p.ring + (bh * 2 + (un.c & 1)) * PN;
-                            if (un.c == 0 && src) src += bh * PN;
-                            if (un.c == sh.nc - 1 && dst) dst += bh * PN;
-                            uint8_t *srow = sSb + (n >> 6) * 8192;
-                            const int chunk = (n & 63) >> 3, sub = (n & 7) * 2;
-#pragma unroll 4
-                            for (int q = 0; q < 32; ++q) {
-                                const int pp = wg * 32 + q;
-                                const float old = src ? __ldcg(src + (size_t)pp * N + n) : 0.f;
-                                const float nw = fmaf(dchunk, old, __uint_as_float(dv[q]));
-                                if (dst) __stcg(dst + (size_t)pp * N + n, nw);
-                                *reinterpret_cast<__nv_bfloat16 *>(srow + pp * 128 + ((chunk ^ (pp & 7)) << 4) + sub) =
-                                    __float2bfloat16_rn(old);
+                        const size_t PN = (size_t)kP * N;
+                        const float *src = (un.c == 0) ? p.init : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
+                        float *dst = (un.c == sh.nc - 1) ? p.fin : p.ring + (bh * 2 + (un.c & 1)) * PN;
+                        if (un.c == 0 && src) src += bh * PN;
+                        if (un.c == sh.nc - 1 && dst) dst += bh * PN;
+                        uint8_t *srow = sSp + (n >> 6) * 8192;
+                        const int chunk = (n & 63) >> 3, sub = (n & 7) * 2;
+                        // 16 columns at a time: the accumulator slice and 16 loads are in flight
+                        // before the matching stores (src and dst may not be proven disjoint)
+                        // 32 columns at a time: the accumulator slice and 32 ring loads are in flight
+                        // before the matching stores (src and dst may not be proven disjoint)
+#pragma unroll 1
+                        for (int q0 = 0; q0 < kP; q0 += 32) {
+                            uint32_t dv[32];
+                            tmem_ld16(tD + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[0]));
+                            tmem_ld16(tD + q0 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[16]));
+                            float old[32];
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                old[q] = (src && n < N) ? __ldcg(src + (size_t)(q0 + q) * N + n) : 0.f;
+                            tmem_wait_ld();
+                            if (q0 == 0) SSD_TRACE_POINT(12);
+                            if (n < N) {
+#pragma unroll
+                                for (int q = 0; q < 32; ++q) {
+                                    const int pp = q0 + q;
+                                    const float nw = fmaf(dchunk, old[q], __uint_as_float(dv[q]));
+                                    if (dst) __stcg(dst + (size_t)pp * N + n, nw);
+                                    *reinterpret_cast<__nv_bfloat16 *>(srow + pp * 128 + ((chunk ^ (pp & 7)) << 4) +
+                                                                       sub) = __float2bfloat16_rn(old[q]);
+                                }
                             }
                         }
                     }
-                    __threadfence();
                     fence_view_async_shared();
-                    named_bar_sync(kSimtBar, kSimtThreads);
-                    if (tid == 0 && un.c < sh.nc - 1) st_release_gpu(p.ready + bh, un.c + 1);
+                    named_bar_sync(wg_bar, kWgThreads);
+                    SSD_TRACE_POINT(13);
+                    // the barrier orders every thread's ring stores before this thread's
+                    // GPU-scope fence, which publishes them with the flag (fences are cumulative)
+                    if (wtid == 0 && un.c < sh.nc - 1) {
+                        __threadfence();
+                        st_release_gpu(p.ready + bh, un.c + 1);
+                    }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars.s_full[buf]);
+                    if (lane == 0) mbar_arrive(&pb.s_full);
                 } else {
                     // entering state S~_{c-1} -> bf16 K-major tile
-                    if (tid == 0 && un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
-                    named_bar_sync(kSimtBar, kSimtThreads);
+                    if (wtid == 0 && un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
+                    named_bar_sync(wg_bar, kWgThreads);
+                    SSD_TRACE_POINT(5);
                     const size_t PN = (size_t)kP * N;
                     const float *src = (un.c == 0) ? (p.init ? p.init + bh * PN : nullptr)
                                                    : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
-                    for (int idx = tid; idx < kP * NK * 8; idx += kSimtThreads) {
-                        const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (src && n < N) {
-                            const float4 a = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n));
-                            const float4 bq = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
-                            v.x = pack_bf16x2(a.x, a.y);
-                            v.y = pack_bf16x2(a.z, a.w);
-                            v.z = pack_bf16x2(bq.x, bq.y);
-                            v.w = pack_bf16x2(bq.z, bq.w);
+                    const int nchunks = kP * NK * 8;  // 16-byte chunks of 8 values
+                    {
+                        const int base = 0;
+                        float4 lo[8], hi[8];
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const int idx = base + wtid + r * kWgThreads;
+                            const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
+                            lo[r] = hi[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (idx < nchunks && src && n < N) {
+                                lo[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n));
+                                hi[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
+                            }
                         }
-                        *reinterpret_cast<uint4 *>(sSb + (n >> 6) * 8192 + pr * 128 + ((((n & 63) >> 3) ^ (pr & 7)) << 4)) =
-                            v;
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const int idx = base + wtid + r * kWgThreads;
+                            const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
+                            if (idx >= nchunks) continue;
+                            uint4 v;
+                            v.x = pack_bf16x2(lo[r].x, lo[r].y);
+                            v.y = pack_bf16x2(lo[r].z, lo[r].w);
+                            v.z = pack_bf16x2(hi[r].x, hi[r].y);
+                            v.w = pack_bf16x2(hi[r].z, hi[r].w);
+                            *reinterpret_cast<uint4 *>(sSp + (n >> 6) * 8192 + pr * 128 +
+                                                       ((((n & 63) >> 3) ^ (pr & 7)) << 4)) = v;
+                        }
                     }
                     fence_view_async_shared();
-                    named_bar_sync(kSimtBar, kSimtThreads);
-                    if (tid == 0) st_release_gpu(p.cons + bh, un.c + 1);
+                    named_bar_sync(wg_bar, kWgThreads);
+                    if (wtid == 0) st_release_gpu(p.cons + bh, un.c + 1);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars.s_full[buf]);
+                    if (lane == 0) mbar_arrive(&pb.s_full);
                 }
 
+                SSD_TRACE_POINT(6);
                 // Y *= exp(s_j): stage 4's decay from the chunk start
-                wait_bar(&bars.inter_done[buf], par_of(use), abort, p.status);
+                wait_bar(&pb.inter_done, par_of(use), abort, p.status);
+                SSD_TRACE_POINT(7);
                 fence_after_sync();
                 const float sj = sJb[j];
                 {
                     const float e = expf(sj);
-                    uint32_t v[16];
+                    uint32_t v[64];
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const uint32_t ta = tY + wg * 32 + hf * 16 + lane_base;
-                        tmem_ld16(ta, v);
-                        tmem_wait_ld();
+                    for (int q0 = 0; q0 < kP; q0 += 16)
+                        tmem_ld16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * e);
-                        tmem_st16(ta, v);
-                    }
+                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * e);
+#pragma unroll
+                    for (int q0 = 0; q0 < kP; q0 += 16)
+                        tmem_st16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
                 }
-                // decay mask into TMEM, one K-half of 128 columns at a time
+                SSD_TRACE_POINT(8);
+                // decay mask into TMEM, one 128-token K-half at a time
                 const float Dh = p.D[h];
                 const int nhalf = first ? 1 : 2;
                 for (int hf = 0; hf < nhalf; ++hf) {
-                    if (mcnt[hf] > 0) wait_bar(&bars.m_free[hf], par_of(mcnt[hf] - 1), abort, p.status);
+                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
                     fence_after_sync();
-                    for (int sl = wg; sl < 4; sl += 2) {
-                        const int i0 = hf * 128 + sl * 32;
-                        uint32_t gv[32];
-                        tmem_ld16(tmem + kColG + i0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&gv[0]));
-                        tmem_ld16(tmem + kColG + i0 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&gv[16]));
+#pragma unroll 1
+                    for (int sp = 0; sp < 4; sp += 2) {
+                        uint32_t gv[64];
+#pragma unroll
+                        for (int q0 = 0; q0 < 64; q0 += 16)
+                            tmem_ld16(tmem + kColG + hf * 128 + sp * 32 + q0 + lane_base,
+                                      *reinterpret_cast<uint32_t(*)[16]>(&gv[q0]));
                         tmem_wait_ld();
-                        uint32_t o[16];
-                        if (i0 + 31 < j) {
-                            const float rf = expf(sj - sJb[i0 + 31]);
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                const float a = __uint_as_float(gv[2 * q]) * (rf * sFb[i0 + 2 * q]);
-                                const float bb = __uint_as_float(gv[2 * q + 1]) * (rf * sFb[i0 + 2 * q + 1]);
-                                o[q] = pack_bf16x2(a, bb);
+                        for (int ss = 0; ss < 2; ++ss) {
+                            const int sl = sp + ss;
+                            const int i0 = hf * 128 + sl * 32;
+                            const uint32_t *g = gv + ss * 32;
+                            uint32_t o[16];
+                            if (i0 + 31 < j) {
+                                // below the diagonal block: row factor x column factor, both <= 1
+                                const float rf = expf(sj - sJb[i0 + 31]);
+                                const float4 *f4 = reinterpret_cast<const float4 *>(sFb + i0);
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const float4 f = f4[q];
+                                    const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
+                                    const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
+                                    const float2 m0 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
+                                    const float2 m1 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
+                                    o[2 * q] = pack_bf16x2(m0.x, m0.y);
+                                    o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
+                                }
+                            } else if (i0 > j) {
+#pragma unroll
+                                for (int q = 0; q < 16; ++q) o[q] = 0u;
+                            } else {
+                                // the diagonal 32x32 block: one exponential per element
+#pragma unroll
+                                for (int q = 0; q < 16; ++q) {
+                                    const int ia = i0 + 2 * q, ib = ia + 1;
+                                    float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
+                                    float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
+                                    if (ia == j) a += Dh;
+                                    if (ib == j) bb += Dh;
+                                    o[q] = pack_bf16x2(a, bb);
+                                }
                             }
-                        } else if (i0 > j) {
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) o[q] = 0u;
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                const int ia = i0 + 2 * q, ib = ia + 1;
-                                float a = (ia <= j) ? __uint_as_float(gv[2 * q]) * expf(sj - sJb[ia]) : 0.f;
-                                float bb = (ib <= j) ? __uint_as_float(gv[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
-                                if (ia == j) a += Dh;
-                                if (ib == j) bb += Dh;
-                                o[q] = pack_bf16x2(a, bb);
-                            }
+                            tmem_st16(tM + sl * 16 + lane_base, o);
                         }
-                        tmem_st16(tmem + kColM + hf * 64 + (sl * 32) / 2 + lane_base, o);
                     }
                     tmem_wait_st();
                     fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars.m_full[hf]);
-                    ++mcnt[hf];
+                    if (lane == 0) mbar_arrive(&pb.m_full);
+                    ++mcnt;
                 }
-                // stage 5: y = bf16(Y)
-                wait_bar(&bars.mx_done[buf], par_of(use), abort, p.status);
+                SSD_TRACE_POINT(9);
+                // stage 5: y = bf16(Y), staged in the S~ buffer (its inter-chunk product is done)
+                // in the 128-byte-swizzled layout and written by one TMA store
+                wait_bar(&pb.mx_done, par_of(use), abort, p.status);
+                SSD_TRACE_POINT(10);
                 fence_after_sync();
                 {
-                    uint32_t v[32];
-                    tmem_ld16(tY + wg * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld16(tY + wg * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_wait_ld();
-                    if (j < un.len) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(
-                            p.y + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP + wg * 32);
+                    uint32_t v[64];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                            w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                            w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                            w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                            dst[q] = w;
-                        }
+                    for (int q0 = 0; q0 < kP; q0 += 16)
+                        tmem_ld16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
+                    tmem_wait_ld();
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.y_free);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+                        w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+                        w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+                        w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+                        *reinterpret_cast<uint4 *>(sSp + lrow * 128 + ((q ^ (lrow & 7)) << 4)) = w;
+                    }
+                    fence_view_async_shared();
+                    named_bar_sync(wg_bar, kWgThreads);
+                    if (wtid == kWgThreads - 1) {
+                        tma_store_4d(&mY, sSp, 0, h, un.t0 + un.row0, un.b);
+                        bulk_commit();
                     }
                 }
-                fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.y_free[buf]);
+                SSD_TRACE_POINT(11);
+#ifdef SSD_TRACE
+                if (ssd_trace_buffer && wtid == 0 && trace_i < 60)
+                    ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 16 + 14] =
+                        ((unsigned long long)h << 32) | ((unsigned long long)un.c << 8) | (first ? 1 : 0);
+                ++trace_i;
+#endif
             }
         }
     }
+    if (warp < 8 && (tid & (kWgThreads - 1)) == kWgThreads - 1) bulk_wait_all();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -584,8 +716,9 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, con
     const uint64_t dx[4] = {(uint64_t)sh.P, (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sx[3] = {(uint64_t)sh.P * 2, (uint64_t)sh.H * sh.P * 2, (uint64_t)sh.T * sh.H * sh.P * 2};
     const uint32_t box_x[4] = {64, 1, kRows, 1};
+    CUtensorMap mY;
     if (!make_map_bf16(&mC, C, 4, dbc, sbc, box_bc) || !make_map_bf16(&mB, B, 4, dbc, sbc, box_bc) ||
-        !make_map_bf16(&mX, x, 4, dx, sx, box_x))
+        !make_map_bf16(&mX, x, 4, dx, sx, box_x) || !make_map_bf16(&mY, y, 4, dx, sx, box_x))
         return cudaErrorInvalidValue;
     Params p;
     p.sh = sh;
@@ -608,7 +741,7 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, con
         cudaFuncSetAttribute(ssd_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = min(p.n_units, device_sm_count());
-    ssd_fused_kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, p);
+    ssd_fused_kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, p);
     return cudaGetLastError();
 }
 

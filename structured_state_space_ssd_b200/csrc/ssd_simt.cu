@@ -34,11 +34,22 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restri
     {
         const int h0 = blockIdx.z * 32;
         const int hn = min(32, sh.H - h0);
-        for (int idx = threadIdx.x; idx < sh.Q * 32; idx += blockDim.x) {
-            const int i = idx >> 5, hh = idx & 31;
-            float v = 0.f;
-            if (i < len && hh < hn) v = dt[((size_t)b * sh.T + t0 + i) * sh.H + h0 + hh] * A[h0 + hh];
-            tile[i * 33 + hh] = v;
+        // eight loads in flight per thread (rows i .. i+7*8 of one head column)
+        for (int base = threadIdx.x; base < sh.Q * 32; base += 8 * blockDim.x) {
+            float v[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int idx = base + r * blockDim.x;
+                const int i = idx >> 5, hh = idx & 31;
+                v[r] = (idx < sh.Q * 32 && i < len && hh < hn)
+                           ? dt[((size_t)b * sh.T + t0 + i) * sh.H + h0 + hh] * A[h0 + hh]
+                           : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int idx = base + r * blockDim.x;
+                if (idx < sh.Q * 32) tile[(idx >> 5) * 33 + (idx & 31)] = v[r];
+            }
         }
         __syncthreads();
         for (int hh = warp; hh < hn; hh += nwarps) {
