@@ -205,6 +205,33 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# Rank plumbing (one process per GPU; no collective on the data path)
+# ---------------------------------------------------------------------------
+def rank_inputs(w, rank: int):
+    """Inputs of this rank's batch: the workload's own seed on rank 0, a distinct seed elsewhere."""
+    from structured_state_space_ssd_b200.inputs import make_inputs, workload_inputs
+    if rank == 0:
+        return workload_inputs(w)
+    return make_inputs(w.batch, w.T, w.H, w.P, w.N, w.G, w.dtype, w.seed + 7919 * rank, w.with_init)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(w, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes one batch of the workload per step."""
+    return w.tokens * world / (ms_per_step * 1e-3)
+
+
 def config_of(w, n):
     return {"workload": w.name, "batch": w.batch, "seq_len": w.T, "heads": w.H, "head_dim": w.P,
             "state_dim": w.N, "groups": w.G, "chunk": w.Q, "init_state": w.with_init,
@@ -216,7 +243,7 @@ def config_of(w, n):
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
-    from structured_state_space_ssd_b200.inputs import HEADLINE, WORKLOADS, workload_inputs
+    from structured_state_space_ssd_b200.inputs import HEADLINE, WORKLOADS
     w = WORKLOADS[args.workload or HEADLINE]
     if args.impl == "reference":
         run_reference(args, w)
@@ -237,7 +264,7 @@ def main():
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     S.load()
-    host = workload_inputs(w) if world == 1 else _rank_inputs(w, rank)
+    host = rank_inputs(w, rank)
     d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
     y = torch.empty_like(d["x"])
     fin = torch.empty((w.batch, w.H, w.P, w.N), dtype=torch.float32, device=dev)
@@ -276,14 +303,10 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    total_ms = sum(per_step)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(per_step), dev)
     ms_per_step = total_ms / args.steps
     tokens = w.tokens * world
-    value = tokens / (ms_per_step * 1e-3)
+    value = job_tokens_per_s(w, world, ms_per_step)
 
     # --- end to end: pinned host inputs in, y and final_state out, every step
     e2e_steps = args.e2e_steps or args.steps
@@ -312,11 +335,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank == 0:
@@ -391,11 +411,6 @@ def _traffic_from_profiles(kernel, w):
     with open(path) as f:
         t = json.load(f)
     return t.get(w.name, {}).get(kernel)
-
-
-def _rank_inputs(w, rank):
-    from structured_state_space_ssd_b200.inputs import make_inputs
-    return make_inputs(w.batch, w.T, w.H, w.P, w.N, w.G, w.dtype, w.seed + 7919 * rank, w.with_init)
 
 
 if __name__ == "__main__":
