@@ -132,6 +132,29 @@ SSD_API const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, in
  */
 SSD_API int ssd_fwd_check(const void *workspace, void *stream);
 
+/*
+ * ssd_fwd for callers that cannot allocate device memory when they run the
+ * layer (an engine that fixes every buffer before serving, a framework whose
+ * allocator owns the device, a loop that must never reach cudaMalloc).  The
+ * paper has no counterpart to this entry point; it only changes where the
+ * scratch lives.
+ *
+ * Same arguments, results and conventions as ssd_fwd, without the workspace:
+ * the library uses its own scratch, a static device array of
+ * SSD_NO_ALLOC_SCRATCH_BYTES bytes present on every GPU that loads the
+ * library until the process exits.  Problems whose ssd_fwd_workspace_bytes
+ * exceeds that size are rejected with SSD_ERR_UNSUPPORTED before anything is
+ * launched.  The first call on each device looks up the array's device
+ * address (and may load the library's device code there), so make it before
+ * any stream capture.  All calls on a device share the array and it keeps
+ * the last call's contents (each call clears what it needs); calls whose GPU
+ * work overlaps, e.g. on two streams, race on it.  Nothing is allocated.
+ */
+#define SSD_NO_ALLOC_SCRATCH_BYTES (32u << 20)
+SSD_API int ssd_fwd_no_alloc(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                     const float *D, int Q, const float *init_state, void *y, float *final_state,
+                     int batch, int T, int H, int P, int G, int N, int dtype, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

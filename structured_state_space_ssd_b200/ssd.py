@@ -23,7 +23,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
-           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version")
+           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc")
 
 
 class SSDError(RuntimeError):
