@@ -40,21 +40,35 @@
 #include "tma_host.h"
 
 // Optional phase timestamps for performance work: compiled in only with
-// -DSSD_TRACE, which also provides ssd_trace_buffer (one 16-slot record per
+// -DSSD_TRACE, which also provides ssd_trace_buffer (one 32-slot record per
 // head and pipeline).  Production builds contain no trace code.
 #ifdef SSD_TRACE
 __device__ unsigned long long *ssd_trace_buffer = nullptr;
 #define SSD_TRACE_POINT(ev)                                                                                    \
     do {                                                                                                       \
-        if (ssd_trace_buffer && wtid == 0 && trace_i < 60) {                                                   \
+        if (ssd_trace_buffer && wtid == 0 && trace_i < 30) {                                                   \
             unsigned long long t_;                                                                             \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                           \
-            ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 16 + (ev)] = t_;               \
+            ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 32 + (ev)] = t_;               \
         }                                                                                                      \
     } while (0)
 #else
 #define SSD_TRACE_POINT(ev) \
     do {                    \
+    } while (0)
+#endif
+#ifdef SSD_TRACE
+// waits until the values v[0..n) have arrived, then records event ev
+#define SSD_TRACE_ARRIVED(v, n, ev)                              \
+    do {                                                         \
+        float acc_ = 0.f;                                        \
+        for (int i_ = 0; i_ < (n); ++i_) acc_ += (v)[i_];        \
+        if (acc_ == -1.2345e-30f) ssd_trace_buffer[0] = 1;       \
+        SSD_TRACE_POINT(ev);                                     \
+    } while (0)
+#else
+#define SSD_TRACE_ARRIVED(v, n, ev) \
+    do {                            \
     } while (0)
 #endif
 
@@ -64,8 +78,10 @@ using namespace tc;
 
 namespace fz {
 
-constexpr int kWgThreads = 128;              // one warpgroup: the 128 TMEM lanes
-constexpr int kThreads = 2 * kWgThreads + 64; // warps 0-7: two warpgroups; warps 8-9: issuers
+constexpr int kWgThreads = 128;                  // one warpgroup: the 128 TMEM lanes
+constexpr int kPipeThreads = 2 * kWgThreads;     // two warpgroups per head pipeline, each half the columns
+constexpr int kSimtWarps = 2 * kPipeThreads / 32;  // warps 0-15: CUDA-core work of pipelines 0 and 1
+constexpr int kThreads = 2 * kPipeThreads + 128;  // + warps 16-17: issuers, 18-19: publishers
 constexpr int kRows = 128;
 constexpr int kP = 64;
 
@@ -86,7 +102,6 @@ constexpr uint32_t kOffJ = kOffS + 2 * 16384;  // per pipeline, 2 buffers: s val
 constexpr uint32_t kOffF = kOffJ + 4 * 1024;   // per pipeline, 2 buffers: column factors (256 floats)
 constexpr uint32_t kSmemBytes = kOffF + 4 * 1024 + 1024;
 
-constexpr uint32_t kBarPolls = 1u << 22;
 constexpr uint32_t kFlagPolls = 1u << 22;
 
 struct Params {
@@ -123,13 +138,14 @@ struct PipeBars {
     uint64_t m_free;      // product reading it done
     uint64_t mx_done;     // every product of the head done
     uint64_t y_free;      // output accumulator drained (4 warp arrivals)
+    uint64_t ring_done;   // ring stores issued (first half) / ring loads consumed (second half)
 };
 
 struct Bars {
     uint64_t cb;          // C and B tiles landed (TMA)
     uint64_t g_done;      // G = C B^T in TMEM
     uint64_t unit_full;   // unit id posted (issuer 0)
-    uint64_t unit_empty;  // unit id read (8 CUDA-core warps + issuer 1)
+    uint64_t unit_empty;  // unit id read (16 CUDA-core warps, issuer 1, 2 publishers)
     uint64_t unit_done;   // both pipelines finished the unit (2 issuer arrivals)
     PipeBars pb[2];
 };
@@ -162,10 +178,16 @@ __device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
 }
 
 // Bounded mbarrier wait that gives up at once after any wait in the CTA failed.
+// Each poll parks the warp for up to kSuspendNs, so the bound is about
+// kWaitPolls * kSuspendNs (~2 s) of waiting, after which the status word
+// records SSD_ERR_TIMEOUT.
+constexpr uint32_t kSuspendNs = 100000;
+constexpr uint32_t kWaitPolls = 20000;
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int *status) {
-    for (uint32_t i = 0; i < kBarPolls; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (*abort) return false;
     }
     atomicExch(status, SSD_ERR_TIMEOUT);
     *abort = 1;
@@ -217,13 +239,14 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         s_abort = 0;
         uint64_t *all = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(Bars) / 8); ++i) mbar_init(&all[i], 1);
-        mbar_init(&bars.unit_empty, 9);
+        mbar_init(&bars.unit_empty, kSimtWarps + 3);
         mbar_init(&bars.unit_done, 2);
         for (int q = 0; q < 2; ++q) {
-            mbar_init(&bars.pb[q].xd_full, 4);
-            mbar_init(&bars.pb[q].s_full, 4);
-            mbar_init(&bars.pb[q].m_full, 4);
-            mbar_init(&bars.pb[q].y_free, 4);
+            mbar_init(&bars.pb[q].xd_full, kPipeThreads / 32);
+            mbar_init(&bars.pb[q].s_full, kPipeThreads / 32);
+            mbar_init(&bars.pb[q].m_full, kPipeThreads / 32);
+            mbar_init(&bars.pb[q].y_free, kPipeThreads / 32);
+            mbar_init(&bars.pb[q].ring_done, kPipeThreads / 32);
         }
         mbar_fence_init();
     }
@@ -232,13 +255,52 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     fence_after_sync();
     const uint32_t tmem = tslot;
 
-    if (warp >= 8) {
+    if (warp >= kSimtWarps + 2) {
         // ------------------------------------------------------------------
-        // Issuer warps: warp 8 drives pipeline 0 and also hands out units,
-        // loads C/B and forms G; warp 9 drives pipeline 1.  The whole warp
+        // Publisher warps: warp 18 + pl makes pipeline pl's chain hand-offs
+        // visible, so that neither the CUDA-core warps nor the issuer wait
+        // for the GPU-scope fence.  After a first half's ring stores it
+        // releases `ready` (S~_c readable); after a second half consumed
+        // S~_{c-1} it releases `cons` (the ring slot may be rewritten).  The
+        // warps' arrival on ring_done orders their accesses before this
+        // thread's fence and flag.
+        // ------------------------------------------------------------------
+        const int pl = warp - kSimtWarps - 2;
+        PipeBars &pb = bars.pb[pl];
+        uint32_t ucnt = 0, rcnt = 0;
+        for (;;) {
+            wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
+            ++ucnt;
+            const int u = s_unit;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.unit_empty);
+            if (u >= p.n_units) break;
+            const Unit un = decode(u, p);
+            if (un.row0 >= un.len) continue;
+            const bool first = (un.r == 0);
+            for (int h = un.h0 + pl; h < un.h1; h += 2, ++rcnt) {
+                wait_bar(&pb.ring_done, par_of(rcnt), abort, p.status);
+                if (lane == 0) {
+                    const size_t bh = (size_t)un.b * sh.H + h;
+                    if (first) {
+                        if (un.c < sh.nc - 1) {
+                            __threadfence();
+                            st_release_gpu(p.ready + bh, un.c + 1);
+                        }
+                    } else {
+                        st_release_gpu(p.cons + bh, un.c + 1);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    } else if (warp >= kSimtWarps) {
+        // ------------------------------------------------------------------
+        // Issuer warps: warp 16 drives pipeline 0 and also hands out units,
+        // loads C/B and forms G; warp 17 drives pipeline 1.  The whole warp
         // follows the control flow and waits; lane 0 alone issues.
         // ------------------------------------------------------------------
-        const int pl = warp - 8;
+        const int pl = warp - kSimtWarps;
         const bool leader = (lane == 0);
         PipeBars &pb = bars.pb[pl];
         uint8_t *sXp = smem + kOffX + pl * 32768;
@@ -381,11 +443,14 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------------
-        // CUDA-core warpgroups: warpgroup pl serves pipeline pl
+        // CUDA-core warps: warps 8pl..8pl+7 serve pipeline pl as two
+        // warpgroups; warpgroup `half` takes columns [32 half, 32 half + 32)
+        // of every 64-wide tile and every other 32-column slab of the mask.
         // ------------------------------------------------------------------
-        const int pl = warp >> 2;
-        const int wtid = tid & (kWgThreads - 1);
-        const int lrow = wtid;  // TMEM lane = row within the half
+        const int pl = warp >> 3;
+        const int half = (warp >> 2) & 1;
+        const int wtid = tid & (kPipeThreads - 1);
+        const int lrow = ((warp & 3) << 5) + lane;  // TMEM lane = row within the chunk half
         const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
         const int wg_bar = 1 + pl;
         PipeBars &pb = bars.pb[pl];
@@ -421,35 +486,122 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 float *sJb = sJp + jb * 256;
                 float *sFb = sFp + jb * 256;
                 const size_t bh = (size_t)un.b * sh.H + h;
+                const size_t PN = (size_t)kP * N;
                 SSD_TRACE_POINT(0);
                 // the previous head's y tile left the S~ buffer before it is overwritten (the
-                // stores are issued by the warpgroup's last thread, never by the thread that
+                // stores are issued by the pipeline's last thread, never by the thread that
                 // fences and publishes states, whose GPU-scope fence would wait for them)
-                if (wtid == kWgThreads - 1) bulk_wait_read();
+                if (wtid == kPipeThreads - 1) bulk_wait_read();
                 SSD_TRACE_POINT(1);
                 wait_bar(&pb.j_full[jb], par_of(use >> 1), abort, p.status);
-                for (int i = wtid; i < kcols; i += kWgThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
-                named_bar_sync(wg_bar, kWgThreads);
+                for (int i = wtid; i < kcols; i += kPipeThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
+                // the entering state S~_{c-1} is read once it is published (chunk 0 reads the initial
+                // state).  A second half asks here whether it is, a first half after its decay: if so
+                // its loads are in flight during the mask, else the mask is done while waiting
+                bool rdy = false;
+                if (!first && wtid == 0) rdy = un.c == 0 || ld_acquire_gpu(p.ready + bh) >= un.c;
+                rdy = named_bar_or(wg_bar, kPipeThreads, rdy);
                 SSD_TRACE_POINT(2);
+                const float *src = (un.c == 0) ? (p.init ? p.init + bh * PN : nullptr)
+                                               : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
+                const float sj = sJb[j];
+                const float Dh = p.D[h];
+                const float s_end = sJb[Q - 1];
+
+                // decay mask for 32-column slabs sl = half, half + 2 of K-half hf, into TMEM, in
+                // 16-column pieces (few live registers: the entering state may be in flight)
+                auto mask_half = [&](int hf) {
+#pragma unroll 1
+                    for (int sl = half; sl < 4; sl += 2) {
+                        const int i0 = hf * 128 + sl * 32;
+                        if (i0 > j) {
+                            uint32_t z[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) z[q] = 0u;
+                            tmem_st8(tM + sl * 16 + lane_base, z);
+                            tmem_st8(tM + sl * 16 + 8 + lane_base, z);
+                            continue;
+                        }
+                        const bool below = i0 + 31 < j;
+                        // below the diagonal block: row factor x column factor, both <= 1
+                        const float rf = below ? expf(sj - sJb[i0 + 31]) : 0.f;
+#pragma unroll 1
+                        for (int pc = 0; pc < 2; ++pc) {
+                            const int c0 = i0 + pc * 16;
+                            uint32_t g[16], o[8];
+                            tmem_ld16(tmem + kColG + c0 + lane_base, g);
+                            tmem_wait_ld();
+                            if (below) {
+                                const float4 *f4 = reinterpret_cast<const float4 *>(sFb + c0);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const float4 f = f4[q];
+                                    const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
+                                    const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
+                                    const float2 m0 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
+                                    const float2 m1 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
+                                    o[2 * q] = pack_bf16x2(m0.x, m0.y);
+                                    o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
+                                }
+                            } else {
+                                // the diagonal 32x32 block: one exponential per element
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    const int ia = c0 + 2 * q, ib = ia + 1;
+                                    float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
+                                    float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
+                                    if (ia == j) a += Dh;
+                                    if (ib == j) bb += Dh;
+                                    o[q] = pack_bf16x2(a, bb);
+                                }
+                            }
+                            tmem_st8(tM + sl * 16 + pc * 8 + lane_base, o);
+                        }
+                    }
+                    tmem_wait_st();
+                };
+                // Y *= exp(s_j) (stage 4's decay from the chunk start), then hand mask K-half 0 to
+                // the issuer: its product accumulates onto the scaled Y
+                auto scale_and_release_mask = [&]() {
+                    wait_bar(&pb.inter_done, par_of(use), abort, p.status);
+                    fence_after_sync();
+                    const float e = expf(sj);
+                    uint32_t v[32];
+                    tmem_ld16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                    tmem_ld16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * e);
+                    tmem_st16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                    tmem_st16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+                    tmem_wait_st();
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.m_full);
+                    ++mcnt;
+                };
 
                 if (first) {
                     // x_i * exp(s_end - s_i) for the chunk state: rows 0..127 into the S~ buffer
                     // (rows 0..127 of the X tile stay undecayed for the masked product), rows 128.. in place
                     wait_bar(&pb.x_full, par_of(use), abort, p.status);
-                    const float s_end = sJb[Q - 1];
+                    SSD_TRACE_POINT(21);
 #pragma unroll 1
-                    for (int base = wtid; base < Q * 8; base += 4 * kWgThreads) {
+                    for (int base = wtid; base < Q * 8; base += 4 * kPipeThreads) {
                         uint4 v[4];
                         float w[4];
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            const int idx = base + r * kWgThreads;
+                            const int idx = min(base + r * kPipeThreads, Q * 8 - 1);
                             v[r] = *reinterpret_cast<const uint4 *>(sXp + idx * 16);
                             w[r] = expf(s_end - sJb[idx >> 3]);
                         }
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            const int idx = base + r * kWgThreads;
+                            const int idx = base + r * kPipeThreads;
+                            if (idx >= Q * 8) continue;
                             uint4 o;
                             o.x = pack_bf16x2(bf16lo(v[r].x) * w[r], bf16hi(v[r].x) * w[r]);
                             o.y = pack_bf16x2(bf16lo(v[r].y) * w[r], bf16hi(v[r].y) * w[r]);
@@ -462,80 +614,83 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.xd_full);
                     SSD_TRACE_POINT(3);
-                    // stage 3: S~_c = exp(s_end) S~_{c-1} + S_c
+                    // mask K-half 0 (the whole K range of a first half) while the state product runs
+                    // and before waiting on the chain, so that the chain's path holds no mask work
+                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
+                    SSD_TRACE_POINT(22);
+                    fence_after_sync();
+                    mask_half(0);
+                    // S~_{c-1} must be published and the outgoing ring slot free of readers
                     if (wtid == 0) {
                         if (un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
                         if (p.halves == 2 && un.c >= 2) wait_flag(p.cons + bh, un.c, abort, p.status);
                     }
+                    named_bar_sync(wg_bar, kPipeThreads);
+                    SSD_TRACE_POINT(15);
+                    // this thread's 32 columns of S~_{c-1} (lane n; [p][n] like the initial state)
+                    const int n = lrow;
+                    float old[32];
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        old[q] = (src && n < N) ? __ldcg(src + (size_t)(half * 32 + q) * N + n) : 0.f;
                     SSD_TRACE_POINT(4);
+                    SSD_TRACE_ARRIVED(old, 32, 8);
+                    // stage 3: S~_c = exp(s_end) S~_{c-1} + S_c; S~_{c-1} in bf16 is this head's
+                    // inter-chunk operand (the decayed rows left the S~ buffer with the state product)
                     wait_bar(&pb.d_done, par_of(r0use), abort, p.status);
                     ++r0use;
-                    named_bar_sync(wg_bar, kWgThreads);
-                    SSD_TRACE_POINT(5);
+                    named_bar_sync(wg_bar, kPipeThreads);
                     fence_after_sync();
+                    SSD_TRACE_POINT(5);
                     {
+                        // the outgoing state goes to the ring or, after the last chunk, to the final state
                         const float dchunk = expf(s_end);
-                        const int n = lrow;
-                        const size_t PN = (size_t)kP * N;
-                        const float *src = (un.c == 0) ? p.init : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
-                        float *dst = (un.c == sh.nc - 1) ? p.fin : p.ring + (bh * 2 + (un.c & 1)) * PN;
-                        if (un.c == 0 && src) src += bh * PN;
-                        if (un.c == sh.nc - 1 && dst) dst += bh * PN;
-                        uint8_t *srow = sSp + (n >> 6) * 8192;
-                        const int chunk = (n & 63) >> 3, sub = (n & 7) * 2;
-                        // 16 columns at a time: the accumulator slice and 16 loads are in flight
-                        // before the matching stores (src and dst may not be proven disjoint)
-                        // 32 columns at a time: the accumulator slice and 32 ring loads are in flight
-                        // before the matching stores (src and dst may not be proven disjoint)
-#pragma unroll 1
-                        for (int q0 = 0; q0 < kP; q0 += 32) {
-                            uint32_t dv[32];
-                            tmem_ld16(tD + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[0]));
-                            tmem_ld16(tD + q0 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&dv[16]));
-                            float old[32];
+                        float *dst = (un.c == sh.nc - 1) ? (p.fin ? p.fin + bh * PN : nullptr)
+                                                         : p.ring + (bh * 2 + (un.c & 1)) * PN;
 #pragma unroll
-                            for (int q = 0; q < 32; ++q)
-                                old[q] = (src && n < N) ? __ldcg(src + (size_t)(q0 + q) * N + n) : 0.f;
+                        for (int q0 = 0; q0 < 32; q0 += 16) {
+                            uint32_t dv[16];
+                            tmem_ld16(tmem + kColD + pl * 64 + half * 32 + q0 + lane_base, dv);
                             tmem_wait_ld();
-                            if (q0 == 0) SSD_TRACE_POINT(12);
-                            if (n < N) {
+                            if (n < N && dst) {
 #pragma unroll
-                                for (int q = 0; q < 32; ++q) {
-                                    const int pp = q0 + q;
-                                    const float nw = fmaf(dchunk, old[q], __uint_as_float(dv[q]));
-                                    if (dst) __stcg(dst + (size_t)pp * N + n, nw);
-                                    *reinterpret_cast<__nv_bfloat16 *>(srow + pp * 128 + ((chunk ^ (pp & 7)) << 4) +
-                                                                       sub) = __float2bfloat16_rn(old[q]);
-                                }
+                                for (int q = 0; q < 16; ++q)
+                                    __stcg(dst + (size_t)(half * 32 + q0 + q) * N + n,
+                                           fmaf(dchunk, old[q0 + q], __uint_as_float(dv[q])));
+                            }
+                        }
+                        // the publisher warp releases the stores
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&pb.ring_done);
+                        // S~_{c-1} in bf16 into column n of the S~ tile ([p][n], 128-byte swizzled)
+                        if (n < N) {
+                            uint8_t *srow = sSp + (n >> 6) * 8192;
+                            const int chunk = (n & 63) >> 3, sub = (n & 7) * 2;
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) {
+                                const int pp = half * 32 + q;
+                                *reinterpret_cast<__nv_bfloat16 *>(srow + pp * 128 + ((chunk ^ (pp & 7)) << 4) + sub) =
+                                    __float2bfloat16_rn(old[q]);
                             }
                         }
                     }
+                    SSD_TRACE_POINT(12);
                     fence_view_async_shared();
-                    named_bar_sync(wg_bar, kWgThreads);
+                    named_bar_sync(wg_bar, kPipeThreads);
                     SSD_TRACE_POINT(13);
-                    // the barrier orders every thread's ring stores before this thread's
-                    // GPU-scope fence, which publishes them with the flag (fences are cumulative)
-                    if (wtid == 0 && un.c < sh.nc - 1) {
-                        __threadfence();
-                        st_release_gpu(p.ready + bh, un.c + 1);
-                    }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.s_full);
+                    SSD_TRACE_POINT(6);
+                    scale_and_release_mask();
+                    SSD_TRACE_POINT(7);
                 } else {
-                    // entering state S~_{c-1} -> bf16 K-major tile
-                    if (wtid == 0 && un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
-                    named_bar_sync(wg_bar, kWgThreads);
-                    SSD_TRACE_POINT(5);
-                    const size_t PN = (size_t)kP * N;
-                    const float *src = (un.c == 0) ? (p.init ? p.init + bh * PN : nullptr)
-                                                   : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
-                    const int nchunks = kP * NK * 8;  // 16-byte chunks of 8 values
-                    {
-                        const int base = 0;
-                        float4 lo[8], hi[8];
+                    // this thread's pieces of S~_{c-1} ([p][n]: 8 consecutive n of one row p each)
+                    const int nchunks = kP * NK * 8;
+                    float4 lo[4], hi[4];
+                    auto load_pieces = [&]() {
 #pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            const int idx = base + wtid + r * kWgThreads;
+                        for (int r = 0; r < 4; ++r) {
+                            const int idx = wtid + r * kPipeThreads;
                             const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
                             lo[r] = hi[r] = make_float4(0.f, 0.f, 0.f, 0.f);
                             if (idx < nchunks && src && n < N) {
@@ -543,102 +698,50 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                                 hi[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
                             }
                         }
-#pragma unroll
-                        for (int r = 0; r < 8; ++r) {
-                            const int idx = base + wtid + r * kWgThreads;
-                            const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
-                            if (idx >= nchunks) continue;
-                            uint4 v;
-                            v.x = pack_bf16x2(lo[r].x, lo[r].y);
-                            v.y = pack_bf16x2(lo[r].z, lo[r].w);
-                            v.z = pack_bf16x2(hi[r].x, hi[r].y);
-                            v.w = pack_bf16x2(hi[r].z, hi[r].w);
-                            *reinterpret_cast<uint4 *>(sSp + (n >> 6) * 8192 + pr * 128 +
-                                                       ((((n & 63) >> 3) ^ (pr & 7)) << 4)) = v;
-                        }
+                    };
+                    auto mask0 = [&]() {
+                        if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
+                        fence_after_sync();
+                        mask_half(0);
+                    };
+                    if (rdy) {
+                        load_pieces();
+                        mask0();
+                    } else {
+                        mask0();
+                        if (wtid == 0) wait_flag(p.ready + bh, un.c, abort, p.status);
+                        named_bar_sync(wg_bar, kPipeThreads);
+                        load_pieces();
                     }
+                    SSD_TRACE_POINT(3);
+                    SSD_TRACE_ARRIVED(reinterpret_cast<const float *>(lo), 16, 8);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int idx = wtid + r * kPipeThreads;
+                        const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
+                        if (idx >= nchunks) continue;
+                        uint4 v;
+                        v.x = pack_bf16x2(lo[r].x, lo[r].y);
+                        v.y = pack_bf16x2(lo[r].z, lo[r].w);
+                        v.z = pack_bf16x2(hi[r].x, hi[r].y);
+                        v.w = pack_bf16x2(hi[r].z, hi[r].w);
+                        *reinterpret_cast<uint4 *>(sSp + (n >> 6) * 8192 + pr * 128 +
+                                                   ((((n & 63) >> 3) ^ (pr & 7)) << 4)) = v;
+                    }
+                    // the publisher warp releases the ring slot: this warp's loads are consumed
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.ring_done);
                     fence_view_async_shared();
-                    named_bar_sync(wg_bar, kWgThreads);
-                    if (wtid == 0) st_release_gpu(p.cons + bh, un.c + 1);
+                    named_bar_sync(wg_bar, kPipeThreads);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.s_full);
-                }
-
-                SSD_TRACE_POINT(6);
-                // Y *= exp(s_j): stage 4's decay from the chunk start
-                wait_bar(&pb.inter_done, par_of(use), abort, p.status);
-                SSD_TRACE_POINT(7);
-                fence_after_sync();
-                const float sj = sJb[j];
-                {
-                    const float e = expf(sj);
-                    uint32_t v[64];
-#pragma unroll
-                    for (int q0 = 0; q0 < kP; q0 += 16)
-                        tmem_ld16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 64; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * e);
-#pragma unroll
-                    for (int q0 = 0; q0 < kP; q0 += 16)
-                        tmem_st16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
-                }
-                SSD_TRACE_POINT(8);
-                // decay mask into TMEM, one 128-token K-half at a time
-                const float Dh = p.D[h];
-                const int nhalf = first ? 1 : 2;
-                for (int hf = 0; hf < nhalf; ++hf) {
-                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
+                    SSD_TRACE_POINT(6);
+                    scale_and_release_mask();
+                    SSD_TRACE_POINT(7);
+                    // mask K-half 1 once the product of K-half 0 has read the mask buffer
+                    wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
                     fence_after_sync();
-#pragma unroll 1
-                    for (int sp = 0; sp < 4; sp += 2) {
-                        uint32_t gv[64];
-#pragma unroll
-                        for (int q0 = 0; q0 < 64; q0 += 16)
-                            tmem_ld16(tmem + kColG + hf * 128 + sp * 32 + q0 + lane_base,
-                                      *reinterpret_cast<uint32_t(*)[16]>(&gv[q0]));
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int ss = 0; ss < 2; ++ss) {
-                            const int sl = sp + ss;
-                            const int i0 = hf * 128 + sl * 32;
-                            const uint32_t *g = gv + ss * 32;
-                            uint32_t o[16];
-                            if (i0 + 31 < j) {
-                                // below the diagonal block: row factor x column factor, both <= 1
-                                const float rf = expf(sj - sJb[i0 + 31]);
-                                const float4 *f4 = reinterpret_cast<const float4 *>(sFb + i0);
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const float4 f = f4[q];
-                                    const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
-                                    const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
-                                    const float2 m0 = mul_f32x2(
-                                        make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
-                                    const float2 m1 = mul_f32x2(
-                                        make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
-                                    o[2 * q] = pack_bf16x2(m0.x, m0.y);
-                                    o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
-                                }
-                            } else if (i0 > j) {
-#pragma unroll
-                                for (int q = 0; q < 16; ++q) o[q] = 0u;
-                            } else {
-                                // the diagonal 32x32 block: one exponential per element
-#pragma unroll
-                                for (int q = 0; q < 16; ++q) {
-                                    const int ia = i0 + 2 * q, ib = ia + 1;
-                                    float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
-                                    float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
-                                    if (ia == j) a += Dh;
-                                    if (ib == j) bb += Dh;
-                                    o[q] = pack_bf16x2(a, bb);
-                                }
-                            }
-                            tmem_st16(tM + sl * 16 + lane_base, o);
-                        }
-                    }
-                    tmem_wait_st();
+                    mask_half(1);
                     fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.m_full);
@@ -651,41 +754,41 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 SSD_TRACE_POINT(10);
                 fence_after_sync();
                 {
-                    uint32_t v[64];
-#pragma unroll
-                    for (int q0 = 0; q0 < kP; q0 += 16)
-                        tmem_ld16(tY + q0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[q0]));
+                    uint32_t v[32];
+                    tmem_ld16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                    tmem_ld16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
                     tmem_wait_ld();
                     fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.y_free);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < 4; ++q) {
                         uint4 w;
                         w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
                         w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
                         w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
                         w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                        *reinterpret_cast<uint4 *>(sSp + lrow * 128 + ((q ^ (lrow & 7)) << 4)) = w;
+                        const int qq = half * 4 + q;  // 16-byte chunk of the 128-byte row
+                        *reinterpret_cast<uint4 *>(sSp + lrow * 128 + ((qq ^ (lrow & 7)) << 4)) = w;
                     }
                     fence_view_async_shared();
-                    named_bar_sync(wg_bar, kWgThreads);
-                    if (wtid == kWgThreads - 1) {
+                    named_bar_sync(wg_bar, kPipeThreads);
+                    if (wtid == kPipeThreads - 1) {
                         tma_store_4d(&mY, sSp, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
                     }
                 }
                 SSD_TRACE_POINT(11);
 #ifdef SSD_TRACE
-                if (ssd_trace_buffer && wtid == 0 && trace_i < 60)
-                    ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 16 + 14] =
+                if (ssd_trace_buffer && wtid == 0 && trace_i < 30)
+                    ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 32 + 14] =
                         ((unsigned long long)h << 32) | ((unsigned long long)un.c << 8) | (first ? 1 : 0);
                 ++trace_i;
 #endif
             }
         }
     }
-    if (warp < 8 && (tid & (kWgThreads - 1)) == kWgThreads - 1) bulk_wait_all();
+    if (warp < kSimtWarps && (tid & (kPipeThreads - 1)) == kPipeThreads - 1) bulk_wait_all();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
