@@ -495,12 +495,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 SSD_TRACE_POINT(1);
                 wait_bar(&pb.j_full[jb], par_of(use >> 1), abort, p.status);
                 for (int i = wtid; i < kcols; i += kPipeThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
-                // the entering state S~_{c-1} is read once it is published (chunk 0 reads the initial
-                // state).  A second half asks here whether it is, a first half after its decay: if so
-                // its loads are in flight during the mask, else the mask is done while waiting
-                bool rdy = false;
-                if (!first && wtid == 0) rdy = un.c == 0 || ld_acquire_gpu(p.ready + bh) >= un.c;
-                rdy = named_bar_or(wg_bar, kPipeThreads, rdy);
+                named_bar_sync(wg_bar, kPipeThreads);
                 SSD_TRACE_POINT(2);
                 const float *src = (un.c == 0) ? (p.init ? p.init + bh * PN : nullptr)
                                                : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
@@ -514,51 +509,46 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 #pragma unroll 1
                     for (int sl = half; sl < 4; sl += 2) {
                         const int i0 = hf * 128 + sl * 32;
+                        uint32_t o[16];
                         if (i0 > j) {
-                            uint32_t z[8];
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) z[q] = 0u;
-                            tmem_st8(tM + sl * 16 + lane_base, z);
-                            tmem_st8(tM + sl * 16 + 8 + lane_base, z);
+                            for (int q = 0; q < 16; ++q) o[q] = 0u;
+                            tmem_st16(tM + sl * 16 + lane_base, o);
                             continue;
                         }
-                        const bool below = i0 + 31 < j;
-                        // below the diagonal block: row factor x column factor, both <= 1
-                        const float rf = below ? expf(sj - sJb[i0 + 31]) : 0.f;
-#pragma unroll 1
-                        for (int pc = 0; pc < 2; ++pc) {
-                            const int c0 = i0 + pc * 16;
-                            uint32_t g[16], o[8];
-                            tmem_ld16(tmem + kColG + c0 + lane_base, g);
-                            tmem_wait_ld();
-                            if (below) {
-                                const float4 *f4 = reinterpret_cast<const float4 *>(sFb + c0);
+                        uint32_t g[32];
+                        tmem_ld16(tmem + kColG + i0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+                        tmem_ld16(tmem + kColG + i0 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+                        tmem_wait_ld();
+                        if (i0 + 31 < j) {
+                            // below the diagonal block: row factor x column factor, both <= 1
+                            const float rf = expf(sj - sJb[i0 + 31]);
+                            const float4 *f4 = reinterpret_cast<const float4 *>(sFb + i0);
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const float4 f = f4[q];
-                                    const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
-                                    const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
-                                    const float2 m0 = mul_f32x2(
-                                        make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
-                                    const float2 m1 = mul_f32x2(
-                                        make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
-                                    o[2 * q] = pack_bf16x2(m0.x, m0.y);
-                                    o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
-                                }
-                            } else {
-                                // the diagonal 32x32 block: one exponential per element
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) {
-                                    const int ia = c0 + 2 * q, ib = ia + 1;
-                                    float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
-                                    float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
-                                    if (ia == j) a += Dh;
-                                    if (ib == j) bb += Dh;
-                                    o[q] = pack_bf16x2(a, bb);
-                                }
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 f = f4[q];
+                                const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
+                                const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
+                                const float2 m0 = mul_f32x2(
+                                    make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
+                                const float2 m1 = mul_f32x2(
+                                    make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
+                                o[2 * q] = pack_bf16x2(m0.x, m0.y);
+                                o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
                             }
-                            tmem_st8(tM + sl * 16 + pc * 8 + lane_base, o);
+                        } else {
+                            // the diagonal 32x32 block: one exponential per element
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                const int ia = i0 + 2 * q, ib = ia + 1;
+                                float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
+                                float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
+                                if (ia == j) a += Dh;
+                                if (ib == j) bb += Dh;
+                                o[q] = pack_bf16x2(a, bb);
+                            }
                         }
+                        tmem_st16(tM + sl * 16 + lane_base, o);
                     }
                     tmem_wait_st();
                 };
@@ -684,34 +674,25 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     scale_and_release_mask();
                     SSD_TRACE_POINT(7);
                 } else {
+                    // mask K-half 0 first, then wait for the entering state (chunk 0 reads the
+                    // initial state)
+                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
+                    fence_after_sync();
+                    mask_half(0);
+                    if (wtid == 0 && un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
+                    named_bar_sync(wg_bar, kPipeThreads);
                     // this thread's pieces of S~_{c-1} ([p][n]: 8 consecutive n of one row p each)
                     const int nchunks = kP * NK * 8;
                     float4 lo[4], hi[4];
-                    auto load_pieces = [&]() {
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int idx = wtid + r * kPipeThreads;
-                            const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
-                            lo[r] = hi[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (idx < nchunks && src && n < N) {
-                                lo[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n));
-                                hi[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
-                            }
+                    for (int r = 0; r < 4; ++r) {
+                        const int idx = wtid + r * kPipeThreads;
+                        const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
+                        lo[r] = hi[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (idx < nchunks && src && n < N) {
+                            lo[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n));
+                            hi[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
                         }
-                    };
-                    auto mask0 = [&]() {
-                        if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
-                        fence_after_sync();
-                        mask_half(0);
-                    };
-                    if (rdy) {
-                        load_pieces();
-                        mask0();
-                    } else {
-                        mask0();
-                        if (wtid == 0) wait_flag(p.ready + bh, un.c, abort, p.status);
-                        named_bar_sync(wg_bar, kPipeThreads);
-                        load_pieces();
                     }
                     SSD_TRACE_POINT(3);
                     SSD_TRACE_ARRIVED(reinterpret_cast<const float *>(lo), 16, 8);
@@ -733,7 +714,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (lane == 0) mbar_arrive(&pb.ring_done);
                     fence_view_async_shared();
                     named_bar_sync(wg_bar, kPipeThreads);
-                    __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.s_full);
                     SSD_TRACE_POINT(6);
                     scale_and_release_mask();
