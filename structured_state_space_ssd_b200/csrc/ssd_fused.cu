@@ -112,7 +112,8 @@ struct Params {
     float *fin;         // [b][H][P][N] or null
     float *ring;        // [b][H][2][P][N]
     int *ready;         // [b*H]: chunks whose outgoing state is published
-    int *cons;          // [b*H]: chunks whose second half has read its entering state
+    int *cons;          // [b*H]: second halves that have read their entering state (a count: second
+                        // halves of different chunks finish in any order)
     int *counter;       // unit dispenser
     int *status;
     __nv_bfloat16 *y;
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             st_release_gpu(p.ready + bh, un.c + 1);
                         }
                     } else {
-                        st_release_gpu(p.cons + bh, un.c + 1);
+                        red_release_add_gpu(p.cons + bh, 1);
                     }
                 }
                 __syncwarp();
@@ -472,9 +473,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
             if (un.row0 >= un.len) {
-                // no rows: release the (unread) entering state of every head for the slot's next writer
+                // no rows: count the (unread) entering state of every head as read
                 if (tid == 0)
-                    for (int h = un.h0; h < un.h1; ++h) st_release_gpu(p.cons + un.b * sh.H + h, un.c + 1);
+                    for (int h = un.h0; h < un.h1; ++h) red_release_add_gpu(p.cons + un.b * sh.H + h, 1);
                 continue;
             }
             const bool first = (un.r == 0);
@@ -610,7 +611,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     SSD_TRACE_POINT(22);
                     fence_after_sync();
                     mask_half(0);
-                    // S~_{c-1} must be published and the outgoing ring slot free of readers
+                    // S~_{c-1} must be published and the outgoing ring slot free of readers: the slot
+                    // held S~_{c-2}, read by the second half of chunk c-1, so wait until the second
+                    // halves of chunks 0..c-1 have all read theirs
                     if (wtid == 0) {
                         if (un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
                         if (p.halves == 2 && un.c >= 2) wait_flag(p.cons + bh, un.c, abort, p.status);
