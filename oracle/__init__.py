@@ -20,6 +20,9 @@ the "Transformers are SSMs" pages:
 * :func:`ssd_chunked_fwd` -- the block decomposition, stages 0 to 5 in the
   pages' order (section "The Block-Decomposition SSD Algorithm"), returning
   its intermediates (chunk states, propagated states) for diagnosis.
+* :func:`ssd_ref_step` -- one token of the recurrence (the autoregressive
+  mode: the same equation advanced by a single step, as the English note's
+  section "Working Through Four Tokens" does by hand), in numpy.
 
 Discretisation (the pages never write it): ``a_t = exp(dt_t * A_h)``, input
 term ``B_t x_t^T`` without a dt factor, skip ``D_h * x_t``, initial state
@@ -221,3 +224,31 @@ def ssd_chunked_fwd(x, dt, A, B, C, D, Q: int, init_state=None):
                 state = np.prod(ac) * state + S[b, c, h]                 # stage 3
             fin[b, h] = state
     return y, fin, S, S_prev
+
+
+def ssd_ref_step(state, x, dt, A, B, C, D):
+    """One autoregressive step of the recurrence in fp64 (numpy).
+
+    Layouts: state [b,H,P,N], x [b,H,P], dt [b,H], A [H], B/C [b,G,N], D [H].
+    For every (batch b, head h), with g = h // (H // G)::
+
+        a = exp(dt[b, h] * A[h])
+        S = a * state[b, h] + outer(x[b, h], B[b, g])      # S is [P, N]
+        y[b, h] = S @ C[b, g] + D[h] * x[b, h]
+
+    Returns (new_state, y); the input state is not modified.
+    """
+    state, x, dt, A, B, C, D = (_f64(v) for v in (state, x, dt, A, B, C, D))
+    batch, H, P, N = state.shape
+    G = B.shape[1]
+    assert x.shape == (batch, H, P) and dt.shape == (batch, H) and A.shape == (H,) and D.shape == (H,)
+    assert B.shape == (batch, G, N) and C.shape == B.shape and H % G == 0
+    new = np.empty_like(state)
+    y = np.empty((batch, H, P))
+    for b in range(batch):
+        for h in range(H):
+            g = h // (H // G)
+            a = np.exp(dt[b, h] * A[h])
+            new[b, h] = a * state[b, h] + np.outer(x[b, h], B[b, g])
+            y[b, h] = new[b, h] @ C[b, g] + D[h] * x[b, h]
+    return new, y
