@@ -392,6 +392,7 @@ def main():
             "gpu_launches": S.ssd_fwd_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
             * args.steps,
         }
+        line["decode_step"] = measure_decode(w, host, dev, stream, flush, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(host, w)
         print(json.dumps(line), flush=True)
@@ -401,6 +402,59 @@ def main():
 
 def _stage_uses_tensor_cores(name, w):
     return False
+
+
+def measure_decode(w, host, dev, stream, flush, peaks, steps=50, resident_steps=200):
+    """The decode step (one token of the recurrence, ssd_step) on the workload's batch, heads and state.
+
+    Each step reads and writes the whole fp32 state, so it is HBM-bound when the state is cold
+    (L2 flushed before every timed step) and L2-bound inside a decode loop that keeps it resident.
+    """
+    import torch
+    from structured_state_space_ssd_b200 import ssd as S
+    b, H, P, G, N = w.batch, w.H, w.P, w.G, w.N
+    gen = torch.Generator().manual_seed(w.seed + 99)
+    state = torch.randn((b, H, P, N), generator=gen).to(dev)
+    x, dt, B, C = (host[k][:, 0].contiguous().to(dev) for k in ("x", "dt", "B", "C"))
+    A, D = host["A"].to(dev), host["D"].to(dev)
+    y = torch.empty_like(x)
+    es = x.element_size()
+    alg = 2 * state.numel() * 4 + 2 * x.numel() * es + 2 * B.numel() * es + dt.numel() * 4 + 2 * H * 4
+
+    def one():
+        S.ssd_step(state, x, dt, A, B, C, D, y=y, stream=stream)
+
+    for _ in range(5):
+        flush.zero_()
+        one()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    cold_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    # a decode loop as a user runs it: the steps captured once in a CUDA graph and replayed, so that
+    # the host does not pace the launches
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream(dev)
+        for _ in range(resident_steps):
+            S.ssd_step(state, x, dt, A, B, C, D, y=y, stream=cap)
+    graph.replay()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    graph.replay()
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    warm_ms = r0.elapsed_time(r1) / resident_steps
+    del graph
+    gbps = alg / (cold_ms * 1e-3) / 1e9
+    return {"state_shape": [b, H, P, N], "dtype": w.dtype, "alg_bytes": alg,
+            "us_per_step_cold": cold_ms * 1e3, "GBps_cold": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"],
+            "us_per_step_l2_resident": warm_ms * 1e3, "l2_resident_loop": f"{resident_steps} steps in one CUDA graph",
+            "GBps_l2_resident": alg / (warm_ms * 1e-3) / 1e9, "launches_per_step": 1}
 
 
 def _traffic_from_profiles(kernel, w):

@@ -155,6 +155,35 @@ SSD_API int ssd_fwd_no_alloc(const void *x, const float *dt, const float *A, con
                      const float *D, int Q, const float *init_state, void *y, float *final_state,
                      int batch, int T, int H, int P, int G, int N, int dtype, void *stream);
 
+/*
+ * One autoregressive (decode) step of the same recurrence, in place: for
+ * every batch row b and head h, with g = h / (H / G),
+ *
+ *     state[b][h] = exp(dt[b][h] * A[h]) * state[b][h] + x[b][h] B[b][g]^T
+ *     y[b][h]     = state[b][h] C[b][g] + D[h] * x[b][h]
+ *
+ * (the recurrent mode: "Transformers are SSMs", analysis page, section "The
+ * Scalar-Identity SSM"; the English note's section "Working Through Four
+ * Tokens" advances it one token at a time).  Calling it for t = 0 .. T-1 from
+ * state = init_state gives the y and final_state of ssd_fwd over those T
+ * tokens, up to rounding.
+ *
+ *   state  [batch][H][P][N]   fp32    h_{t-1} on entry, h_t on return
+ *   x      [batch][H][P]      dtype   this token's input
+ *   dt     [batch][H]         fp32    step sizes
+ *   A, D   [H]                fp32
+ *   B, C   [batch][G][N]      dtype
+ *   y      [batch][H][P]      dtype   output (written)
+ *
+ * Limits: batch, H, G, P, N >= 1, H % G == 0, N <= 1024 (else
+ * SSD_ERR_UNSUPPORTED), batch and H <= 65535.  Pointers aligned to their
+ * element size; y and the state must not overlap each other or an input.  No
+ * workspace, no host synchronisation.  Returns SSD_OK, SSD_ERR_INVALID_ARG,
+ * SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
+ */
+SSD_API int ssd_step(float *state, const void *x, const float *dt, const float *A, const void *B, const void *C,
+             const float *D, void *y, int batch, int H, int P, int G, int N, int dtype, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

@@ -23,7 +23,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
-           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc")
+           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc",
+           "ssd_step")
 
 
 class SSDError(RuntimeError):
@@ -64,6 +65,8 @@ def load():
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_version.argtypes = []
     lib.ssd_version.restype = i
+    lib.ssd_step.argtypes = [vp, vp, fp, fp, vp, vp, fp, vp, i, i, i, i, i, i, vp]
+    lib.ssd_step.restype = i
     _lib = lib
     return lib
 
@@ -183,3 +186,42 @@ def ssd_fwd_check(workspace, stream=None) -> int:
         stream = torch.cuda.current_stream(workspace.device)
     handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
     return int(load().ssd_fwd_check(_ptr(workspace), ctypes.c_void_p(handle)))
+
+
+def ssd_step(state, x, dt, A, B, C, D, *, y=None, stream=None):
+    """One decode step on the GPU: updates ``state`` in place and returns y.
+
+    state [b,H,P,N] fp32, x [b,H,P] and B/C [b,G,N] (fp32 or bf16, one dtype),
+    dt [b,H], A [H], D [H] fp32 -- contiguous CUDA tensors on one device.
+    Runs on ``stream`` (default: the current torch stream) without host sync.
+    """
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_step needs CUDA tensors (there is no CPU path)")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    code = _dtype_code(x.dtype)
+    named = dict(state=state, x=x, dt=dt, A=A, B=B, C=C, D=D)
+    for k, t in named.items():
+        if t.device != dev:
+            raise ValueError(f"{k} is on {t.device}, x on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{k} must be contiguous")
+    if B.dtype != x.dtype or C.dtype != x.dtype:
+        raise TypeError("x, B and C must share one dtype")
+    for k in ("state", "dt", "A", "D"):
+        if named[k].dtype != torch.float32:
+            raise TypeError(f"{k} must be float32")
+    if tuple(state.shape) != (b, H, P, N) or tuple(dt.shape) != (b, H) or tuple(A.shape) != (H,) \
+            or tuple(D.shape) != (H,) or tuple(C.shape) != (b, G, N):
+        raise ValueError("expected state [b,H,P,N], dt [b,H], A and D [H], B and C [b,G,N]")
+    if y is None:
+        y = torch.empty_like(x)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    rc = load().ssd_step(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                         b, H, P, G, N, code, ctypes.c_void_p(handle))
+    if rc != 0:
+        raise SSDError(rc, "ssd_step")
+    return y

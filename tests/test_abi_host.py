@@ -97,3 +97,27 @@ def _call(lib, **over):
 ])
 def test_invalid_arguments_are_rejected_on_the_host(lib, over, code):
     assert _call(lib, **over) == code
+
+
+def _step(lib, **over):
+    """ssd_step with fake (never dereferenced) pointers; only validation runs."""
+    args = dict(state=0x100000, x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, y=0x70000,
+                batch=1, H=2, P=16, G=1, N=16, dtype=0, stream=None)
+    args.update(over)
+    v = lambda a: None if a is None else ctypes.c_void_p(a)  # noqa: E731
+    return lib.ssd_step(v(args["state"]), v(args["x"]), v(args["dt"]), v(args["A"]), v(args["B"]), v(args["C"]),
+                        v(args["D"]), v(args["y"]), args["batch"], args["H"], args["P"], args["G"], args["N"],
+                        args["dtype"], v(args["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(state=None), 1), (dict(x=None), 1), (dict(dt=None), 1), (dict(A=None), 1), (dict(B=None), 1),
+    (dict(C=None), 1), (dict(D=None), 1), (dict(y=None), 1),
+    (dict(batch=0), 1), (dict(H=0), 1), (dict(P=0), 1), (dict(N=0), 1), (dict(G=0), 1), (dict(H=3, G=2), 1),
+    (dict(dtype=4), 1), (dict(N=1025), 2),
+    (dict(x=0x10002), 1),                 # fp32 tensor not 4-byte aligned
+    (dict(y=0x100000 + 64), 1),           # y inside the state
+    (dict(y=0x10000), 1),                 # y aliases x
+])
+def test_step_rejects_invalid_arguments_on_the_host(lib, over, code):
+    assert _step(lib, **over) == code
