@@ -23,6 +23,10 @@ the "Transformers are SSMs" pages:
 * :func:`ssd_ref_step` -- one token of the recurrence (the autoregressive
   mode: the same equation advanced by a single step, as the English note's
   section "Working Through Four Tokens" does by hand), in numpy.
+* :func:`ref_gate_norm` -- the Mamba-2 block's step after the layer: the
+  output gated by Swish of a parallel branch z, then GroupNorm (analysis
+  page, section "The Mamba-2 Architecture", paragraphs "Gating" and "Extra
+  normalization"), in numpy.
 
 Discretisation (the pages never write it): ``a_t = exp(dt_t * A_h)``, input
 term ``B_t x_t^T`` without a dt factor, skip ``D_h * x_t``, initial state
@@ -252,3 +256,28 @@ def ssd_ref_step(state, x, dt, A, B, C, D):
             new[b, h] = a * state[b, h] + np.outer(x[b, h], B[b, g])
             y[b, h] = new[b, h] @ C[b, g] + D[h] * x[b, h]
     return new, y
+
+
+def ref_gate_norm(y, z, ngroups, eps=1e-5, weight=None, bias=None):
+    """Gate then GroupNorm in fp64 (numpy), per token.
+
+    y, z [..., channels] (channels = H * P, the layer's output flattened per token);
+    weight, bias [channels] or None (1 and 0).  With g = y * silu(z) = y * z / (1 + exp(-z)),
+    the channels of each token split into ``ngroups`` contiguous groups, and per group::
+
+        out = (g - mean(g)) / sqrt(var(g) + eps) * weight + bias       (var: population variance)
+    """
+    y, z = _f64(y), _f64(z)
+    shape = y.shape
+    ch = shape[-1]
+    assert z.shape == shape and ch % ngroups == 0
+    g = y * z / (1.0 + np.exp(-z))
+    gg = g.reshape(-1, ngroups, ch // ngroups)
+    mean = gg.mean(axis=2, keepdims=True)
+    var = ((gg - mean) ** 2).mean(axis=2, keepdims=True)
+    out = ((gg - mean) / np.sqrt(var + eps)).reshape(shape)
+    if weight is not None:
+        out = out * _f64(weight)
+    if bias is not None:
+        out = out + _f64(bias)
+    return out
