@@ -393,6 +393,7 @@ def main():
             * args.steps,
         }
         line["decode_step"] = measure_decode(w, host, dev, stream, flush, peaks)
+        line["gate_norm"] = measure_gate_norm(w, y, dev, stream, flush, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(host, w)
         print(json.dumps(line), flush=True)
@@ -455,6 +456,36 @@ def measure_decode(w, host, dev, stream, flush, peaks, steps=50, resident_steps=
             "us_per_step_cold": cold_ms * 1e3, "GBps_cold": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"],
             "us_per_step_l2_resident": warm_ms * 1e3, "l2_resident_loop": f"{resident_steps} steps in one CUDA graph",
             "GBps_l2_resident": alg / (warm_ms * 1e-3) / 1e9, "launches_per_step": 1}
+
+
+def measure_gate_norm(w, y, dev, stream, flush, peaks, steps=20):
+    """The block's step after the layer (Swish gate by z, GroupNorm with a group per head) on this
+    workload's output y, L2 flushed before each launch: one read of y and z, one write."""
+    import torch
+    from structured_state_space_ssd_b200 import ssd as S
+    gen = torch.Generator().manual_seed(w.seed + 7)
+    yv = y.view(-1, w.H * w.P)  # per token: all heads' channels
+    z = torch.randn(tuple(yv.shape), generator=gen).to(y.dtype).to(dev)
+    out = torch.empty_like(yv)
+    alg = 3 * y.numel() * y.element_size()
+
+    def one():
+        S.ssd_gate_norm(yv, z, w.H, 1e-5, out=out, stream=stream)
+
+    for _ in range(3):
+        flush.zero_()
+        one()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    gbps = alg / (ms * 1e-3) / 1e9
+    return {"rows": y.numel() // (w.H * w.P), "channels": w.H * w.P, "ngroups": w.H, "dtype": w.dtype,
+            "alg_bytes": alg, "us_per_launch": ms * 1e3, "GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"]}
 
 
 def _traffic_from_profiles(kernel, w):

@@ -184,6 +184,27 @@ SSD_API int ssd_fwd_no_alloc(const void *x, const float *dt, const float *A, con
 SSD_API int ssd_step(float *state, const void *x, const float *dt, const float *A, const void *B, const void *C,
              const float *D, void *y, int batch, int H, int P, int G, int N, int dtype, void *stream);
 
+/*
+ * The Mamba-2 block's step after the layer: the output gated by the Swish of
+ * a parallel branch z, then GroupNorm ("Transformers are SSMs", analysis page,
+ * section "The Mamba-2 Architecture", paragraphs "Gating" and "Extra
+ * normalization").  Per token (row), with g = y * silu(z) = y * z / (1 + e^-z)
+ * and the channels split into ngroups contiguous groups,
+ *
+ *     out = (g - mean(g)) / sqrt(var(g) + eps) * weight + bias      (per group, population variance)
+ *
+ *   y, z, out  [rows][channels]  dtype   y is ssd_fwd's output viewed as [batch*T][H*P]
+ *   weight     [channels]        fp32    NULL = 1
+ *   bias       [channels]        fp32    NULL = 0
+ *
+ * Limits: rows >= 0, channels >= 1, channels % ngroups == 0, channels /
+ * ngroups <= 4096 (else SSD_ERR_UNSUPPORTED), eps >= 0.  out may be y
+ * (in place) but must not otherwise overlap y or z.  Returns SSD_OK,
+ * SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
+ */
+SSD_API int ssd_gate_norm(const void *y, const void *z, const float *weight, const float *bias, void *out,
+                  long long rows, int channels, int ngroups, float eps, int dtype, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

@@ -24,7 +24,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
            "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc",
-           "ssd_step")
+           "ssd_step", "ssd_gate_norm")
 
 
 class SSDError(RuntimeError):
@@ -67,6 +67,8 @@ def load():
     lib.ssd_version.restype = i
     lib.ssd_step.argtypes = [vp, vp, fp, fp, vp, vp, fp, vp, i, i, i, i, i, i, vp]
     lib.ssd_step.restype = i
+    lib.ssd_gate_norm.argtypes = [vp, vp, fp, fp, vp, ctypes.c_longlong, i, i, ctypes.c_float, i, vp]
+    lib.ssd_gate_norm.restype = i
     _lib = lib
     return lib
 
@@ -225,3 +227,34 @@ def ssd_step(state, x, dt, A, B, C, D, *, y=None, stream=None):
     if rc != 0:
         raise SSDError(rc, "ssd_step")
     return y
+
+
+def ssd_gate_norm(y, z, ngroups: int, eps: float = 1e-5, weight=None, bias=None, *, out=None, stream=None):
+    """Swish gate then GroupNorm on the GPU: ``out = GroupNorm(y * silu(z))`` per token.
+
+    y and z have one shape [..., channels] and dtype (fp32 or bf16); the channels of each token split
+    into ``ngroups`` contiguous groups.  weight, bias: fp32 [channels] or None.  ``out`` may be y.
+    """
+    dev = y.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_gate_norm needs CUDA tensors (there is no CPU path)")
+    if z.shape != y.shape or z.dtype != y.dtype or z.device != dev:
+        raise ValueError("y and z must have one shape, dtype and device")
+    ch = y.shape[-1]
+    for k, t in (("y", y), ("z", z), ("weight", weight), ("bias", bias)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{k} must be contiguous")
+    for k, t in (("weight", weight), ("bias", bias)):
+        if t is not None and (t.dtype != torch.float32 or t.numel() != ch or t.device != dev):
+            raise ValueError(f"{k} must be a float32 [{ch}] tensor on {dev}")
+    if out is None:
+        out = torch.empty_like(y)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    rows = y.numel() // ch
+    rc = load().ssd_gate_norm(_ptr(y), _ptr(z), _ptr(weight), _ptr(bias), _ptr(out), rows, ch, int(ngroups),
+                              float(eps), _dtype_code(y.dtype), ctypes.c_void_p(handle))
+    if rc != 0:
+        raise SSDError(rc, "ssd_gate_norm")
+    return out

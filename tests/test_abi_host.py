@@ -121,3 +121,26 @@ def _step(lib, **over):
 ])
 def test_step_rejects_invalid_arguments_on_the_host(lib, over, code):
     assert _step(lib, **over) == code
+
+
+def _gn(lib, **over):
+    """ssd_gate_norm with fake (never dereferenced) pointers; only validation runs."""
+    args = dict(y=0x100000, z=0x200000, w=None, b=None, out=0x300000, rows=4, ch=64, ng=4, eps=1e-5, dtype=1,
+                stream=None)
+    args.update(over)
+    v = lambda a: None if a is None else ctypes.c_void_p(a)  # noqa: E731
+    return lib.ssd_gate_norm(v(args["y"]), v(args["z"]), v(args["w"]), v(args["b"]), v(args["out"]), args["rows"],
+                             args["ch"], args["ng"], ctypes.c_float(args["eps"]), args["dtype"], v(args["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(y=None), 1), (dict(z=None), 1), (dict(out=None), 1), (dict(rows=-1), 1), (dict(ch=0), 1),
+    (dict(ng=0), 1), (dict(ng=5), 1), (dict(eps=-1.0), 1), (dict(dtype=3), 1),
+    (dict(ch=8192, ng=1), 2),             # a group larger than the kernel holds
+    (dict(y=0x100001), 1),                # bf16 tensor not 2-byte aligned
+    (dict(out=0x200000), 1),              # out aliases z
+    (dict(out=0x100000 + 64), 1),         # out partly overlaps y
+    (dict(rows=0), 0),                    # nothing to do
+])
+def test_gate_norm_rejects_invalid_arguments_on_the_host(lib, over, code):
+    assert _gn(lib, **over) == code
