@@ -820,7 +820,7 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, con
     p.y = y;
     p.NK = (sh.N + 63) / 64;
     p.halves = sh.Q / kRows;
-    p.heads_per_unit = min(8, sh.heads_per_group);
+    p.heads_per_unit = min(4, sh.heads_per_group);
     p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
     p.n_units = sh.nc * sh.batch * sh.G * p.blocks_per_group * p.halves;
     cudaError_t e =
