@@ -30,7 +30,9 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
+// z * sigmoid(z) with the fast exponential and reciprocal: the kernel is otherwise bound by issue,
+// not by memory (for very negative z the reciprocal of an infinite denominator is 0)
+__device__ __forceinline__ float silu(float z) { return z * __frcp_rn(1.f + __expf(-z)); }
 
 template <typename T>
 __global__ void __launch_bounds__(kGnWarps * 32)
@@ -118,16 +120,18 @@ __device__ __forceinline__ void store8<float>(float *p, const float (&v)[8]) {
 
 // Groups of 8 * L channels (L = 1, 2, .., 32 lanes per group, 32 / L groups per warp): every lane
 // holds 8 consecutive channels in registers, the group's sums are shuffle reductions over its L lanes.
+// Groups are numbered in memory order (token-major), so a group's channels start at unit * gs and its
+// channel offset within the token is (unit % ngroups) * gs (32-bit arithmetic when it fits).
 template <typename T, int L>
 __global__ void __launch_bounds__(kGnWarps * 32)
     gate_norm_small_kernel(const T *y, const T *__restrict__ z, const float *__restrict__ weight,
-                           const float *__restrict__ bias, T *out, long long units, int C, float eps) {
+                           const float *__restrict__ bias, T *out, long long units, int ngroups, float eps) {
     constexpr int gs = 8 * L;
     const long long t = (long long)blockIdx.x * kGnWarps * 32 + threadIdx.x;
-    const long long unit = t / L;  // (token, group), in channel order
+    const long long unit = t / L;
     const bool active = unit < units;
-    const int sub = (int)(t % L);
-    const size_t base = (size_t)(active ? unit : 0) * gs + sub * 8;  // groups tile each row contiguously
+    const int sub = (int)(t & (L - 1));
+    const size_t base = (size_t)(active ? unit : 0) * gs + sub * 8;
     float g[8], zv[8];
     float sum = 0.f;
     if (active) {
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(kGnWarps * 32)
     }
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float mean = sum / gs;
+    const float mean = sum * (1.f / gs);
     float sq = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -151,24 +155,28 @@ __global__ void __launch_bounds__(kGnWarps * 32)
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     if (!active) return;
-    const float rstd = rsqrtf(sq / gs + eps);
-    const int c = (int)(base % C);
+    const float rstd = rsqrtf(sq * (1.f / gs) + eps);
+    if (weight || bias) {
+        const int grp = units < (1LL << 31) ? (int)unit % ngroups : (int)(unit % ngroups);
+        const int c = grp * gs + sub * 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        g[i] = (g[i] - mean) * rstd;
-        if (weight) g[i] *= weight[c + i];
-        if (bias) g[i] += bias[c + i];
+        for (int i = 0; i < 8; ++i)
+            g[i] = fmaf((g[i] - mean) * rstd, weight ? weight[c + i] : 1.f, bias ? bias[c + i] : 0.f);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[i] = (g[i] - mean) * rstd;
     }
     store8<T>(out + base, g);
 }
 
 template <typename T, int L>
 cudaError_t launch_small(const void *y, const void *z, const float *weight, const float *bias, void *out,
-                         long long units, int C, float eps, cudaStream_t st) {
+                         long long units, int ngroups, float eps, cudaStream_t st) {
     const long long threads = units * L;
     const long long blocks = (threads + kGnWarps * 32 - 1) / (kGnWarps * 32);
     gate_norm_small_kernel<T, L><<<(unsigned)blocks, kGnWarps * 32, 0, st>>>(
-        static_cast<const T *>(y), static_cast<const T *>(z), weight, bias, static_cast<T *>(out), units, C, eps);
+        static_cast<const T *>(y), static_cast<const T *>(z), weight, bias, static_cast<T *>(out), units, ngroups,
+        eps);
     return cudaGetLastError();
 }
 
@@ -179,12 +187,12 @@ cudaError_t launch_gate_norm(const void *y, const void *z, const float *weight, 
     const long long units = rows * ngroups;
     if (vec_ok) {
         switch (gs) {
-            case 8: return launch_small<T, 1>(y, z, weight, bias, out, units, C, eps, st);
-            case 16: return launch_small<T, 2>(y, z, weight, bias, out, units, C, eps, st);
-            case 32: return launch_small<T, 4>(y, z, weight, bias, out, units, C, eps, st);
-            case 64: return launch_small<T, 8>(y, z, weight, bias, out, units, C, eps, st);
-            case 128: return launch_small<T, 16>(y, z, weight, bias, out, units, C, eps, st);
-            case 256: return launch_small<T, 32>(y, z, weight, bias, out, units, C, eps, st);
+            case 8: return launch_small<T, 1>(y, z, weight, bias, out, units, ngroups, eps, st);
+            case 16: return launch_small<T, 2>(y, z, weight, bias, out, units, ngroups, eps, st);
+            case 32: return launch_small<T, 4>(y, z, weight, bias, out, units, ngroups, eps, st);
+            case 64: return launch_small<T, 8>(y, z, weight, bias, out, units, ngroups, eps, st);
+            case 128: return launch_small<T, 16>(y, z, weight, bias, out, units, ngroups, eps, st);
+            case 256: return launch_small<T, 32>(y, z, weight, bias, out, units, ngroups, eps, st);
             default: break;
         }
     }

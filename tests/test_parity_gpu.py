@@ -178,3 +178,33 @@ def test_status_word_is_clear_after_a_run(cuda_device):
                      device=cuda_device)
     ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], 64, None, workspace=ws)
     assert ssd_fwd_check(ws) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_forward_replays_from_a_cuda_graph(dtype, cuda_device):
+    # a serving loop captures the forward once and replays it: same launches, same results
+    inp = make_inputs(2, 600, 8, 64, 128, 2, dtype, seed=31, with_init=True)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    from structured_state_space_ssd_b200.ssd import ssd_fwd_workspace_bytes
+    ws = torch.empty(ssd_fwd_workspace_bytes(2, 600, 8, 64, 2, 128, 256, d["x"].dtype), dtype=torch.uint8,
+                     device=cuda_device)
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((2, 8, 64, 128), dtype=torch.float32, device=cuda_device)
+
+    def fwd():
+        ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], 256, d["init_state"], y=y, final_state=fin,
+                workspace=ws, stream=torch.cuda.current_stream(cuda_device))
+
+    fwd()
+    torch.cuda.synchronize(cuda_device)
+    y_eager, f_eager = y.clone(), fin.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fwd()
+    for _ in range(2):
+        y.zero_()
+        fin.zero_()
+        graph.replay()
+        torch.cuda.synchronize(cuda_device)
+        assert torch.equal(y, y_eager) and torch.equal(fin, f_eager)
+    del graph
