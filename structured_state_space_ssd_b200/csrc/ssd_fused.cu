@@ -23,18 +23,23 @@
 //    decay mask M = G o exp(s_j - s_i) (+ D_h on the diagonal) written by the
 //    CUDA cores into TMEM as the bf16 A operand, Y += M X (stage 1), y = bf16(Y)
 //    (stage 5).
-//  * Second-half units read S~_{c-1} from the ring and then release the
-//    slot; a first-half unit overwrites a slot only after both readers of its
-//    previous content are done.  Every wait is bounded: on expiry the status
-//    word is set to SSD_ERR_TIMEOUT and the CTA finishes without waiting.
+//  * Second-half units read S~_{c-1} from the ring and count themselves as
+//    done with it; a first-half unit overwrites a slot only after every
+//    second half up to the previous chunk has read (a count, since second
+//    halves of different chunks finish in any order).  Every wait is
+//    bounded: on expiry the status word is set to SSD_ERR_TIMEOUT and the
+//    CTA finishes without waiting.
 //
-// Warp roles: each CTA runs two head pipelines side by side.  Pipeline pl
-// takes every other head of a unit; its CUDA-core warpgroup (warps 4pl..4pl+3,
-// covering the 128 TMEM lanes) and its issuer warp (8 + pl; one lane issues
-// TMA loads and tcgen05.mma) hand the pipeline's own X tile, state tile,
-// decay mask (one 128-token K-half at a time) and accumulators back and forth
-// through mbarriers, so that one pipeline's CUDA-core work overlaps the other's
-// tensor-core products.  C, B and G are shared by the unit's heads.
+// Warp roles: each CTA runs two head pipelines side by side; pipeline pl
+// takes every other head of a unit (units hold up to 4 heads).  Its eight
+// CUDA-core warps (warps 8pl..8pl+7: two warpgroups, each covering the 128
+// TMEM lanes and half of every tile's columns), its issuer warp (16 + pl;
+// one lane issues TMA loads and tcgen05.mma) and its publisher warp (18 + pl;
+// the GPU-scope fences and flags of the state hand-off) pass the pipeline's
+// own X tile, state tile, decay mask (one 128-token K-half at a time) and
+// accumulators back and forth through mbarriers, so that one pipeline's
+// CUDA-core work overlaps the other's tensor-core products.  C, B and G are
+// shared by the unit's heads.
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
