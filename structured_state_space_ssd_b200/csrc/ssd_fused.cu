@@ -265,11 +265,12 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // ------------------------------------------------------------------
         // Publisher warps: warp 18 + pl makes pipeline pl's chain hand-offs
         // visible, so that neither the CUDA-core warps nor the issuer wait
-        // for the GPU-scope fence.  After a first half's ring stores it
+        // for a GPU-scope release.  After a first half's ring stores it
         // releases `ready` (S~_c readable); after a second half consumed
-        // S~_{c-1} it releases `cons` (the ring slot may be rewritten).  The
-        // warps' arrival on ring_done orders their accesses before this
-        // thread's fence and flag.
+        // S~_{c-1} it adds one to `cons` (the ring slot may be rewritten).
+        // The warps' arrival on ring_done (a CTA-scope release, acquired by
+        // this thread's wait) puts their accesses before this thread's
+        // GPU-scope release, which carries them along (release is cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
         PipeBars &pb = bars.pb[pl];
@@ -289,10 +290,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 if (lane == 0) {
                     const size_t bh = (size_t)un.b * sh.H + h;
                     if (first) {
-                        if (un.c < sh.nc - 1) {
-                            __threadfence();
-                            st_release_gpu(p.ready + bh, un.c + 1);
-                        }
+                        if (un.c < sh.nc - 1) st_release_gpu(p.ready + bh, un.c + 1);
                     } else {
                         red_release_add_gpu(p.cons + bh, 1);
                     }
