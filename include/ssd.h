@@ -205,6 +205,42 @@ SSD_API int ssd_step(float *state, const void *x, const float *dt, const float *
 SSD_API int ssd_gate_norm(const void *y, const void *z, const float *weight, const float *bias, void *out,
                   long long rows, int channels, int ngroups, float eps, int dtype, void *stream);
 
+/*
+ * Sequence split: contiguous shards of one sequence (on one GPU or one per
+ * worker) run ssd_fwd from a zero state at the same time and exchange only
+ * their states.  Workers process contiguous shards and pass recurrent states
+ * between them, communication linear in the number of workers (the paper's
+ * claim summary on its reproduction page); it is the block decomposition of
+ * "Transformers are SSMs" (analysis page, section "The Block-Decomposition
+ * SSD Algorithm", stages 3 and 4) one level up, shards in the place of
+ * chunks.  For shard k of K, with sigma_t the inclusive sum of dt_u * A_h
+ * over the shard's tokens up to t:
+ *
+ *   1. ssd_fwd(shard, init_state = NULL)  -> y0, fin0
+ *   2. ssd_split_logdecay                 -> sig [batch][H][T_shard], total [batch][H]
+ *   3. exchange (fin0, total) of every shard, shard order, into
+ *      fin0_all [K][batch][H][P][N] and total_all [K][batch][H]
+ *   4. ssd_split_combine(k)               -> s_in = state entering shard k (fold of the
+ *      earlier shards over init_state) and the shard's true final state
+ *   5. ssd_split_correct                  -> y += exp(sigma_t) s_in C_t, in place
+ *
+ * gives the y and final_state of ssd_fwd over the whole sequence (up to
+ * rounding; bf16 y is rounded once more).  Layouts as for ssd_fwd; all
+ * pointers are device pointers; sig, total, s_in are fp32.
+ *
+ * ssd_split_logdecay: dt [batch][T][H], A [H] -> sig, total.  T >= 1.
+ * ssd_split_combine: init_state and final_state may be NULL (zero / not written).
+ * ssd_split_correct: y [batch][T][H][P] (dtype, updated in place), C [batch][T][G][N]
+ * (dtype), sig, s_in [batch][H][P][N].  Limits P <= 128, N <= 256.
+ * Each returns SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
+ */
+SSD_API int ssd_split_logdecay(const float *dt, const float *A, float *sig, float *total, int batch, int T, int H,
+                       void *stream);
+SSD_API int ssd_split_combine(const float *fin0_all, const float *total_all, const float *init_state, int k,
+                      int shards, float *s_in, float *final_state, int batch, int H, int P, int N, void *stream);
+SSD_API int ssd_split_correct(void *y, const void *C, const float *sig, const float *s_in, int batch, int T, int H,
+                      int P, int G, int N, int dtype, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

@@ -24,7 +24,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
            "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc",
-           "ssd_step", "ssd_gate_norm")
+           "ssd_step", "ssd_gate_norm", "ssd_split_logdecay", "ssd_split_combine", "ssd_split_correct")
 
 
 class SSDError(RuntimeError):
@@ -69,6 +69,12 @@ def load():
     lib.ssd_step.restype = i
     lib.ssd_gate_norm.argtypes = [vp, vp, fp, fp, vp, ctypes.c_longlong, i, i, ctypes.c_float, i, vp]
     lib.ssd_gate_norm.restype = i
+    lib.ssd_split_logdecay.argtypes = [fp, fp, fp, fp, i, i, i, vp]
+    lib.ssd_split_logdecay.restype = i
+    lib.ssd_split_combine.argtypes = [fp, fp, fp, i, i, fp, fp, i, i, i, i, vp]
+    lib.ssd_split_combine.restype = i
+    lib.ssd_split_correct.argtypes = [vp, vp, fp, fp, i, i, i, i, i, i, i, vp]
+    lib.ssd_split_correct.restype = i
     _lib = lib
     return lib
 
@@ -258,3 +264,76 @@ def ssd_gate_norm(y, z, ngroups: int, eps: float = 1e-5, weight=None, bias=None,
     if rc != 0:
         raise SSDError(rc, "ssd_gate_norm")
     return out
+
+
+# --- sequence split: shards of one sequence run at once and exchange only their states ---------------
+
+def _handle(stream, dev):
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def ssd_split_logdecay(dt, A, *, stream=None):
+    """Per-token inclusive log-decay prefix of a shard: returns (sig [b,H,T], total [b,H]) fp32."""
+    b, T, H = dt.shape
+    sig = torch.empty((b, H, T), dtype=torch.float32, device=dt.device)
+    total = torch.empty((b, H), dtype=torch.float32, device=dt.device)
+    rc = load().ssd_split_logdecay(_ptr(dt), _ptr(A), _ptr(sig), _ptr(total), b, T, H, _handle(stream, dt.device))
+    if rc != 0:
+        raise SSDError(rc, "ssd_split_logdecay")
+    return sig, total
+
+
+def ssd_split_combine(fin0_all, total_all, k: int, init_state=None, *, stream=None):
+    """State entering shard k and the shard's true final state, from every shard's zero-start final state
+    fin0_all [K,b,H,P,N] and total log decay total_all [K,b,H] (shard order)."""
+    K, b, H, P, N = fin0_all.shape
+    s_in = torch.empty((b, H, P, N), dtype=torch.float32, device=fin0_all.device)
+    fin = torch.empty_like(s_in)
+    rc = load().ssd_split_combine(_ptr(fin0_all), _ptr(total_all), _ptr(init_state), int(k), K, _ptr(s_in),
+                                  _ptr(fin), b, H, P, N, _handle(stream, fin0_all.device))
+    if rc != 0:
+        raise SSDError(rc, "ssd_split_combine")
+    return s_in, fin
+
+
+def ssd_split_correct(y, C, sig, s_in, *, stream=None):
+    """y += exp(sig_t) s_in C_t in place (y [b,T,H,P], C [b,T,G,N]); returns y."""
+    b, T, H, P = y.shape
+    G, N = C.shape[2], C.shape[3]
+    rc = load().ssd_split_correct(_ptr(y), _ptr(C), _ptr(sig), _ptr(s_in), b, T, H, P, G, N, _dtype_code(y.dtype),
+                                  _handle(stream, y.device))
+    if rc != 0:
+        raise SSDError(rc, "ssd_split_correct")
+    return y
+
+
+def exchange_shard_states(fin0, total, group=None):
+    """All-gather every worker's (zero-start final state, total log decay) in rank order: the one exchange
+    of the sequence split.  Returns (fin0_all [K,...], total_all [K,...])."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    fin0_all = torch.empty((world,) + tuple(fin0.shape), dtype=fin0.dtype, device=fin0.device)
+    total_all = torch.empty((world,) + tuple(total.shape), dtype=total.dtype, device=total.device)
+    dist.all_gather(list(fin0_all.unbind(0)), fin0.contiguous(), group=group)
+    dist.all_gather(list(total_all.unbind(0)), total.contiguous(), group=group)
+    return fin0_all, total_all
+
+
+def ssd_fwd_sequence_parallel(x, dt, A, B, C, D, Q: int, init_state=None, group=None):
+    """This worker's shard of a sequence split across the workers of ``group`` (rank order = shard order).
+
+    Every worker passes its contiguous shard (x [b,T_k,H,P], dt, B, C) and the same A, D and
+    init_state (the state before the whole sequence, or None).  Returns (y_k, final_state_k): y of the
+    shard and the state after it, as ssd_fwd over the whole sequence would give them; the last worker's
+    final_state is the sequence's.
+    """
+    import torch.distributed as dist
+    k = dist.get_rank(group)
+    y, fin0 = ssd_fwd(x, dt, A, B, C, D, Q, None)
+    sig, total = ssd_split_logdecay(dt, A)
+    fin0_all, total_all = exchange_shard_states(fin0, total, group)
+    s_in, fin = ssd_split_combine(fin0_all, total_all, k, init_state)
+    ssd_split_correct(y, C, sig, s_in)
+    return y, fin

@@ -144,3 +144,17 @@ def _gn(lib, **over):
 ])
 def test_gate_norm_rejects_invalid_arguments_on_the_host(lib, over, code):
     assert _gn(lib, **over) == code
+
+
+@pytest.mark.parametrize("call,code", [
+    (lambda L, v: L.ssd_split_logdecay(None, v(1), v(2), v(3), 1, 8, 2, None), 1),
+    (lambda L, v: L.ssd_split_logdecay(v(4), v(8), v(12), v(16), 1, 0, 2, None), 1),          # T < 1
+    (lambda L, v: L.ssd_split_combine(v(4), v(8), None, 2, 2, v(12), None, 1, 2, 4, 4, None), 1),  # k >= K
+    (lambda L, v: L.ssd_split_combine(v(4), v(8), None, -1, 2, v(12), None, 1, 2, 4, 4, None), 1),
+    (lambda L, v: L.ssd_split_correct(v(4), v(8), v(12), v(16), 1, 8, 3, 4, 2, 4, 0, None), 1),  # H % G
+    (lambda L, v: L.ssd_split_correct(v(4), v(8), v(12), v(16), 1, 8, 2, 4, 1, 512, 0, None), 2),  # N > 256
+    (lambda L, v: L.ssd_split_correct(v(4), v(8), v(12), v(16), 1, 0, 2, 4, 1, 4, 0, None), 0),  # nothing to do
+])
+def test_split_entry_points_validate_on_the_host(lib, call, code):
+    v = lambda a: ctypes.c_void_p(0x100000 * a)  # noqa: E731  (never dereferenced)
+    assert call(lib, v) == code

@@ -56,3 +56,32 @@ def test_single_process_reduction_is_identity():
     w = WORKLOADS["mamba2_2p7b_layer"]
     assert bench.job_tokens_per_s(w, 1, 1.0) == w.tokens / 1e-3
     assert bench.rank_inputs(WORKLOADS["tiny_f32"], 0)["x"].shape == (1, 256, 2, 16)
+
+
+def _exchange_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from structured_state_space_ssd_b200.ssd import exchange_shard_states
+        fin0 = torch.full((2, 3, 4, 5), float(rank + 1))   # [b, H, P, N]
+        total = torch.full((2, 3), -0.5 * (rank + 1))      # [b, H]
+        fin0_all, total_all = exchange_shard_states(fin0, total)
+        out[rank] = (fin0_all[:, 0, 0, 0, 0].tolist(), total_all[:, 0, 0].tolist(), tuple(fin0_all.shape))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_split_exchange_stacks_states_in_rank_order():
+    # the one collective of the sequence split: every rank sees every shard's state, shard k at index k
+    world = 3
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_exchange_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert set(res) == {0, 1, 2}
+    for rank in range(world):
+        fins, totals, shape = res[rank]
+        assert fins == [1.0, 2.0, 3.0]
+        assert totals == [-0.5, -1.0, -1.5]
+        assert shape == (3, 2, 3, 4, 5)
