@@ -274,8 +274,19 @@ def _handle(stream, dev):
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _check_cuda_f32(**named):
+    for k, t in named.items():
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError(f"{k} must be a CUDA tensor (there is no CPU path)")
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError(f"{k} must be a contiguous float32 tensor")
+
+
 def ssd_split_logdecay(dt, A, *, stream=None):
     """Per-token inclusive log-decay prefix of a shard: returns (sig [b,H,T], total [b,H]) fp32."""
+    _check_cuda_f32(dt=dt, A=A)
     b, T, H = dt.shape
     sig = torch.empty((b, H, T), dtype=torch.float32, device=dt.device)
     total = torch.empty((b, H), dtype=torch.float32, device=dt.device)
@@ -288,7 +299,10 @@ def ssd_split_logdecay(dt, A, *, stream=None):
 def ssd_split_combine(fin0_all, total_all, k: int, init_state=None, *, stream=None):
     """State entering shard k and the shard's true final state, from every shard's zero-start final state
     fin0_all [K,b,H,P,N] and total log decay total_all [K,b,H] (shard order)."""
+    _check_cuda_f32(fin0_all=fin0_all, total_all=total_all, init_state=init_state)
     K, b, H, P, N = fin0_all.shape
+    if tuple(total_all.shape) != (K, b, H) or (init_state is not None and tuple(init_state.shape) != (b, H, P, N)):
+        raise ValueError("expected total_all [K,b,H] and init_state [b,H,P,N] matching fin0_all [K,b,H,P,N]")
     s_in = torch.empty((b, H, P, N), dtype=torch.float32, device=fin0_all.device)
     fin = torch.empty_like(s_in)
     rc = load().ssd_split_combine(_ptr(fin0_all), _ptr(total_all), _ptr(init_state), int(k), K, _ptr(s_in),
@@ -300,8 +314,13 @@ def ssd_split_combine(fin0_all, total_all, k: int, init_state=None, *, stream=No
 
 def ssd_split_correct(y, C, sig, s_in, *, stream=None):
     """y += exp(sig_t) s_in C_t in place (y [b,T,H,P], C [b,T,G,N]); returns y."""
+    _check_cuda_f32(sig=sig, s_in=s_in)
+    if C.dtype != y.dtype or not (y.is_contiguous() and C.is_contiguous()) or y.device != C.device:
+        raise TypeError("y and C must be contiguous tensors of one dtype on one device")
     b, T, H, P = y.shape
     G, N = C.shape[2], C.shape[3]
+    if tuple(sig.shape) != (b, H, T) or tuple(s_in.shape) != (b, H, P, N):
+        raise ValueError("expected sig [b,H,T] and s_in [b,H,P,N]")
     rc = load().ssd_split_correct(_ptr(y), _ptr(C), _ptr(sig), _ptr(s_in), b, T, H, P, G, N, _dtype_code(y.dtype),
                                   _handle(stream, y.device))
     if rc != 0:
