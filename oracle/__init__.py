@@ -23,6 +23,14 @@ the "Transformers are SSMs" pages:
 * :func:`ssd_ref_step` -- one token of the recurrence (the autoregressive
   mode: the same equation advanced by a single step, as the English note's
   section "Working Through Four Tokens" does by hand), in numpy.
+* :func:`ssd_ref_bwd` -- the gradients of the layer (x, dt, A, B, C, D and
+  the initial state) for given output gradients: the adjoint of the
+  recurrence stepped in reverse, in numpy.  The pages print no backward; the
+  gradient is unique, and its pins are central finite differences of
+  :func:`ssd_ref_fwd`, the adjoint identity of the linear map and closed
+  forms (``tests/test_oracle_bwd.py``).
+* :func:`ssd_ref_bwd_at` -- the same gradients at a few tokens from explicit
+  sums (no state history), for checks at full problem sizes.
 * :func:`ref_gate_norm` -- the Mamba-2 block's step after the layer: the
   output gated by Swish of a parallel branch z, then GroupNorm (analysis
   page, section "The Mamba-2 Architecture", paragraphs "Gating" and "Extra
@@ -280,4 +288,128 @@ def ref_gate_norm(y, z, ngroups, eps=1e-5, weight=None, bias=None):
         out = out * _f64(weight)
     if bias is not None:
         out = out + _f64(bias)
+    return out
+
+
+def _bwd_args(x, dt, A, B, C, D, dy, init_state, dfinal_state):
+    x, dt, A, B, C, D, dy, init_state, dfinal_state = (
+        _f64(v) for v in (x, dt, A, B, C, D, dy, init_state, dfinal_state))
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt.shape == (batch, T, H) and A.shape == (H,) and D.shape == (H,) and dy.shape == x.shape
+    assert B.shape == (batch, T, G, N) and C.shape == B.shape and H % G == 0
+    for st in (init_state, dfinal_state):
+        assert st is None or st.shape == (batch, H, P, N)
+    return x, dt, A, B, C, D, dy, init_state, dfinal_state
+
+
+def ssd_ref_bwd(x, dt, A, B, C, D, dy, init_state=None, dfinal_state=None):
+    """Reverse-mode gradient of the token-by-token recurrence (fp64, numpy).
+
+    The pages give the forward only (analysis page, section "The SSM as a
+    Matrix Transformation", equation (2), scalar-identity case); they motivate
+    training speed but print no backward algorithm.  The gradient of a
+    function is unique, so this oracle is the adjoint of that recurrence,
+    taken step by step in reverse order.  With the loss
+    ``L = sum(dy * y) + sum(dfinal_state * final_state)`` and, per (b, h), the
+    states ``h_t = a_t h_{t-1} + x_t B_t^T`` (``a_t = exp(dt_t A_h)``,
+    ``h_{-1}`` the initial state), the adjoint ``g_t = dL/dh_t`` obeys::
+
+        g_{T-1} = dfinal + dy_{T-1} C_{T-1}^T
+        g_t     = a_{t+1} g_{t+1} + dy_t C_t^T
+
+    and every input gradient is local to its token::
+
+        dx_t      = g_t B_t + D_h dy_t
+        dB_t      = sum over the group's heads of g_t^T x_t
+        dC_t      = sum over the group's heads of h_t^T dy_t
+        dlog a_t  = <g_t, a_t h_{t-1}>            (a_t = exp(dt_t A_h))
+        ddt_t     = A_h dlog a_t,   dA_h = sum_{b,t} dt_t dlog a_t
+        dD_h      = sum_{b,t} <dy_t, x_t>,   dinit = a_0 g_0
+
+    Every state of a batch row is kept ([T, H, P, N] fp64): small problems
+    only.  Returns a dict with dx [b,T,H,P], ddt [b,T,H], dA [H], dB, dC
+    [b,T,G,N], dD [H] and dinit_state [b,H,P,N], all fp64.
+    """
+    x, dt, A, B, C, D, dy, init_state, dfinal_state = _bwd_args(x, dt, A, B, C, D, dy, init_state, dfinal_state)
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    hpg = H // G
+    grp = np.arange(H) // hpg
+    out = {"dx": np.zeros_like(x), "ddt": np.zeros_like(dt), "dA": np.zeros(H), "dB": np.zeros_like(B),
+           "dC": np.zeros_like(C), "dD": np.zeros(H), "dinit_state": np.zeros((batch, H, P, N))}
+    for b in range(batch):
+        Bh, Ch = B[b][:, grp, :], C[b][:, grp, :]          # [T, H, N]: each head's group row
+        a = np.exp(dt[b] * A[None, :])                      # [T, H]
+        h0 = np.zeros((H, P, N)) if init_state is None else init_state[b]
+        states = np.empty((T, H, P, N))
+        S = h0
+        for t in range(T):
+            S = a[t][:, None, None] * S + x[b, t][:, :, None] * Bh[t][:, None, :]
+            states[t] = S
+        g = np.zeros((H, P, N)) if dfinal_state is None else dfinal_state[b].copy()
+        for t in range(T - 1, -1, -1):
+            g = g + dy[b, t][:, :, None] * Ch[t][:, None, :]          # g_t
+            out["dx"][b, t] = np.einsum("hpn,hn->hp", g, Bh[t]) + D[:, None] * dy[b, t]
+            out["dB"][b, t] = np.einsum("hpn,hp->hn", g, x[b, t]).reshape(G, hpg, N).sum(axis=1)
+            out["dC"][b, t] = np.einsum("hpn,hp->hn", states[t], dy[b, t]).reshape(G, hpg, N).sum(axis=1)
+            prev = states[t - 1] if t > 0 else h0
+            dlog = a[t] * np.einsum("hpn,hpn->h", g, prev)
+            out["ddt"][b, t] = A * dlog
+            out["dA"] += dt[b, t] * dlog
+            out["dD"] += np.einsum("hp,hp->h", dy[b, t], x[b, t])
+            g = a[t][:, None, None] * g                                 # carried to t-1
+        out["dinit_state"][b] = g
+    return out
+
+
+def ssd_ref_bwd_at(x, dt, A, B, C, D, dy, b, tokens, init_state=None, dfinal_state=None):
+    """The same gradients at chosen tokens of batch row ``b``, from explicit sums (fp64).
+
+    Instead of stepping the recurrence, each needed state is written out as
+    the sum it stands for (the unrolled form of equation (2), section "The SSM
+    as a Matrix Transformation"), with the decay products
+    ``a_{u+1} ... a_t = exp(sigma_t - sigma_u)`` from the running sum
+    ``sigma_t = sum_{v<=t} dt_v A_h`` (the log-space products of section "The
+    Scalar-Identity SSM")::
+
+        h_t = sum_{u<=t} exp(sigma_t - sigma_u) x_u B_u^T + exp(sigma_t) h_{-1}
+        g_t = sum_{k>=t} exp(sigma_k - sigma_t) dy_k C_k^T + exp(sigma_{T-1} - sigma_t) dfinal
+
+    and the per-token gradients follow as in :func:`ssd_ref_bwd`.  Costs
+    O(T P N) per head and token, with no state history: usable at full
+    problem sizes on a few tokens.  Returns a dict with dx [k,H,P], ddt [k,H],
+    dB, dC [k,G,N] for the k listed tokens.
+    """
+    x, dt, A, B, C, D, dy, init_state, dfinal_state = _bwd_args(x, dt, A, B, C, D, dy, init_state, dfinal_state)
+    _, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    hpg = H // G
+    tokens = [int(t) for t in tokens]
+    k = len(tokens)
+    out = {"dx": np.zeros((k, H, P)), "ddt": np.zeros((k, H)), "dB": np.zeros((k, G, N)), "dC": np.zeros((k, G, N))}
+    for h in range(H):
+        gi = h // hpg
+        sig = np.cumsum(dt[b, :, h] * A[h])                 # sigma_t
+        xs, dys = x[b, :, h, :], dy[b, :, h, :]
+        Bs, Cs = B[b, :, gi, :], C[b, :, gi, :]
+        for i, t in enumerate(tokens):
+            def state_at(u):
+                if u < 0:
+                    return np.zeros((P, N)) if init_state is None else init_state[b, h]
+                w = np.exp(sig[u] - sig[:u + 1])
+                st = (xs[:u + 1] * w[:, None]).T @ Bs[:u + 1]
+                if init_state is not None:
+                    st = st + np.exp(sig[u]) * init_state[b, h]
+                return st
+            w = np.exp(sig[t:] - sig[t])
+            g = (dys[t:] * w[:, None]).T @ Cs[t:]
+            if dfinal_state is not None:
+                g = g + np.exp(sig[T - 1] - sig[t]) * dfinal_state[b, h]
+            ht = state_at(t)
+            a_t = np.exp(dt[b, t, h] * A[h])
+            out["dx"][i, h] = g @ Bs[t] + D[h] * dys[t]
+            out["dB"][i, gi] += xs[t] @ g
+            out["dC"][i, gi] += dys[t] @ ht
+            out["ddt"][i, h] = A[h] * a_t * np.sum(g * state_at(t - 1))
     return out

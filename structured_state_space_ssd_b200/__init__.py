@@ -6,9 +6,9 @@ marshals torch tensors into it.  Importing this package loads nothing: the
 library is opened on the first call, and a missing or unloadable library is
 an error, never a fallback.
 """
-from .inputs import HEADLINE, WORKLOADS, Workload, make_inputs, workload_inputs  # noqa: F401
+from .inputs import HEADLINE, WORKLOADS, Workload, make_inputs, make_output_grads, workload_inputs  # noqa: F401
 
-__all__ = ["HEADLINE", "WORKLOADS", "Workload", "make_inputs", "workload_inputs",
+__all__ = ["HEADLINE", "WORKLOADS", "Workload", "make_inputs", "make_output_grads", "workload_inputs",
            "ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_status_string", "SSDError"]
 
 

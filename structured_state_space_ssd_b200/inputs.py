@@ -101,3 +101,22 @@ def make_inputs(batch: int, T: int, H: int, P: int, N: int, G: int, dtype: str =
 def workload_inputs(w: Workload) -> dict:
     """Inputs of a named workload, drawn with its own seed."""
     return make_inputs(w.batch, w.T, w.H, w.P, w.N, w.G, w.dtype, w.seed, w.with_init)
+
+
+def make_output_grads(batch: int, T: int, H: int, P: int, N: int, dtype: str = "bf16", seed: int = 0,
+                      with_dfinal: bool = False) -> dict:
+    """Draw the gradients arriving at the layer's outputs for a backward pass.
+
+    Returns CPU tensors ``dy`` [b,T,H,P] ~ N(0, 1) in the dtype of y (rounded once
+    to bf16 for bf16 problems) and ``dfinal_state`` [b,H,P,N] ~ N(0, 0.1^2) in fp32,
+    or None.  The seed stream is separate from :func:`make_inputs`'.
+    """
+    if dtype not in ("f32", "bf16"):
+        raise ValueError(f"dtype must be 'f32' or 'bf16', got {dtype!r}")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7_000_003)
+    dy = torch.randn(batch, T, H, P, generator=g)
+    dfin = (0.1 * torch.randn(batch, H, P, N, generator=g)) if with_dfinal else None
+    if dtype == "bf16":
+        dy = dy.bfloat16()
+    return {"dy": dy, "dfinal_state": dfin}
