@@ -394,6 +394,7 @@ def main():
         }
         line["decode_step"] = measure_decode(w, host, dev, stream, flush, peaks)
         line["gate_norm"] = measure_gate_norm(w, y, dev, stream, flush, peaks)
+        line["backward"] = measure_backward(w, d, dev, stream, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(host, w)
         print(json.dumps(line), flush=True)
@@ -486,6 +487,46 @@ def measure_gate_norm(w, y, dev, stream, flush, peaks, steps=20):
     gbps = alg / (ms * 1e-3) / 1e9
     return {"rows": y.numel() // (w.H * w.P), "channels": w.H * w.P, "ngroups": w.H, "dtype": w.dtype,
             "alg_bytes": alg, "us_per_launch": ms * 1e3, "GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"]}
+
+
+def measure_backward(w, d, dev, stream, flush, steps=5):
+    """The layer's backward (ssd_bwd: every input gradient for given dy and dfinal) on this workload,
+    L2 flushed before each call.  It runs on the CUDA cores in fp32, so its bound is the FFMA rate:
+    148 SMs x 128 lanes x 2 flops per cycle at the clock's maximum (74.4 TFLOP/s at 1965 MHz)."""
+    import torch
+    from structured_state_space_ssd_b200 import ssd as S
+    from structured_state_space_ssd_b200.inputs import make_output_grads
+    g = make_output_grads(w.batch, w.T, w.H, w.P, w.N, w.dtype, seed=w.seed, with_dfinal=True)
+    dy, dfin = g["dy"].to(dev), g["dfinal_state"].to(dev)
+    ws = torch.empty(S.ssd_bwd_workspace_bytes(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, dy.dtype), dtype=torch.uint8,
+                     device=dev)
+    Q, H, P, N, G = w.Q, w.H, w.P, w.N, w.G
+    # block-form work per (batch, chunk): C B^T per group; the masked Q x Q products for dx, for
+    # W = dy x^T and for dB, dC; five Q x N x P state products (forward and backward chunk states, the
+    # state terms of dx, dB and dC)
+    per_chunk = 2 * Q * Q * N * G + 2 * (2 * Q * Q * P * H) + 2 * (2 * Q * Q * N * H) + 5 * (2 * Q * N * P * H)
+    alg_flops = per_chunk * w.batch * w.nc
+
+    def one():
+        S.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], dy, Q, d["init_state"], dfin, workspace=ws,
+                  stream=stream)
+
+    for _ in range(3):
+        flush.zero_()
+        one()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    peak = 148 * 128 * 2 * 1.965e9
+    return {"ms": ms, "tokens_per_s": w.tokens / (ms * 1e-3), "alg_flops": alg_flops,
+            "tflops": alg_flops / (ms * 1e-3) / 1e12, "bound": "alu",
+            "frac_of_fp32_ffma_peak": alg_flops / (ms * 1e-3) / peak, "launches_per_call": 11,
+            "with": "init_state and dfinal_state"}
 
 
 def _traffic_from_profiles(kernel, w):

@@ -241,6 +241,42 @@ SSD_API int ssd_split_combine(const float *fin0_all, const float *total_all, con
 SSD_API int ssd_split_correct(void *y, const void *C, const float *sig, const float *s_in, int batch, int T, int H,
                       int P, int G, int N, int dtype, void *stream);
 
+/*
+ * Backward pass: the gradients of L = sum(dy * y) + sum(dfinal_state * final_state)
+ * with respect to every input of ssd_fwd, for the same problem.  The pages
+ * print the forward only ("Transformers are SSMs", analysis page, section
+ * "The SSM as a Matrix Transformation", equation (2), and the chunked form of
+ * section "The Block-Decomposition SSD Algorithm"); this is the unique
+ * gradient of that function, organised by the same chunks.  Per (b, h), with
+ * the adjoint g_t = dL/dh_t of the state h_t [P][N] (g_{T-1} = dfinal + dy C^T,
+ * g_t = a_{t+1} g_{t+1} + dy_t C_t^T):
+ *
+ *   dx_t   = g_t B_t + D_h dy_t                     [batch][T][H][P], dtype
+ *   dB_t   = sum over the group's heads of g_t^T x_t    [batch][T][G][N], dtype
+ *   dC_t   = sum over the group's heads of h_t^T dy_t   [batch][T][G][N], dtype
+ *   ddt_t  = A_h <g_t, a_t h_{t-1}>                 [batch][T][H], fp32
+ *   dA_h   = sum_{b,t} dt_t <g_t, a_t h_{t-1}>      [H], fp32
+ *   dD_h   = sum_{b,t} <dy_t, x_t>                  [H], fp32
+ *   dinit  = a_0 g_0                                [batch][H][P][N], fp32 (NULL: not written)
+ *
+ * Inputs as for ssd_fwd, plus dy [batch][T][H][P] in the dtype of x and
+ * dfinal_state [batch][H][P][N] fp32 (NULL: zero).  init_state NULL means
+ * zero.  All pointers are device pointers, 4-byte (fp32) or 2-byte (bf16)
+ * aligned; workspace 256-byte aligned with at least ssd_bwd_workspace_bytes()
+ * bytes (0 there: invalid dimensions).  Outputs may not overlap any input,
+ * one another or the workspace.  Every kernel runs on the CUDA cores in fp32
+ * (sums over the sequence for dt, A and D in fp64), in a fixed order: results
+ * are bitwise reproducible.  Same dimension limits as ssd_fwd, plus batch,
+ * H <= 65535.  Asynchronous on `stream`; 11 launches (none when T == 0, where
+ * dA = dD = 0 and dinit = dfinal).  Returns SSD_OK, SSD_ERR_INVALID_ARG,
+ * SSD_ERR_UNSUPPORTED or SSD_ERR_CUDA.
+ */
+SSD_API size_t ssd_bwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
+SSD_API int ssd_bwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
+                    int Q, const float *init_state, const void *dy, const float *dfinal_state, void *dx, float *ddt,
+                    float *dA, void *dB, void *dC, float *dD, float *dinit_state, int batch, int T, int H, int P,
+                    int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

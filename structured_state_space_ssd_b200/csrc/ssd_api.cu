@@ -8,7 +8,8 @@
 namespace ssd {
 cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const Shape &sh, cudaStream_t st);
 template <typename T>
-cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st);
+cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st,
+                               bool from_start);
 cudaError_t launch_state_passing(float *S, const float *s, const float *init, float *fin, const Shape &sh,
                                  cudaStream_t st);
 template <typename T>
@@ -23,14 +24,9 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, con
 
 using ssd::Shape;
 
-namespace {
+namespace ssd {
 
-constexpr int kVersion = 200;  // 0.2.0
-constexpr int kMaxP = 128, kMaxN = 256, kMaxQ = 256;
-constexpr int64_t kMaxElems = int64_t(1) << 46;
-constexpr int kMaxStages = 8;
-
-// Validates the dimensions; fills `sh` on success.
+// Validates the dimensions of a forward or backward call; fills `sh` on success.
 int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, Shape *sh) {
     if (batch < 1 || T < 0 || H < 1 || P < 1 || G < 1 || N < 1 || Q < 1) return SSD_ERR_INVALID_ARG;
     if (H % G != 0) return SSD_ERR_INVALID_ARG;
@@ -50,6 +46,14 @@ int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, S
     sh->heads_per_group = H / G;
     return SSD_OK;
 }
+
+}  // namespace ssd
+
+namespace {
+
+constexpr int kVersion = 200;  // 0.2.0
+constexpr int kMaxStages = 8;
+using ssd::check_dims;
 
 ssd::Path choose_path(const Shape &sh, int dtype) {
     return ssd::fused_supported(sh, dtype) ? ssd::kPathFused : ssd::kPathSimt;
@@ -85,7 +89,8 @@ int run_simt(const Shape &sh, const T *x, const float *dt, const float *A, const
     float *S = reinterpret_cast<float *>(ws + w.state_off);
     if (!mk.mark(0, st)) return SSD_ERR_CUDA;
     if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(1, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st) != cudaSuccess || !mk.mark(2, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st, false) != cudaSuccess || !mk.mark(2, st))
+        return SSD_ERR_CUDA;
     if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || !mk.mark(3, st)) return SSD_ERR_CUDA;
     if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || !mk.mark(4, st))
         return SSD_ERR_CUDA;

@@ -1,0 +1,610 @@
+// ssd_bwd.cu -- the SSD layer backward on the CUDA cores: gradients of
+// (y, final_state) with respect to x, dt, A, B, C, D and the initial state.
+//
+// The pages give the forward only ("Transformers are SSMs", analysis page,
+// section "The Block-Decomposition SSD Algorithm"); the backward here is the
+// gradient of that function, organised by the same chunk decomposition.  With
+// s_i the inclusive log-decay prefix of a chunk (s_end its last value), Hin_c
+// the state entering chunk c and dHout_c the gradient arriving at the state
+// that leaves it:
+//
+//   dHout_{nc-1} = dfinal,   dHout_{c-1} = exp(s_end,c) dHout_c + sum_i exp(s_i) dy_i C_i^T
+//   dinit = dHout_{-1}
+//   dx_r  = exp(s_end - s_r) dHout_c B_r + sum_{i>=r} exp(s_i - s_r) (B_r . C_i) dy_i + D_h dy_r
+//   dB_r  = sum over heads of [exp(s_end - s_r) x_r^T dHout_c + sum_{i>=r} exp(s_i - s_r) (x_r . dy_i) C_i]
+//   dC_r  = sum over heads of [exp(s_r) dy_r^T Hin_c + sum_{i<=r} exp(s_r - s_i) (dy_r . x_i) B_i]
+//
+// and the decays enter through the per-token gradient of the running
+// log-decay sigma_t = sum_{u<=t} dt_u A_h of the whole sequence:
+//
+//   dsigma_t = C_t . dC_t^(h) - B_t . dB_t^(h)   (+ <dfinal, final> at the last token)
+//   d(dt_u A_h) = sum_{t>=u} dsigma_t,   ddt_u = A_h d(dt_u A_h),   dA_h = sum dt_u d(dt_u A_h)
+//
+// where dB^(h), dC^(h) are one head's terms before the sum over its group.
+// The three products above share one masked-scan kernel (the forward's
+// chunk_scan shape with the roles of its operands exchanged); the chunk sums
+// and the forward states reuse the forward's CUDA-core kernels.  Every
+// reduction runs in a fixed order: results are bitwise reproducible.
+#include "ssd_common.cuh"
+
+namespace ssd {
+cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const Shape &sh, cudaStream_t st);
+template <typename T>
+cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st,
+                               bool from_start);
+cudaError_t launch_state_passing(float *S, const float *s, const float *init, float *fin, const Shape &sh,
+                                 cudaStream_t st);
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Workspace of one backward call (all offsets 256-byte aligned).
+// ---------------------------------------------------------------------------
+struct BwdWorkspace {
+    size_t s_off;     // float s[batch][H][nc][Q]
+    size_t hin_off;   // float Hin[batch][nc][H][P][N]: chunk states, then the state entering each chunk
+    size_t gout_off;  // float G[batch][nc][H][P][N]: chunk sums of dy C^T, then dHout of each chunk
+    size_t fin_off;   // float final[batch][H][P][N]
+    size_t dbh_off;   // float dB^(h)[batch][T][H][N]
+    size_t dch_off;   // float dC^(h)[batch][T][H][N]
+    size_t dsig_off;  // float dsigma[batch][H][T]
+    size_t pa_off;    // double dA partial[batch][H]
+    size_t pd_off;    // double dD partial[batch][H]
+    size_t total;
+};
+
+BwdWorkspace bwd_layout(const Shape &s) {
+    BwdWorkspace w;
+    const size_t bh = (size_t)s.batch * s.H, PN = (size_t)s.P * s.N;
+    const size_t states = sizeof(float) * (size_t)s.batch * s.nc * s.H * PN;
+    const size_t perhead = sizeof(float) * (size_t)s.batch * s.T * s.H * s.N;
+    size_t off = 0;
+    w.s_off = off;
+    off = align256(off + sizeof(float) * bh * s.nc * s.Q);
+    w.hin_off = off;
+    off = align256(off + states);
+    w.gout_off = off;
+    off = align256(off + states);
+    w.fin_off = off;
+    off = align256(off + sizeof(float) * bh * PN);
+    w.dbh_off = off;
+    off = align256(off + perhead);
+    w.dch_off = off;
+    off = align256(off + perhead);
+    w.dsig_off = off;
+    off = align256(off + sizeof(float) * bh * s.T);
+    w.pa_off = off;
+    off = align256(off + sizeof(double) * bh);
+    w.pd_off = off;
+    off = align256(off + sizeof(double) * bh);
+    w.total = off;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// Reverse state passing, in place on the chunk sums G_c = sum_i exp(s_i) dy_i C_i^T:
+// slot c receives dHout_c, and dinit (if requested) receives dHout_{-1}.
+// grid (ceil(P*N/256), H, batch); the loads of up to 8 chunks go out ahead of
+// the dependent chain, as in the forward's state passing.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) state_passing_bwd_kernel(float *__restrict__ Gs, const float *__restrict__ s,
+                                                                const float *__restrict__ dfin,
+                                                                float *__restrict__ dinit, Shape sh) {
+    const int PN = sh.P * sh.N;
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    const int h = blockIdx.y, b = blockIdx.z;
+    if (e >= PN) return;
+    float run = dfin ? dfin[((size_t)b * sh.H + h) * PN + e] : 0.f;
+    const float *sb = s + ((size_t)b * sh.H + h) * sh.nc * sh.Q;
+    const size_t cstride = (size_t)sh.H * PN;
+    float *base = Gs + ((size_t)b * sh.nc * sh.H + h) * PN + e;
+    for (int cend = sh.nc; cend > 0; cend -= 8) {
+        const int cn = min(8, cend), c0 = cend - cn;
+        float loc[8], dec[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < cn) {
+                loc[k] = base[(size_t)(c0 + k) * cstride];
+                dec[k] = expf(sb[(size_t)(c0 + k) * sh.Q + sh.Q - 1]);
+            }
+        }
+#pragma unroll
+        for (int k = 7; k >= 0; --k) {
+            if (k < cn) {
+                base[(size_t)(c0 + k) * cstride] = run;
+                run = fmaf(dec[k], run, loc[k]);
+            }
+        }
+    }
+    if (dinit) dinit[((size_t)b * sh.H + h) * PN + e] = run;
+}
+
+// ---------------------------------------------------------------------------
+// Masked scan over one chunk, one head and a 64-row tile:
+//
+//   out_r[w] = e_r * sum_k R_r[k] St[k][w]
+//            + sum_{i in chunk, i >= r (kAnti) or i <= r} exp(+-(s_i - s_r)) (R_r . K_i) V_i[w]
+//            + D_h V_r[w]                                          (when D is given)
+//
+// with e_r = exp(s_end - s_r) (kAnti: the state arrives at the chunk's end)
+// or exp(s_r) (the state enters at its start).  Operands are rows of
+// [batch][T][*] tensors: R and K have KD columns, V has W; each is either a
+// head's slice (row length H*KD or H*W) or its group's (G*KD or G*W).  St is
+// the [P][N] state of the (batch, chunk, head), read as [W][KD] or [KD][W].
+// grid (nc * ceil(Q/64), H, batch), 256 threads as 16 (w) x 16 (rows); each
+// thread owns 4 rows x RW columns.
+// ---------------------------------------------------------------------------
+struct ScanArgs {
+    const void *R, *K, *V;
+    int r_head, k_head, v_head;  // 1: the head's slice, 0: the group's
+    const float *St;             // [batch][nc][H][P*N]
+    int st_kw;                   // 1: St is [KD][W], 0: [W][KD]
+    int KD, W;
+    const float *D;              // skip factor per head, or null
+    void *out;                   // [batch][T][H][W]
+};
+
+template <typename T, typename TO, int RW, bool kAnti>
+__global__ void __launch_bounds__(256) masked_scan_kernel(ScanArgs a, const float *__restrict__ s, Shape sh) {
+    extern __shared__ float smem[];
+    const int KD = a.KD, W = a.W, KP = KD + 1;
+    float *Rs = smem;              // [64][KD+1]
+    float *Ks = Rs + 64 * KP;      // [32][KD+1]
+    float *Vs = Ks + 32 * KP;      // [32][W]
+    float *Ms = Vs + 32 * W;       // [64][33]
+    float *sr = Ms + 64 * 33;      // [64]
+    float *sc = sr + 64;           // [32]
+    float *Ss = sc + 32;           // [W][33]
+    const int tiles = (sh.Q + 63) >> 6;
+    const int c = blockIdx.x / tiles, jt = blockIdx.x - c * tiles;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int g = h / sh.heads_per_group;
+    const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0);
+    const int j0 = jt * 64;
+    if (j0 >= len) return;
+    const int jn = min(64, len - j0);
+    const float *sch = s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+    const T *Rp = static_cast<const T *>(a.R);
+    const T *Kp = static_cast<const T *>(a.K);
+    const T *Vp = static_cast<const T *>(a.V);
+    const size_t r_ld = (size_t)(a.r_head ? sh.H : sh.G) * KD, r_off = (size_t)(a.r_head ? h : g) * KD;
+    const size_t k_ld = (size_t)(a.k_head ? sh.H : sh.G) * KD, k_off = (size_t)(a.k_head ? h : g) * KD;
+    const size_t v_ld = (size_t)(a.v_head ? sh.H : sh.G) * W, v_off = (size_t)(a.v_head ? h : g) * W;
+    const size_t row0 = (size_t)b * sh.T + t0;  // token index of the chunk's first row
+
+    for (int idx = threadIdx.x; idx < 64 * KD; idx += 256) {
+        const int jj = idx / KD, k = idx - jj * KD;
+        Rs[jj * KP + k] = (jj < jn) ? to_f32(Rp[(row0 + j0 + jj) * r_ld + r_off + k]) : 0.f;
+    }
+    if (threadIdx.x < 64) sr[threadIdx.x] = (threadIdx.x < jn) ? sch[j0 + threadIdx.x] : 0.f;
+    __syncthreads();
+
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][RW];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int k = 0; k < RW; ++k) acc[r][k] = 0.f;
+
+    // the state term, 32 of the KD contraction indices at a time
+    const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
+    for (int k0 = 0; k0 < KD; k0 += 32) {
+        for (int idx = threadIdx.x; idx < W * 32; idx += 256) {
+            int w, kk;
+            if (a.st_kw) {  // [KD][W]: consecutive threads along w
+                kk = idx / W;
+                w = idx - kk * W;
+            } else {        // [W][KD]: consecutive threads along k
+                w = idx >> 5;
+                kk = idx & 31;
+            }
+            const int k = k0 + kk;
+            float v = 0.f;
+            if (k < KD) v = a.st_kw ? Sp[(size_t)k * W + w] : Sp[(size_t)w * KD + k];
+            Ss[w * 33 + kk] = v;
+        }
+        __syncthreads();
+        const int klim = min(32, KD - k0);
+        for (int kk = 0; kk < klim; ++kk) {
+            float rv[4], sv[RW];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) rv[r] = Rs[(ty + 16 * r) * KP + k0 + kk];
+#pragma unroll
+            for (int k = 0; k < RW; ++k) {
+                const int w = tx + 16 * k;
+                sv[k] = (w < W) ? Ss[w * 33 + kk] : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int k = 0; k < RW; ++k) acc[r][k] = fmaf(rv[r], sv[k], acc[r][k]);
+        }
+        __syncthreads();
+    }
+    {
+        const float s_end = sch[sh.Q - 1];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float sj = sr[ty + 16 * r];
+            const float e = kAnti ? expf(s_end - sj) : expf(sj);
+#pragma unroll
+            for (int k = 0; k < RW; ++k) acc[r][k] *= e;
+        }
+    }
+
+    // the masked quadratic term over the chunk's other rows
+    const int ibeg = kAnti ? j0 : 0;
+    const int iend = kAnti ? len : j0 + jn;
+    for (int i0 = ibeg; i0 < iend; i0 += 32) {
+        for (int idx = threadIdx.x; idx < 32 * KD; idx += 256) {
+            const int ii = idx / KD, k = idx - ii * KD, i = i0 + ii;
+            Ks[ii * KP + k] = (i < iend) ? to_f32(Kp[(row0 + i) * k_ld + k_off + k]) : 0.f;
+        }
+        for (int idx = threadIdx.x; idx < 32 * W; idx += 256) {
+            const int ii = idx / W, w = idx - ii * W, i = i0 + ii;
+            Vs[idx] = (i < iend) ? to_f32(Vp[(row0 + i) * v_ld + v_off + w]) : 0.f;
+        }
+        if (threadIdx.x < 32) sc[threadIdx.x] = (i0 + threadIdx.x < iend) ? sch[i0 + threadIdx.x] : 0.f;
+        __syncthreads();
+        {
+            const int jj = threadIdx.x >> 2, ib = (threadIdx.x & 3) * 8;
+            float dot[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dot[e] = 0.f;
+            for (int k = 0; k < KD; ++k) {
+                const float rv = Rs[jj * KP + k];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dot[e] = fmaf(rv, Ks[(ib + e) * KP + k], dot[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int ii = ib + e, i = i0 + ii, j = j0 + jj;
+                const bool ok = jj < jn && i < iend && (kAnti ? i >= j : i <= j);
+                Ms[jj * 33 + ii] = ok ? expf(kAnti ? sc[ii] - sr[jj] : sr[jj] - sc[ii]) * dot[e] : 0.f;
+            }
+        }
+        __syncthreads();
+        for (int ii = 0; ii < 32; ++ii) {
+            float mv[4], vv[RW];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) mv[r] = Ms[(ty + 16 * r) * 33 + ii];
+#pragma unroll
+            for (int k = 0; k < RW; ++k) {
+                const int w = tx + 16 * k;
+                vv[k] = (w < W) ? Vs[ii * W + w] : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int k = 0; k < RW; ++k) acc[r][k] = fmaf(mv[r], vv[k], acc[r][k]);
+        }
+        __syncthreads();
+    }
+
+    const float Dh = a.D ? a.D[h] : 0.f;
+    TO *out = static_cast<TO *>(a.out);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int jj = ty + 16 * r;
+        if (jj >= jn) continue;
+        const size_t tok = row0 + j0 + jj;
+        TO *orow = out + (tok * sh.H + h) * W;
+#pragma unroll
+        for (int k = 0; k < RW; ++k) {
+            const int w = tx + 16 * k;
+            if (w >= W) continue;
+            float v = acc[r][k];
+            if (a.D) v = fmaf(Dh, to_f32(Vp[tok * v_ld + v_off + w]), v);
+            orow[w] = from_f32<TO>(v);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Sum over each group's heads: dB = sum_h dB^(h), dC = sum_h dC^(h) (in the
+// input dtype), and each head's dsigma_t = C_t . dC^(h)_t - B_t . dB^(h)_t.
+// One warp per (batch, token, group); lanes stride the N columns; heads in
+// ascending order.  256 threads per block.
+// ---------------------------------------------------------------------------
+constexpr int kMaxNPerLane = kMaxN / 32;
+
+template <typename T>
+__global__ void __launch_bounds__(256) group_reduce_kernel(const float *__restrict__ dBh, const float *__restrict__ dCh,
+                                                           const T *__restrict__ Bm, const T *__restrict__ Cm,
+                                                           T *__restrict__ dB, T *__restrict__ dC,
+                                                           float *__restrict__ dsig, Shape sh) {
+    const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long units = (long long)sh.batch * sh.T * sh.G;
+    if (unit >= units) return;
+    const int lane = threadIdx.x & 31;
+    const int g = (int)(unit % sh.G);
+    const long long tok = unit / sh.G;  // b * T + t
+    const int b = (int)(tok / sh.T), t = (int)(tok - (long long)b * sh.T);
+    const size_t grow = (size_t)unit * sh.N;  // row (b, t, g) of B, C, dB, dC
+    float bv[kMaxNPerLane], cv[kMaxNPerLane], sb[kMaxNPerLane], sc[kMaxNPerLane];
+#pragma unroll
+    for (int m = 0; m < kMaxNPerLane; ++m) {
+        const int n = lane + 32 * m;
+        const bool ok = n < sh.N;
+        bv[m] = ok ? to_f32(Bm[grow + n]) : 0.f;
+        cv[m] = ok ? to_f32(Cm[grow + n]) : 0.f;
+        sb[m] = 0.f;
+        sc[m] = 0.f;
+    }
+    for (int hh = 0; hh < sh.heads_per_group; ++hh) {
+        const int h = g * sh.heads_per_group + hh;
+        const size_t hrow = ((size_t)tok * sh.H + h) * sh.N;
+        float d = 0.f;
+#pragma unroll
+        for (int m = 0; m < kMaxNPerLane; ++m) {
+            const int n = lane + 32 * m;
+            if (n < sh.N) {
+                const float db = dBh[hrow + n], dc = dCh[hrow + n];
+                sb[m] += db;
+                sc[m] += dc;
+                d = fmaf(cv[m], dc, d);
+                d = fmaf(-bv[m], db, d);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (lane == 0) dsig[((size_t)b * sh.H + h) * sh.T + t] = d;
+    }
+#pragma unroll
+    for (int m = 0; m < kMaxNPerLane; ++m) {
+        const int n = lane + 32 * m;
+        if (n < sh.N) {
+            dB[grow + n] = from_f32<T>(sb[m]);
+            dC[grow + n] = from_f32<T>(sc[m]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per (head, batch): the suffix sums of dsigma over the whole sequence (fp64),
+// plus <dfinal, final> at the last token, give d(dt_u A_h); write
+// ddt = A_h d(dt A), and the batch row's shares of dA = sum dt d(dt A) and
+// dD = sum <dy, x> (fp64).  grid (H, batch), 256 threads: each thread owns a
+// contiguous run of tokens, a block scan of the run totals gives each run the
+// sum of the runs after it.
+// ---------------------------------------------------------------------------
+constexpr int kDtThreads = 256;
+
+__device__ double block_sum(double v, double *red) {
+    red[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = kDtThreads / 2; o > 0; o >>= 1) {
+        if ((int)threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+        __syncthreads();
+    }
+    const double r = red[0];
+    __syncthreads();
+    return r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__restrict__ dsig,
+                                                             const float *__restrict__ dt,
+                                                             const float *__restrict__ A, const T *__restrict__ x,
+                                                             const T *__restrict__ dy,
+                                                             const float *__restrict__ dfin,
+                                                             const float *__restrict__ fin, float *__restrict__ ddt,
+                                                             double *__restrict__ pa, double *__restrict__ pd,
+                                                             Shape sh) {
+    __shared__ double red[kDtThreads];
+    __shared__ double suf[kDtThreads];
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const size_t bh = (size_t)b * sh.H + h;
+    const size_t PN = (size_t)sh.P * sh.N;
+    double fd = 0.0;
+    if (dfin)
+        for (size_t e = tid; e < PN; e += kDtThreads) fd += (double)dfin[bh * PN + e] * (double)fin[bh * PN + e];
+    const double fdot = block_sum(fd, red);
+
+    const float *ds = dsig + bh * sh.T;
+    const int run = (sh.T + kDtThreads - 1) / kDtThreads;
+    const int t0 = min(sh.T, tid * run), t1 = min(sh.T, t0 + run);
+    double part = 0.0;
+    for (int t = t0; t < t1; ++t) part += (double)ds[t];
+    suf[tid] = part;
+    __syncthreads();
+    // inclusive suffix scan of the run totals
+    for (int o = 1; o < kDtThreads; o <<= 1) {
+        const double v = tid + o < kDtThreads ? suf[tid + o] : 0.0;
+        __syncthreads();
+        suf[tid] += v;
+        __syncthreads();
+    }
+    double acc = (tid + 1 < kDtThreads ? suf[tid + 1] : 0.0) + fdot;
+    const double Ah = (double)A[h];
+    double da = 0.0;
+    for (int t = t1 - 1; t >= t0; --t) {
+        acc += (double)ds[t];
+        const size_t it = ((size_t)b * sh.T + t) * sh.H + h;
+        ddt[it] = (float)(Ah * acc);
+        da += (double)dt[it] * acc;
+    }
+    const double dA_part = block_sum(da, red);
+
+    double dd = 0.0;
+    const long long TP = (long long)sh.T * sh.P;
+    for (long long idx = tid; idx < TP; idx += kDtThreads) {
+        const int t = (int)(idx / sh.P), p = (int)(idx - (long long)t * sh.P);
+        const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + p;
+        dd += (double)to_f32(dy[off]) * (double)to_f32(x[off]);
+    }
+    const double dD_part = block_sum(dd, red);
+    if (tid == 0) {
+        pa[bh] = dA_part;
+        pd[bh] = dD_part;
+    }
+}
+
+// dA[h] = sum_b pa[b][h], dD[h] = sum_b pd[b][h], in batch order.
+__global__ void __launch_bounds__(256) param_reduce_kernel(const double *__restrict__ pa,
+                                                           const double *__restrict__ pd, float *__restrict__ dA,
+                                                           float *__restrict__ dD, int batch, int H) {
+    const int h = blockIdx.x * 256 + threadIdx.x;
+    if (h >= H) return;
+    double sa = 0.0, sd = 0.0;
+    for (int b = 0; b < batch; ++b) {
+        sa += pa[(size_t)b * H + h];
+        sd += pd[(size_t)b * H + h];
+    }
+    dA[h] = (float)sa;
+    dD[h] = (float)sd;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+int pow2_ceil(int v) {
+    int r = 1;
+    while (r < v) r <<= 1;
+    return r;
+}
+
+size_t scan_smem_bytes(int KD, int W) {
+    return sizeof(float) * ((size_t)96 * (KD + 1) + (size_t)32 * W + 64 * 33 + 96 + (size_t)W * 33);
+}
+
+template <typename T, typename TO, int RW, bool kAnti>
+cudaError_t launch_scan_rw(const ScanArgs &a, const float *s, const Shape &sh, cudaStream_t st) {
+    const size_t smem = scan_smem_bytes(a.KD, a.W);
+    auto k = masked_scan_kernel<T, TO, RW, kAnti>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = (sh.Q + 63) / 64;
+    k<<<dim3(sh.nc * tiles, sh.H, sh.batch), 256, smem, st>>>(a, s, sh);
+    return cudaGetLastError();
+}
+
+template <typename T, typename TO, bool kAnti>
+cudaError_t launch_scan(const ScanArgs &a, const float *s, const Shape &sh, cudaStream_t st) {
+    switch (pow2_ceil((a.W + 15) / 16)) {
+        case 1: return launch_scan_rw<T, TO, 1, kAnti>(a, s, sh, st);
+        case 2: return launch_scan_rw<T, TO, 2, kAnti>(a, s, sh, st);
+        case 4: return launch_scan_rw<T, TO, 4, kAnti>(a, s, sh, st);
+        case 8: return launch_scan_rw<T, TO, 8, kAnti>(a, s, sh, st);
+        default: return launch_scan_rw<T, TO, 16, kAnti>(a, s, sh, st);
+    }
+}
+
+bool is_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || !na || !nb) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+template <typename T>
+int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const T *B, const T *C, const float *D,
+            const float *init, const T *dy, const float *dfin, T *dx, float *ddt, float *dA, T *dB, T *dC,
+            float *dD, float *dinit, char *ws, const BwdWorkspace &w, cudaStream_t st) {
+    float *s = reinterpret_cast<float *>(ws + w.s_off);
+    float *Hin = reinterpret_cast<float *>(ws + w.hin_off);
+    float *Gout = reinterpret_cast<float *>(ws + w.gout_off);
+    float *fin = reinterpret_cast<float *>(ws + w.fin_off);
+    float *dBh = reinterpret_cast<float *>(ws + w.dbh_off);
+    float *dCh = reinterpret_cast<float *>(ws + w.dch_off);
+    float *dsig = reinterpret_cast<float *>(ws + w.dsig_off);
+    double *pa = reinterpret_cast<double *>(ws + w.pa_off);
+    double *pd = reinterpret_cast<double *>(ws + w.pd_off);
+    if (launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    // forward states: Hin_c, and the final state when a final-state gradient is given
+    if (launch_chunk_state<T>(x, B, s, Hin, sh, st, false) != cudaSuccess) return SSD_ERR_CUDA;
+    if (launch_state_passing(Hin, s, init, dfin ? fin : nullptr, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    // backward states: sum_i exp(s_i) dy_i C_i^T per chunk, then dHout_c and dinit
+    if (launch_chunk_state<T>(dy, C, s, Gout, sh, st, true) != cudaSuccess) return SSD_ERR_CUDA;
+    const int PN = sh.P * sh.N;
+    state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    // dx: rows of B against columns of C, values dy, state dHout as [P][N] = [W][KD], skip D dy
+    ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx};
+    if (launch_scan<T, T, true>(ax, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    // dB^(h): rows of x against columns of dy, values C, state dHout as [P][N] = [KD][W]
+    ScanArgs ab{x, dy, C, 1, 1, 0, Gout, 1, sh.P, sh.N, nullptr, dBh};
+    if (launch_scan<T, float, true>(ab, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    // dC^(h): rows of dy against columns of x, values B, state Hin as [P][N] = [KD][W]
+    ScanArgs ac{dy, x, B, 1, 1, 0, Hin, 1, sh.P, sh.N, nullptr, dCh};
+    if (launch_scan<T, float, false>(ac, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    const long long units = (long long)sh.batch * sh.T * sh.G;
+    group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    dt_scan_kernel<T><<<dim3(sh.H, sh.batch), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    param_reduce_kernel<<<(sh.H + 255) / 256, 256, 0, st>>>(pa, pd, dA, dD, sh.batch, sh.H);
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" size_t ssd_bwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
+    ssd::Shape sh;
+    if (ssd::check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
+    return ssd::bwd_layout(sh).total;
+}
+
+extern "C" int ssd_bwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
+                       int Q, const float *init_state, const void *dy, const float *dfinal_state, void *dx,
+                       float *ddt, float *dA, void *dB, void *dC, float *dD, float *dinit_state, int batch, int T,
+                       int H, int P, int G, int N, int dtype, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+    ssd::Shape sh;
+    int rc = ssd::check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
+    if (rc != SSD_OK) return rc;
+    if ((T > 0 && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC)) || !A || !D || !dA || !dD ||
+        !workspace)
+        return SSD_ERR_INVALID_ARG;
+    if (batch > 65535 || H > 65535) return SSD_ERR_UNSUPPORTED;
+    const size_t es = (dtype == SSD_BF16) ? 2 : 4;
+    using ssd::is_aligned;
+    if (!is_aligned(x, es) || !is_aligned(B, es) || !is_aligned(C, es) || !is_aligned(dy, es) ||
+        !is_aligned(dx, es) || !is_aligned(dB, es) || !is_aligned(dC, es) || !is_aligned(dt, 4) ||
+        !is_aligned(A, 4) || !is_aligned(D, 4) || !is_aligned(ddt, 4) || !is_aligned(dA, 4) || !is_aligned(dD, 4) ||
+        !is_aligned(init_state, 4) || !is_aligned(dfinal_state, 4) || !is_aligned(dinit_state, 4) ||
+        !is_aligned(workspace, 256))
+        return SSD_ERR_INVALID_ARG;
+    const ssd::BwdWorkspace w = ssd::bwd_layout(sh);
+    if (workspace_bytes < w.total) return SSD_ERR_INVALID_ARG;
+    // outputs may not overlap any input or one another
+    const size_t xb = es * (size_t)batch * T * H * P, bcb = es * (size_t)batch * T * G * N;
+    const size_t tb = sizeof(float) * (size_t)batch * T * H, hb = sizeof(float) * H;
+    const size_t sb = sizeof(float) * (size_t)batch * H * P * N;
+    const void *ins[] = {x, dt, A, B, C, D, init_state, dy, dfinal_state};
+    const size_t insz[] = {xb, tb, hb, bcb, bcb, hb, sb, xb, sb};
+    const void *outs[] = {dx, ddt, dA, dB, dC, dD, dinit_state, workspace};
+    const size_t outsz[] = {xb, tb, hb, bcb, bcb, hb, sb, w.total};
+    for (int i = 0; i < 8; ++i) {
+        for (int j = 0; j < 9; ++j)
+            if (ssd::ranges_overlap(outs[i], outsz[i], ins[j], insz[j])) return SSD_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 8; ++j)
+            if (ssd::ranges_overlap(outs[i], outsz[i], outs[j], outsz[j])) return SSD_ERR_INVALID_ARG;
+    }
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // final = init: the gradient passes straight through; nothing else depends on the inputs
+        if (cudaMemsetAsync(dA, 0, hb, st) != cudaSuccess || cudaMemsetAsync(dD, 0, hb, st) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        if (!dinit_state) return SSD_OK;
+        cudaError_t e = dfinal_state
+                            ? cudaMemcpyAsync(dinit_state, dfinal_state, sb, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(dinit_state, 0, sb, st);
+        return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    }
+    char *ws = static_cast<char *>(workspace);
+    if (dtype == SSD_BF16) {
+        using bf = __nv_bfloat16;
+        return ssd::run_bwd<bf>(sh, static_cast<const bf *>(x), dt, A, static_cast<const bf *>(B),
+                                static_cast<const bf *>(C), D, init_state, static_cast<const bf *>(dy),
+                                dfinal_state, static_cast<bf *>(dx), ddt, dA, static_cast<bf *>(dB),
+                                static_cast<bf *>(dC), dD, dinit_state, ws, w, st);
+    }
+    return ssd::run_bwd<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
+                               static_cast<const float *>(C), D, init_state, static_cast<const float *>(dy),
+                               dfinal_state, static_cast<float *>(dx), ddt, dA, static_cast<float *>(dB),
+                               static_cast<float *>(dC), dD, dinit_state, ws, w, st);
+}

@@ -45,6 +45,14 @@ struct Workspace {
     size_t total;
 };
 
+// Dimension limits shared by the forward and backward entry points.
+constexpr int kMaxP = 128, kMaxN = 256, kMaxQ = 256;
+constexpr int64_t kMaxElems = int64_t(1) << 46;
+
+// Validates the dimensions of a forward or backward call; fills `sh` on success
+// (ssd_api.cu).
+int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, Shape *sh);
+
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 inline Workspace workspace_layout(const Shape &s, Path path) {

@@ -95,15 +95,17 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restri
 // ---------------------------------------------------------------------------
 // Stage 2: chunk-final states from a zero start,
 //   S_c[p][n] = sum_i exp(s_end - s_i) * x_i[p] * B_i[n].
+// With from_start the weights are exp(s_i) instead (the decay from the chunk's
+// start): the backward pass's chunk sums of dy_i C_i^T use this form.
 // grid (nc, H, batch), 256 threads as 16 (n) x 16 (p); each thread owns an
 // RP x RN register tile.  Rows are staged through shared memory 32 at a time.
 // ---------------------------------------------------------------------------
 template <typename T, int RP, int RN>
 __global__ void __launch_bounds__(256) chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ Bm,
                                                           const float *__restrict__ s, float *__restrict__ S,
-                                                          Shape sh) {
+                                                          Shape sh, bool from_start) {
     extern __shared__ float smem[];
-    float *Xs = smem;               // [32][P], already scaled by the decay to the chunk end
+    float *Xs = smem;               // [32][P], already scaled by the decay weight
     float *Bs = smem + 32 * sh.P;   // [32][N]
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / sh.heads_per_group;
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(const T *__restrict__ 
             const int ii = idx / sh.P, p = idx - ii * sh.P, i = i0 + ii;
             float v = 0.f;
             if (i < len)
-                v = to_f32(x[(((size_t)b * sh.T + t0 + i) * sh.H + h) * sh.P + p]) * expf(s_end - sc[i]);
+                v = to_f32(x[(((size_t)b * sh.T + t0 + i) * sh.H + h) * sh.P + p]) *
+                    expf(from_start ? sc[i] : s_end - sc[i]);
             Xs[idx] = v;
         }
         for (int idx = threadIdx.x; idx < 32 * sh.N; idx += 256) {
@@ -359,34 +362,35 @@ cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const
 
 template <typename T, int RP, int RN>
 static cudaError_t launch_state_rprn(const T *x, const T *B, const float *s, float *S, const Shape &sh,
-                                     cudaStream_t st) {
+                                     cudaStream_t st, bool from_start) {
     const size_t smem = sizeof(float) * 32 * (size_t)(sh.P + sh.N);
     auto k = chunk_state_kernel<T, RP, RN>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<dim3(sh.nc, sh.H, sh.batch), 256, smem, st>>>(x, B, s, S, sh);
+    k<<<dim3(sh.nc, sh.H, sh.batch), 256, smem, st>>>(x, B, s, S, sh, from_start);
     return cudaGetLastError();
 }
 
 template <typename T, int RP>
 static cudaError_t launch_state_rp(const T *x, const T *B, const float *s, float *S, const Shape &sh,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, bool from_start) {
     switch (pow2_at_least((sh.N + 15) / 16)) {
-        case 1: return launch_state_rprn<T, RP, 1>(x, B, s, S, sh, st);
-        case 2: return launch_state_rprn<T, RP, 2>(x, B, s, S, sh, st);
-        case 4: return launch_state_rprn<T, RP, 4>(x, B, s, S, sh, st);
-        case 8: return launch_state_rprn<T, RP, 8>(x, B, s, S, sh, st);
-        default: return launch_state_rprn<T, RP, 16>(x, B, s, S, sh, st);
+        case 1: return launch_state_rprn<T, RP, 1>(x, B, s, S, sh, st, from_start);
+        case 2: return launch_state_rprn<T, RP, 2>(x, B, s, S, sh, st, from_start);
+        case 4: return launch_state_rprn<T, RP, 4>(x, B, s, S, sh, st, from_start);
+        case 8: return launch_state_rprn<T, RP, 8>(x, B, s, S, sh, st, from_start);
+        default: return launch_state_rprn<T, RP, 16>(x, B, s, S, sh, st, from_start);
     }
 }
 
 template <typename T>
-cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st) {
+cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S, const Shape &sh, cudaStream_t st,
+                               bool from_start) {
     switch (pow2_at_least((sh.P + 15) / 16)) {
-        case 1: return launch_state_rp<T, 1>(x, B, s, S, sh, st);
-        case 2: return launch_state_rp<T, 2>(x, B, s, S, sh, st);
-        case 4: return launch_state_rp<T, 4>(x, B, s, S, sh, st);
-        default: return launch_state_rp<T, 8>(x, B, s, S, sh, st);
+        case 1: return launch_state_rp<T, 1>(x, B, s, S, sh, st, from_start);
+        case 2: return launch_state_rp<T, 2>(x, B, s, S, sh, st, from_start);
+        case 4: return launch_state_rp<T, 4>(x, B, s, S, sh, st, from_start);
+        default: return launch_state_rp<T, 8>(x, B, s, S, sh, st, from_start);
     }
 }
 
@@ -421,9 +425,9 @@ cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D
 }
 
 template cudaError_t launch_chunk_state<float>(const float *, const float *, const float *, float *, const Shape &,
-                                               cudaStream_t);
+                                               cudaStream_t, bool);
 template cudaError_t launch_chunk_state<__nv_bfloat16>(const __nv_bfloat16 *, const __nv_bfloat16 *, const float *,
-                                                       float *, const Shape &, cudaStream_t);
+                                                       float *, const Shape &, cudaStream_t, bool);
 template cudaError_t launch_chunk_scan<float>(const float *, const float *, const float *, const float *,
                                               const float *, const float *, float *, const Shape &, cudaStream_t);
 template cudaError_t launch_chunk_scan<__nv_bfloat16>(const __nv_bfloat16 *, const __nv_bfloat16 *,

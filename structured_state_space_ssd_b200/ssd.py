@@ -24,7 +24,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
            "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc",
-           "ssd_step", "ssd_gate_norm", "ssd_split_logdecay", "ssd_split_combine", "ssd_split_correct")
+           "ssd_step", "ssd_gate_norm", "ssd_split_logdecay", "ssd_split_combine", "ssd_split_correct",
+           "ssd_bwd", "ssd_bwd_workspace_bytes")
 
 
 class SSDError(RuntimeError):
@@ -75,6 +76,10 @@ def load():
     lib.ssd_split_combine.restype = i
     lib.ssd_split_correct.argtypes = [vp, vp, fp, fp, i, i, i, i, i, i, i, vp]
     lib.ssd_split_correct.restype = i
+    lib.ssd_bwd.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, vp, fp, fp, vp, vp, fp, fp] + [i] * 7 + [vp, sz, vp]
+    lib.ssd_bwd.restype = i
+    lib.ssd_bwd_workspace_bytes.argtypes = [i] * 8
+    lib.ssd_bwd_workspace_bytes.restype = sz
     _lib = lib
     return lib
 
@@ -356,3 +361,91 @@ def ssd_fwd_sequence_parallel(x, dt, A, B, C, D, Q: int, init_state=None, group=
     s_in, fin = ssd_split_combine(fin0_all, total_all, k, init_state)
     ssd_split_correct(y, C, sig, s_in)
     return y, fin
+
+
+# --- backward pass and the autograd wrapper -----------------------------------------------------------
+
+def ssd_bwd_workspace_bytes(batch, T, H, P, G, N, Q, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else _dtype_code(dtype)
+    return int(load().ssd_bwd_workspace_bytes(batch, T, H, P, G, N, Q, code))
+
+
+def ssd_bwd(x, dt, A, B, C, D, dy, Q: int = 256, init_state=None, dfinal_state=None, *, need_dinit: bool = True,
+            workspace=None, stream=None):
+    """Gradients of ``sum(dy * y) + sum(dfinal_state * final_state)`` for ``ssd_fwd``'s inputs, on the GPU.
+
+    Inputs as for :func:`ssd_fwd`, plus dy [b,T,H,P] in x's dtype and dfinal_state [b,H,P,N] fp32
+    (None: zero).  Returns a dict with dx [b,T,H,P], dB, dC [b,T,G,N] (x's dtype), ddt [b,T,H],
+    dA [H], dD [H] and dinit_state [b,H,P,N] (fp32; None unless ``need_dinit``).
+    Runs on ``stream`` (default: the current torch stream) without host sync.
+    """
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_bwd needs CUDA tensors (there is no CPU path)")
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    code = _dtype_code(x.dtype)
+    named = dict(x=x, dt=dt, A=A, B=B, C=C, D=D, dy=dy, init_state=init_state, dfinal_state=dfinal_state)
+    for k, t in named.items():
+        if t is None:
+            continue
+        if t.device != dev:
+            raise ValueError(f"{k} is on {t.device}, x on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{k} must be contiguous")
+    if B.dtype != x.dtype or C.dtype != x.dtype or dy.dtype != x.dtype:
+        raise TypeError("x, B, C and dy must share one dtype")
+    for k in ("dt", "A", "D", "init_state", "dfinal_state"):
+        if named[k] is not None and named[k].dtype != torch.float32:
+            raise TypeError(f"{k} must be float32")
+    if tuple(dt.shape) != (b, T, H) or tuple(A.shape) != (H,) or tuple(D.shape) != (H,) or dy.shape != x.shape:
+        raise ValueError("dt must be [b,T,H]; A and D must be [H]; dy must match x")
+    if tuple(B.shape) != (b, T, G, N) or tuple(C.shape) != (b, T, G, N):
+        raise ValueError("B and C must be [b,T,G,N]")
+    for k in ("init_state", "dfinal_state"):
+        if named[k] is not None and tuple(named[k].shape) != (b, H, P, N):
+            raise ValueError(f"{k} must be [b,H,P,N]")
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty_like(x), "ddt": torch.empty((b, T, H), **f32), "dA": torch.empty((H,), **f32),
+           "dB": torch.empty_like(B), "dC": torch.empty_like(C), "dD": torch.empty((H,), **f32),
+           "dinit_state": torch.empty((b, H, P, N), **f32) if need_dinit else None}
+    lib = load()
+    need = int(lib.ssd_bwd_workspace_bytes(b, T, H, P, G, N, int(Q), code))
+    if need == 0:
+        raise SSDError(1, "ssd_bwd_workspace_bytes")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    rc = lib.ssd_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(Q), _ptr(init_state), _ptr(dy),
+                     _ptr(dfinal_state), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dB"]),
+                     _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dinit_state"]), b, T, H, P, G, N, code,
+                     _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                     _handle(stream, dev))
+    if rc != 0:
+        raise SSDError(rc, "ssd_bwd")
+    return out
+
+
+class _SSDLayer(torch.autograd.Function):
+    """ssd_fwd forward, ssd_bwd backward; no arithmetic of its own."""
+
+    @staticmethod
+    def forward(ctx, x, dt, A, B, C, D, init_state, Q):
+        y, fin = ssd_fwd(x, dt, A, B, C, D, Q, init_state)
+        ctx.Q = Q
+        ctx.save_for_backward(x, dt, A, B, C, D, init_state)
+        return y, fin
+
+    @staticmethod
+    def backward(ctx, dy, dfin):
+        x, dt, A, B, C, D, init_state = ctx.saved_tensors
+        dy = torch.zeros_like(x) if dy is None else dy.to(x.dtype).contiguous()
+        dfin = None if dfin is None else dfin.float().contiguous()
+        need_dinit = init_state is not None and ctx.needs_input_grad[6]
+        g = ssd_bwd(x, dt, A, B, C, D, dy, ctx.Q, init_state, dfin, need_dinit=need_dinit)
+        return g["dx"], g["ddt"], g["dA"], g["dB"], g["dC"], g["dD"], g["dinit_state"], None
+
+
+def ssd_layer(x, dt, A, B, C, D, Q: int = 256, init_state=None):
+    """Differentiable SSD layer: returns ``(y, final_state)`` like :func:`ssd_fwd`, with gradients for every
+    tensor input through :func:`ssd_bwd` (torch autograd only records the call)."""
+    return _SSDLayer.apply(x, dt, A, B, C, D, init_state, int(Q))

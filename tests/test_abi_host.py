@@ -158,3 +158,44 @@ def test_gate_norm_rejects_invalid_arguments_on_the_host(lib, over, code):
 def test_split_entry_points_validate_on_the_host(lib, call, code):
     v = lambda a: ctypes.c_void_p(0x100000 * a)  # noqa: E731  (never dereferenced)
     assert call(lib, v) == code
+
+
+def test_bwd_workspace_bytes(lib):
+    f = lib.ssd_bwd_workspace_bytes
+    w = f(4, 2048, 80, 64, 1, 128, 256, 1)
+    # two sets of chunk states and the per-head dB, dC terms at least
+    assert w % 256 == 0 and w >= 2 * (4 * 8 * 80 * 64 * 128 * 4) + 2 * (4 * 2048 * 80 * 128 * 4)
+    assert f(4, 2048, 80, 64, 3, 128, 256, 1) == 0      # H % G != 0
+    assert f(4, 2048, 80, 256, 1, 128, 256, 1) == 0     # P above the limit
+    assert f(1, 0, 2, 16, 1, 16, 64, 0) > 0             # empty sequence is valid
+
+
+def _bwd(lib, **over):
+    """ssd_bwd with fake (never dereferenced) pointers; only validation runs."""
+    args = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, Q=64, init=None, dy=0x70000,
+                dfin=None, dx=0x80000, ddt=0x90000, dA=0xa0000, dB=0xb0000, dC=0xc0000, dD=0xd0000, dinit=None,
+                batch=1, T=256, H=2, P=16, G=1, N=16, dtype=0, ws=0x100000, wsb=1 << 40, stream=None)
+    args.update(over)
+    v = lambda a: None if a is None else ctypes.c_void_p(a)  # noqa: E731
+    a = args
+    return lib.ssd_bwd(v(a["x"]), v(a["dt"]), v(a["A"]), v(a["B"]), v(a["C"]), v(a["D"]), a["Q"], v(a["init"]),
+                       v(a["dy"]), v(a["dfin"]), v(a["dx"]), v(a["ddt"]), v(a["dA"]), v(a["dB"]), v(a["dC"]),
+                       v(a["dD"]), v(a["dinit"]), a["batch"], a["T"], a["H"], a["P"], a["G"], a["N"], a["dtype"],
+                       v(a["ws"]), ctypes.c_size_t(a["wsb"]), v(a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(x=None), 1), (dict(dy=None), 1), (dict(dx=None), 1), (dict(ddt=None), 1), (dict(dA=None), 1),
+    (dict(dB=None), 1), (dict(dC=None), 1), (dict(dD=None), 1), (dict(ws=None), 1),
+    (dict(H=3, G=2), 1), (dict(dtype=5), 1), (dict(Q=0), 1), (dict(P=256), 2), (dict(batch=70000), 2),
+    (dict(wsb=16), 1),                                    # workspace too small
+    (dict(ws=0x100010), 1),                               # workspace not 256-byte aligned
+    (dict(dtype=1, x=0x10001), 1),                        # bf16 tensor not 2-byte aligned
+    (dict(dx=0x10000), 1),                                # dx aliases x
+    (dict(dB=0x70000 + 64), 1),                           # dB inside dy
+    (dict(dfin=0x200000, dinit=0x200000), 1),             # dinit aliases dfinal
+    (dict(dC=0xb0000), 1),                                # two outputs on one buffer
+    (dict(dD=0x100000 + 256), 1),                         # an output inside the workspace
+])
+def test_bwd_rejects_invalid_arguments_on_the_host(lib, over, code):
+    assert _bwd(lib, **over) == code
