@@ -131,8 +131,19 @@ __global__ void __launch_bounds__(256) state_passing_bwd_kernel(float *__restric
 // [batch][T][*] tensors: R and K have KD columns, V has W; each is either a
 // head's slice (row length H*KD or H*W) or its group's (G*KD or G*W).  St is
 // the [P][N] state of the (batch, chunk, head), read as [W][KD] or [KD][W].
-// grid (nc * ceil(Q/64), H, batch), 256 threads as 16 (w) x 16 (rows); each
-// thread owns 4 rows x RW columns.
+// grid (nc * ceil(Q/64), H, batch), 256 threads.
+//
+// Shared memory, fp32 (KD4 = KD rounded up to 4; KP = KD4 + 4 keeps rows
+// 16-byte aligned and puts eight consecutive rows on distinct bank quads;
+// W64 = 64 RV >= W; SW = W64 + 4):
+//   Rs [64][KP] the tile's rows of R     Ks [32][KP]  32 columns' rows of K
+//   Vs [32][W64] their rows of V         Ss [32][SW]  32 contraction rows of the state
+//   Ms [64][36] the masked weights of the 64 x 32 block;  sr [64], sc [32] prefix sums
+// The output belongs to 16 (tx) x 16 (ty) threads: rows ty + 16 rr (rr < 4),
+// columns 64 v + 4 tx + e (v < RV, e < 4), read as float4 rows of V and of the
+// state.  The 64 x 32 dot products belong to 32 (rg) x 8 (cg) threads: rows
+// rg + 32 p (p < 2), columns cg + 8 q (q < 4), float4 along the contraction.
+// Every shared-memory operand is then used by at least two FMAs per load.
 // ---------------------------------------------------------------------------
 struct ScanArgs {
     const void *R, *K, *V;
@@ -142,19 +153,36 @@ struct ScanArgs {
     int KD, W;
     const float *D;              // skip factor per head, or null
     void *out;                   // [batch][T][H][W]
+    int vec;                     // R, K, V rows load as 16-byte vectors (aligned, KD and W multiples of it)
+    int st_vec;                  // the state loads as float4 (its rows' lengths multiples of 4)
 };
 
-template <typename T, typename TO, int RW, bool kAnti>
+constexpr int kMsLd = 36;  // row length of Ms (32 columns, padded to keep float4 rows aligned)
+
+// 16-byte asynchronous copy global -> shared (zero-filled when src_bytes is 0), and its group fences.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+template <typename T, typename TO, int RV, bool kAnti>
 __global__ void __launch_bounds__(256) masked_scan_kernel(ScanArgs a, const float *__restrict__ s, Shape sh) {
-    extern __shared__ float smem[];
-    const int KD = a.KD, W = a.W, KP = KD + 1;
-    float *Rs = smem;              // [64][KD+1]
-    float *Ks = Rs + 64 * KP;      // [32][KD+1]
-    float *Vs = Ks + 32 * KP;      // [32][W]
-    float *Ms = Vs + 32 * W;       // [64][33]
-    float *sr = Ms + 64 * 33;      // [64]
+    extern __shared__ __align__(16) float smem[];
+    const int KD = a.KD, W = a.W;
+    const int KD4 = (KD + 3) & ~3, KP = KD4 + 4;
+    constexpr int W64 = 64 * RV, SW = W64 + 4;
+    float *Rs = smem;              // [64][KP]
+    float *Ks = Rs + 64 * KP;      // [32][KP]
+    float *Vs = Ks + 32 * KP;      // [32][W64]
+    float *Ss = Vs + 32 * W64;     // [32][SW]
+    float *Ms = Ss + 32 * SW;      // [64][kMsLd]
+    float *sr = Ms + 64 * kMsLd;   // [64]
     float *sc = sr + 64;           // [32]
-    float *Ss = sc + 32;           // [W][33]
+    float *sq = sc + 32;           // [kMaxQ]: the chunk's prefix sums
+    T *KsRaw = reinterpret_cast<T *>(sq + kMaxQ);  // [32][KD] next column tile as copied (vec only)
+    T *VsRaw = KsRaw + 32 * KD;                    // [32][W]
     const int tiles = (sh.Q + 63) >> 6;
     const int c = blockIdx.x / tiles, jt = blockIdx.x - c * tiles;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -172,52 +200,71 @@ __global__ void __launch_bounds__(256) masked_scan_kernel(ScanArgs a, const floa
     const size_t v_ld = (size_t)(a.v_head ? sh.H : sh.G) * W, v_off = (size_t)(a.v_head ? h : g) * W;
     const size_t row0 = (size_t)b * sh.T + t0;  // token index of the chunk's first row
 
-    for (int idx = threadIdx.x; idx < 64 * KD; idx += 256) {
-        const int jj = idx / KD, k = idx - jj * KD;
-        Rs[jj * KP + k] = (jj < jn) ? to_f32(Rp[(row0 + j0 + jj) * r_ld + r_off + k]) : 0.f;
-    }
+    stage_rows<T>(Rs, KP, Rp + (row0 + j0) * r_ld + r_off, r_ld, 64, jn, KD, KD4, a.vec);
     if (threadIdx.x < 64) sr[threadIdx.x] = (threadIdx.x < jn) ? sch[j0 + threadIdx.x] : 0.f;
+    for (int i = threadIdx.x; i < sh.Q; i += 256) sq[i] = sch[i];
     __syncthreads();
 
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][RW];
+    float acc[4][RV][4];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int k = 0; k < RW; ++k) acc[r][k] = 0.f;
+        for (int v = 0; v < RV; ++v)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[r][v][e] = 0.f;
 
     // the state term, 32 of the KD contraction indices at a time
     const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
     for (int k0 = 0; k0 < KD; k0 += 32) {
-        for (int idx = threadIdx.x; idx < W * 32; idx += 256) {
-            int w, kk;
-            if (a.st_kw) {  // [KD][W]: consecutive threads along w
-                kk = idx / W;
-                w = idx - kk * W;
-            } else {        // [W][KD]: consecutive threads along k
-                w = idx >> 5;
-                kk = idx & 31;
+        if (a.st_kw) {  // [KD][W]: rows k0.. of the state, lanes along w
+            stage_rows<float>(Ss, SW, Sp + (size_t)k0 * W, W, 32, KD - k0, W, W64, a.st_vec);
+        } else if (a.st_vec) {  // [W][KD], KD a multiple of 4: float4 along k, stored transposed
+            const int total = W64 * 8;  // (row w, quad of k) pairs of the slab
+            for (int base = threadIdx.x; base < total; base += 4 * 256) {
+                float4 u[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int idx = base + q * 256, w = idx >> 3, k = k0 + 4 * (idx & 7);
+                    u[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (idx < total && w < W && k < KD)
+                        u[q] = *reinterpret_cast<const float4 *>(Sp + (size_t)w * KD + k);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int idx = base + q * 256, w = idx >> 3, kk = 4 * (idx & 7);
+                    if (idx < total) {
+                        Ss[kk * SW + w] = u[q].x;
+                        Ss[(kk + 1) * SW + w] = u[q].y;
+                        Ss[(kk + 2) * SW + w] = u[q].z;
+                        Ss[(kk + 3) * SW + w] = u[q].w;
+                    }
+                }
             }
-            const int k = k0 + kk;
-            float v = 0.f;
-            if (k < KD) v = a.st_kw ? Sp[(size_t)k * W + w] : Sp[(size_t)w * KD + k];
-            Ss[w * 33 + kk] = v;
+        } else {        // [W][KD]: a warp reads 8 consecutive k of 4 rows
+            for (int idx = threadIdx.x; idx < 32 * W64; idx += 256) {
+                const int lane = idx & 31, grp = idx >> 5;
+                const int kk = (lane & 7) + 8 * (grp & 3), w = (lane >> 3) + 4 * (grp >> 2), k = k0 + kk;
+                Ss[kk * SW + w] = (k < KD && w < W) ? Sp[(size_t)w * KD + k] : 0.f;
+            }
         }
         __syncthreads();
         const int klim = min(32, KD - k0);
         for (int kk = 0; kk < klim; ++kk) {
-            float rv[4], sv[RW];
+            float rv[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) rv[r] = Rs[(ty + 16 * r) * KP + k0 + kk];
 #pragma unroll
-            for (int k = 0; k < RW; ++k) {
-                const int w = tx + 16 * k;
-                sv[k] = (w < W) ? Ss[w * 33 + kk] : 0.f;
+            for (int v = 0; v < RV; ++v) {
+                const float4 sv = *reinterpret_cast<const float4 *>(Ss + kk * SW + 64 * v + 4 * tx);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    acc[r][v][0] = fmaf(rv[r], sv.x, acc[r][v][0]);
+                    acc[r][v][1] = fmaf(rv[r], sv.y, acc[r][v][1]);
+                    acc[r][v][2] = fmaf(rv[r], sv.z, acc[r][v][2]);
+                    acc[r][v][3] = fmaf(rv[r], sv.w, acc[r][v][3]);
+                }
             }
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int k = 0; k < RW; ++k) acc[r][k] = fmaf(rv[r], sv[k], acc[r][k]);
         }
         __syncthreads();
     }
@@ -228,55 +275,128 @@ __global__ void __launch_bounds__(256) masked_scan_kernel(ScanArgs a, const floa
             const float sj = sr[ty + 16 * r];
             const float e = kAnti ? expf(s_end - sj) : expf(sj);
 #pragma unroll
-            for (int k = 0; k < RW; ++k) acc[r][k] *= e;
+            for (int v = 0; v < RV; ++v)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[r][v][q] *= e;
         }
     }
 
     // the masked quadratic term over the chunk's other rows
     const int ibeg = kAnti ? j0 : 0;
     const int iend = kAnti ? len : j0 + jn;
+    const int rg = threadIdx.x >> 3, cg = threadIdx.x & 7;
+    // With 16-byte rows the next column tile is copied asynchronously (raw, into KsRaw / VsRaw) while
+    // this one's products run, then widened to fp32 in shared memory.
+    constexpr int VE = 16 / (int)sizeof(T);
+    const bool pipe = a.vec;
+    auto issue = [&](int i0n) {
+        const int valid = iend - i0n, kcr = KD / VE, vcr = W / VE;
+        for (int idx = threadIdx.x; idx < 32 * kcr; idx += 256) {
+            const int r = idx / kcr, kc = idx - r * kcr;
+            const bool ok = r < valid;
+            cp_async16(KsRaw + r * KD + kc * VE, ok ? Kp + (row0 + i0n + r) * k_ld + k_off + kc * VE : Kp, ok ? 16 : 0);
+        }
+        for (int idx = threadIdx.x; idx < 32 * vcr; idx += 256) {
+            const int r = idx / vcr, vc = idx - r * vcr;
+            const bool ok = r < valid;
+            cp_async16(VsRaw + r * W + vc * VE, ok ? Vp + (row0 + i0n + r) * v_ld + v_off + vc * VE : Vp, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    if (pipe) {
+        for (int idx = threadIdx.x; idx < 32 * (W64 - W); idx += 256) {  // padding columns stay zero
+            const int r = idx / (W64 - W);
+            Vs[r * W64 + W + (idx - r * (W64 - W))] = 0.f;
+        }
+        if (ibeg < iend) issue(ibeg);
+    }
     for (int i0 = ibeg; i0 < iend; i0 += 32) {
-        for (int idx = threadIdx.x; idx < 32 * KD; idx += 256) {
-            const int ii = idx / KD, k = idx - ii * KD, i = i0 + ii;
-            Ks[ii * KP + k] = (i < iend) ? to_f32(Kp[(row0 + i) * k_ld + k_off + k]) : 0.f;
+        if (pipe) {
+            cp_async_wait_all();
+            __syncthreads();
+            const int kcr = KD / VE, vcr = W / VE;
+            for (int idx = threadIdx.x; idx < 32 * kcr; idx += 256) {
+                const int r = idx / kcr, kc = idx - r * kcr;
+                float f[VE];
+                unpack16(*reinterpret_cast<const uint4 *>(KsRaw + r * KD + kc * VE), f, T());
+                float4 *d = reinterpret_cast<float4 *>(Ks + r * KP + kc * VE);
+#pragma unroll
+                for (int e = 0; e < VE / 4; ++e) d[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+            }
+            for (int idx = threadIdx.x; idx < 32 * vcr; idx += 256) {
+                const int r = idx / vcr, vc = idx - r * vcr;
+                float f[VE];
+                unpack16(*reinterpret_cast<const uint4 *>(VsRaw + r * W + vc * VE), f, T());
+                float4 *d = reinterpret_cast<float4 *>(Vs + r * W64 + vc * VE);
+#pragma unroll
+                for (int e = 0; e < VE / 4; ++e) d[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+            }
+            if (threadIdx.x < 32) sc[threadIdx.x] = (i0 + threadIdx.x < iend) ? sq[i0 + threadIdx.x] : 0.f;
+            __syncthreads();
+            if (i0 + 32 < iend) issue(i0 + 32);
+        } else {
+            stage_rows<T>(Ks, KP, Kp + (row0 + i0) * k_ld + k_off, k_ld, 32, iend - i0, KD, KD4, false);
+            stage_rows<T>(Vs, W64, Vp + (row0 + i0) * v_ld + v_off, v_ld, 32, iend - i0, W, W64, false);
+            if (threadIdx.x < 32) sc[threadIdx.x] = (i0 + threadIdx.x < iend) ? sq[i0 + threadIdx.x] : 0.f;
+            __syncthreads();
         }
-        for (int idx = threadIdx.x; idx < 32 * W; idx += 256) {
-            const int ii = idx / W, w = idx - ii * W, i = i0 + ii;
-            Vs[idx] = (i < iend) ? to_f32(Vp[(row0 + i) * v_ld + v_off + w]) : 0.f;
-        }
-        if (threadIdx.x < 32) sc[threadIdx.x] = (i0 + threadIdx.x < iend) ? sch[i0 + threadIdx.x] : 0.f;
-        __syncthreads();
         {
-            const int jj = threadIdx.x >> 2, ib = (threadIdx.x & 3) * 8;
-            float dot[8];
+            float dot[2][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dot[e] = 0.f;
-            for (int k = 0; k < KD; ++k) {
-                const float rv = Rs[jj * KP + k];
+            for (int p = 0; p < 2; ++p)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dot[e] = fmaf(rv, Ks[(ib + e) * KP + k], dot[e]);
+                for (int q = 0; q < 4; ++q) dot[p][q] = 0.f;
+            const float *ra_p = Rs + rg * KP, *rb_p = Rs + (rg + 32) * KP;
+            for (int k = 0; k < KD4; k += 4) {
+                const float4 ra = *reinterpret_cast<const float4 *>(ra_p + k);
+                const float4 rb = *reinterpret_cast<const float4 *>(rb_p + k);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 kv = *reinterpret_cast<const float4 *>(Ks + (cg + 8 * q) * KP + k);
+                    float d0 = dot[0][q], d1 = dot[1][q];
+                    d0 = fmaf(ra.x, kv.x, d0);
+                    d1 = fmaf(rb.x, kv.x, d1);
+                    d0 = fmaf(ra.y, kv.y, d0);
+                    d1 = fmaf(rb.y, kv.y, d1);
+                    d0 = fmaf(ra.z, kv.z, d0);
+                    d1 = fmaf(rb.z, kv.z, d1);
+                    d0 = fmaf(ra.w, kv.w, d0);
+                    d1 = fmaf(rb.w, kv.w, d1);
+                    dot[0][q] = d0;
+                    dot[1][q] = d1;
+                }
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int ii = ib + e, i = i0 + ii, j = j0 + jj;
-                const bool ok = jj < jn && i < iend && (kAnti ? i >= j : i <= j);
-                Ms[jj * 33 + ii] = ok ? expf(kAnti ? sc[ii] - sr[jj] : sr[jj] - sc[ii]) * dot[e] : 0.f;
+            for (int p = 0; p < 2; ++p) {
+                const int jj = rg + 32 * p, j = j0 + jj;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int ii = cg + 8 * q, i = i0 + ii;
+                    const bool ok = jj < jn && i < iend && (kAnti ? i >= j : i <= j);
+                    Ms[jj * kMsLd + ii] = ok ? expf(kAnti ? sc[ii] - sr[jj] : sr[jj] - sc[ii]) * dot[p][q] : 0.f;
+                }
             }
         }
         __syncthreads();
-        for (int ii = 0; ii < 32; ++ii) {
-            float mv[4], vv[RW];
+        for (int ii = 0; ii < 32; ii += 4) {
+            float4 mv[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) mv[r] = Ms[(ty + 16 * r) * 33 + ii];
+            for (int r = 0; r < 4; ++r) mv[r] = *reinterpret_cast<const float4 *>(Ms + (ty + 16 * r) * kMsLd + ii);
 #pragma unroll
-            for (int k = 0; k < RW; ++k) {
-                const int w = tx + 16 * k;
-                vv[k] = (w < W) ? Vs[ii * W + w] : 0.f;
+            for (int e2 = 0; e2 < 4; ++e2) {
+#pragma unroll
+                for (int v = 0; v < RV; ++v) {
+                    const float4 vv = *reinterpret_cast<const float4 *>(Vs + (ii + e2) * W64 + 64 * v + 4 * tx);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float m = e2 == 0 ? mv[r].x : e2 == 1 ? mv[r].y : e2 == 2 ? mv[r].z : mv[r].w;
+                        acc[r][v][0] = fmaf(m, vv.x, acc[r][v][0]);
+                        acc[r][v][1] = fmaf(m, vv.y, acc[r][v][1]);
+                        acc[r][v][2] = fmaf(m, vv.z, acc[r][v][2]);
+                        acc[r][v][3] = fmaf(m, vv.w, acc[r][v][3]);
+                    }
+                }
             }
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int k = 0; k < RW; ++k) acc[r][k] = fmaf(mv[r], vv[k], acc[r][k]);
         }
         __syncthreads();
     }
@@ -290,12 +410,15 @@ __global__ void __launch_bounds__(256) masked_scan_kernel(ScanArgs a, const floa
         const size_t tok = row0 + j0 + jj;
         TO *orow = out + (tok * sh.H + h) * W;
 #pragma unroll
-        for (int k = 0; k < RW; ++k) {
-            const int w = tx + 16 * k;
-            if (w >= W) continue;
-            float v = acc[r][k];
-            if (a.D) v = fmaf(Dh, to_f32(Vp[tok * v_ld + v_off + w]), v);
-            orow[w] = from_f32<TO>(v);
+        for (int v = 0; v < RV; ++v) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int w = 64 * v + 4 * tx + e;
+                if (w >= W) continue;
+                float val = acc[r][v][e];
+                if (a.D) val = fmaf(Dh, to_f32(Vp[tok * v_ld + v_off + w]), val);
+                orow[w] = from_f32<TO>(val);
+            }
         }
     }
 }
@@ -458,20 +581,16 @@ __global__ void __launch_bounds__(256) param_reduce_kernel(const double *__restr
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-int pow2_ceil(int v) {
-    int r = 1;
-    while (r < v) r <<= 1;
-    return r;
+size_t scan_smem_bytes(int KD, int W, size_t es, bool vec) {
+    const size_t KP = (size_t)((KD + 3) & ~3) + 4, W64 = (size_t)64 * ((W + 63) / 64);
+    const size_t raw = vec ? 32 * (size_t)(KD + W) * es : 0;
+    return sizeof(float) * (96 * KP + 32 * W64 + 32 * (W64 + 4) + 64 * kMsLd + 96 + kMaxQ) + raw;
 }
 
-size_t scan_smem_bytes(int KD, int W) {
-    return sizeof(float) * ((size_t)96 * (KD + 1) + (size_t)32 * W + 64 * 33 + 96 + (size_t)W * 33);
-}
-
-template <typename T, typename TO, int RW, bool kAnti>
-cudaError_t launch_scan_rw(const ScanArgs &a, const float *s, const Shape &sh, cudaStream_t st) {
-    const size_t smem = scan_smem_bytes(a.KD, a.W);
-    auto k = masked_scan_kernel<T, TO, RW, kAnti>;
+template <typename T, typename TO, int RV, bool kAnti>
+cudaError_t launch_scan_rv(const ScanArgs &a, const float *s, const Shape &sh, cudaStream_t st) {
+    const size_t smem = scan_smem_bytes(a.KD, a.W, sizeof(T), a.vec != 0);
+    auto k = masked_scan_kernel<T, TO, RV, kAnti>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = (sh.Q + 63) / 64;
@@ -481,12 +600,11 @@ cudaError_t launch_scan_rw(const ScanArgs &a, const float *s, const Shape &sh, c
 
 template <typename T, typename TO, bool kAnti>
 cudaError_t launch_scan(const ScanArgs &a, const float *s, const Shape &sh, cudaStream_t st) {
-    switch (pow2_ceil((a.W + 15) / 16)) {
-        case 1: return launch_scan_rw<T, TO, 1, kAnti>(a, s, sh, st);
-        case 2: return launch_scan_rw<T, TO, 2, kAnti>(a, s, sh, st);
-        case 4: return launch_scan_rw<T, TO, 4, kAnti>(a, s, sh, st);
-        case 8: return launch_scan_rw<T, TO, 8, kAnti>(a, s, sh, st);
-        default: return launch_scan_rw<T, TO, 16, kAnti>(a, s, sh, st);
+    switch ((a.W + 63) / 64) {
+        case 1: return launch_scan_rv<T, TO, 1, kAnti>(a, s, sh, st);
+        case 2: return launch_scan_rv<T, TO, 2, kAnti>(a, s, sh, st);
+        case 3: return launch_scan_rv<T, TO, 3, kAnti>(a, s, sh, st);
+        default: return launch_scan_rv<T, TO, 4, kAnti>(a, s, sh, st);
     }
 }
 
@@ -520,14 +638,19 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     const int PN = sh.P * sh.N;
     state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    // 16-byte operand loads need 16-byte aligned tensors whose rows are whole vectors
+    constexpr int VE = 16 / (int)sizeof(T);
+    const bool al = is_aligned(x, 16) && is_aligned(dy, 16) && is_aligned(B, 16) && is_aligned(C, 16);
+    const int vec = al && sh.P % VE == 0 && sh.N % VE == 0;
+    const int st_vec = sh.P % 4 == 0 && sh.N % 4 == 0;
     // dx: rows of B against columns of C, values dy, state dHout as [P][N] = [W][KD], skip D dy
-    ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx};
+    ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx, vec, st_vec};
     if (launch_scan<T, T, true>(ax, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     // dB^(h): rows of x against columns of dy, values C, state dHout as [P][N] = [KD][W]
-    ScanArgs ab{x, dy, C, 1, 1, 0, Gout, 1, sh.P, sh.N, nullptr, dBh};
+    ScanArgs ab{x, dy, C, 1, 1, 0, Gout, 1, sh.P, sh.N, nullptr, dBh, vec, st_vec};
     if (launch_scan<T, float, true>(ab, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     // dC^(h): rows of dy against columns of x, values B, state Hin as [P][N] = [KD][W]
-    ScanArgs ac{dy, x, B, 1, 1, 0, Hin, 1, sh.P, sh.N, nullptr, dCh};
+    ScanArgs ac{dy, x, B, 1, 1, 0, Hin, 1, sh.P, sh.N, nullptr, dCh, vec, st_vec};
     if (launch_scan<T, float, false>(ac, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     const long long units = (long long)sh.batch * sh.T * sh.G;
     group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);

@@ -19,6 +19,68 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(v);
 }
 
+// 16 bytes of T as fp32: four floats or eight bf16 (a bf16 is the top half of its fp32).
+__device__ __forceinline__ void unpack16(const uint4 &u, float *f, float) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 &u, float *f, __nv_bfloat16) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// dst[r * dld + k] = src[r * ld + k] as fp32 for r < rows and k < cols, zero for rows r >= valid and
+// for columns k in [cols, cols_pad).  With vec (src and ld 16-byte aligned, cols a multiple of the
+// vector) each thread issues up to four 16-byte loads before it stores any.  All 256 threads call it.
+template <typename T>
+__device__ __forceinline__ void stage_rows(float *dst, int dld, const T *src, size_t ld, int rows, int valid,
+                                           int cols, int cols_pad, bool vec) {
+    if (vec) {
+        constexpr int VE = 16 / (int)sizeof(T);
+        const int cpr = cols / VE, total = rows * cpr;
+        for (int base = threadIdx.x; base < total; base += 4 * 256) {
+            uint4 u[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int idx = base + q * 256;
+                const int r = idx / cpr, kc = idx - r * cpr;
+                u[q] = make_uint4(0u, 0u, 0u, 0u);
+                if (idx < total && r < valid)
+                    u[q] = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)r * ld + (size_t)kc * VE));
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int idx = base + q * 256;
+                if (idx < total) {
+                    const int r = idx / cpr, kc = idx - r * cpr;
+                    float f[VE];
+                    unpack16(u[q], f, T());
+                    float4 *d = reinterpret_cast<float4 *>(dst + r * dld + kc * VE);
+#pragma unroll
+                    for (int e = 0; e < VE / 4; ++e)
+                        d[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+                }
+            }
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < rows * cols; idx += 256) {
+            const int r = idx / cols, k = idx - r * cols;
+            dst[r * dld + k] = r < valid ? to_f32(src[(size_t)r * ld + k]) : 0.f;
+        }
+    }
+    const int padc = cols_pad - cols;
+    for (int idx = threadIdx.x; idx < rows * padc; idx += 256) {
+        const int r = idx / padc, k = cols + (idx - r * padc);
+        dst[r * dld + k] = 0.f;
+    }
+}
+
 // Problem shape as every kernel sees it.
 struct Shape {
     int batch, T, H, P, G, N, Q, nc;

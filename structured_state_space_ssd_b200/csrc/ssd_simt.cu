@@ -103,10 +103,11 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(const float *__restri
 template <typename T, int RP, int RN>
 __global__ void __launch_bounds__(256) chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ Bm,
                                                           const float *__restrict__ s, float *__restrict__ S,
-                                                          Shape sh, bool from_start) {
-    extern __shared__ float smem[];
-    float *Xs = smem;               // [32][P], already scaled by the decay weight
+                                                          Shape sh, bool from_start, bool vec) {
+    extern __shared__ __align__(16) float smem[];
+    float *Xs = smem;               // [32][P]
     float *Bs = smem + 32 * sh.P;   // [32][N]
+    float *wr = Bs + 32 * sh.N;     // [32] decay weight of each row
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / sh.heads_per_group;
     const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0);
@@ -120,25 +121,23 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(const T *__restrict__ 
         for (int m = 0; m < RN; ++m) acc[r][m] = 0.f;
 
     for (int i0 = 0; i0 < len; i0 += 32) {
-        for (int idx = threadIdx.x; idx < 32 * sh.P; idx += 256) {
-            const int ii = idx / sh.P, p = idx - ii * sh.P, i = i0 + ii;
-            float v = 0.f;
-            if (i < len)
-                v = to_f32(x[(((size_t)b * sh.T + t0 + i) * sh.H + h) * sh.P + p]) *
-                    expf(from_start ? sc[i] : s_end - sc[i]);
-            Xs[idx] = v;
-        }
-        for (int idx = threadIdx.x; idx < 32 * sh.N; idx += 256) {
-            const int ii = idx / sh.N, n = idx - ii * sh.N, i = i0 + ii;
-            Bs[idx] = (i < len) ? to_f32(Bm[(((size_t)b * sh.T + t0 + i) * sh.G + g) * sh.N + n]) : 0.f;
+        // rows i0 .. i0+31 of x and B (16-byte loads when the rows allow), and each row's weight
+        stage_rows<T>(Xs, sh.P, x + (((size_t)b * sh.T + t0 + i0) * sh.H + h) * sh.P, (size_t)sh.H * sh.P, 32,
+                      len - i0, sh.P, sh.P, vec);
+        stage_rows<T>(Bs, sh.N, Bm + (((size_t)b * sh.T + t0 + i0) * sh.G + g) * sh.N, (size_t)sh.G * sh.N, 32,
+                      len - i0, sh.N, sh.N, vec);
+        if (threadIdx.x < 32) {
+            const int i = i0 + threadIdx.x;
+            wr[threadIdx.x] = (i < len) ? expf(from_start ? sc[i] : s_end - sc[i]) : 0.f;
         }
         __syncthreads();
         for (int ii = 0; ii < 32; ++ii) {
             float xv[RP], bv[RN];
+            const float wi = wr[ii];
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const int p = ty + 16 * r;
-                xv[r] = (p < sh.P) ? Xs[ii * sh.P + p] : 0.f;
+                xv[r] = (p < sh.P) ? Xs[ii * sh.P + p] * wi : 0.f;
             }
 #pragma unroll
             for (int m = 0; m < RN; ++m) {
@@ -363,11 +362,15 @@ cudaError_t launch_chunk_cumsum(const float *dt, const float *A, float *s, const
 template <typename T, int RP, int RN>
 static cudaError_t launch_state_rprn(const T *x, const T *B, const float *s, float *S, const Shape &sh,
                                      cudaStream_t st, bool from_start) {
-    const size_t smem = sizeof(float) * 32 * (size_t)(sh.P + sh.N);
+    const size_t smem = sizeof(float) * (32 * (size_t)(sh.P + sh.N) + 32);
     auto k = chunk_state_kernel<T, RP, RN>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<dim3(sh.nc, sh.H, sh.batch), 256, smem, st>>>(x, B, s, S, sh, from_start);
+    // 16-byte row loads: aligned tensors whose rows (P and N elements) are whole vectors
+    constexpr int VE = 16 / (int)sizeof(T);
+    const bool vec = reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(B) % 16 == 0 &&
+                     sh.P % VE == 0 && sh.N % VE == 0;
+    k<<<dim3(sh.nc, sh.H, sh.batch), 256, smem, st>>>(x, B, s, S, sh, from_start, vec);
     return cudaGetLastError();
 }
 
