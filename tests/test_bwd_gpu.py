@@ -127,3 +127,59 @@ def test_full_size_layer_on_sampled_tokens(cuda_device):
     _check("dD", got["dD"], np.einsum("bthp,bthp->h", dy, x), w.dtype)
     dt, A = inp["dt"].double().numpy(), inp["A"].double().numpy()
     _check("dA", got["dA"], np.einsum("bth,bth->h", dt, got["ddt"].astype(np.float64) / A), w.dtype)
+
+
+def test_backward_replays_from_a_cuda_graph(cuda_device):
+    # a training step captured once and replayed: same launches, same gradients
+    from structured_state_space_ssd_b200.ssd import ssd_bwd_workspace_bytes
+    inp = make_inputs(2, 600, 8, 64, 128, 2, "bf16", seed=45, with_init=True)
+    grads = make_output_grads(2, 600, 8, 64, 128, "bf16", seed=45, with_dfinal=True)
+    d, g = _to(cuda_device, inp), _to(cuda_device, grads)
+    ws = torch.empty(ssd_bwd_workspace_bytes(2, 600, 8, 64, 2, 128, 256, torch.bfloat16), dtype=torch.uint8,
+                     device=cuda_device)
+
+    def bwd():
+        return ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], g["dy"], 256, d["init_state"],
+                       g["dfinal_state"], workspace=ws, stream=torch.cuda.current_stream(cuda_device))
+
+    eager = {k: v.clone() for k, v in bwd().items()}
+    torch.cuda.synchronize(cuda_device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out = bwd()
+    for _ in range(2):
+        for v in out.values():
+            v.zero_()
+        graph.replay()
+        torch.cuda.synchronize(cuda_device)
+        for k, v in eager.items():
+            assert torch.equal(out[k], v), k
+    del graph
+
+
+@pytest.mark.parametrize("split", [300, 512])
+def test_backward_of_a_split_sequence_matches_the_whole(split, cuda_device):
+    # chain rule across a cut at token `split` (inside a chunk, or on a chunk boundary): the second part's
+    # backward from the first part's final state hands its initial-state gradient to the first part as
+    # its final-state gradient; per-token gradients concatenate, dA and dD add
+    b, T, H, P, N, G, Q = 2, 900, 4, 64, 128, 2, 256
+    inp = make_inputs(b, T, H, P, N, G, "f32", seed=46, with_init=True)
+    grads = make_output_grads(b, T, H, P, N, "f32", seed=46, with_dfinal=True)
+    d, g = _to(cuda_device, inp), _to(cuda_device, grads)
+    full = ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], g["dy"], Q, d["init_state"], g["dfinal_state"])
+
+    def part(lo, hi):
+        return {k: d[k][:, lo:hi].contiguous() for k in ("x", "dt", "B", "C")}, g["dy"][:, lo:hi].contiguous()
+
+    p1, dy1 = part(0, split)
+    p2, dy2 = part(split, T)
+    _, fin1 = ssd_fwd(p1["x"], p1["dt"], d["A"], p1["B"], p1["C"], d["D"], Q, d["init_state"])
+    g2 = ssd_bwd(p2["x"], p2["dt"], d["A"], p2["B"], p2["C"], d["D"], dy2, Q, fin1, g["dfinal_state"])
+    g1 = ssd_bwd(p1["x"], p1["dt"], d["A"], p1["B"], p1["C"], d["D"], dy1, Q, d["init_state"], g2["dinit_state"])
+    torch.cuda.synchronize(cuda_device)
+    for name in ("dx", "ddt", "dB", "dC"):
+        joined = torch.cat([g1[name], g2[name]], dim=1)
+        _check(name, joined.cpu().numpy(), full[name].double().cpu().numpy(), "f32")
+    for name in ("dA", "dD"):
+        _check(name, (g1[name] + g2[name]).cpu().numpy(), full[name].double().cpu().numpy(), "f32")
+    _check("dinit_state", g1["dinit_state"].cpu().numpy(), full["dinit_state"].double().cpu().numpy(), "f32")
