@@ -489,6 +489,15 @@ def measure_gate_norm(w, y, dev, stream, flush, peaks, steps=20):
             "alg_bytes": alg, "us_per_launch": ms * 1e3, "GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"]}
 
 
+def backward_alg_flops(w):
+    """Block-form work of the backward per call: per (batch, chunk), C B^T once per group; the masked
+    Q x Q products for dx and for W = dy x^T, and those of W with C and B for dB and dC; five Q x N x P
+    state products (forward and backward chunk states, the state terms of dx, dB and dC)."""
+    Q, H, P, N, G = w.Q, w.H, w.P, w.N, w.G
+    per_chunk = 2 * Q * Q * N * G + 2 * (2 * Q * Q * P * H) + 2 * (2 * Q * Q * N * H) + 5 * (2 * Q * N * P * H)
+    return per_chunk * w.batch * w.nc
+
+
 def measure_backward(w, d, dev, stream, flush, steps=5):
     """The layer's backward (ssd_bwd: every input gradient for given dy and dfinal) on this workload,
     L2 flushed before each call.  It runs on the CUDA cores in fp32, so its bound is the FFMA rate:
@@ -500,12 +509,8 @@ def measure_backward(w, d, dev, stream, flush, steps=5):
     dy, dfin = g["dy"].to(dev), g["dfinal_state"].to(dev)
     ws = torch.empty(S.ssd_bwd_workspace_bytes(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, dy.dtype), dtype=torch.uint8,
                      device=dev)
-    Q, H, P, N, G = w.Q, w.H, w.P, w.N, w.G
-    # block-form work per (batch, chunk): C B^T per group; the masked Q x Q products for dx, for
-    # W = dy x^T and for dB, dC; five Q x N x P state products (forward and backward chunk states, the
-    # state terms of dx, dB and dC)
-    per_chunk = 2 * Q * Q * N * G + 2 * (2 * Q * Q * P * H) + 2 * (2 * Q * Q * N * H) + 5 * (2 * Q * N * P * H)
-    alg_flops = per_chunk * w.batch * w.nc
+    Q = w.Q
+    alg_flops = backward_alg_flops(w)
 
     def one():
         S.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], dy, Q, d["init_state"], dfin, workspace=ws,
