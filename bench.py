@@ -531,7 +531,7 @@ def measure_backward(w, d, dev, stream, flush, steps=5):
     return {"ms": ms, "tokens_per_s": w.tokens / (ms * 1e-3), "alg_flops": alg_flops,
             "tflops": alg_flops / (ms * 1e-3) / 1e12, "bound": "alu",
             "frac_of_fp32_ffma_peak": alg_flops / (ms * 1e-3) / peak, "launches_per_call": 11,
-            "with": "init_state and dfinal_state"}
+            "with": "dfinal_state and init_state" if w.with_init else "dfinal_state (the workload has no init_state)"}
 
 
 def _traffic_from_profiles(kernel, w):
