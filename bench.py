@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-workloads", action="store_true")
     return ap.parse_args()
 
 
@@ -81,10 +82,8 @@ def algorithmic(w):
               + state * (2 if w.with_init else 1))
     per_chunk = 2 * Q * Q * N * G + 2 * Q * Q * P * H + 4 * Q * N * P * H + 2 * N * P * H
     flops = b * nc * per_chunk
-    # the fused kernel reads the prefix sums s in place of dt: same size per token
-    fused_bytes = bytes_ - 4 * b * T * H + 4 * b * H * nc * Q
     stages = {
-        "ssd_fused": ("pass", (fused_bytes, flops)),
+        "ssd_fused": ("pass", (bytes_, flops)),
         "ssd_chunk_cumsum": ("hbm", 4 * b * T * H + 4 * H + 4 * b * H * nc * Q),
         "ssd_chunk_state": ("flop", b * nc * 2 * Q * N * P * H),
         "ssd_state_passing": ("hbm", 2 * 4 * b * nc * H * P * N + state * (2 if w.with_init else 1)),
@@ -360,8 +359,7 @@ def main():
             roof = {"bound": "hbm", "achieved": amount / (dom_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s"}
         else:
-            tc = _stage_uses_tensor_cores(dom, w) or both is not None
-            if tc:
+            if both is not None:
                 roof = {"bound": "tensor", "achieved": amount / (dom_ms * 1e-3) / 1e12,
                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
             else:
@@ -392,6 +390,8 @@ def main():
             "gpu_launches": S.ssd_fwd_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
             * args.steps,
         }
+        if world == 1 and not args.no_workloads:
+            line["workloads"] = measure_workloads(w, dev, stream, flush, peaks)
         line["decode_step"] = measure_decode(w, host, dev, stream, flush, peaks)
         line["gate_norm"] = measure_gate_norm(w, y, dev, stream, flush, peaks)
         line["backward"] = measure_backward(w, d, dev, stream, flush)
@@ -402,8 +402,43 @@ def main():
         dist.destroy_process_group()
 
 
-def _stage_uses_tensor_cores(name, w):
-    return False
+def measure_workloads(headline, dev, stream, flush, peaks, steps=10, warmup=3):
+    """Every other bf16 workload of the configuration list, timed like the headline (L2 flushed between
+    steps, CUDA events recorded by the library around its kernels).  Their inputs are drawn on the GPU
+    (same distributions as the seeded CPU draws the parity tests use): only time is measured here."""
+    import torch
+    from structured_state_space_ssd_b200 import ssd as S
+    from structured_state_space_ssd_b200.inputs import WORKLOADS, make_inputs
+    out = {}
+    for name, w in WORKLOADS.items():
+        if name == headline.name or w.dtype != "bf16":
+            continue
+        d = make_inputs(w.batch, w.T, w.H, w.P, w.N, w.G, w.dtype, w.seed, w.with_init, device=str(dev))
+        y = torch.empty_like(d["x"])
+        fin = torch.empty((w.batch, w.H, w.P, w.N), dtype=torch.float32, device=dev)
+        ws = torch.empty(S.ssd_fwd_workspace_bytes(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype),
+                         dtype=torch.uint8, device=dev)
+        names = S.ssd_fwd_stage_names(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
+        per_step, per_stage = [], [[] for _ in names]
+        for k in range(warmup + steps):
+            flush.zero_()
+            ms = []
+            S.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], w.Q, d["init_state"], y=y, final_state=fin,
+                      workspace=ws, stream=stream, stage_ms=ms)
+            if k >= warmup:
+                per_step.append(ms[-1])
+                for i in range(len(names)):
+                    per_stage[i].append(ms[i])
+        ms_step = sum(per_step) / len(per_step)
+        alg_bytes, alg_flops, _ = algorithmic(w)
+        t_roof = max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flops / (peaks["bf16_tflops"] * 1e12))
+        out[name] = {"ms_per_step": ms_step, "tokens_per_s": w.tokens / (ms_step * 1e-3),
+                     "tflops": alg_flops / (ms_step * 1e-3) / 1e12,
+                     "pass_roofline": {"roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step},
+                     "kernels_ms": {n: sum(v) / len(v) for n, v in zip(names, per_stage)}}
+        del d, y, fin, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def measure_decode(w, host, dev, stream, flush, peaks, steps=50, resident_steps=200):

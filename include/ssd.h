@@ -133,6 +133,24 @@ SSD_API const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, in
 SSD_API int ssd_fwd_check(const void *workspace, void *stream);
 
 /*
+ * Test hook of the bounded waits (no counterpart on the pages): ssd_fwd on
+ * the fused tensor-core path, except that the block owning chunk
+ * `withhold_c` of sequence (withhold_b, withhold_h) never publishes its
+ * outgoing state, and every wait on another block's flag gives up after
+ * `flag_polls` polls (about 0.1-1 us each).  The blocks waiting for that
+ * state then give up, ssd_fwd_check reports SSD_ERR_TIMEOUT, the kernel still
+ * finishes (every block drains its own copies and products before it exits)
+ * and the device stays usable; y and final_state are not valid.  Arguments as
+ * for ssd_fwd plus the three indices (in range) and flag_polls >= 1; returns
+ * SSD_ERR_UNSUPPORTED for problems that do not take the fused path.
+ */
+SSD_API int ssd_fwd_withhold_publish(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                                     const float *D, int Q, const float *init_state, void *y, float *final_state,
+                                     int batch, int T, int H, int P, int G, int N, int dtype, void *workspace,
+                                     size_t workspace_bytes, void *stream, int withhold_b, int withhold_h,
+                                     int withhold_c, unsigned flag_polls);
+
+/*
  * ssd_fwd for callers that cannot allocate device memory when they run the
  * layer (an engine that fixes every buffer before serving, a framework whose
  * allocator owns the device, a loop that must never reach cudaMalloc).  The
@@ -154,6 +172,15 @@ SSD_API int ssd_fwd_check(const void *workspace, void *stream);
 SSD_API int ssd_fwd_no_alloc(const void *x, const float *dt, const float *A, const void *B, const void *C,
                      const float *D, int Q, const float *init_state, void *y, float *final_state,
                      int batch, int T, int H, int P, int G, int N, int dtype, void *stream);
+
+/*
+ * ssd_fwd_check for ssd_fwd_no_alloc, whose callers hold no workspace
+ * pointer: waits for `stream`, then reads the status word the last
+ * ssd_fwd_no_alloc on the current device left in the library's scratch
+ * (SSD_OK or SSD_ERR_TIMEOUT).  Returns SSD_ERR_CUDA if the wait or the copy
+ * fails.  Allocates nothing.
+ */
+SSD_API int ssd_fwd_no_alloc_check(void *stream);
 
 /*
  * One autoregressive (decode) step of the same recurrence, in place: for

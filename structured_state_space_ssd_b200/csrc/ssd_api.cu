@@ -16,10 +16,10 @@ template <typename T>
 cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D, const float *s,
                               const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
 bool fused_supported(const Shape &sh, int dtype);
-cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, const __nv_bfloat16 *C,
-                             const float *D, const float *s, const float *init, float *fin, float *ring, int *ready,
-                             int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
-                             cudaStream_t st);
+cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
+                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
+                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
+                             const FusedDebug *dbg, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -67,14 +67,15 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 }
 
 const char *const kSimtStages[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan"};
-const char *const kFusedStages[] = {"ssd_chunk_cumsum", "ssd_fused"};
+const char *const kFusedStages[] = {"ssd_fused"};
 
 int launch_count(const Shape &sh, ssd::Path path) {
     if (sh.T == 0) return 0;
-    return path == ssd::kPathFused ? 2 : 4;
+    return path == ssd::kPathFused ? 1 : 4;
 }
 
-// Optional per-kernel event marks: ev[0] before the first kernel, ev[k+1] after kernel k.
+// Optional event marks: ev[0] at the start of the call (before the workspace
+// clear), ev[1] before the first kernel, ev[k+2] after kernel k.
 struct Marks {
     cudaEvent_t *ev = nullptr;
     int n = 0;
@@ -87,26 +88,24 @@ int run_simt(const Shape &sh, const T *x, const float *dt, const float *A, const
              const Marks &mk) {
     float *s = reinterpret_cast<float *>(ws + w.s_off);
     float *S = reinterpret_cast<float *>(ws + w.state_off);
-    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(1, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st, false) != cudaSuccess || !mk.mark(2, st))
+    if (!mk.mark(1, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(2, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_state<T>(x, B, s, S, sh, st, false) != cudaSuccess || !mk.mark(3, st))
         return SSD_ERR_CUDA;
-    if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || !mk.mark(3, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || !mk.mark(4, st))
+    if (ssd::launch_state_passing(S, s, init, fin, sh, st) != cudaSuccess || !mk.mark(4, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_chunk_scan<T>(x, B, C, D, s, S, y, sh, st) != cudaSuccess || !mk.mark(5, st))
         return SSD_ERR_CUDA;
     return SSD_OK;
 }
 
 int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
               const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
-              const ssd::Workspace &w, cudaStream_t st, const Marks &mk) {
-    float *s = reinterpret_cast<float *>(ws + w.s_off);
-    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess || !mk.mark(1, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_ssd_fused(x, B, C, D, s, init, fin, reinterpret_cast<float *>(ws + w.ring_off),
+              const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg) {
+    if (!mk.mark(1, st)) return SSD_ERR_CUDA;
+    if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, reinterpret_cast<float *>(ws + w.ring_off),
                               reinterpret_cast<int *>(ws + w.ready_off), reinterpret_cast<int *>(ws + w.cons_off),
                               reinterpret_cast<int *>(ws + w.counter_off), reinterpret_cast<int *>(ws + w.status_off),
-                              y, sh, st) != cudaSuccess ||
+                              y, sh, dbg, st) != cudaSuccess ||
         !mk.mark(2, st))
         return SSD_ERR_CUDA;
     return SSD_OK;
@@ -114,7 +113,8 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
 
 int fwd_impl(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
              const float *init_state, void *y, float *final_state, int batch, int T, int H, int P, int G, int N,
-             int dtype, void *workspace, size_t workspace_bytes, void *stream, const Marks &mk) {
+             int dtype, void *workspace, size_t workspace_bytes, void *stream, const Marks &mk,
+             const ssd::FusedDebug *dbg = nullptr) {
     Shape sh;
     int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
     if (rc != SSD_OK) return rc;
@@ -135,11 +135,13 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
                    overlaps(y, ybytes, C, bcbytes)))
         return SSD_ERR_INVALID_ARG;
 
+    if (dbg && path != ssd::kPathFused) return SSD_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
+    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
     if (cudaMemsetAsync(ws, 0, w.clear_bytes, st) != cudaSuccess) return SSD_ERR_CUDA;
     if (T == 0) {
-        if (!mk.mark(0, st)) return SSD_ERR_CUDA;
+        if (!mk.mark(1, st)) return SSD_ERR_CUDA;
         if (!final_state) return SSD_OK;
         const size_t fb = sizeof(float) * (size_t)batch * H * P * N;
         cudaError_t e = init_state ? cudaMemcpyAsync(final_state, init_state, fb, cudaMemcpyDeviceToDevice, st)
@@ -149,7 +151,7 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     if (path == ssd::kPathFused)
         return run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
                          static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
-                         final_state, ws, w, st, mk);
+                         final_state, ws, w, st, mk, dbg);
     if (dtype == SSD_BF16)
         return run_simt<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
                                        static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C),
@@ -194,34 +196,54 @@ int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B,
                   int Q, const float *init_state, void *y, float *final_state, int batch, int T, int H, int P,
                   int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream, float *stage_ms,
                   int max_stages, float *total_ms) {
-    thread_local cudaEvent_t events[kMaxStages + 1];
-    thread_local int events_device = -1;
+    // One set of events per device, created on that device the first time this
+    // host thread times a call there, kept until the process exits.
+    constexpr int kMaxDevices = 64;
+    thread_local cudaEvent_t events[kMaxDevices][kMaxStages + 2];
+    thread_local bool created[kMaxDevices] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
-    if (events_device != dev) {
-        for (int i = 0; i <= kMaxStages; ++i)
-            if (cudaEventCreate(&events[i]) != cudaSuccess) return SSD_ERR_CUDA;
-        events_device = dev;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSD_ERR_CUDA;
+    if (!created[dev]) {
+        for (int i = 0; i < kMaxStages + 2; ++i)
+            if (cudaEventCreate(&events[dev][i]) != cudaSuccess) return SSD_ERR_CUDA;
+        created[dev] = true;
     }
     Shape sh;
     int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
     if (rc != SSD_OK) return rc;
     const int k = launch_count(sh, choose_path(sh, dtype));
     Marks mk;
-    mk.ev = events;
-    mk.n = k + 1;
+    mk.ev = events[dev];
+    mk.n = k + 2;
     rc = fwd_impl(x, dt, A, B, C, D, Q, init_state, y, final_state, batch, T, H, P, G, N, dtype, workspace,
                   workspace_bytes, stream, mk);
     if (rc != SSD_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
     for (int i = 0; i < k && i < max_stages && stage_ms; ++i)
-        if (cudaEventElapsedTime(&stage_ms[i], events[i], events[i + 1]) != cudaSuccess) return SSD_ERR_CUDA;
+        if (cudaEventElapsedTime(&stage_ms[i], events[dev][i + 1], events[dev][i + 2]) != cudaSuccess)
+            return SSD_ERR_CUDA;
     if (total_ms) {
         *total_ms = 0.f;
-        if (k > 0 && cudaEventElapsedTime(total_ms, events[0], events[k]) != cudaSuccess) return SSD_ERR_CUDA;
+        if (k > 0 && cudaEventElapsedTime(total_ms, events[dev][0], events[dev][k + 1]) != cudaSuccess)
+            return SSD_ERR_CUDA;
     }
     return SSD_OK;
+}
+
+int ssd_fwd_withhold_publish(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                             const float *D, int Q, const float *init_state, void *y, float *final_state, int batch,
+                             int T, int H, int P, int G, int N, int dtype, void *workspace, size_t workspace_bytes,
+                             void *stream, int withhold_b, int withhold_h, int withhold_c, unsigned flag_polls) {
+    if (withhold_b < 0 || withhold_b >= batch || withhold_h < 0 || withhold_h >= H || withhold_c < 0 ||
+        flag_polls == 0)
+        return SSD_ERR_INVALID_ARG;
+    ssd::FusedDebug dbg;
+    dbg.flag_polls = flag_polls;
+    dbg.withhold_bh = withhold_b * H + withhold_h;
+    dbg.withhold_c = withhold_c;
+    return fwd_impl(x, dt, A, B, C, D, Q, init_state, y, final_state, batch, T, H, P, G, N, dtype, workspace,
+                    workspace_bytes, stream, Marks{}, &dbg);
 }
 
 int ssd_fwd_check(const void *workspace, void *stream) {

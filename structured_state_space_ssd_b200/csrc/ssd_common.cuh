@@ -89,8 +89,18 @@ struct Shape {
 
 // The two launch sequences: stage-per-kernel on CUDA cores (any shape and
 // dtype within the limits) or the fused tensor-core kernel (bf16, P = 64,
-// N in {64, 128}, Q in {128, 256}).
+// N a multiple of 16 up to 128, Q in {128, 256}).
 enum Path { kPathSimt = 0, kPathFused = 1 };
+
+// Test hooks of the fused kernel's hand-off (ssd_fwd_withhold_publish):
+// each wait on another CTA's flag gives up after flag_polls polls (0: the
+// default bound), and the owner of chunk withhold_c of sequence withhold_bh
+// (batch * H + head) never publishes its state (-1: every owner publishes).
+struct FusedDebug {
+    unsigned flag_polls;
+    int withhold_bh;
+    int withhold_c;
+};
 
 // Workspace carve-up, computed identically by ssd_fwd_workspace_bytes and ssd_fwd.
 // The front 256-byte block holds the status word and the unit counter; it and
@@ -99,11 +109,11 @@ struct Workspace {
     size_t status_off;  // int status word
     size_t counter_off; // int unit counter (fused path)
     size_t ready_off;   // int ready[batch * H] (fused path)
-    size_t cons_off;    // int cons[batch * H] (fused path)
+    size_t cons_off;    // int cons[batch * H][2] (fused path)
     size_t clear_bytes; // bytes from offset 0 cleared per call
-    size_t s_off;       // float s[batch][H][nc][Q]: inclusive log-decay prefix sums per chunk
+    size_t s_off;       // CUDA-core path: float s[batch][H][nc][Q], inclusive log-decay prefix sums per chunk
     size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
-    size_t ring_off;    // fused path: float ring[batch][H][2][P][N], outgoing states of the last two chunks
+    size_t ring_off;    // fused path: float ring[batch][H][2][N][P], outgoing states of the last two chunks
     size_t total;
 };
 
@@ -126,11 +136,11 @@ inline Workspace workspace_layout(const Shape &s, Path path) {
     w.ready_off = off;
     off += sizeof(int) * bh;
     w.cons_off = off;
-    off += sizeof(int) * bh;
+    off += sizeof(int) * bh * 2;
     off = align256(off);
     w.clear_bytes = (path == kPathFused) ? off : 256;
     w.s_off = off;
-    off = align256(off + sizeof(float) * bh * s.nc * s.Q);
+    if (path != kPathFused) off = align256(off + sizeof(float) * bh * s.nc * s.Q);
     w.state_off = w.ring_off = off;
     if (path == kPathFused)
         off = align256(off + sizeof(float) * bh * 2 * s.P * s.N);

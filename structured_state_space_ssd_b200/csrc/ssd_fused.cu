@@ -1,81 +1,51 @@
 // ssd_fused.cu -- the bf16 SSD forward as one persistent tensor-core kernel.
 //
 // "Transformers are SSMs" (analysis page, section "The Block-Decomposition SSD
-// Algorithm") computes the layer in stages: the quadratic masked form inside
-// each chunk of Q tokens (stage 1), chunk-final states (stage 2), the scalar
-// recurrence of those states across chunks (stage 3), the inter-chunk output
-// (stage 4) and the sum (stage 5).  This kernel runs stages 1-5 for every
-// chunk, every head and both 128-row halves of a chunk without sending the
-// fp32 chunk states through HBM:
+// Algorithm") computes the layer in stages: chunk prefix sums of the
+// log-decay (stage 0), the quadratic masked form inside each chunk of Q
+// tokens (stage 1), chunk-final states (stage 2), the scalar recurrence of
+// those states across chunks (stage 3), the inter-chunk output (stage 4) and
+// the sum (stage 5).  This kernel runs every stage in one launch; nothing but
+// the chained fp32 states (an L2-resident ring) leaves the SM.
 //
-//  * A work unit is (chunk c, batch b, group g, block of heads, half r).
+// Blocks of 128 rows.  A chunk of Q = 256 tokens is two blocks, and the
+// second block reaches the first through the state at the chunk's midpoint
+// instead of through the off-diagonal block of the quadratic form: the same
+// block decomposition applied once more inside the chunk, so the function is
+// unchanged and only the diagonal 128 x 128 blocks of the semiseparable
+// matrix are ever formed.  With s the inclusive prefix sum of dt*A from the
+// chunk start, r the block's first row (s_{-1} = 0) and x~_i the rows
+// scaled by a decay:
+//
+//   entering state  E   = exp(s_{r-1}) S~_{c-1} + B_{<r}^T (exp(s_{r-1} - s_i) x_i)
+//   output          y_j = exp(s_j - s_{r-1}) C_j E^T
+//                         + sum_{r <= i <= j} exp(s_j - s_i) (C_j . B_i) x_i + D_h x_j
+//   chunk state     S~_c = exp(s_end - s_{r-1}) E + B_{>=r}^T (exp(s_end - s_i) x_i)   (last block)
+//
+//  * A work unit is (chunk c, batch b, group g, block of heads, block r).
 //    Units are handed out by an atomic counter in chunk-major order, so a
-//    unit only ever waits for units handed out before it (which are running
-//    or done): there is no deadlock however many CTAs are resident.
-//  * First-half units (rows 0..127) own the chunk state: per head they form
-//    S_c = B_c^T (exp(s_end - s_i) x_i) on the tensor cores (stage 2), wait
-//    for the state S~_{c-1} entering the chunk (published by the first-half
-//    unit of chunk c-1), publish S~_c = exp(s_end) S~_{c-1} + S_c (stage 3)
-//    into a two-slot fp32 ring that stays in L2, and write final_state for
-//    the last chunk.
-//  * Every unit then produces its 128 output rows per head: G = C_r B^T once
-//    per unit into TMEM, Y = exp(s_j) C_r S~_{c-1}^T (stage 4), the causal
-//    decay mask M = G o exp(s_j - s_i) (+ D_h on the diagonal) written by the
-//    CUDA cores into TMEM as the bf16 A operand, Y += M X (stage 1), y = bf16(Y)
-//    (stage 5).
-//  * Second-half units read S~_{c-1} from the ring and count themselves as
-//    done with it; a first-half unit overwrites a slot only after every
-//    second half up to the previous chunk has read (a count, since second
-//    halves of different chunks finish in any order).  Every wait is
-//    bounded: on expiry the status word is set to SSD_ERR_TIMEOUT and the
-//    CTA finishes without waiting.
+//    unit only ever waits for units handed out before it: there is no
+//    deadlock however many CTAs are resident.
+//  * The last block of a chunk owns the chunk state: it waits for S~_{c-1}
+//    (published by the owner of chunk c-1), forms E and S~_c, and writes
+//    S~_c into a two-slot fp32 ring (or final_state after the last chunk).
+//    Other blocks only read S~_{c-1} and count themselves as done with it;
+//    an owner overwrites a slot only after every reader of the chunk before
+//    has read it.  Every wait on another CTA is bounded: on expiry the
+//    status word is set to SSD_ERR_TIMEOUT and the waits that follow give up
+//    at once (the CTA's own barriers are still waited for, so nothing it
+//    issued is in flight when it exits).
 //
-// Warp roles: each CTA runs two head pipelines side by side; pipeline pl
-// takes every other head of a unit (units hold up to 4 heads).  Its eight
-// CUDA-core warps (warps 8pl..8pl+7: two warpgroups, each covering the 128
-// TMEM lanes and half of every tile's columns), its issuer warp (16 + pl;
-// one lane issues TMA loads and tcgen05.mma) and its publisher warp (18 + pl;
-// the GPU-scope fences and flags of the state hand-off) pass the pipeline's
-// own X tile, state tile, decay mask (one 128-token K-half at a time) and
-// accumulators back and forth through mbarriers, so that one pipeline's
-// CUDA-core work overlaps the other's tensor-core products.  C, B and G are
-// shared by the unit's heads.
+// Warp roles: two head pipelines per CTA, pipeline pl taking every other head
+// of a unit.  Its eight CUDA-core warps (two warpgroups over the 128 TMEM
+// lanes) form the prefix sums, scale x, build the decay mask, move the states
+// and drain the accumulators; its issuer warp (16 + pl) loads x with TMA and
+// issues tcgen05.mma; its publisher warp (18 + pl) makes the state hand-offs
+// visible to other CTAs.  C, B and G = C B^T (the block's 128 x 128) are shared
+// by the unit's heads.
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
-
-// Optional phase timestamps for performance work: compiled in only with
-// -DSSD_TRACE, which also provides ssd_trace_buffer (one 32-slot record per
-// head and pipeline).  Production builds contain no trace code.
-#ifdef SSD_TRACE
-__device__ unsigned long long *ssd_trace_buffer = nullptr;
-#define SSD_TRACE_POINT(ev)                                                                                    \
-    do {                                                                                                       \
-        if (ssd_trace_buffer && wtid == 0 && trace_i < 30) {                                                   \
-            unsigned long long t_;                                                                             \
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                           \
-            ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 32 + (ev)] = t_;               \
-        }                                                                                                      \
-    } while (0)
-#else
-#define SSD_TRACE_POINT(ev) \
-    do {                    \
-    } while (0)
-#endif
-#ifdef SSD_TRACE
-// waits until the values v[0..n) have arrived, then records event ev
-#define SSD_TRACE_ARRIVED(v, n, ev)                              \
-    do {                                                         \
-        float acc_ = 0.f;                                        \
-        for (int i_ = 0; i_ < (n); ++i_) acc_ += (v)[i_];        \
-        if (acc_ == -1.2345e-30f) ssd_trace_buffer[0] = 1;       \
-        SSD_TRACE_POINT(ev);                                     \
-    } while (0)
-#else
-#define SSD_TRACE_ARRIVED(v, n, ev) \
-    do {                            \
-    } while (0)
-#endif
 
 namespace ssd {
 
@@ -83,68 +53,70 @@ using namespace tc;
 
 namespace fz {
 
-constexpr int kWgThreads = 128;                  // one warpgroup: the 128 TMEM lanes
-constexpr int kPipeThreads = 2 * kWgThreads;     // two warpgroups per head pipeline, each half the columns
-constexpr int kSimtWarps = 2 * kPipeThreads / 32;  // warps 0-15: CUDA-core work of pipelines 0 and 1
-constexpr int kThreads = 2 * kPipeThreads + 128;  // + warps 16-17: issuers, 18-19: publishers
-constexpr int kRows = 128;
-constexpr int kP = 64;
+constexpr int kRows = 128;                         // rows of a block: one TMEM lane each
+constexpr int kP = 64;                             // head dimension of this path
+constexpr int kPipeThreads = 256;                  // two warpgroups per head pipeline
+constexpr int kPipeWarps = kPipeThreads / 32;
+constexpr int kSimtWarps = 2 * kPipeWarps;         // warps 0-15: CUDA-core work of pipelines 0 and 1
+constexpr int kThreads = 32 * kSimtWarps + 128;    // + warps 16-17: issuers, 18-19: publishers
+constexpr float kLog2e = 1.4426950408889634f;
 
-// TMEM columns (512 allocated).  Pipeline pl owns D[pl], M[pl] and Y[pl].
+// TMEM columns (512 allocated).  G is the unit's C B^T block (fp32).  Per
+// pipeline: accumulator A holds the pre-block state, then the inter-chunk
+// product; accumulator B holds the block's own state contribution, then the
+// masked product; M holds the bf16 decay mask (the A operand of M X).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColG = 0;    // G: 128 (first half) or 256 (second half) fp32 columns
-constexpr uint32_t kColD = 128;  // first half only: chunk-state accumulators, 64 columns per pipeline
-constexpr uint32_t kColM = 256;  // decay mask (one 128-token K-half, bf16 pairs), 64 columns per pipeline
-constexpr uint32_t kColY = 384;  // output accumulators, 64 columns per pipeline
+constexpr uint32_t kColG = 0;
+__device__ __forceinline__ uint32_t col_acc_a(int pl) { return 128u + 192u * pl; }
+__device__ __forceinline__ uint32_t col_acc_b(int pl) { return 192u + 192u * pl; }
+__device__ __forceinline__ uint32_t col_mask(int pl) { return 256u + 192u * pl; }
 
-// Shared memory (bytes from a 1 KiB-aligned base)
-constexpr uint32_t kOffC = 0;                  // C rows of the half: 2 K-atoms x 128 rows x 128 B
-constexpr uint32_t kOffB = 32768;              // B rows 0..Q-1: 2 K-atoms x 256 rows x 128 B
-constexpr uint32_t kOffX = kOffB + 65536;      // per pipeline: X rows 0..Q-1, 256 rows x 128 B
-constexpr uint32_t kOffS = kOffX + 2 * 32768;  // per pipeline: S~ tile (2 atoms x 64 rows x 128 B), or
-                                               // the decayed X rows 0..127 before the chunk-state product
-constexpr uint32_t kOffJ = kOffS + 2 * 16384;  // per pipeline, 2 buffers: s values (256 floats)
-constexpr uint32_t kOffF = kOffJ + 4 * 1024;   // per pipeline, 2 buffers: column factors (256 floats)
-constexpr uint32_t kSmemBytes = kOffF + 4 * 1024 + 1024;
+// Shared memory, from a 1 KiB-aligned base.  Tiles are bf16 rows of 128 bytes
+// in the 128-byte-swizzled layout TMA writes (8-row atoms of 1 KiB).
+constexpr uint32_t kOffC = 0;           // C rows of the block: NK atoms x 128 rows
+constexpr uint32_t kOffB = 32768;       // B rows 0..Q-1: 2 atoms of 256 rows (atom stride 32 KiB)
+constexpr uint32_t kOffPipe = 98304;    // per pipeline: x rows 0..127 | W | x rows 128..255, 16 KiB each
+constexpr uint32_t kPipeBytes = 49152;  // W: scaled x rows, then the entering-state tile [n][p]
+constexpr uint32_t kOffAux = kOffPipe + 2 * kPipeBytes;
+constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units), column factors, warp totals
+constexpr uint32_t kSmemBytes = kOffAux + 2 * kAuxFloats * 4 + 1024;
 
-constexpr uint32_t kFlagPolls = 1u << 22;
+constexpr uint32_t kDefaultFlagPolls = 1u << 22;
 
 struct Params {
     Shape sh;
-    const float *s;     // [b][H][nc][Q] per-chunk inclusive prefix sums of dt*A
+    const float *dt;    // [b][T][H]
+    const float *A;     // [H]
     const float *D;     // [H]
     const float *init;  // [b][H][P][N] or null
     float *fin;         // [b][H][P][N] or null
-    float *ring;        // [b][H][2][P][N]
+    float *ring;        // [b][H][2][P/4][N][4]: outgoing states of the last two chunks (see ring_quad)
     int *ready;         // [b*H]: chunks whose outgoing state is published
-    int *cons;          // [b*H]: second halves that have read their entering state (a count: second
-                        // halves of different chunks finish in any order)
+    int *cons;          // [b*H][2]: per ring slot, non-owner blocks that have read it (a count)
     int *counter;       // unit dispenser
     int *status;
     __nv_bfloat16 *y;
-    int NK;             // 64-wide K-atoms along N (C and the S~ tile)
+    int NK;             // 64-wide K-atoms along N
     int halves;         // Q / 128
     int heads_per_unit;
     int blocks_per_group;
     int n_units;
+    uint32_t flag_polls;  // bound of each wait on another CTA's flag
+    int withhold_bh;      // test hook: the owner of (b*H + h, chunk) below never publishes (-1: none)
+    int withhold_c;
 };
 
-// One head pipeline: its issuer warp and its warpgroup.  Barriers signalled
-// once per head of the pipeline are waited with parity (use & 1), `use`
-// counting the pipeline's earlier heads; both sides keep identical counters.
+// One head pipeline.  Barriers signalled once per head of the pipeline are
+// waited with parity (count & 1); both sides keep identical counters.
 struct PipeBars {
-    uint64_t x_full;      // X tile landed (TMA)
-    uint64_t x_free;      // products reading the X tile done
-    uint64_t j_full[2];   // s values landed (bulk copy), double-buffered
-    uint64_t xd_full;     // first half: decayed X written (4 warp arrivals)
-    uint64_t d_done;      // first half: chunk-state product done
-    uint64_t s_full;      // S~ tile written (4 warp arrivals)
-    uint64_t inter_done;  // inter-chunk product done
-    uint64_t m_full;      // one mask K-half written (4 warp arrivals)
-    uint64_t m_free;      // product reading it done
-    uint64_t mx_done;     // every product of the head done
-    uint64_t y_free;      // output accumulator drained (4 warp arrivals)
-    uint64_t ring_done;   // ring stores issued (first half) / ring loads consumed (second half)
+    uint64_t x_full;     // x rows landed (TMA)
+    uint64_t xd_full;    // owner: scaled x rows written (8 warp arrivals)
+    uint64_t d_done;     // owner: state products done
+    uint64_t m_full;     // decay mask written (8 warp arrivals)
+    uint64_t s_full;     // entering-state tile written, state accumulators read (8 warp arrivals)
+    uint64_t mx_done;    // every product of the head done
+    uint64_t acc_free;   // accumulators drained (8 warp arrivals)
+    uint64_t ring_done;  // ring stores issued (owner) / ring loads consumed (others), for the publisher
 };
 
 struct Bars {
@@ -152,12 +124,14 @@ struct Bars {
     uint64_t g_done;      // G = C B^T in TMEM
     uint64_t unit_full;   // unit id posted (issuer 0)
     uint64_t unit_empty;  // unit id read (16 CUDA-core warps, issuer 1, 2 publishers)
-    uint64_t unit_done;   // both pipelines finished the unit (2 issuer arrivals)
+    uint64_t unit_done;   // both pipelines finished the unit's products (2 issuer arrivals)
     PipeBars pb[2];
 };
 
 struct Unit {
     int b, c, g, h0, h1, r, t0, len, row0;
+    bool rows;   // the block has rows (the last chunk may be short)
+    bool owner;  // the chunk's last block with rows: it carries the chunk state
 };
 
 __device__ __forceinline__ Unit decode(int u, const Params &p) {
@@ -176,6 +150,8 @@ __device__ __forceinline__ Unit decode(int u, const Params &p) {
     un.t0 = un.c * p.sh.Q;
     un.len = min(p.sh.Q, p.sh.T - un.t0);
     un.row0 = un.r * kRows;
+    un.rows = un.row0 < un.len;
+    un.owner = un.rows && un.r == ((un.len - 1) >> 7);
     return un;
 }
 
@@ -183,39 +159,78 @@ __device__ __forceinline__ uint8_t *align_1k(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Bounded mbarrier wait that gives up at once after any wait in the CTA failed.
-// Each poll parks the warp for up to kSuspendNs, so the bound is about
-// kWaitPolls * kSuspendNs (~2 s) of waiting, after which the status word
-// records SSD_ERR_TIMEOUT.
-constexpr uint32_t kSuspendNs = 100000;
-constexpr uint32_t kWaitPolls = 20000;
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int *status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
-        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
-        if (*abort) return false;
+// Wait on one of the CTA's own mbarriers.  Its producers are this CTA's own
+// warps, TMA and tensor cores, which always finish, so the wait is never cut
+// short by a timeout on another CTA's flag.  The bound (about 2 s) only turns
+// a defect of the kernel itself into a status instead of a hang; once one such
+// wait has expired (`broken`), the CTA's later waits give up after about 1 ms
+// so that the kernel still ends in bounded time.
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kBrokenWaitNs = 1000000ull;
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void wait_bar(uint64_t *bar, uint32_t parity, int *status, volatile int *broken) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_ns(), limit = *broken ? kBrokenWaitNs : kWaitNs;
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return;
+        if (global_ns() - t0 > limit) break;
     }
     atomicExch(status, SSD_ERR_TIMEOUT);
-    *abort = 1;
-    return false;
+    *broken = 1;
 }
 
-// Bounded wait for a GPU-scope counter to reach `target` (acquire).
-__device__ __forceinline__ bool wait_flag(const int *flag, int target, volatile int *abort, int *status) {
-    for (uint32_t i = 0; i < kFlagPolls; ++i) {
-        if (ld_acquire_gpu(flag) >= target) return true;
-        if (*abort || ld_relaxed_gpu(status) != 0) {
+// Bounded wait for another CTA's counter to reach `target` (acquire).  Gives
+// up at once when a wait anywhere has already given up.
+__device__ __forceinline__ void wait_flag(const int *flag, int target, uint32_t polls, volatile int *abort,
+                                          int *status) {
+    if (*abort) return;
+    for (uint32_t i = 0; i < polls; ++i) {
+        if (ld_acquire_gpu(flag) >= target) return;
+        if (ld_relaxed_gpu(status) != 0) {
             *abort = 1;
-            return false;
+            return;
         }
         __nanosleep(64);
     }
     atomicExch(status, SSD_ERR_TIMEOUT);
     *abort = 1;
-    return false;
 }
 
-__device__ __forceinline__ uint32_t par_of(uint32_t use) { return use & 1u; }
+__device__ __forceinline__ uint32_t par(uint32_t n) { return n & 1u; }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ void sts128(uint8_t *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
+}
+
+// The fp32 chunk states in the ring are stored in quads of p: entry (n, p) of
+// a slot sits at float4 index (p / 4) * N + n, component p % 4.  A warp's 32
+// lanes (32 consecutive n, one TMEM lane each) then move 512 contiguous bytes
+// per 16-byte access.
+__device__ __forceinline__ size_t ring_quad(int N, int n, int quad) { return (size_t)quad * N + n; }
+
+// Eight bf16 scaled by w (fp32 products, one rounding to bf16).
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
+    const float2 ww = make_float2(w, w);
+    uint4 o;
+    float2 a;
+    a = mul_f32x2(make_float2(bf16lo(v.x), bf16hi(v.x)), ww);
+    o.x = pack_bf16x2(a.x, a.y);
+    a = mul_f32x2(make_float2(bf16lo(v.y), bf16hi(v.y)), ww);
+    o.y = pack_bf16x2(a.x, a.y);
+    a = mul_f32x2(make_float2(bf16lo(v.z), bf16hi(v.z)), ww);
+    o.z = pack_bf16x2(a.x, a.y);
+    a = mul_f32x2(make_float2(bf16lo(v.w), bf16hi(v.w)), ww);
+    o.w = pack_bf16x2(a.x, a.y);
+    return o;
+}
 
 }  // namespace fz
 
@@ -232,27 +247,29 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     __shared__ Bars bars;
     __shared__ uint32_t tslot;
     __shared__ int s_unit;
-    __shared__ int s_abort;
+    __shared__ int s_abort, s_broken;
     volatile int *abort = &s_abort;
+    volatile int *broken = &s_broken;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const Shape sh = p.sh;
-    const int Q = sh.Q, N = sh.N, NK = p.NK;
+    const int N = sh.N, NK = p.NK;
 
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     if (tid == 0) {
         s_abort = 0;
+        s_broken = 0;
         uint64_t *all = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(Bars) / 8); ++i) mbar_init(&all[i], 1);
         mbar_init(&bars.unit_empty, kSimtWarps + 3);
         mbar_init(&bars.unit_done, 2);
         for (int q = 0; q < 2; ++q) {
-            mbar_init(&bars.pb[q].xd_full, kPipeThreads / 32);
-            mbar_init(&bars.pb[q].s_full, kPipeThreads / 32);
-            mbar_init(&bars.pb[q].m_full, kPipeThreads / 32);
-            mbar_init(&bars.pb[q].y_free, kPipeThreads / 32);
-            mbar_init(&bars.pb[q].ring_done, kPipeThreads / 32);
+            mbar_init(&bars.pb[q].xd_full, kPipeWarps);
+            mbar_init(&bars.pb[q].m_full, kPipeWarps);
+            mbar_init(&bars.pb[q].s_full, kPipeWarps);
+            mbar_init(&bars.pb[q].acc_free, kPipeWarps);
+            mbar_init(&bars.pb[q].ring_done, kPipeWarps);
         }
         mbar_fence_init();
     }
@@ -263,36 +280,37 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 
     if (warp >= kSimtWarps + 2) {
         // ------------------------------------------------------------------
-        // Publisher warps: warp 18 + pl makes pipeline pl's chain hand-offs
-        // visible, so that neither the CUDA-core warps nor the issuer wait
-        // for a GPU-scope release.  After a first half's ring stores it
-        // releases `ready` (S~_c readable); after a second half consumed
-        // S~_{c-1} it adds one to `cons` (the ring slot may be rewritten).
-        // The warps' arrival on ring_done (a CTA-scope release, acquired by
-        // this thread's wait) puts their accesses before this thread's
-        // GPU-scope release, which carries them along (release is cumulative).
+        // Publisher warps: warp 18 + pl makes pipeline pl's hand-offs visible
+        // to other CTAs, so that neither the CUDA-core warps nor the issuer
+        // wait for a GPU-scope release.  After an owner's ring stores it
+        // releases `ready` (S~_c readable); after another block read S~_{c-1}
+        // it adds one to `cons` (the slot may be rewritten).  The warps'
+        // arrival on ring_done (a CTA-scope release, acquired by this
+        // thread's wait) puts their accesses before this thread's GPU-scope
+        // release, which carries them along (release is cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
         PipeBars &pb = bars.pb[pl];
         uint32_t ucnt = 0, rcnt = 0;
         for (;;) {
-            wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
+            wait_bar(&bars.unit_full, par(ucnt), p.status, broken);
             ++ucnt;
             const int u = s_unit;
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.unit_empty);
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
-            if (un.row0 >= un.len) continue;
-            const bool first = (un.r == 0);
+            if (!un.rows) continue;
             for (int h = un.h0 + pl; h < un.h1; h += 2, ++rcnt) {
-                wait_bar(&pb.ring_done, par_of(rcnt), abort, p.status);
+                wait_bar(&pb.ring_done, par(rcnt), p.status, broken);
                 if (lane == 0) {
-                    const size_t bh = (size_t)un.b * sh.H + h;
-                    if (first) {
-                        if (un.c < sh.nc - 1) st_release_gpu(p.ready + bh, un.c + 1);
-                    } else {
-                        red_release_add_gpu(p.cons + bh, 1);
+                    const int bh = un.b * sh.H + h;
+                    if (un.owner) {
+                        const bool withheld = (bh == p.withhold_bh && un.c == p.withhold_c);
+                        if (un.c < sh.nc - 1 && !withheld) st_release_gpu(p.ready + bh, un.c + 1);
+                    } else if (un.c > 0) {
+                        // chunk c read slot (c-1) & 1 (chunk 0 read the initial state)
+                        red_release_add_gpu(p.cons + 2 * bh + ((un.c - 1) & 1), 1);
                     }
                 }
                 __syncwarp();
@@ -301,39 +319,40 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     } else if (warp >= kSimtWarps) {
         // ------------------------------------------------------------------
         // Issuer warps: warp 16 drives pipeline 0 and also hands out units,
-        // loads C/B and forms G; warp 17 drives pipeline 1.  The whole warp
-        // follows the control flow and waits; lane 0 alone issues.
+        // loads C and B and forms G; warp 17 drives pipeline 1.  The whole
+        // warp follows the control flow and waits; lane 0 alone issues.
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps;
         const bool leader = (lane == 0);
         PipeBars &pb = bars.pb[pl];
-        uint8_t *sXp = smem + kOffX + pl * 32768;
-        uint8_t *sSp = smem + kOffS + pl * 16384;
-        float *sJp = reinterpret_cast<float *>(smem + kOffJ) + pl * 512;
-        const uint32_t tY = tmem + kColY + pl * 64, tM = tmem + kColM + pl * 64, tD = tmem + kColD + pl * 64;
+        uint8_t *sXlo = smem + kOffPipe + pl * kPipeBytes;
+        uint8_t *sW = sXlo + 16384;
+        uint8_t *sXhi = sXlo + 32768;
+        const uint32_t tA = tmem + col_acc_a(pl), tB = tmem + col_acc_b(pl), tM = tmem + col_mask(pl);
         if (leader && pl == 0) {
             tma_prefetch_desc(&mC);
             tma_prefetch_desc(&mB);
             tma_prefetch_desc(&mX);
+            tma_prefetch_desc(&mY);
         }
-        uint32_t use = 0, r0use = 0, mcnt = 0, ucnt = 0, cbcnt = 0, units_done = 0;
-        const uint32_t idG0 = idesc_bf16_f32(kRows, kRows, 0, 0);
-        const uint32_t idG1 = idesc_bf16_f32(kRows, 2 * kRows, 0, 0);
-        const uint32_t idInter = idesc_bf16_f32(kRows, kP, 0, 0);
-        const uint32_t idState = idesc_bf16_f32(kRows, kP, 1, 1);
-        const uint32_t idMX = idesc_bf16_f32(kRows, kP, 0, 1);
+        const uint32_t idG = idesc_bf16_f32(kRows, kRows, 0, 0);    // C (K-major) x B (K-major)
+        const uint32_t idState = idesc_bf16_f32(kRows, kP, 1, 1);   // B^T (MN-major) x scaled x (MN-major)
+        const uint32_t idInter = idesc_bf16_f32(kRows, kP, 0, 1);   // C (K-major) x state tile [n][p]
+        const uint32_t idMX = idesc_bf16_f32(kRows, kP, 0, 1);      // mask (TMEM) x x rows [i][p]
+        uint32_t use = 0, ocnt = 0, ucnt = 0, cbcnt = 0, udone = 0;
+        int next_u = -1;
         for (;;) {
             int u = 0;
             if (pl == 0) {
-                if (ucnt > 0) wait_bar(&bars.unit_empty, par_of(ucnt - 1), abort, p.status);
+                if (ucnt > 0) wait_bar(&bars.unit_empty, par(ucnt - 1), p.status, broken);
                 if (leader) {
-                    u = atomicAdd(p.counter, 1);
+                    u = (next_u >= 0) ? next_u : atomicAdd(p.counter, 1);
                     s_unit = u;
                     mbar_arrive(&bars.unit_full);
                 }
                 u = __shfl_sync(0xffffffffu, u, 0);
             } else {
-                wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
+                wait_bar(&bars.unit_full, par(ucnt), p.status, broken);
                 u = s_unit;
                 __syncwarp();
                 if (leader) mbar_arrive(&bars.unit_empty);
@@ -341,440 +360,438 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             ++ucnt;
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
-            if (un.row0 >= un.len) continue;
-            const bool first = (un.r == 0);
-            const int qbox = Q / kRows;
+            if (!un.rows) {
+                next_u = -1;
+                continue;
+            }
             if (pl == 0) {
                 // both pipelines are done with the previous unit's C, B and G
-                if (units_done > 0) wait_bar(&bars.unit_done, par_of(units_done - 1), abort, p.status);
+                if (udone > 0) wait_bar(&bars.unit_done, par(udone - 1), p.status, broken);
                 if (leader) {
-                    mbar_arrive_expect_tx(&bars.cb, (uint32_t)(NK + 2 * qbox) * 16384u);
+                    const uint32_t bboxes = (un.r == 1) ? 2u : 1u;
+                    mbar_arrive_expect_tx(&bars.cb, (uint32_t)(NK + 2 * bboxes) * 16384u);
                     for (int k = 0; k < NK; ++k)
                         tma_load_4d(sC + k * 16384, &mC, &bars.cb, k * 64, un.g, un.t0 + un.row0, un.b);
                     for (int k = 0; k < 2; ++k)
-                        for (int q = 0; q < qbox; ++q)
+                        for (uint32_t q = 0; q < bboxes; ++q)
                             tma_load_4d(sB + k * 32768 + q * 16384, &mB, &bars.cb, k * 64, un.g,
-                                        un.t0 + q * kRows, un.b);
+                                        un.t0 + (int)q * kRows, un.b);
+                    // claim the next unit now and warm L2 with its first tiles
+                    next_u = atomicAdd(p.counter, 1);
+                    if (next_u < p.n_units) {
+                        const Unit nx = decode(next_u, p);
+                        if (nx.rows) {
+                            for (int k = 0; k < NK; ++k)
+                                tma_prefetch_4d(&mC, k * 64, nx.g, nx.t0 + nx.row0, nx.b);
+                            for (int k = 0; k < 2; ++k)
+                                for (int q = 0; q <= nx.r; ++q)
+                                    tma_prefetch_4d(&mB, k * 64, nx.g, nx.t0 + q * kRows, nx.b);
+                            for (int hh = nx.h0; hh < min(nx.h0 + 2, nx.h1); ++hh)
+                                for (int q = 0; q <= nx.r; ++q)
+                                    tma_prefetch_4d(&mX, 0, hh, nx.t0 + q * kRows, nx.b);
+                        }
+                    }
                 }
+                next_u = __shfl_sync(0xffffffffu, next_u, 0);
             }
-            ++units_done;
-            wait_bar(&bars.cb, par_of(cbcnt++), abort, p.status);
+            ++udone;
+            wait_bar(&bars.cb, par(cbcnt++), p.status, broken);
             fence_after_sync();
             if (pl == 0) {
-                // G = C_r B^T  (rows of this half x columns 0 .. end of this half)
+                // G = C_r B_r^T: the block's rows against its own columns, K = N
                 if (leader) {
                     for (int kk = 0; kk < NK * 4; ++kk) {
                         const int atom = kk >> 2, kin = kk & 3;
-                        mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
-                               smem_desc_sw128(smem_u32(sB) + atom * 32768 + kin * 32, 16, 1024),
-                               first ? idG0 : idG1, kk > 0);
+                        mma_ss(tmem + kColG,
+                               smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
+                               smem_desc_sw128(smem_u32(sB) + atom * 32768 + un.row0 * 128 + kin * 32, 16, 1024),
+                               idG, kk > 0);
                     }
                     mma_commit(&bars.g_done);
                 }
                 __syncwarp();
             }
+            uint8_t *sXr = (un.r == 1) ? sXhi : sXlo;  // x rows of this block
             bool any = false;
             for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
                 any = true;
-                const int jb = use & 1;
-                // this head's X rows 0..Q-1 and s values; warm L2 for the pipeline's next head
-                if (use > 0) wait_bar(&pb.x_free, par_of(use - 1), abort, p.status);
+                // this head's x rows; warm L2 for the pipeline's next head
+                if (use > 0) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
                 if (leader) {
-                    mbar_arrive_expect_tx(&pb.x_full, (uint32_t)qbox * 16384u);
-                    for (int q = 0; q < qbox; ++q)
-                        tma_load_4d(sXp + q * 16384, &mX, &pb.x_full, 0, h, un.t0 + q * kRows, un.b);
-                    mbar_arrive_expect_tx(&pb.j_full[jb], (uint32_t)Q * 4u);
-                    bulk_load(sJp + jb * 256, p.s + (((size_t)un.b * sh.H + h) * sh.nc + un.c) * Q,
-                              (uint32_t)Q * 4u, &pb.j_full[jb]);
+                    const uint32_t xboxes = (un.r == 1) ? 2u : 1u;
+                    mbar_arrive_expect_tx(&pb.x_full, xboxes * 16384u);
+                    tma_load_4d(sXlo, &mX, &pb.x_full, 0, h, un.t0, un.b);
+                    if (un.r == 1) tma_load_4d(sXhi, &mX, &pb.x_full, 0, h, un.t0 + kRows, un.b);
                     if (h + 2 < un.h1)
-                        for (int q = 0; q < qbox; ++q) tma_prefetch_4d(&mX, 0, h + 2, un.t0 + q * kRows, un.b);
+                        for (uint32_t q = 0; q < xboxes; ++q)
+                            tma_prefetch_4d(&mX, 0, h + 2, un.t0 + (int)q * kRows, un.b);
                 }
                 __syncwarp();
-                if (first) {
-                    // stage 2: D = B_c^T (decayed X), M = n (128), N = p, K = Q tokens; the decayed
-                    // rows 0..127 sit in the S~ buffer, rows 128.. were decayed in place
-                    wait_bar(&pb.xd_full, par_of(r0use), abort, p.status);
+                if (un.owner) {
+                    // stages 2-3 products: S_pre = B_{<r}^T (scaled rows before the block) into A,
+                    // S_own = B_r^T (scaled rows of the block) into B; M = n, N = p, K = tokens
+                    wait_bar(&pb.x_full, par(use), p.status, broken);
+                    wait_bar(&pb.xd_full, par(ocnt), p.status, broken);
+                    if (use > 0) wait_bar(&pb.acc_free, par(use - 1), p.status, broken);
                     fence_after_sync();
                     if (leader) {
-                        for (int kk = 0; kk < Q / 16; ++kk) {
-                            const uint32_t xb = (kk < 8) ? smem_u32(sSp) + kk * 2048 : smem_u32(sXp) + kk * 2048;
-                            mma_ss(tD, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
-                                   smem_desc_sw128(xb, 16, 1024), idState, kk > 0);
-                        }
+                        if (un.r == 1)
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_ss(tA, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
+                                       smem_desc_sw128(smem_u32(sXlo) + kk * 2048, 16, 1024), idState, kk > 0);
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(tB, smem_desc_sw128(smem_u32(sB) + un.row0 * 128 + kk * 2048, 32768, 1024),
+                                   smem_desc_sw128(smem_u32(sW) + kk * 2048, 16, 1024), idState, kk > 0);
                         mma_commit(&pb.d_done);
                     }
                     __syncwarp();
-                    ++r0use;
+                    ++ocnt;
                 }
-                // stage 4 product: Y = C_r S~^T
-                wait_bar(&pb.s_full, par_of(use), abort, p.status);
-                if (use > 0) wait_bar(&pb.y_free, par_of(use - 1), abort, p.status);
+                // stage 4 product: Y_inter = C_r E^T into A (E: the entering-state tile [n][p] in W)
+                wait_bar(&pb.s_full, par(use), p.status, broken);
+                if (!un.owner && use > 0) wait_bar(&pb.acc_free, par(use - 1), p.status, broken);
                 fence_after_sync();
                 if (leader) {
                     for (int kk = 0; kk < NK * 4; ++kk) {
                         const int atom = kk >> 2, kin = kk & 3;
-                        mma_ss(tY, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
-                               smem_desc_sw128(smem_u32(sSp) + atom * 8192 + kin * 32, 16, 1024), idInter, kk > 0);
+                        mma_ss(tA, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
+                               smem_desc_sw128(smem_u32(sW) + kk * 2048, 16, 1024), idInter, kk > 0);
                     }
-                    mma_commit(&pb.inter_done);
                 }
                 __syncwarp();
-                // stage 1 product: Y += M X, one 128-token K-half at a time
-                const int nhalf = first ? 1 : 2;
-                for (int hf = 0; hf < nhalf; ++hf) {
-                    wait_bar(&pb.m_full, par_of(mcnt), abort, p.status);
-                    if (hf == 0 && !first) wait_bar(&pb.x_full, par_of(use), abort, p.status);
-                    fence_after_sync();
-                    if (leader) {
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tY, tM + kk * 8, smem_desc_sw128(smem_u32(sXp) + (hf * 8 + kk) * 2048, 16, 1024),
-                                   idMX, 1);
-                        mma_commit(&pb.m_free);
-                    }
-                    __syncwarp();
-                    ++mcnt;
-                }
+                // stage 1 product: Y_intra = M X_r into B
+                wait_bar(&pb.m_full, par(use), p.status, broken);
+                if (!un.owner) wait_bar(&pb.x_full, par(use), p.status, broken);
+                fence_after_sync();
                 if (leader) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tB, tM + kk * 8, smem_desc_sw128(smem_u32(sXr) + kk * 2048, 16, 1024), idMX,
+                               kk > 0);
                     mma_commit(&pb.mx_done);
-                    mma_commit(&pb.x_free);
                 }
                 __syncwarp();
             }
             // this pipeline is done with the unit once its last products completed
-            if (any) wait_bar(&pb.mx_done, par_of(use - 1), abort, p.status);
+            if (any) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
             if (leader) mbar_arrive(&bars.unit_done);
             __syncwarp();
         }
     } else {
         // ------------------------------------------------------------------
-        // CUDA-core warps: warps 8pl..8pl+7 serve pipeline pl as two
-        // warpgroups; warpgroup `half` takes columns [32 half, 32 half + 32)
-        // of every 64-wide tile and every other 32-column slab of the mask.
+        // CUDA-core warps: warps 8pl..8pl+7 serve pipeline pl.  Thread wtid
+        // owns token wtid of the chunk for the prefix sums; for tile work,
+        // warp quarter q (warp & 3) owns TMEM lanes 32q..32q+31 (rows of
+        // the block, or n of a state) and warpgroup `half` owns columns
+        // 32 half .. 32 half + 31 of every 64-wide tile.
         // ------------------------------------------------------------------
         const int pl = warp >> 3;
-        const int half = (warp >> 2) & 1;
-        const int wtid = tid & (kPipeThreads - 1);
-        const int lrow = ((warp & 3) << 5) + lane;  // TMEM lane = row within the chunk half
-        const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
-        const int wg_bar = 1 + pl;
+        const int pw = warp & 7;
+        const int half = pw >> 2;
+        const int quarter = warp & 3;
+        const int wtid = pw * 32 + lane;
+        const int lrow = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const int bar_id = 1 + pl;
         PipeBars &pb = bars.pb[pl];
-        uint8_t *sXp = smem + kOffX + pl * 32768;
-        uint8_t *sSp = smem + kOffS + pl * 16384;
-        float *sJp = reinterpret_cast<float *>(smem + kOffJ) + pl * 512;
-        float *sFp = reinterpret_cast<float *>(smem + kOffF) + pl * 512;
-        const uint32_t tY = tmem + kColY + pl * 64, tM = tmem + kColM + pl * 64, tD = tmem + kColD + pl * 64;
-        uint32_t use = 0, r0use = 0, mcnt = 0, ucnt = 0, gcnt = 0;
-#ifdef SSD_TRACE
-        int trace_i = 0;
-#endif
+        uint8_t *sXlo = smem + kOffPipe + pl * kPipeBytes;
+        uint8_t *sW = sXlo + 16384;
+        uint8_t *sXhi = sXlo + 32768;
+        float *sJ = reinterpret_cast<float *>(smem + kOffAux) + pl * kAuxFloats;  // s in log2 units
+        float *sF = sJ + 256;                                                     // column factors
+        float *sTot = sF + 256;                                                   // warp totals
+        const uint32_t tA = tmem + col_acc_a(pl), tB = tmem + col_acc_b(pl), tM = tmem + col_mask(pl);
+        const size_t PN = (size_t)kP * N;
+        uint32_t use = 0, ocnt = 0, ucnt = 0, gcnt = 0;
         for (;;) {
-            wait_bar(&bars.unit_full, par_of(ucnt), abort, p.status);
+            wait_bar(&bars.unit_full, par(ucnt), p.status, broken);
             ++ucnt;
             const int u = s_unit;
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.unit_empty);
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
-            if (un.row0 >= un.len) {
-                // no rows: count the (unread) entering state of every head as read
-                if (tid == 0)
-                    for (int h = un.h0; h < un.h1; ++h) red_release_add_gpu(p.cons + un.b * sh.H + h, 1);
-                continue;
-            }
-            const bool first = (un.r == 0);
-            const int j = un.row0 + lrow;  // this thread's row within the chunk
-            const int kcols = un.row0 + kRows;
-            wait_bar(&bars.g_done, par_of(gcnt++), abort, p.status);
-            for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
-                const int jb = use & 1;
-                float *sJb = sJp + jb * 256;
-                float *sFb = sFp + jb * 256;
-                const size_t bh = (size_t)un.b * sh.H + h;
-                const size_t PN = (size_t)kP * N;
-                SSD_TRACE_POINT(0);
-                // the previous head's y tile left the S~ buffer before it is overwritten (the
-                // stores are issued by the pipeline's last thread, never by the thread that
-                // fences and publishes states, whose GPU-scope fence would wait for them)
+            if (!un.rows) continue;
+            const uint32_t gphase = gcnt++;
+            int h = un.h0 + pl;
+            if (h >= un.h1) continue;
+            const bool own = un.owner;
+            const int end = un.len - 1;
+            const int j = un.row0 + lrow;  // this thread's row of the chunk
+            // dt of this token, A and D for the pipeline's first head of the unit
+            const float *dtp = p.dt + ((size_t)un.b * sh.T + un.t0 + wtid) * sh.H;
+            float dt_cur = (wtid < un.len) ? __ldg(dtp + h) : 0.f;
+            float a_cur = __ldg(p.A + h), d_cur = __ldg(p.D + h);
+            bool first_head = true;
+            for (; h < un.h1; h += 2, ++use) {
+                const int bh = un.b * sh.H + h;
+                // the y tile of the pipeline's previous head has left W (its store was issued by this
+                // thread); the scan's barrier below publishes that to the pipeline
                 if (wtid == kPipeThreads - 1) bulk_wait_read();
-                SSD_TRACE_POINT(1);
-                wait_bar(&pb.j_full[jb], par_of(use >> 1), abort, p.status);
-                for (int i = wtid; i < kcols; i += kPipeThreads) sFb[i] = expf(sJb[i | 31] - sJb[i]);
-                named_bar_sync(wg_bar, kPipeThreads);
-                SSD_TRACE_POINT(2);
-                const float *src = (un.c == 0) ? (p.init ? p.init + bh * PN : nullptr)
-                                               : p.ring + (bh * 2 + ((un.c - 1) & 1)) * PN;
-                const float sj = sJb[j];
-                const float Dh = p.D[h];
-                const float s_end = sJb[Q - 1];
+                // ---- stage 0: inclusive prefix sums of dt*A over the chunk, in log2 units
+                float v = dt_cur * (a_cur * kLog2e);
+                const float Dh = d_cur;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float t = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += t;
+                }
+                if (lane == 31) sTot[pw] = v;
+                named_bar_sync(bar_id, kPipeThreads);
+                // the next head's dt, A and D, in flight while this head is processed
+                if (h + 2 < un.h1) {
+                    dt_cur = (wtid < un.len) ? __ldg(dtp + h + 2) : 0.f;
+                    a_cur = __ldg(p.A + h + 2);
+                    d_cur = __ldg(p.D + h + 2);
+                }
+                float pre = 0.f;
+                for (int w = 0; w < pw; ++w) pre += sTot[w];
+                const float s_mine = pre + v;
+                sJ[wtid] = s_mine;
+                // column factor exp(s_{i|31} - s_i) <= 1 of the mask's blocks below the diagonal
+                sF[wtid] = ex2(__shfl_sync(0xffffffffu, s_mine, 31) - s_mine);
+                named_bar_sync(bar_id, kPipeThreads);
+                const float s_end = sJ[end];
+                const float s_ref = (un.r == 1) ? sJ[kRows - 1] : 0.f;  // s_{r-1}
+                const float sj = sJ[j];
 
-                // decay mask for 32-column slabs sl = half, half + 2 of K-half hf, into TMEM, in
-                // 16-column pieces (few live registers: the entering state may be in flight)
-                auto mask_half = [&](int hf) {
-#pragma unroll 1
-                    for (int sl = half; sl < 4; sl += 2) {
-                        const int i0 = hf * 128 + sl * 32;
-                        uint32_t o[16];
-                        if (i0 > j) {
+                // ---- owner: rows scaled by their decay to the state's end (stage 2 operand)
+                if (own) {
+                    wait_bar(&pb.x_full, par(use), p.status, broken);
+                    if (un.r == 1) {
+                        // rows 0..127 in place (to row 127: S_pre), rows 128..255 into W (to the end)
+                        const int row = wtid;
+                        const bool lo = row < kRows;
+                        const float w = ex2((lo ? s_ref : s_end) - sJ[row]);
+                        const uint8_t *src = (lo ? sXlo : sXhi);
+                        uint8_t *dst = lo ? sXlo : sW;
+                        const int rr = row & (kRows - 1);
+                        uint4 xv[8];
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) o[q] = 0u;
-                            tmem_st16(tM + sl * 16 + lane_base, o);
-                            continue;
-                        }
-                        uint32_t g[32];
-                        tmem_ld16(tmem + kColG + i0 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
-                        tmem_ld16(tmem + kColG + i0 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
-                        tmem_wait_ld();
-                        if (i0 + 31 < j) {
-                            // below the diagonal block: row factor x column factor, both <= 1
-                            const float rf = expf(sj - sJb[i0 + 31]);
-                            const float4 *f4 = reinterpret_cast<const float4 *>(sFb + i0);
+                        for (int k = 0; k < 8; ++k) xv[k] = lds128(src + swz(rr, k));
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 f = f4[q];
-                                const float2 w0 = mul_f32x2(make_float2(rf, rf), make_float2(f.x, f.y));
-                                const float2 w1 = mul_f32x2(make_float2(rf, rf), make_float2(f.z, f.w));
-                                const float2 m0 = mul_f32x2(
-                                    make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
-                                const float2 m1 = mul_f32x2(
-                                    make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])), w1);
-                                o[2 * q] = pack_bf16x2(m0.x, m0.y);
-                                o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
-                            }
-                        } else {
-                            // the diagonal 32x32 block: one exponential per element
+                        for (int k = 0; k < 8; ++k) sts128(dst + swz(rr, k), scale_bf16x8(xv[k], w));
+                    } else {
+                        // the only block: rows 0..127 into W (to the end); x stays unscaled for M X
+                        const int rr = wtid & (kRows - 1), k0 = (wtid >> 7) * 4;
+                        const float w = ex2(s_end - sJ[rr]);
+                        uint4 xv[4];
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                const int ia = i0 + 2 * q, ib = ia + 1;
-                                float a = (ia <= j) ? __uint_as_float(g[2 * q]) * expf(sj - sJb[ia]) : 0.f;
-                                float bb = (ib <= j) ? __uint_as_float(g[2 * q + 1]) * expf(sj - sJb[ib]) : 0.f;
-                                if (ia == j) a += Dh;
-                                if (ib == j) bb += Dh;
-                                o[q] = pack_bf16x2(a, bb);
-                            }
-                        }
-                        tmem_st16(tM + sl * 16 + lane_base, o);
-                    }
-                    tmem_wait_st();
-                };
-                // Y *= exp(s_j) (stage 4's decay from the chunk start), then hand mask K-half 0 to
-                // the issuer: its product accumulates onto the scaled Y
-                auto scale_and_release_mask = [&]() {
-                    wait_bar(&pb.inter_done, par_of(use), abort, p.status);
-                    fence_after_sync();
-                    const float e = expf(sj);
-                    uint32_t v[32];
-                    tmem_ld16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_wait_ld();
+                        for (int k = 0; k < 4; ++k) xv[k] = lds128(sXlo + swz(rr, k0 + k));
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * e);
-                    tmem_st16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_st16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_wait_st();
-                    fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.m_full);
-                    ++mcnt;
-                };
-
-                if (first) {
-                    // x_i * exp(s_end - s_i) for the chunk state: rows 0..127 into the S~ buffer
-                    // (rows 0..127 of the X tile stay undecayed for the masked product), rows 128.. in place
-                    wait_bar(&pb.x_full, par_of(use), abort, p.status);
-                    SSD_TRACE_POINT(21);
-#pragma unroll 1
-                    for (int base = wtid; base < Q * 8; base += 4 * kPipeThreads) {
-                        uint4 v[4];
-                        float w[4];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int idx = min(base + r * kPipeThreads, Q * 8 - 1);
-                            v[r] = *reinterpret_cast<const uint4 *>(sXp + idx * 16);
-                            w[r] = expf(s_end - sJb[idx >> 3]);
-                        }
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int idx = base + r * kPipeThreads;
-                            if (idx >= Q * 8) continue;
-                            uint4 o;
-                            o.x = pack_bf16x2(bf16lo(v[r].x) * w[r], bf16hi(v[r].x) * w[r]);
-                            o.y = pack_bf16x2(bf16lo(v[r].y) * w[r], bf16hi(v[r].y) * w[r]);
-                            o.z = pack_bf16x2(bf16lo(v[r].z) * w[r], bf16hi(v[r].z) * w[r]);
-                            o.w = pack_bf16x2(bf16lo(v[r].w) * w[r], bf16hi(v[r].w) * w[r]);
-                            *reinterpret_cast<uint4 *>(((idx >> 3) < kRows ? sSp : sXp) + idx * 16) = o;
-                        }
+                        for (int k = 0; k < 4; ++k) sts128(sW + swz(rr, k0 + k), scale_bf16x8(xv[k], w));
                     }
                     fence_view_async_shared();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.xd_full);
-                    SSD_TRACE_POINT(3);
-                    // mask K-half 0 (the whole K range of a first half) while the state product runs
-                    // and before waiting on the chain, so that the chain's path holds no mask work
-                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
-                    SSD_TRACE_POINT(22);
-                    fence_after_sync();
-                    mask_half(0);
-                    // S~_{c-1} must be published and the outgoing ring slot free of readers: the slot
-                    // held S~_{c-2}, read by the second half of chunk c-1, so wait until the second
-                    // halves of chunks 0..c-1 have all read theirs
-                    if (wtid == 0) {
-                        if (un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
-                        if (p.halves == 2 && un.c >= 2) wait_flag(p.cons + bh, un.c, abort, p.status);
-                    }
-                    named_bar_sync(wg_bar, kPipeThreads);
-                    SSD_TRACE_POINT(15);
-                    // this thread's 32 columns of S~_{c-1} (lane n; [p][n] like the initial state)
-                    const int n = lrow;
-                    float old[32];
+                }
+
+                // ---- stage 1 mask M[j][i] = exp(s_j - s_i) G[j][i] for i <= j (+ D_h at i = j), bf16 in
+                // TMEM.  Warpgroup 0 builds each row's diagonal 32-column slab (one exponential per
+                // element), warpgroup 1 the slabs below it (row factor x column factor, both <= 1) and
+                // the zero slabs above it.
+                if (first_head) wait_bar(&bars.g_done, par(gphase), p.status, broken);
+                fence_after_sync();
+                {
+                    const int dq = quarter;  // diagonal slab of this warp's rows
+                    if (half == 0) {
+                        uint32_t g[32], o[16];
+                        tmem_ld16(tmem + kColG + dq * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+                        tmem_ld16(tmem + kColG + dq * 32 + 16 + lane_base,
+                                  *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+                        tmem_wait_ld();
+                        const float2 *sc = reinterpret_cast<const float2 *>(sJ + un.row0 + dq * 32);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        old[q] = (src && n < N) ? __ldcg(src + (size_t)(half * 32 + q) * N + n) : 0.f;
-                    SSD_TRACE_POINT(4);
-                    SSD_TRACE_ARRIVED(old, 32, 8);
-                    // stage 3: S~_c = exp(s_end) S~_{c-1} + S_c; S~_{c-1} in bf16 is this head's
-                    // inter-chunk operand (the decayed rows left the S~ buffer with the state product)
-                    wait_bar(&pb.d_done, par_of(r0use), abort, p.status);
-                    ++r0use;
-                    named_bar_sync(wg_bar, kPipeThreads);
-                    fence_after_sync();
-                    SSD_TRACE_POINT(5);
-                    {
-                        // the outgoing state goes to the ring or, after the last chunk, to the final state
-                        const float dchunk = expf(s_end);
-                        float *dst = (un.c == sh.nc - 1) ? (p.fin ? p.fin + bh * PN : nullptr)
-                                                         : p.ring + (bh * 2 + (un.c & 1)) * PN;
+                        for (int q = 0; q < 16; ++q) {
+                            const float2 si = sc[q];
+                            float a = (2 * q <= lane) ? __uint_as_float(g[2 * q]) * ex2(sj - si.x) : 0.f;
+                            float b = (2 * q + 1 <= lane) ? __uint_as_float(g[2 * q + 1]) * ex2(sj - si.y) : 0.f;
+                            if (2 * q == lane) a += Dh;
+                            if (2 * q + 1 == lane) b += Dh;
+                            o[q] = pack_bf16x2(a, b);
+                        }
+                        tmem_st16(tM + dq * 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+                    } else {
+#pragma unroll 1
+                        for (int sl = 0; sl < 4; ++sl) {
+                            if (sl == dq) continue;
+                            uint32_t o[16];
+                            if (sl > dq) {
 #pragma unroll
-                        for (int q0 = 0; q0 < 32; q0 += 16) {
-                            uint32_t dv[16];
-                            tmem_ld16(tmem + kColD + pl * 64 + half * 32 + q0 + lane_base, dv);
-                            tmem_wait_ld();
-                            if (n < N && dst) {
+                                for (int q = 0; q < 16; ++q) o[q] = 0u;
+                            } else {
+                                uint32_t g[32];
+                                tmem_ld16(tmem + kColG + sl * 32 + lane_base,
+                                          *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+                                tmem_ld16(tmem + kColG + sl * 32 + 16 + lane_base,
+                                          *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+                                tmem_wait_ld();
+                                const int i0 = un.row0 + sl * 32;
+                                const float rf = ex2(sj - sJ[i0 + 31]);
+                                const float2 rr = make_float2(rf, rf);
+                                const float4 *f4 = reinterpret_cast<const float4 *>(sF + i0);
 #pragma unroll
-                                for (int q = 0; q < 16; ++q)
-                                    __stcg(dst + (size_t)(half * 32 + q0 + q) * N + n,
-                                           fmaf(dchunk, old[q0 + q], __uint_as_float(dv[q])));
+                                for (int q = 0; q < 8; ++q) {
+                                    const float4 f = f4[q];
+                                    const float2 w0 = mul_f32x2(rr, make_float2(f.x, f.y));
+                                    const float2 w1 = mul_f32x2(rr, make_float2(f.z, f.w));
+                                    const float2 m0 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q]), __uint_as_float(g[4 * q + 1])), w0);
+                                    const float2 m1 = mul_f32x2(
+                                        make_float2(__uint_as_float(g[4 * q + 2]), __uint_as_float(g[4 * q + 3])),
+                                        w1);
+                                    o[2 * q] = pack_bf16x2(m0.x, m0.y);
+                                    o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
+                                }
                             }
-                        }
-                        // the publisher warp releases the stores
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&pb.ring_done);
-                        // S~_{c-1} in bf16 into column n of the S~ tile ([p][n], 128-byte swizzled)
-                        if (n < N) {
-                            uint8_t *srow = sSp + (n >> 6) * 8192;
-                            const int chunk = (n & 63) >> 3, sub = (n & 7) * 2;
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) {
-                                const int pp = half * 32 + q;
-                                *reinterpret_cast<__nv_bfloat16 *>(srow + pp * 128 + ((chunk ^ (pp & 7)) << 4) + sub) =
-                                    __float2bfloat16_rn(old[q]);
-                            }
+                            tmem_st16(tM + sl * 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
                         }
                     }
-                    SSD_TRACE_POINT(12);
-                    fence_view_async_shared();
-                    named_bar_sync(wg_bar, kPipeThreads);
-                    SSD_TRACE_POINT(13);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.s_full);
-                    SSD_TRACE_POINT(6);
-                    scale_and_release_mask();
-                    SSD_TRACE_POINT(7);
-                } else {
-                    // mask K-half 0 first, then wait for the entering state (chunk 0 reads the
-                    // initial state)
-                    if (mcnt > 0) wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
-                    fence_after_sync();
-                    mask_half(0);
-                    if (wtid == 0 && un.c > 0) wait_flag(p.ready + bh, un.c, abort, p.status);
-                    named_bar_sync(wg_bar, kPipeThreads);
-                    // this thread's pieces of S~_{c-1} ([p][n]: 8 consecutive n of one row p each)
-                    const int nchunks = kP * NK * 8;
-                    float4 lo[4], hi[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int idx = wtid + r * kPipeThreads;
-                        const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
-                        lo[r] = hi[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (idx < nchunks && src && n < N) {
-                            lo[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n));
-                            hi[r] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)pr * N + n + 4));
-                        }
-                    }
-                    SSD_TRACE_POINT(3);
-                    SSD_TRACE_ARRIVED(reinterpret_cast<const float *>(lo), 16, 8);
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int idx = wtid + r * kPipeThreads;
-                        const int pr = idx / (NK * 8), n = (idx % (NK * 8)) * 8;
-                        if (idx >= nchunks) continue;
-                        uint4 v;
-                        v.x = pack_bf16x2(lo[r].x, lo[r].y);
-                        v.y = pack_bf16x2(lo[r].z, lo[r].w);
-                        v.z = pack_bf16x2(hi[r].x, hi[r].y);
-                        v.w = pack_bf16x2(hi[r].z, hi[r].w);
-                        *reinterpret_cast<uint4 *>(sSp + (n >> 6) * 8192 + pr * 128 +
-                                                   ((((n & 63) >> 3) ^ (pr & 7)) << 4)) = v;
-                    }
-                    // the publisher warp releases the ring slot: this warp's loads are consumed
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.ring_done);
-                    fence_view_async_shared();
-                    named_bar_sync(wg_bar, kPipeThreads);
-                    if (lane == 0) mbar_arrive(&pb.s_full);
-                    SSD_TRACE_POINT(6);
-                    scale_and_release_mask();
-                    SSD_TRACE_POINT(7);
-                    // mask K-half 1 once the product of K-half 0 has read the mask buffer
-                    wait_bar(&pb.m_free, par_of(mcnt - 1), abort, p.status);
-                    fence_after_sync();
-                    mask_half(1);
+                    tmem_wait_st();
                     fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.m_full);
-                    ++mcnt;
                 }
-                SSD_TRACE_POINT(9);
-                // stage 5: y = bf16(Y), staged in the S~ buffer (its inter-chunk product is done)
-                // in the 128-byte-swizzled layout and written by one TMA store
-                wait_bar(&pb.mx_done, par_of(use), abort, p.status);
-                SSD_TRACE_POINT(10);
-                fence_after_sync();
-                {
-                    uint32_t v[32];
-                    tmem_ld16(tY + half * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld16(tY + half * 32 + 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_wait_ld();
+                first_head = false;
+
+                // ---- stage 3: the state entering the chunk (published by the owner of chunk c-1);
+                // an owner that writes the ring also waits until the slot it overwrites (S~_{c-2})
+                // has been read by the other block of chunk c-1.  Reads are counted per slot: the
+                // non-owners of chunks 1, 3, 5, ... read slot 0 and those of chunks 2, 4, ... slot 1,
+                // so slot c & 1 has had c / 2 reads once chunk c-1's is in (a single count could be
+                // reached early by chunk c's own reader, which reads the other slot).
+                const bool writes_ring = own && un.c < sh.nc - 1;
+                if (wtid == 0) {
+                    if (un.c > 0) wait_flag(p.ready + bh, un.c, p.flag_polls, abort, p.status);
+                    if (writes_ring && p.halves == 2 && un.c >= 2)
+                        wait_flag(p.cons + 2 * bh + (un.c & 1), un.c / 2, p.flag_polls, abort, p.status);
+                }
+                named_bar_sync(bar_id, kPipeThreads);
+                // this thread's 32 entries of S~_{c-1}: state row n = lrow, p in [32 half, 32 half + 32)
+                const int n = lrow;
+                const bool nv = n < N;
+                float old[32];
+                if (un.c == 0) {
+                    const float *src = p.init ? p.init + (size_t)bh * PN + (size_t)(half * 32) * N + n : nullptr;
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) old[q] = (src && nv) ? __ldg(src + (size_t)q * N) : 0.f;
+                } else {
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * 2 + ((un.c - 1) & 1)) * PN);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 t = nv ? __ldcg(src + ring_quad(N, n, half * 8 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        old[4 * q] = t.x;
+                        old[4 * q + 1] = t.y;
+                        old[4 * q + 2] = t.z;
+                        old[4 * q + 3] = t.w;
+                    }
+                }
+                if (own) {
+                    wait_bar(&pb.d_done, par(ocnt), p.status, broken);
+                    ++ocnt;
+                    fence_after_sync();
+                    if (un.r == 1) {
+                        // E = exp(s_127) S~_{c-1} + S_pre
+                        const float e_start = ex2(s_ref);
+#pragma unroll
+                        for (int q0 = 0; q0 < 32; q0 += 16) {
+                            uint32_t t[16];
+                            tmem_ld16(tA + half * 32 + q0 + lane_base, t);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) old[q0 + q] = fmaf(e_start, old[q0 + q], __uint_as_float(t[q]));
+                        }
+                    }
+                }
+                // E in bf16 into row n of the tile [n][p] (128-byte swizzled), the B operand of stage 4;
+                // handed to the issuer before the outgoing state is formed
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    uint4 t;
+                    t.x = pack_bf16x2(old[8 * k + 0], old[8 * k + 1]);
+                    t.y = pack_bf16x2(old[8 * k + 2], old[8 * k + 3]);
+                    t.z = pack_bf16x2(old[8 * k + 4], old[8 * k + 5]);
+                    t.w = pack_bf16x2(old[8 * k + 6], old[8 * k + 7]);
+                    if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
+                    sts128(sW + swz(n, half * 4 + k), t);
+                }
+                fence_view_async_shared();
+                if (!own) {
+                    // the ring entries are in registers: the publisher may count the slot as read
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&pb.ring_done);
+                        mbar_arrive(&pb.s_full);
+                    }
+                } else {
+                    // S~_c = exp(s_end - s_{r-1}) E + S_own, to the ring or to final_state.  S_own is read
+                    // from TMEM before s_full, after which the issuer overwrites that accumulator.
+                    const float e_rest = ex2(s_end - s_ref);
+#pragma unroll
+                    for (int q0 = 0; q0 < 32; q0 += 16) {
+                        uint32_t t[16];
+                        tmem_ld16(tB + half * 32 + q0 + lane_base, t);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) old[q0 + q] = fmaf(e_rest, old[q0 + q], __uint_as_float(t[q]));
+                    }
                     fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.y_free);
+                    if (lane == 0) mbar_arrive(&pb.s_full);
+                    if (nv && writes_ring) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * 2 + (un.c & 1)) * PN);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-                        w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-                        w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-                        w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-                        const int qq = half * 4 + q;  // 16-byte chunk of the 128-byte row
-                        *reinterpret_cast<uint4 *>(sSp + lrow * 128 + ((qq ^ (lrow & 7)) << 4)) = w;
+                        for (int q = 0; q < 8; ++q)
+                            __stcg(dst + ring_quad(N, n, half * 8 + q),
+                                   make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                    } else if (nv && p.fin) {
+                        float *fin = p.fin + (size_t)bh * PN + (size_t)(half * 32) * N + n;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) fin[(size_t)q * N] = old[q];
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.ring_done);  // the publisher releases the stores
+                }
+
+                // ---- stages 4-5: y_j = exp(s_j - s_{r-1}) Y_inter + Y_intra (the D skip is in the mask),
+                // staged as bf16 in W (128-byte swizzled [j][p]; its state tile has been consumed) and
+                // written by one TMA store (rows past T are clipped)
+                wait_bar(&pb.mx_done, par(use), p.status, broken);
+                fence_after_sync();
+                {
+                    const float ej = ex2(sj - s_ref);
+#pragma unroll
+                    for (int q0 = 0; q0 < 32; q0 += 16) {
+                        uint32_t a[16], b[16];
+                        tmem_ld16(tA + half * 32 + q0 + lane_base, a);
+                        tmem_ld16(tB + half * 32 + q0 + lane_base, b);
+                        tmem_wait_ld();
+                        uint32_t o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float2 r = fma_f32x2(make_float2(ej, ej),
+                                                       make_float2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])),
+                                                       make_float2(__uint_as_float(b[2 * q]), __uint_as_float(b[2 * q + 1])));
+                            o[q] = pack_bf16x2(r.x, r.y);
+                        }
+                        const int ch = half * 4 + q0 / 8;
+                        sts128(sW + swz(lrow, ch), make_uint4(o[0], o[1], o[2], o[3]));
+                        sts128(sW + swz(lrow, ch + 1), make_uint4(o[4], o[5], o[6], o[7]));
+                    }
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.acc_free);
                     fence_view_async_shared();
-                    named_bar_sync(wg_bar, kPipeThreads);
+                    named_bar_sync(bar_id, kPipeThreads);
                     if (wtid == kPipeThreads - 1) {
-                        tma_store_4d(&mY, sSp, 0, h, un.t0 + un.row0, un.b);
+                        tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
                     }
                 }
-                SSD_TRACE_POINT(11);
-#ifdef SSD_TRACE
-                if (ssd_trace_buffer && wtid == 0 && trace_i < 30)
-                    ssd_trace_buffer[((size_t)blockIdx.x * 2 + pl) * 1024 + trace_i * 32 + 14] =
-                        ((unsigned long long)h << 32) | ((unsigned long long)un.c << 8) | (first ? 1 : 0);
-                ++trace_i;
-#endif
             }
         }
+        if (wtid == kPipeThreads - 1) bulk_wait_all();
     }
-    if (warp < kSimtWarps && (tid & (kPipeThreads - 1)) == kPipeThreads - 1) bulk_wait_all();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
@@ -784,7 +801,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 bool fused_supported(const Shape &sh, int dtype) {
-    return dtype == SSD_BF16 && sh.P == kP && (sh.N == 64 || sh.N == 128) && (sh.Q == 128 || sh.Q == 256);
+    return dtype == SSD_BF16 && sh.P == kP && sh.N >= 16 && sh.N <= 128 && sh.N % 16 == 0 &&
+           (sh.Q == 128 || sh.Q == 256);
 }
 
 static int device_sm_count() {
@@ -794,24 +812,33 @@ static int device_sm_count() {
     return n;
 }
 
-cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, const __nv_bfloat16 *C,
-                             const float *D, const float *s, const float *init, float *fin, float *ring, int *ready,
-                             int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
-                             cudaStream_t st) {
+// Heads per work unit: enough to amortise the unit's C, B and G over several
+// heads, few enough that every SM gets several units.
+static int heads_per_unit(const Shape &sh) {
+    const int hpg = sh.heads_per_group;
+    if (hpg <= 8) return hpg;
+    const int blocks = (hpg + 7) / 8;
+    return (hpg + blocks - 1) / blocks;
+}
+
+cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
+                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
+                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
+                             const FusedDebug *dbg, cudaStream_t st) {
     CUtensorMap mC, mB, mX;
     const uint64_t dbc[4] = {(uint64_t)sh.N, (uint64_t)sh.G, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sbc[3] = {(uint64_t)sh.N * 2, (uint64_t)sh.G * sh.N * 2, (uint64_t)sh.T * sh.G * sh.N * 2};
-    const uint32_t box_bc[4] = {64, 1, kRows, 1};
+    const uint32_t box[4] = {64, 1, kRows, 1};
     const uint64_t dx[4] = {(uint64_t)sh.P, (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sx[3] = {(uint64_t)sh.P * 2, (uint64_t)sh.H * sh.P * 2, (uint64_t)sh.T * sh.H * sh.P * 2};
-    const uint32_t box_x[4] = {64, 1, kRows, 1};
     CUtensorMap mY;
-    if (!make_map_bf16(&mC, C, 4, dbc, sbc, box_bc) || !make_map_bf16(&mB, B, 4, dbc, sbc, box_bc) ||
-        !make_map_bf16(&mX, x, 4, dx, sx, box_x) || !make_map_bf16(&mY, y, 4, dx, sx, box_x))
+    if (!make_map_bf16(&mC, C, 4, dbc, sbc, box) || !make_map_bf16(&mB, B, 4, dbc, sbc, box) ||
+        !make_map_bf16(&mX, x, 4, dx, sx, box) || !make_map_bf16(&mY, y, 4, dx, sx, box))
         return cudaErrorInvalidValue;
     Params p;
     p.sh = sh;
-    p.s = s;
+    p.dt = dt;
+    p.A = A;
     p.D = D;
     p.init = init;
     p.fin = fin;
@@ -823,9 +850,12 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const __nv_bfloat16 *B, con
     p.y = y;
     p.NK = (sh.N + 63) / 64;
     p.halves = sh.Q / kRows;
-    p.heads_per_unit = min(4, sh.heads_per_group);
+    p.heads_per_unit = heads_per_unit(sh);
     p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
     p.n_units = sh.nc * sh.batch * sh.G * p.blocks_per_group * p.halves;
+    p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
+    p.withhold_bh = dbg ? dbg->withhold_bh : -1;
+    p.withhold_c = dbg ? dbg->withhold_c : -1;
     cudaError_t e =
         cudaFuncSetAttribute(ssd_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;

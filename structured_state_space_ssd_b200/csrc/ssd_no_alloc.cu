@@ -61,3 +61,14 @@ extern "C" int ssd_fwd_no_alloc(const void *x, const float *dt, const float *A, 
     return ssd_fwd(x, dt, A, B, C, D, Q, init_state, y, final_state, batch, T, H, P, G, N, dtype, ws,
                    (size_t)SSD_NO_ALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" int ssd_fwd_no_alloc_check(void *stream) {
+    void *ws = nullptr;
+    const int rc = scratch_of_current_device(&ws);
+    if (rc != SSD_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    int status = 0;
+    if (cudaMemcpy(&status, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    return status;
+}

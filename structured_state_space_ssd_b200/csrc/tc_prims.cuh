@@ -322,6 +322,28 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
     return c;
 }
 
+// Packed fp32x2 fused multiply-add a * b + c (one instruction for two lanes of data on sm_100).
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+    unsigned long long ra, rb, rc, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+
+// 2^x by the hardware's base-2 exponential instruction (PTX ex2.approx.ftz.f32).
+// The tensor-core path keeps its log-decays in base-2 units (scaled by log2 e
+// once, where the prefix sums are formed), so exp(s_a - s_b) is ex2 of a
+// difference, one instruction.  Subnormal results flush to zero.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

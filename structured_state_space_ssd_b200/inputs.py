@@ -75,24 +75,28 @@ HEADLINE = "mamba2_2p7b_layer"
 
 
 def make_inputs(batch: int, T: int, H: int, P: int, N: int, G: int, dtype: str = "bf16",
-                seed: int = 0, with_init: bool = False) -> dict:
-    """Draw one problem's inputs on the CPU (see the module docstring).
+                seed: int = 0, with_init: bool = False, device: str = "cpu") -> dict:
+    """Draw one problem's inputs (see the module docstring).
 
-    Returns a dict of CPU tensors: x [b,T,H,P], dt [b,T,H], A [H], B, C
+    Returns a dict of tensors: x [b,T,H,P], dt [b,T,H], A [H], B, C
     [b,T,G,N], D [H] and init_state [b,H,P,N] or None.  x/B/C have dtype
-    ``torch.float32`` or ``torch.bfloat16``; the rest are fp32.
+    ``torch.float32`` or ``torch.bfloat16``; the rest are fp32.  With the
+    default ``device="cpu"`` the draws are reproducible across machines (every
+    parity test uses them); another device draws the same distributions with
+    that device's generator, for timing runs that need no oracle.
     """
     if dtype not in ("f32", "bf16"):
         raise ValueError(f"dtype must be 'f32' or 'bf16', got {dtype!r}")
-    g = torch.Generator(device="cpu")
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
-    x = torch.randn(batch, T, H, P, generator=g)
-    B = torch.randn(batch, T, G, N, generator=g) / math.sqrt(N)
-    C = torch.randn(batch, T, G, N, generator=g) / math.sqrt(N)
-    dt = torch.nn.functional.softplus(torch.randn(batch, T, H, generator=g) + DT_BIAS)
-    A = -torch.exp(torch.empty(H).uniform_(math.log(1.0), math.log(16.0), generator=g))
-    D = torch.randn(H, generator=g)
-    init = (0.1 * torch.randn(batch, H, P, N, generator=g)) if with_init else None
+    kw = dict(generator=g, device=device)
+    x = torch.randn(batch, T, H, P, **kw)
+    B = torch.randn(batch, T, G, N, **kw) / math.sqrt(N)
+    C = torch.randn(batch, T, G, N, **kw) / math.sqrt(N)
+    dt = torch.nn.functional.softplus(torch.randn(batch, T, H, **kw) + DT_BIAS)
+    A = -torch.exp(torch.empty(H, device=device).uniform_(math.log(1.0), math.log(16.0), generator=g))
+    D = torch.randn(H, **kw)
+    init = (0.1 * torch.randn(batch, H, P, N, **kw)) if with_init else None
     if dtype == "bf16":
         x, B, C = x.bfloat16(), B.bfloat16(), C.bfloat16()
     return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D, "init_state": init}

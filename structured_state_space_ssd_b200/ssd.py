@@ -23,9 +23,9 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
 
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
-           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_status_string", "ssd_version", "ssd_fwd_no_alloc",
-           "ssd_step", "ssd_gate_norm", "ssd_split_logdecay", "ssd_split_combine", "ssd_split_correct",
-           "ssd_bwd", "ssd_bwd_workspace_bytes")
+           "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_fwd_withhold_publish", "ssd_status_string", "ssd_version",
+           "ssd_fwd_no_alloc", "ssd_fwd_no_alloc_check", "ssd_step", "ssd_gate_norm", "ssd_split_logdecay",
+           "ssd_split_combine", "ssd_split_correct", "ssd_bwd", "ssd_bwd_workspace_bytes")
 
 
 class SSDError(RuntimeError):
@@ -62,6 +62,12 @@ def load():
     lib.ssd_fwd_stage_name.restype = ctypes.c_char_p
     lib.ssd_fwd_check.argtypes = [vp, vp]
     lib.ssd_fwd_check.restype = i
+    lib.ssd_fwd_withhold_publish.argtypes = lib.ssd_fwd.argtypes + [i, i, i, ctypes.c_uint]
+    lib.ssd_fwd_withhold_publish.restype = i
+    lib.ssd_fwd_no_alloc.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, i, i, i, i, i, i, i, vp]
+    lib.ssd_fwd_no_alloc.restype = i
+    lib.ssd_fwd_no_alloc_check.argtypes = [vp]
+    lib.ssd_fwd_no_alloc_check.restype = i
     lib.ssd_status_string.argtypes = [i]
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_version.argtypes = []

@@ -54,6 +54,8 @@ def test_no_alloc_matches_ssd_fwd_on_two_calls_in_a_row(name, cuda_device):
         rc = f(_p(d["x"]), _p(d["dt"]), _p(d["A"]), _p(d["B"]), _p(d["C"]), _p(d["D"]), w.Q, _p(d["init_state"]),
                _p(y), _p(fin), w.batch, w.T, w.H, w.P, w.G, w.N, code, ctypes.c_void_p(stream.cuda_stream))
         assert rc == 0, S.status_string(rc)
+        # the status word lives in the library's scratch: this is how such a caller reads it
+        assert S.load().ssd_fwd_no_alloc_check(ctypes.c_void_p(stream.cuda_stream)) == 0
         torch.cuda.synchronize(cuda_device)
         assert_close(y.float().cpu().numpy(), y_ref, w.dtype, f"{name} y, call {call}")
         assert_close(fin.cpu().numpy(), fin_ref, w.dtype, f"{name} final_state, call {call}")
