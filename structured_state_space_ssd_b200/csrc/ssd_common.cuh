@@ -113,7 +113,7 @@ struct Workspace {
     size_t clear_bytes; // bytes from offset 0 cleared per call
     size_t s_off;       // CUDA-core path: float s[batch][H][nc][Q], inclusive log-decay prefix sums per chunk
     size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
-    size_t ring_off;    // fused path: float ring[batch][H][2][N][P], outgoing states of the last two chunks
+    size_t ring_off;    // fused path: float ring[batch][H][2][P/4][N][4], outgoing states of the last two chunks
     size_t total;
 };
 

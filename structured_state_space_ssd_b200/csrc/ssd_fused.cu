@@ -116,7 +116,6 @@ struct PipeBars {
     uint64_t s_full;     // entering-state tile written, state accumulators read (8 warp arrivals)
     uint64_t mx_done;    // every product of the head done
     uint64_t acc_free;   // accumulators drained (8 warp arrivals)
-    uint64_t ring_done;  // ring stores issued (owner) / ring loads consumed (others), for the publisher
 };
 
 struct Bars {
@@ -248,6 +247,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     __shared__ uint32_t tslot;
     __shared__ int s_unit;
     __shared__ int s_abort, s_broken;
+    // per pipeline, for its publisher: warps that finished an owner's ring stores, and warps that
+    // finished reading another block's state from the ring (8 per head in either case)
+    __shared__ uint32_t s_owned[2], s_copied[2];
     volatile int *abort = &s_abort;
     volatile int *broken = &s_broken;
 
@@ -260,6 +262,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     if (tid == 0) {
         s_abort = 0;
         s_broken = 0;
+        s_owned[0] = s_owned[1] = s_copied[0] = s_copied[1] = 0;
         uint64_t *all = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(Bars) / 8); ++i) mbar_init(&all[i], 1);
         mbar_init(&bars.unit_empty, kSimtWarps + 3);
@@ -269,7 +272,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             mbar_init(&bars.pb[q].m_full, kPipeWarps);
             mbar_init(&bars.pb[q].s_full, kPipeWarps);
             mbar_init(&bars.pb[q].acc_free, kPipeWarps);
-            mbar_init(&bars.pb[q].ring_done, kPipeWarps);
         }
         mbar_fence_init();
     }
@@ -283,15 +285,27 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // Publisher warps: warp 18 + pl makes pipeline pl's hand-offs visible
         // to other CTAs, so that neither the CUDA-core warps nor the issuer
         // wait for a GPU-scope release.  After an owner's ring stores it
-        // releases `ready` (S~_c readable); after another block read S~_{c-1}
-        // it adds one to `cons` (the slot may be rewritten).  The warps'
-        // arrival on ring_done (a CTA-scope release, acquired by this
-        // thread's wait) puts their accesses before this thread's GPU-scope
-        // release, which carries them along (release is cumulative).
+        // releases `ready` (S~_c readable); once another block's copy of
+        // S~_{c-1} has been read it adds one to that slot's `cons` (the
+        // slot may be rewritten).  The warps signal through CTA-scope release
+        // counts in shared memory, acquired here, which puts their stores
+        // before this thread's GPU-scope release (release is cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
-        PipeBars &pb = bars.pb[pl];
-        uint32_t ucnt = 0, rcnt = 0;
+        uint32_t ucnt = 0, ocnt = 0, tcnt = 0;
+        // bounded wait for one of this pipeline's shared-memory counts to reach `target`
+        auto wait_count = [&](const uint32_t *cnt, uint32_t target) {
+            if (ld_acquire_cta_shared(cnt) >= target) return;
+            const uint64_t t0 = global_ns(), limit = *broken ? kBrokenWaitNs : kWaitNs;
+            while (ld_acquire_cta_shared(cnt) < target) {
+                if (global_ns() - t0 > limit) {
+                    atomicExch(p.status, SSD_ERR_TIMEOUT);
+                    *broken = 1;
+                    return;
+                }
+                __nanosleep(32);
+            }
+        };
         for (;;) {
             wait_bar(&bars.unit_full, par(ucnt), p.status, broken);
             ++ucnt;
@@ -301,17 +315,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             if (u >= p.n_units) break;
             const Unit un = decode(u, p);
             if (!un.rows) continue;
-            for (int h = un.h0 + pl; h < un.h1; h += 2, ++rcnt) {
-                wait_bar(&pb.ring_done, par(rcnt), p.status, broken);
-                if (lane == 0) {
-                    const int bh = un.b * sh.H + h;
-                    if (un.owner) {
-                        const bool withheld = (bh == p.withhold_bh && un.c == p.withhold_c);
-                        if (un.c < sh.nc - 1 && !withheld) st_release_gpu(p.ready + bh, un.c + 1);
-                    } else if (un.c > 0) {
-                        // chunk c read slot (c-1) & 1 (chunk 0 read the initial state)
-                        red_release_add_gpu(p.cons + 2 * bh + ((un.c - 1) & 1), 1);
-                    }
+            for (int h = un.h0 + pl; h < un.h1; h += 2) {
+                const int bh = un.b * sh.H + h;
+                if (un.owner) {
+                    wait_count(&s_owned[pl], kPipeWarps * ++ocnt);
+                    const bool withheld = (bh == p.withhold_bh && un.c == p.withhold_c);
+                    if (lane == 0 && un.c < sh.nc - 1 && !withheld) st_release_gpu(p.ready + bh, un.c + 1);
+                } else if (un.c > 0) {
+                    // chunk c has read slot (c-1) & 1 (chunk 0 reads the initial state)
+                    wait_count(&s_copied[pl], kPipeWarps * ++tcnt);
+                    if (lane == 0) red_release_add_gpu(p.cons + 2 * bh + ((un.c - 1) & 1), 1);
                 }
                 __syncwarp();
             }
@@ -411,7 +424,10 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
                 __syncwarp();
             }
-            uint8_t *sXr = (un.r == 1) ? sXhi : sXlo;  // x rows of this block
+            // x rows of this block; the entering-state tile: W for an owner, the unused x buffer for
+            // another block (so that it need not wait for the previous head's y tile to leave W)
+            uint8_t *sXr = (un.r == 1) ? sXhi : sXlo;
+            uint8_t *sE = un.owner ? sW : sXhi;
             bool any = false;
             for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
                 any = true;
@@ -447,7 +463,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     __syncwarp();
                     ++ocnt;
                 }
-                // stage 4 product: Y_inter = C_r E^T into A (E: the entering-state tile [n][p] in W)
+                // stage 4 product: Y_inter = C_r E^T into A (E: the entering-state tile [n][p])
                 wait_bar(&pb.s_full, par(use), p.status, broken);
                 if (!un.owner && use > 0) wait_bar(&pb.acc_free, par(use - 1), p.status, broken);
                 fence_after_sync();
@@ -455,7 +471,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     for (int kk = 0; kk < NK * 4; ++kk) {
                         const int atom = kk >> 2, kin = kk & 3;
                         mma_ss(tA, smem_desc_sw128(smem_u32(sC) + atom * 16384 + kin * 32, 16, 1024),
-                               smem_desc_sw128(smem_u32(sW) + kk * 2048, 16, 1024), idInter, kk > 0);
+                               smem_desc_sw128(smem_u32(sE) + kk * 2048, 16, 1024), idInter, kk > 0);
                     }
                 }
                 __syncwarp();
@@ -482,16 +498,20 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // owns token wtid of the chunk for the prefix sums; for tile work,
         // warp quarter q (warp & 3) owns TMEM lanes 32q..32q+31 (rows of
         // the block, or n of a state) and warpgroup `half` owns columns
-        // 32 half .. 32 half + 31 of every 64-wide tile.
+        // 32 half .. 32 half + 31 of every 64-wide tile.  One thread (`ctl`,
+        // the first of warpgroup 1, whose warp has the least mask work) waits
+        // on other CTAs' flags and issues the y stores.
         // ------------------------------------------------------------------
         const int pl = warp >> 3;
         const int pw = warp & 7;
         const int half = pw >> 2;
         const int quarter = warp & 3;
         const int wtid = pw * 32 + lane;
+        const bool ctl = (wtid == kPipeThreads / 2);
         const int lrow = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const int bar_id = 1 + pl;
+        const int bar_id = 1 + pl;       // the pipeline's 256 threads
+        const int bar_wg1 = 3 + pl;      // its second warpgroup (the one holding ctl)
         PipeBars &pb = bars.pb[pl];
         uint8_t *sXlo = smem + kOffPipe + pl * kPipeBytes;
         uint8_t *sW = sXlo + 16384;
@@ -502,6 +522,25 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         const uint32_t tA = tmem + col_acc_a(pl), tB = tmem + col_acc_b(pl), tM = tmem + col_mask(pl);
         const size_t PN = (size_t)kP * N;
         uint32_t use = 0, ocnt = 0, ucnt = 0, gcnt = 0;
+
+        // stage 0: inclusive prefix sums of dt*A over the chunk, in log2 units, into sJ (and the
+        // mask's column factors exp(s_{i|31} - s_i) <= 1 into sF); every thread of the pipeline
+        auto scan = [&](float dtv, float a) {
+            float v = dtv * (a * kLog2e);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float t = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += t;
+            }
+            if (lane == 31) sTot[pw] = v;
+            named_bar_sync(bar_id, kPipeThreads);
+            float pre = 0.f;
+            for (int w = 0; w < pw; ++w) pre += sTot[w];
+            const float s_mine = pre + v;
+            sJ[wtid] = s_mine;
+            sF[wtid] = ex2(__shfl_sync(0xffffffffu, s_mine, 31) - s_mine);
+            named_bar_sync(bar_id, kPipeThreads);
+        };
         for (;;) {
             wait_bar(&bars.unit_full, par(ucnt), p.status, broken);
             ++ucnt;
@@ -517,50 +556,41 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             const bool own = un.owner;
             const int end = un.len - 1;
             const int j = un.row0 + lrow;  // this thread's row of the chunk
-            // dt of this token, A and D for the pipeline's first head of the unit
             const float *dtp = p.dt + ((size_t)un.b * sh.T + un.t0 + wtid) * sh.H;
-            float dt_cur = (wtid < un.len) ? __ldg(dtp + h) : 0.f;
-            float a_cur = __ldg(p.A + h), d_cur = __ldg(p.D + h);
+            float dt_next = 0.f, a_next = 0.f, d_cur = __ldg(p.D + h);
+            scan((wtid < un.len) ? __ldg(dtp + h) : 0.f, __ldg(p.A + h));
+            // ctl reads `ready` of the pipeline's head early (acquire), so that the wait usually costs
+            // nothing by the time the state is needed (ctl's warp builds only zero mask slabs)
+            int ready_seen = (ctl && un.c > 0) ? ld_acquire_gpu(p.ready + un.b * sh.H + h) : 0;
             bool first_head = true;
             for (; h < un.h1; h += 2, ++use) {
                 const int bh = un.b * sh.H + h;
-                // the y tile of the pipeline's previous head has left W (its store was issued by this
-                // thread); the scan's barrier below publishes that to the pipeline
-                if (wtid == kPipeThreads - 1) bulk_wait_read();
-                // ---- stage 0: inclusive prefix sums of dt*A over the chunk, in log2 units
-                float v = dt_cur * (a_cur * kLog2e);
-                const float Dh = d_cur;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float t = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += t;
-                }
-                if (lane == 31) sTot[pw] = v;
-                named_bar_sync(bar_id, kPipeThreads);
+                const bool has_next = h + 2 < un.h1;
                 // the next head's dt, A and D, in flight while this head is processed
-                if (h + 2 < un.h1) {
-                    dt_cur = (wtid < un.len) ? __ldg(dtp + h + 2) : 0.f;
-                    a_cur = __ldg(p.A + h + 2);
-                    d_cur = __ldg(p.D + h + 2);
+                if (has_next) {
+                    dt_next = (wtid < un.len) ? __ldg(dtp + h + 2) : 0.f;
+                    a_next = __ldg(p.A + h + 2);
                 }
-                float pre = 0.f;
-                for (int w = 0; w < pw; ++w) pre += sTot[w];
-                const float s_mine = pre + v;
-                sJ[wtid] = s_mine;
-                // column factor exp(s_{i|31} - s_i) <= 1 of the mask's blocks below the diagonal
-                sF[wtid] = ex2(__shfl_sync(0xffffffffu, s_mine, 31) - s_mine);
-                named_bar_sync(bar_id, kPipeThreads);
+                const float Dh = d_cur;
+                if (has_next) d_cur = __ldg(p.D + h + 2);
                 const float s_end = sJ[end];
                 const float s_ref = (un.r == 1) ? sJ[kRows - 1] : 0.f;  // s_{r-1}
                 const float sj = sJ[j];
+                const float ej = ex2(sj - s_ref);
+                const bool writes_ring = own && un.c < sh.nc - 1;
 
                 // ---- owner: rows scaled by their decay to the state's end (stage 2 operand)
                 if (own) {
                     wait_bar(&pb.x_full, par(use), p.status, broken);
                     if (un.r == 1) {
-                        // rows 0..127 in place (to row 127: S_pre), rows 128..255 into W (to the end)
+                        // rows 0..127 in place (to row 127: S_pre, warpgroup 0), rows 128..255 into W
+                        // (to the end, warpgroup 1, once the previous y tile has left W)
                         const int row = wtid;
                         const bool lo = row < kRows;
+                        if (!lo) {
+                            if (ctl) bulk_wait_read();
+                            named_bar_sync(bar_wg1, kPipeThreads / 2);
+                        }
                         const float w = ex2((lo ? s_ref : s_end) - sJ[row]);
                         const uint8_t *src = (lo ? sXlo : sXhi);
                         uint8_t *dst = lo ? sXlo : sW;
@@ -572,6 +602,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         for (int k = 0; k < 8; ++k) sts128(dst + swz(rr, k), scale_bf16x8(xv[k], w));
                     } else {
                         // the only block: rows 0..127 into W (to the end); x stays unscaled for M X
+                        if (ctl) bulk_wait_read();
+                        named_bar_sync(bar_id, kPipeThreads);
                         const int rr = wtid & (kRows - 1), k0 = (wtid >> 7) * 4;
                         const float w = ex2(s_end - sJ[rr]);
                         uint4 xv[4];
@@ -586,45 +618,44 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
 
                 // ---- stage 1 mask M[j][i] = exp(s_j - s_i) G[j][i] for i <= j (+ D_h at i = j), bf16 in
-                // TMEM.  Warpgroup 0 builds each row's diagonal 32-column slab (one exponential per
-                // element), warpgroup 1 the slabs below it (row factor x column factor, both <= 1) and
-                // the zero slabs above it.
+                // TMEM, in 32-column slabs: below the diagonal slab a row factor times a column factor
+                // (both <= 1), in it one exponential per element (about three times the work), above
+                // it zeros.  Warpgroup 0 takes the diagonal slab, warpgroup 1 the other three.
+                // an owner's slot count, read (acquire) before the mask for the same reason
+                int cons_seen = 0;
+                if (own && ctl && writes_ring && p.halves == 2 && un.c >= 2)
+                    cons_seen = ld_acquire_gpu(p.cons + 2 * bh + (un.c & 1));
                 if (first_head) wait_bar(&bars.g_done, par(gphase), p.status, broken);
                 fence_after_sync();
                 {
                     const int dq = quarter;  // diagonal slab of this warp's rows
-                    if (half == 0) {
-                        uint32_t g[32], o[16];
-                        tmem_ld16(tmem + kColG + dq * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
-                        tmem_ld16(tmem + kColG + dq * 32 + 16 + lane_base,
-                                  *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
-                        tmem_wait_ld();
-                        const float2 *sc = reinterpret_cast<const float2 *>(sJ + un.row0 + dq * 32);
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const float2 si = sc[q];
-                            float a = (2 * q <= lane) ? __uint_as_float(g[2 * q]) * ex2(sj - si.x) : 0.f;
-                            float b = (2 * q + 1 <= lane) ? __uint_as_float(g[2 * q + 1]) * ex2(sj - si.y) : 0.f;
-                            if (2 * q == lane) a += Dh;
-                            if (2 * q + 1 == lane) b += Dh;
-                            o[q] = pack_bf16x2(a, b);
-                        }
-                        tmem_st16(tM + dq * 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-                    } else {
 #pragma unroll 1
-                        for (int sl = 0; sl < 4; ++sl) {
-                            if (sl == dq) continue;
-                            uint32_t o[16];
-                            if (sl > dq) {
+                    for (int sl = 0; sl < 4; ++sl) {
+                        const bool mine = (half == 0) ? (sl == dq) : (sl != dq);
+                        if (!mine) continue;
+                        uint32_t o[16];
+                        if (sl > dq) {
 #pragma unroll
-                                for (int q = 0; q < 16; ++q) o[q] = 0u;
+                            for (int q = 0; q < 16; ++q) o[q] = 0u;
+                        } else {
+                            uint32_t g[32];
+                            tmem_ld16(tmem + kColG + sl * 32 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
+                            tmem_ld16(tmem + kColG + sl * 32 + 16 + lane_base,
+                                      *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
+                            tmem_wait_ld();
+                            if (sl == dq) {
+                                const float2 *sc = reinterpret_cast<const float2 *>(sJ + un.row0 + dq * 32);
+#pragma unroll
+                                for (int q = 0; q < 16; ++q) {
+                                    const float2 si = sc[q];
+                                    float a = (2 * q <= lane) ? __uint_as_float(g[2 * q]) * ex2(sj - si.x) : 0.f;
+                                    float b =
+                                        (2 * q + 1 <= lane) ? __uint_as_float(g[2 * q + 1]) * ex2(sj - si.y) : 0.f;
+                                    if (2 * q == lane) a += Dh;
+                                    if (2 * q + 1 == lane) b += Dh;
+                                    o[q] = pack_bf16x2(a, b);
+                                }
                             } else {
-                                uint32_t g[32];
-                                tmem_ld16(tmem + kColG + sl * 32 + lane_base,
-                                          *reinterpret_cast<uint32_t(*)[16]>(&g[0]));
-                                tmem_ld16(tmem + kColG + sl * 32 + 16 + lane_base,
-                                          *reinterpret_cast<uint32_t(*)[16]>(&g[16]));
-                                tmem_wait_ld();
                                 const int i0 = un.row0 + sl * 32;
                                 const float rf = ex2(sj - sJ[i0 + 31]);
                                 const float2 rr = make_float2(rf, rf);
@@ -643,8 +674,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                                     o[2 * q + 1] = pack_bf16x2(m1.x, m1.y);
                                 }
                             }
-                            tmem_st16(tM + sl * 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
                         }
+                        tmem_st16(tM + sl * 16 + lane_base, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
                     }
                     tmem_wait_st();
                     fence_before_sync();
@@ -652,23 +683,24 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (lane == 0) mbar_arrive(&pb.m_full);
                 }
                 first_head = false;
+                // the previous y tile has left W before any thread writes W again (the next barrier of
+                // the pipeline publishes this)
+                if (ctl) bulk_wait_read();
 
-                // ---- stage 3: the state entering the chunk (published by the owner of chunk c-1);
-                // an owner that writes the ring also waits until the slot it overwrites (S~_{c-2})
-                // has been read by the other block of chunk c-1.  Reads are counted per slot: the
-                // non-owners of chunks 1, 3, 5, ... read slot 0 and those of chunks 2, 4, ... slot 1,
-                // so slot c & 1 has had c / 2 reads once chunk c-1's is in (a single count could be
-                // reached early by chunk c's own reader, which reads the other slot).
-                const bool writes_ring = own && un.c < sh.nc - 1;
-                if (wtid == 0) {
-                    if (un.c > 0) wait_flag(p.ready + bh, un.c, p.flag_polls, abort, p.status);
-                    if (writes_ring && p.halves == 2 && un.c >= 2)
+                // ---- stage 3: the state entering the block: S~_{c-1} from the ring (published by the
+                // owner of chunk c-1) or the initial state.  A ring slot is overwritten only once the
+                // other block of the chunk before has read it: the non-owners of chunks 1, 3, 5, ... read
+                // slot 0, those of 2, 4, ... slot 1, so slot c & 1 has had c / 2 reads once chunk c-1's
+                // is in (a single count could be reached early by chunk c's own reader, which reads the
+                // other slot).
+                const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
+                const bool nv = n < N;
+                if (ctl) {
+                    if (un.c > 0 && ready_seen < un.c) wait_flag(p.ready + bh, un.c, p.flag_polls, abort, p.status);
+                    if (writes_ring && p.halves == 2 && un.c >= 2 && cons_seen < un.c / 2)
                         wait_flag(p.cons + 2 * bh + (un.c & 1), un.c / 2, p.flag_polls, abort, p.status);
                 }
                 named_bar_sync(bar_id, kPipeThreads);
-                // this thread's 32 entries of S~_{c-1}: state row n = lrow, p in [32 half, 32 half + 32)
-                const int n = lrow;
-                const bool nv = n < N;
                 float old[32];
                 if (un.c == 0) {
                     const float *src = p.init ? p.init + (size_t)bh * PN + (size_t)(half * 32) * N + n : nullptr;
@@ -679,13 +711,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * 2 + ((un.c - 1) & 1)) * PN);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 t = nv ? __ldcg(src + ring_quad(N, n, half * 8 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        const float4 t =
+                            nv ? __ldcg(src + ring_quad(N, n, half * 8 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
                         old[4 * q] = t.x;
                         old[4 * q + 1] = t.y;
                         old[4 * q + 2] = t.z;
                         old[4 * q + 3] = t.w;
                     }
                 }
+                uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
                 if (own) {
                     wait_bar(&pb.d_done, par(ocnt), p.status, broken);
                     ++ocnt;
@@ -699,12 +733,12 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             tmem_ld16(tA + half * 32 + q0 + lane_base, t);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int q = 0; q < 16; ++q) old[q0 + q] = fmaf(e_start, old[q0 + q], __uint_as_float(t[q]));
+                            for (int q = 0; q < 16; ++q)
+                                old[q0 + q] = fmaf(e_start, old[q0 + q], __uint_as_float(t[q]));
                         }
                     }
                 }
-                // E in bf16 into row n of the tile [n][p] (128-byte swizzled), the B operand of stage 4;
-                // handed to the issuer before the outgoing state is formed
+                // E in bf16 into row n of the tile (128-byte swizzled)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     uint4 t;
@@ -713,19 +747,19 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     t.z = pack_bf16x2(old[8 * k + 4], old[8 * k + 5]);
                     t.w = pack_bf16x2(old[8 * k + 6], old[8 * k + 7]);
                     if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
-                    sts128(sW + swz(n, half * 4 + k), t);
+                    sts128(sE + swz(n, half * 4 + k), t);
                 }
                 fence_view_async_shared();
                 if (!own) {
-                    // the ring entries are in registers: the publisher may count the slot as read
                     __syncwarp();
                     if (lane == 0) {
-                        mbar_arrive(&pb.ring_done);
                         mbar_arrive(&pb.s_full);
+                        // the ring entries are consumed: the publisher may count the slot as read
+                        if (un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
                     }
                 } else {
-                    // S~_c = exp(s_end - s_{r-1}) E + S_own, to the ring or to final_state.  S_own is read
-                    // from TMEM before s_full, after which the issuer overwrites that accumulator.
+                    // S~_c = exp(s_end - s_{r-1}) E + S_own.  S_own is read from TMEM before s_full,
+                    // after which the issuer overwrites that accumulator.
                     const float e_rest = ex2(s_end - s_ref);
 #pragma unroll
                     for (int q0 = 0; q0 < 32; q0 += 16) {
@@ -738,28 +772,32 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.s_full);
-                    if (nv && writes_ring) {
+                    if (writes_ring) {
                         float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * 2 + (un.c & 1)) * PN);
+                        if (nv) {
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            __stcg(dst + ring_quad(N, n, half * 8 + q),
-                                   make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                            for (int q = 0; q < 8; ++q)
+                                __stcg(dst + ring_quad(N, n, half * 8 + q),
+                                       make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                        }
                     } else if (nv && p.fin) {
                         float *fin = p.fin + (size_t)bh * PN + (size_t)(half * 32) * N + n;
 #pragma unroll
                         for (int q = 0; q < 32; ++q) fin[(size_t)q * N] = old[q];
                     }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.ring_done);  // the publisher releases the stores
+                    if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
                 }
 
+                // the next head's prefix sums, while this head's products run
+                if (has_next) scan(dt_next, a_next);
+
                 // ---- stages 4-5: y_j = exp(s_j - s_{r-1}) Y_inter + Y_intra (the D skip is in the mask),
-                // staged as bf16 in W (128-byte swizzled [j][p]; its state tile has been consumed) and
-                // written by one TMA store (rows past T are clipped)
+                // staged as bf16 in W (128-byte swizzled [j][p]) and written by one TMA store (rows
+                // past T are clipped)
                 wait_bar(&pb.mx_done, par(use), p.status, broken);
                 fence_after_sync();
                 {
-                    const float ej = ex2(sj - s_ref);
 #pragma unroll
                     for (int q0 = 0; q0 < 32; q0 += 16) {
                         uint32_t a[16], b[16];
@@ -769,9 +807,10 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         uint32_t o[8];
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            const float2 r = fma_f32x2(make_float2(ej, ej),
-                                                       make_float2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])),
-                                                       make_float2(__uint_as_float(b[2 * q]), __uint_as_float(b[2 * q + 1])));
+                            const float2 r =
+                                fma_f32x2(make_float2(ej, ej),
+                                          make_float2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])),
+                                          make_float2(__uint_as_float(b[2 * q]), __uint_as_float(b[2 * q + 1])));
                             o[q] = pack_bf16x2(r.x, r.y);
                         }
                         const int ch = half * 4 + q0 / 8;
@@ -783,14 +822,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (lane == 0) mbar_arrive(&pb.acc_free);
                     fence_view_async_shared();
                     named_bar_sync(bar_id, kPipeThreads);
-                    if (wtid == kPipeThreads - 1) {
+                    if (ctl) {
                         tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
+                        if (has_next && un.c > 0) ready_seen = ld_acquire_gpu(p.ready + bh + 2);
                     }
                 }
             }
         }
-        if (wtid == kPipeThreads - 1) bulk_wait_all();
+        if (ctl) bulk_wait_all();
     }
     fence_before_sync();
     __syncthreads();

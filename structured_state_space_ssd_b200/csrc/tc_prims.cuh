@@ -296,6 +296,25 @@ __device__ __forceinline__ void red_release_add_gpu(int *p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// CTA-scope counters in shared memory (a monotonic count instead of an
+// mbarrier phase, so a waiter that falls behind by several steps still reads
+// an unambiguous value).
+__device__ __forceinline__ void red_release_cta_shared_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_cta_shared(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+// Orders this thread's generic-proxy accesses to global memory with its later
+// async-proxy ones (a bulk copy reading data another CTA published).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
     int v;
     asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

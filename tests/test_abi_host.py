@@ -55,7 +55,8 @@ def test_workspace_bytes(lib):
     w = f(4, 2048, 80, 64, 1, 128, 256, 1)      # fused tensor-core path: flags + the two-slot state ring
     assert w % 256 == 0
     nc = 8
-    assert 4 * 80 * 2 * 64 * 128 * 4 <= w < 4 * 80 * 2 * 64 * 128 * 4 + (1 << 16)
+    ring = 4 * 80 * 2 * 64 * 128 * 4
+    assert ring <= w < ring + (1 << 16)
     w32 = f(4, 2048, 80, 64, 1, 128, 256, 0)    # CUDA-core path: every chunk state
     assert w32 >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
     assert f(0, 2048, 80, 64, 1, 128, 256, 1) == 0      # batch < 1
