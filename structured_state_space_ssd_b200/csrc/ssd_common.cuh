@@ -81,6 +81,9 @@ __device__ __forceinline__ void stage_rows(float *dst, int dld, const T *src, si
     }
 }
 
+// Slots per (batch, head) of the fused path's ring of chunk states.
+constexpr int kRingSlots = 3;
+
 // Problem shape as every kernel sees it.
 struct Shape {
     int batch, T, H, P, G, N, Q, nc;
@@ -109,11 +112,11 @@ struct Workspace {
     size_t status_off;  // int status word
     size_t counter_off; // int unit counter (fused path)
     size_t ready_off;   // int ready[batch * H] (fused path)
-    size_t cons_off;    // int cons[batch * H][2] (fused path)
+    size_t cons_off;    // int cons[batch * H][kRingSlots] (fused path)
     size_t clear_bytes; // bytes from offset 0 cleared per call
     size_t s_off;       // CUDA-core path: float s[batch][H][nc][Q], inclusive log-decay prefix sums per chunk
     size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
-    size_t ring_off;    // fused path: float ring[batch][H][2][P/4][N][4], outgoing states of the last two chunks
+    size_t ring_off;    // fused path: float ring[batch][H][kRingSlots][P/4][N][4], outgoing states of recent chunks
     size_t total;
 };
 
@@ -136,14 +139,14 @@ inline Workspace workspace_layout(const Shape &s, Path path) {
     w.ready_off = off;
     off += sizeof(int) * bh;
     w.cons_off = off;
-    off += sizeof(int) * bh * 2;
+    off += sizeof(int) * bh * kRingSlots;
     off = align256(off);
     w.clear_bytes = (path == kPathFused) ? off : 256;
     w.s_off = off;
     if (path != kPathFused) off = align256(off + sizeof(float) * bh * s.nc * s.Q);
     w.state_off = w.ring_off = off;
     if (path == kPathFused)
-        off = align256(off + sizeof(float) * bh * 2 * s.P * s.N);
+        off = align256(off + sizeof(float) * bh * kRingSlots * s.P * s.N);
     else
         off = align256(off + sizeof(float) * (size_t)s.batch * s.nc * s.H * s.P * s.N);
     w.total = off;

@@ -23,12 +23,12 @@
 //   chunk state     S~_c = exp(s_end - s_{r-1}) E + B_{>=r}^T (exp(s_end - s_i) x_i)   (last block)
 //
 //  * A work unit is (chunk c, batch b, group g, block of heads, block r).
-//    Units are handed out by an atomic counter in chunk-major order, so a
-//    unit only ever waits for units handed out before it: there is no
-//    deadlock however many CTAs are resident.
+//    Units are handed out by an atomic counter in an order (see decode) in
+//    which a unit only ever waits for units handed out before it: there is
+//    no deadlock however many CTAs are resident.
 //  * The last block of a chunk owns the chunk state: it waits for S~_{c-1}
 //    (published by the owner of chunk c-1), forms E and S~_c, and writes
-//    S~_c into a two-slot fp32 ring (or final_state after the last chunk).
+//    S~_c into a three-slot fp32 ring (or final_state after the last chunk).
 //    Other blocks only read S~_{c-1} and count themselves as done with it;
 //    an owner overwrites a slot only after every reader of the chunk before
 //    has read it.  Every wait on another CTA is bounded: on expiry the
@@ -82,6 +82,8 @@ constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units)
 constexpr uint32_t kSmemBytes = kOffAux + 2 * kAuxFloats * 4 + 1024;
 
 constexpr uint32_t kDefaultFlagPolls = 1u << 22;
+// Ring slots per sequence: chunk c's state goes to slot c % kSlots (see the hand-out order in decode).
+constexpr int kSlots = kRingSlots;
 
 struct Params {
     Shape sh;
@@ -90,9 +92,9 @@ struct Params {
     const float *D;     // [H]
     const float *init;  // [b][H][P][N] or null
     float *fin;         // [b][H][P][N] or null
-    float *ring;        // [b][H][2][P/4][N][4]: outgoing states of the last two chunks (see ring_quad)
+    float *ring;        // [b][H][kSlots][P/4][N][4]: outgoing states of recent chunks (see ring_quad)
     int *ready;         // [b*H]: chunks whose outgoing state is published
-    int *cons;          // [b*H][2]: per ring slot, non-owner blocks that have read it (a count)
+    int *cons;          // [b*H][kSlots]: per ring slot, non-owner blocks that have read it (a count)
     int *counter;       // unit dispenser
     int *status;
     __nv_bfloat16 *y;
@@ -100,6 +102,7 @@ struct Params {
     int halves;         // Q / 128
     int heads_per_unit;
     int blocks_per_group;
+    int units_per_role;  // units of one row block of one chunk: batch * G * blocks_per_group
     int n_units;
     uint32_t flag_polls;  // bound of each wait on another CTA's flag
     int withhold_bh;      // test hook: the owner of (b*H + h, chunk) below never publishes (-1: none)
@@ -133,17 +136,42 @@ struct Unit {
     bool owner;  // the chunk's last block with rows: it carries the chunk state
 };
 
+// Hand-out order.  With one row block per chunk (Q = 128) units go chunk by chunk.  With two, the
+// block owning chunk c's state (the last one) is handed out one step ahead of chunk c-1's other block:
+//   [owners of chunk 0] [owners of 1, others of 0] [owners of 2, others of 1] ... [others of nc-1]
+// so that the owners, which carry the inter-chunk chain, run ahead of the blocks that wait for it.
+// Every unit still waits only for units handed out before it: an owner waits for the owner of the
+// chunk before (one step earlier) and for the other block of chunk c-2 to have read the ring slot it
+// overwrites (one step earlier too, with three slots); another block waits for the owner of the chunk
+// before (two steps earlier).  So there is no deadlock however many CTAs are resident.
 __device__ __forceinline__ Unit decode(int u, const Params &p) {
     Unit un;
-    int rem = u;
-    un.r = rem % p.halves;
-    rem /= p.halves;
-    const int hb = rem % p.blocks_per_group;
-    rem /= p.blocks_per_group;
-    un.g = rem % p.sh.G;
-    rem /= p.sh.G;
-    un.b = rem % p.sh.batch;
-    un.c = rem / p.sh.batch;
+    const int M = p.units_per_role;
+    int idx;
+    if (p.halves == 1) {
+        un.r = 0;
+        un.c = u / M;
+        idx = u % M;
+    } else if (u < M) {
+        un.r = 1;
+        un.c = 0;
+        idx = u;
+    } else {
+        const int v = u - M, t = v / (2 * M), j = v % (2 * M);
+        if (t < p.sh.nc - 1 && j < M) {
+            un.r = 1;
+            un.c = t + 1;
+            idx = j;
+        } else {
+            un.r = 0;
+            un.c = t;
+            idx = (t < p.sh.nc - 1) ? j - M : j;
+        }
+    }
+    const int hb = idx % p.blocks_per_group;
+    idx /= p.blocks_per_group;
+    un.g = idx % p.sh.G;
+    un.b = idx / p.sh.G;
     un.h0 = un.g * p.sh.heads_per_group + hb * p.heads_per_unit;
     un.h1 = min(un.h0 + p.heads_per_unit, (un.g + 1) * p.sh.heads_per_group);
     un.t0 = un.c * p.sh.Q;
@@ -324,7 +352,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 } else if (un.c > 0) {
                     // chunk c has read slot (c-1) & 1 (chunk 0 reads the initial state)
                     wait_count(&s_copied[pl], kPipeWarps * ++tcnt);
-                    if (lane == 0) red_release_add_gpu(p.cons + 2 * bh + ((un.c - 1) & 1), 1);
+                    if (lane == 0) red_release_add_gpu(p.cons + kSlots * bh + (un.c - 1) % kSlots, 1);
                 }
                 __syncwarp();
             }
@@ -624,7 +652,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 // an owner's slot count, read (acquire) before the mask for the same reason
                 int cons_seen = 0;
                 if (own && ctl && writes_ring && p.halves == 2 && un.c >= 2)
-                    cons_seen = ld_acquire_gpu(p.cons + 2 * bh + (un.c & 1));
+                    cons_seen = ld_acquire_gpu(p.cons + kSlots * bh + un.c % kSlots);
                 if (first_head) wait_bar(&bars.g_done, par(gphase), p.status, broken);
                 fence_after_sync();
                 {
@@ -688,17 +716,18 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 if (ctl) bulk_wait_read();
 
                 // ---- stage 3: the state entering the block: S~_{c-1} from the ring (published by the
-                // owner of chunk c-1) or the initial state.  A ring slot is overwritten only once the
-                // other block of the chunk before has read it: the non-owners of chunks 1, 3, 5, ... read
-                // slot 0, those of 2, 4, ... slot 1, so slot c & 1 has had c / 2 reads once chunk c-1's
-                // is in (a single count could be reached early by chunk c's own reader, which reads the
-                // other slot).
+                // owner of chunk c-1) or the initial state.  Chunk c's state goes to slot c % kSlots,
+                // which held chunk c - kSlots's, read by the other block of chunk c - kSlots + 1; the
+                // other blocks of chunks k >= 1 read slot (k - 1) % kSlots, so that slot has had
+                // c / kSlots reads once that one is in, and no later reader can add to the count before
+                // this owner publishes.
                 const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
                 const bool nv = n < N;
                 if (ctl) {
                     if (un.c > 0 && ready_seen < un.c) wait_flag(p.ready + bh, un.c, p.flag_polls, abort, p.status);
-                    if (writes_ring && p.halves == 2 && un.c >= 2 && cons_seen < un.c / 2)
-                        wait_flag(p.cons + 2 * bh + (un.c & 1), un.c / 2, p.flag_polls, abort, p.status);
+                    if (writes_ring && p.halves == 2 && un.c >= kSlots && cons_seen < un.c / kSlots)
+                        wait_flag(p.cons + kSlots * bh + un.c % kSlots, un.c / kSlots, p.flag_polls, abort,
+                                  p.status);
                 }
                 named_bar_sync(bar_id, kPipeThreads);
                 float old[32];
@@ -708,7 +737,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     for (int q = 0; q < 32; ++q) old[q] = (src && nv) ? __ldg(src + (size_t)q * N) : 0.f;
                 } else {
                     const float4 *src =
-                        reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * 2 + ((un.c - 1) & 1)) * PN);
+                        reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * kSlots + (un.c - 1) % kSlots) * PN);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 t =
@@ -773,7 +802,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pb.s_full);
                     if (writes_ring) {
-                        float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * 2 + (un.c & 1)) * PN);
+                        float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * kSlots + un.c % kSlots) * PN);
                         if (nv) {
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
@@ -892,7 +921,8 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.halves = sh.Q / kRows;
     p.heads_per_unit = heads_per_unit(sh);
     p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
-    p.n_units = sh.nc * sh.batch * sh.G * p.blocks_per_group * p.halves;
+    p.units_per_role = sh.batch * sh.G * p.blocks_per_group;
+    p.n_units = sh.nc * p.units_per_role * p.halves;
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;

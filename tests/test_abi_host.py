@@ -55,7 +55,7 @@ def test_workspace_bytes(lib):
     w = f(4, 2048, 80, 64, 1, 128, 256, 1)      # fused tensor-core path: flags + the two-slot state ring
     assert w % 256 == 0
     nc = 8
-    ring = 4 * 80 * 2 * 64 * 128 * 4
+    ring = 4 * 80 * 3 * 64 * 128 * 4   # three slots per (batch, head)
     assert ring <= w < ring + (1 << 16)
     w32 = f(4, 2048, 80, 64, 1, 128, 256, 0)    # CUDA-core path: every chunk state
     assert w32 >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
