@@ -18,8 +18,8 @@ cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D
 bool fused_supported(const Shape &sh, int dtype);
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
-                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
-                             const FusedDebug *dbg, cudaStream_t st);
+                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
+                             const Shape &full, int n_half, const FusedDebug *dbg, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -68,10 +68,11 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 const char *const kSimtStages[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan"};
 const char *const kFusedStages[] = {"ssd_fused"};
+const char *const kFusedStages256[] = {"ssd_fused_n0_127", "ssd_fused_n128_255"};
 
 int launch_count(const Shape &sh, ssd::Path path) {
     if (sh.T == 0) return 0;
-    return path == ssd::kPathFused ? 1 : 4;
+    return path == ssd::kPathFused ? ssd::fused_passes(sh) : 4;
 }
 
 // Optional event marks: ev[0] at the start of the call (before the workspace
@@ -102,12 +103,17 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
               const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
               const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg) {
     if (!mk.mark(1, st)) return SSD_ERR_CUDA;
-    if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, reinterpret_cast<float *>(ws + w.ring_off),
-                              reinterpret_cast<int *>(ws + w.ready_off), reinterpret_cast<int *>(ws + w.cons_off),
-                              reinterpret_cast<int *>(ws + w.counter_off), reinterpret_cast<int *>(ws + w.status_off),
-                              y, sh, dbg, st) != cudaSuccess ||
-        !mk.mark(2, st))
-        return SSD_ERR_CUDA;
+    const int passes = ssd::fused_passes(sh);
+    const size_t stride = w.total / passes;  // one pass's counter, flags and ring
+    for (int k = 0; k < passes; ++k) {
+        char *pw = ws + k * stride;
+        if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, reinterpret_cast<float *>(pw + w.ring_off),
+                                  reinterpret_cast<int *>(pw + w.ready_off), reinterpret_cast<int *>(pw + w.cons_off),
+                                  reinterpret_cast<int *>(pw + w.counter_off),
+                                  reinterpret_cast<int *>(ws + w.status_off), y, sh, k, dbg, st) != cudaSuccess ||
+            !mk.mark(2 + k, st))
+            return SSD_ERR_CUDA;
+    }
     return SSD_OK;
 }
 
@@ -140,6 +146,9 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     char *ws = static_cast<char *>(workspace);
     if (!mk.mark(0, st)) return SSD_ERR_CUDA;
     if (cudaMemsetAsync(ws, 0, w.clear_bytes, st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (path == ssd::kPathFused && ssd::fused_passes(sh) == 2 &&
+        cudaMemsetAsync(ws + w.total / 2, 0, w.clear_bytes, st) != cudaSuccess)
+        return SSD_ERR_CUDA;
     if (T == 0) {
         if (!mk.mark(1, st)) return SSD_ERR_CUDA;
         if (!final_state) return SSD_OK;
@@ -182,7 +191,8 @@ const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int
     if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return nullptr;
     const ssd::Path path = choose_path(sh, dtype);
     if (i < 0 || i >= launch_count(sh, path)) return nullptr;
-    return path == ssd::kPathFused ? kFusedStages[i] : kSimtStages[i];
+    if (path != ssd::kPathFused) return kSimtStages[i];
+    return ssd::fused_passes(sh) == 2 ? kFusedStages256[i] : kFusedStages[i];
 }
 
 int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,

@@ -130,7 +130,22 @@ int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, S
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// The fused path runs a 256-wide state as two launches over halves of 128, each with its own
+// counter, flags and ring (one after the other in the workspace); the status word is shared.
+inline int fused_passes(const Shape &s) { return s.N > 128 ? 2 : 1; }
+
+inline Workspace workspace_layout_one(const Shape &s, Path path);
+
 inline Workspace workspace_layout(const Shape &s, Path path) {
+    if (path != kPathFused || fused_passes(s) == 1) return workspace_layout_one(s, path);
+    Shape h = s;
+    h.N = 128;
+    Workspace w = workspace_layout_one(h, path);
+    w.total *= 2;  // pass k's counter, flags and ring sit at k * (total / 2)
+    return w;
+}
+
+inline Workspace workspace_layout_one(const Shape &s, Path path) {
     Workspace w;
     const size_t bh = (size_t)s.batch * s.H;
     w.status_off = 0;

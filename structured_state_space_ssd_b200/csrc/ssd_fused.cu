@@ -107,6 +107,12 @@ struct Params {
     uint32_t flag_polls;  // bound of each wait on another CTA's flag
     int withhold_bh;      // test hook: the owner of (b*H + h, chunk) below never publishes (-1: none)
     int withhold_c;
+    // A state dimension of 256 runs as two launches over n = 0..127 and 128..255 (the state splits
+    // into independent halves, y into the sum of their contributions): sh.N is the half's size,
+    // state_ld the caller's n stride, n_off the half's first n; the second launch has no D skip
+    // (D == null) and adds its result to the y the first one wrote (kernel template argument).
+    int state_ld;
+    int n_off;
 };
 
 // One head pipeline.  Barriers signalled once per head of the pipeline are
@@ -263,6 +269,8 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
 
 using namespace fz;
 
+// kAccum: the second half of a 256-wide state, which adds its y to the first half's.
+template <bool kAccum>
 __global__ void __launch_bounds__(fz::kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                      const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY,
@@ -585,7 +593,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             const int end = un.len - 1;
             const int j = un.row0 + lrow;  // this thread's row of the chunk
             const float *dtp = p.dt + ((size_t)un.b * sh.T + un.t0 + wtid) * sh.H;
-            float dt_next = 0.f, a_next = 0.f, d_cur = __ldg(p.D + h);
+            float dt_next = 0.f, a_next = 0.f, d_cur = p.D ? __ldg(p.D + h) : 0.f;
             scan((wtid < un.len) ? __ldg(dtp + h) : 0.f, __ldg(p.A + h));
             // ctl reads `ready` of the pipeline's head early (acquire), so that the wait usually costs
             // nothing by the time the state is needed (ctl's warp builds only zero mask slabs)
@@ -600,7 +608,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     a_next = __ldg(p.A + h + 2);
                 }
                 const float Dh = d_cur;
-                if (has_next) d_cur = __ldg(p.D + h + 2);
+                if (has_next) d_cur = p.D ? __ldg(p.D + h + 2) : 0.f;
                 const float s_end = sJ[end];
                 const float s_ref = (un.r == 1) ? sJ[kRows - 1] : 0.f;  // s_{r-1}
                 const float sj = sJ[j];
@@ -732,9 +740,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 named_bar_sync(bar_id, kPipeThreads);
                 float old[32];
                 if (un.c == 0) {
-                    const float *src = p.init ? p.init + (size_t)bh * PN + (size_t)(half * 32) * N + n : nullptr;
+                    const size_t ld = p.state_ld;
+                    const float *src =
+                        p.init ? p.init + ((size_t)bh * kP + half * 32) * ld + p.n_off + n : nullptr;
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) old[q] = (src && nv) ? __ldg(src + (size_t)q * N) : 0.f;
+                    for (int q = 0; q < 32; ++q) old[q] = (src && nv) ? __ldg(src + (size_t)q * ld) : 0.f;
                 } else {
                     const float4 *src =
                         reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * kSlots + (un.c - 1) % kSlots) * PN);
@@ -810,9 +820,10 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                                        make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
                         }
                     } else if (nv && p.fin) {
-                        float *fin = p.fin + (size_t)bh * PN + (size_t)(half * 32) * N + n;
+                        const size_t ld = p.state_ld;
+                        float *fin = p.fin + ((size_t)bh * kP + half * 32) * ld + p.n_off + n;
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) fin[(size_t)q * N] = old[q];
+                        for (int q = 0; q < 32; ++q) fin[(size_t)q * ld] = old[q];
                     }
                     __syncwarp();
                     if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
@@ -823,7 +834,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 
                 // ---- stages 4-5: y_j = exp(s_j - s_{r-1}) Y_inter + Y_intra (the D skip is in the mask),
                 // staged as bf16 in W (128-byte swizzled [j][p]) and written by one TMA store (rows
-                // past T are clipped)
+                // past T are clipped).  The second half of a 256-wide state adds the first half's y.
+                uint4 yprev[4];
+                if (kAccum) {
+                    const bool jv = j < un.len;
+                    const uint4 *yp = reinterpret_cast<const uint4 *>(
+                        p.y + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP + half * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yprev[q] = jv ? __ldg(yp + q) : make_uint4(0u, 0u, 0u, 0u);
+                }
                 wait_bar(&pb.mx_done, par(use), p.status, broken);
                 fence_after_sync();
                 {
@@ -836,10 +855,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         uint32_t o[8];
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            const float2 r =
+                            float2 r =
                                 fma_f32x2(make_float2(ej, ej),
                                           make_float2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])),
                                           make_float2(__uint_as_float(b[2 * q]), __uint_as_float(b[2 * q + 1])));
+                            if (kAccum) {
+                                const uint4 &v = yprev[q0 / 8 + q / 4];
+                                const uint32_t w = (q & 3) == 0 ? v.x : (q & 3) == 1 ? v.y : (q & 3) == 2 ? v.z : v.w;
+                                r.x += bf16lo(w);
+                                r.y += bf16hi(w);
+                            }
                             o[q] = pack_bf16x2(r.x, r.y);
                         }
                         const int ch = half * 4 + q0 / 8;
@@ -870,7 +895,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 bool fused_supported(const Shape &sh, int dtype) {
-    return dtype == SSD_BF16 && sh.P == kP && sh.N >= 16 && sh.N <= 128 && sh.N % 16 == 0 &&
+    return dtype == SSD_BF16 && sh.P == kP && ((sh.N >= 16 && sh.N <= 128 && sh.N % 16 == 0) || sh.N == 256) &&
            (sh.Q == 128 || sh.Q == 256);
 }
 
@@ -890,13 +915,21 @@ static int heads_per_unit(const Shape &sh) {
     return (hpg + blocks - 1) / blocks;
 }
 
+// Launches the fused kernel for state columns [n_half * 128, ...) of the problem `full` (all of them
+// when full.N <= 128).  The second half of a 256-wide state adds to the y of the first.
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
-                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y, const Shape &sh,
-                             const FusedDebug *dbg, cudaStream_t st) {
+                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
+                             const Shape &full, int n_half, const FusedDebug *dbg, cudaStream_t st) {
+    Shape sh = full;
+    const int n_off = n_half * 128;
+    if (full.N > 128) sh.N = 128;
     CUtensorMap mC, mB, mX;
     const uint64_t dbc[4] = {(uint64_t)sh.N, (uint64_t)sh.G, (uint64_t)sh.T, (uint64_t)sh.batch};
-    const uint64_t sbc[3] = {(uint64_t)sh.N * 2, (uint64_t)sh.G * sh.N * 2, (uint64_t)sh.T * sh.G * sh.N * 2};
+    const uint64_t sbc[3] = {(uint64_t)full.N * 2, (uint64_t)sh.G * full.N * 2,
+                             (uint64_t)sh.T * sh.G * full.N * 2};
+    B += n_off;
+    C += n_off;
     const uint32_t box[4] = {64, 1, kRows, 1};
     const uint64_t dx[4] = {(uint64_t)sh.P, (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sx[3] = {(uint64_t)sh.P * 2, (uint64_t)sh.H * sh.P * 2, (uint64_t)sh.T * sh.H * sh.P * 2};
@@ -908,7 +941,9 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.sh = sh;
     p.dt = dt;
     p.A = A;
-    p.D = D;
+    p.D = (n_half == 0) ? D : nullptr;
+    p.state_ld = full.N;
+    p.n_off = n_off;
     p.init = init;
     p.fin = fin;
     p.ring = ring;
@@ -926,11 +961,11 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;
-    cudaError_t e =
-        cudaFuncSetAttribute(ssd_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    auto kernel = (n_half > 0) ? ssd_fused_kernel<true> : ssd_fused_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = min(p.n_units, device_sm_count());
-    ssd_fused_kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, p);
+    kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, p);
     return cudaGetLastError();
 }
 

@@ -43,6 +43,9 @@ SMALL = [
     (1, 512, 8, 64, 64, 1, 256, "bf16", False),
     (1, 700, 6, 64, 16, 3, 256, "bf16", True),    # small N, ragged
     (1, 256, 2, 64, 256, 1, 64, "bf16", False),   # largest N in bf16
+    (1, 700, 4, 64, 256, 2, 256, "bf16", True),   # N = 256 on the tensor cores: two half-state launches
+    (2, 333, 2, 64, 256, 1, 128, "bf16", True),   # the same with one row block per chunk, ragged
+    (1, 100, 2, 64, 256, 1, 256, "bf16", True),   # ... and a single short chunk
 ]
 
 
