@@ -19,7 +19,7 @@ bool fused_supported(const Shape &sh, int dtype);
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
                              int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
-                             const Shape &full, int n_half, const FusedDebug *dbg, cudaStream_t st);
+                             const Shape &full, int p_half, int n_half, const FusedDebug *dbg, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -68,7 +68,11 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 const char *const kSimtStages[] = {"ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan"};
 const char *const kFusedStages[] = {"ssd_fused"};
-const char *const kFusedStages256[] = {"ssd_fused_n0_127", "ssd_fused_n128_255"};
+// launch names when the fused path splits the problem: by head columns (P = 128), state columns (N = 256)
+const char *const kFusedStagesP[] = {"ssd_fused_p0_63", "ssd_fused_p64_127"};
+const char *const kFusedStagesN[] = {"ssd_fused_n0_127", "ssd_fused_n128_255"};
+const char *const kFusedStagesPN[] = {"ssd_fused_p0_63_n0_127", "ssd_fused_p64_127_n0_127",
+                                      "ssd_fused_p0_63_n128_255", "ssd_fused_p64_127_n128_255"};
 
 int launch_count(const Shape &sh, ssd::Path path) {
     if (sh.T == 0) return 0;
@@ -103,14 +107,17 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
               const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
               const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg) {
     if (!mk.mark(1, st)) return SSD_ERR_CUDA;
-    const int passes = ssd::fused_passes(sh);
-    const size_t stride = w.total / passes;  // one pass's counter, flags and ring
+    // launch k covers head-column half k % pp and state-column half k / pp: the second state half adds to
+    // the y its first half wrote, so it comes after both head-column launches of that first half
+    const int passes = ssd::fused_passes(sh), pp = ssd::fused_p_passes(sh);
+    const size_t stride = w.total / passes;  // one launch's counter, flags and ring
     for (int k = 0; k < passes; ++k) {
         char *pw = ws + k * stride;
         if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, reinterpret_cast<float *>(pw + w.ring_off),
                                   reinterpret_cast<int *>(pw + w.ready_off), reinterpret_cast<int *>(pw + w.cons_off),
                                   reinterpret_cast<int *>(pw + w.counter_off),
-                                  reinterpret_cast<int *>(ws + w.status_off), y, sh, k, dbg, st) != cudaSuccess ||
+                                  reinterpret_cast<int *>(ws + w.status_off), y, sh, k % pp, k / pp, dbg,
+                                  st) != cudaSuccess ||
             !mk.mark(2 + k, st))
             return SSD_ERR_CUDA;
     }
@@ -146,9 +153,10 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     char *ws = static_cast<char *>(workspace);
     if (!mk.mark(0, st)) return SSD_ERR_CUDA;
     if (cudaMemsetAsync(ws, 0, w.clear_bytes, st) != cudaSuccess) return SSD_ERR_CUDA;
-    if (path == ssd::kPathFused && ssd::fused_passes(sh) == 2 &&
-        cudaMemsetAsync(ws + w.total / 2, 0, w.clear_bytes, st) != cudaSuccess)
-        return SSD_ERR_CUDA;
+    if (path == ssd::kPathFused)
+        for (int k = 1; k < ssd::fused_passes(sh); ++k)
+            if (cudaMemsetAsync(ws + k * (w.total / ssd::fused_passes(sh)), 0, w.clear_bytes, st) != cudaSuccess)
+                return SSD_ERR_CUDA;
     if (T == 0) {
         if (!mk.mark(1, st)) return SSD_ERR_CUDA;
         if (!final_state) return SSD_OK;
@@ -192,7 +200,11 @@ const char *ssd_fwd_stage_name(int batch, int T, int H, int P, int G, int N, int
     const ssd::Path path = choose_path(sh, dtype);
     if (i < 0 || i >= launch_count(sh, path)) return nullptr;
     if (path != ssd::kPathFused) return kSimtStages[i];
-    return ssd::fused_passes(sh) == 2 ? kFusedStages256[i] : kFusedStages[i];
+    const int pp = ssd::fused_p_passes(sh), np = ssd::fused_n_passes(sh);
+    if (pp == 2 && np == 2) return kFusedStagesPN[i];
+    if (pp == 2) return kFusedStagesP[i];
+    if (np == 2) return kFusedStagesN[i];
+    return kFusedStages[i];
 }
 
 int ssd_fwd(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,

@@ -130,18 +130,23 @@ int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, S
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// The fused path runs a 256-wide state as two launches over halves of 128, each with its own
-// counter, flags and ring (one after the other in the workspace); the status word is shared.
-inline int fused_passes(const Shape &s) { return s.N > 128 ? 2 : 1; }
+// The fused path works on 64 head columns and up to 128 state columns per launch: P = 128 runs as two
+// launches over column halves of x and y, N = 256 as two over halves of the state (the second adding to
+// y).  Each launch has its own counter, flags and ring (one after the other in the workspace); the
+// status word is shared.  A head dimension below 64 is zero-padded, so the ring always has 64 rows.
+inline int fused_p_passes(const Shape &s) { return s.P > 64 ? 2 : 1; }
+inline int fused_n_passes(const Shape &s) { return s.N > 128 ? 2 : 1; }
+inline int fused_passes(const Shape &s) { return fused_p_passes(s) * fused_n_passes(s); }
 
 inline Workspace workspace_layout_one(const Shape &s, Path path);
 
 inline Workspace workspace_layout(const Shape &s, Path path) {
-    if (path != kPathFused || fused_passes(s) == 1) return workspace_layout_one(s, path);
+    if (path != kPathFused) return workspace_layout_one(s, path);
     Shape h = s;
-    h.N = 128;
+    h.P = 64;
+    if (h.N > 128) h.N = 128;
     Workspace w = workspace_layout_one(h, path);
-    w.total *= 2;  // pass k's counter, flags and ring sit at k * (total / 2)
+    w.total *= fused_passes(s);  // launch k's counter, flags and ring sit at k * (total / passes)
     return w;
 }
 

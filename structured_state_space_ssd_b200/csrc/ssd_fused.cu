@@ -97,7 +97,7 @@ struct Params {
     int *cons;          // [b*H][kSlots]: per ring slot, non-owner blocks that have read it (a count)
     int *counter;       // unit dispenser
     int *status;
-    __nv_bfloat16 *y;
+    __nv_bfloat16 *y;   // y + p_off (row stride p_full); read back only by the second state half
     int NK;             // 64-wide K-atoms along N
     int halves;         // Q / 128
     int heads_per_unit;
@@ -113,6 +113,11 @@ struct Params {
     // (D == null) and adds its result to the y the first one wrote (kernel template argument).
     int state_ld;
     int n_off;
+    // The tile is 64 columns of p wide: a head dimension below 64 is zero-padded (x loads past P read
+    // zero, y stores past P are clipped, state rows past P are neither read nor written), and P = 128
+    // runs as two launches over columns p_off = 0 and 64 (the rows of the state are independent).
+    int p_full;
+    int p_off;
 };
 
 // One head pipeline.  Barriers signalled once per head of the pipeline are
@@ -741,10 +746,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 float old[32];
                 if (un.c == 0) {
                     const size_t ld = p.state_ld;
+                    const int pv = p.p_full - p.p_off - half * 32;  // valid state rows among this thread's 32
                     const float *src =
-                        p.init ? p.init + ((size_t)bh * kP + half * 32) * ld + p.n_off + n : nullptr;
+                        p.init ? p.init + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n : nullptr;
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) old[q] = (src && nv) ? __ldg(src + (size_t)q * ld) : 0.f;
+                    for (int q = 0; q < 32; ++q) old[q] = (src && nv && q < pv) ? __ldg(src + (size_t)q * ld) : 0.f;
                 } else {
                     const float4 *src =
                         reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * kSlots + (un.c - 1) % kSlots) * PN);
@@ -821,9 +827,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         }
                     } else if (nv && p.fin) {
                         const size_t ld = p.state_ld;
-                        float *fin = p.fin + ((size_t)bh * kP + half * 32) * ld + p.n_off + n;
+                        const int pv = p.p_full - p.p_off - half * 32;
+                        float *fin = p.fin + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n;
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) fin[(size_t)q * ld] = old[q];
+                        for (int q = 0; q < 32; ++q)
+                            if (q < pv) fin[(size_t)q * ld] = old[q];
                     }
                     __syncwarp();
                     if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
@@ -838,10 +846,12 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 uint4 yprev[4];
                 if (kAccum) {
                     const bool jv = j < un.len;
-                    const uint4 *yp = reinterpret_cast<const uint4 *>(
-                        p.y + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP + half * 32);
+                    const int pv = p.p_full - p.p_off - half * 32;
+                    const uint4 *yp = reinterpret_cast<const uint4 *>(  // p.y starts at column p_off
+                        p.y + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * p.p_full + half * 32);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) yprev[q] = jv ? __ldg(yp + q) : make_uint4(0u, 0u, 0u, 0u);
+                    for (int q = 0; q < 4; ++q)
+                        yprev[q] = (jv && 8 * q < pv) ? __ldg(yp + q) : make_uint4(0u, 0u, 0u, 0u);
                 }
                 wait_bar(&pb.mx_done, par(use), p.status, broken);
                 fence_after_sync();
@@ -895,7 +905,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 bool fused_supported(const Shape &sh, int dtype) {
-    return dtype == SSD_BF16 && sh.P == kP && ((sh.N >= 16 && sh.N <= 128 && sh.N % 16 == 0) || sh.N == 256) &&
+    return dtype == SSD_BF16 && sh.P % 8 == 0 && (sh.P <= kP || sh.P == 2 * kP) &&
+           ((sh.N >= 16 && sh.N <= 128 && sh.N % 16 == 0) || sh.N == 256) &&
            (sh.Q == 128 || sh.Q == 256);
 }
 
@@ -915,15 +926,17 @@ static int heads_per_unit(const Shape &sh) {
     return (hpg + blocks - 1) / blocks;
 }
 
-// Launches the fused kernel for state columns [n_half * 128, ...) of the problem `full` (all of them
-// when full.N <= 128).  The second half of a 256-wide state adds to the y of the first.
+// Launches the fused kernel for state columns [n_half * 128, ...) and head columns [p_half * 64, ...)
+// of the problem `full` (all of them when full.N <= 128 and full.P <= 64).  The second half of a
+// 256-wide state adds to the y of the first.
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
                              int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
-                             const Shape &full, int n_half, const FusedDebug *dbg, cudaStream_t st) {
+                             const Shape &full, int p_half, int n_half, const FusedDebug *dbg, cudaStream_t st) {
     Shape sh = full;
-    const int n_off = n_half * 128;
+    const int n_off = n_half * 128, p_off = p_half * kP;
     if (full.N > 128) sh.N = 128;
+    sh.P = kP;
     CUtensorMap mC, mB, mX;
     const uint64_t dbc[4] = {(uint64_t)sh.N, (uint64_t)sh.G, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sbc[3] = {(uint64_t)full.N * 2, (uint64_t)sh.G * full.N * 2,
@@ -931,8 +944,11 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     B += n_off;
     C += n_off;
     const uint32_t box[4] = {64, 1, kRows, 1};
-    const uint64_t dx[4] = {(uint64_t)sh.P, (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
-    const uint64_t sx[3] = {(uint64_t)sh.P * 2, (uint64_t)sh.H * sh.P * 2, (uint64_t)sh.T * sh.H * sh.P * 2};
+    // x and y: the launch's 64 head columns (fewer when P < 64: loads past P read zero, stores are clipped)
+    const uint64_t dx[4] = {(uint64_t)min(kP, full.P - p_off), (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
+    const uint64_t sx[3] = {(uint64_t)full.P * 2, (uint64_t)sh.H * full.P * 2, (uint64_t)sh.T * sh.H * full.P * 2};
+    x += p_off;
+    y += p_off;
     CUtensorMap mY;
     if (!make_map_bf16(&mC, C, 4, dbc, sbc, box) || !make_map_bf16(&mB, B, 4, dbc, sbc, box) ||
         !make_map_bf16(&mX, x, 4, dx, sx, box) || !make_map_bf16(&mY, y, 4, dx, sx, box))
@@ -944,6 +960,8 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.D = (n_half == 0) ? D : nullptr;
     p.state_ld = full.N;
     p.n_off = n_off;
+    p.p_full = full.P;
+    p.p_off = p_off;
     p.init = init;
     p.fin = fin;
     p.ring = ring;

@@ -60,6 +60,9 @@ def test_workspace_bytes(lib):
     w256 = f(8, 4096, 32, 64, 1, 256, 256, 1)   # N = 256: two halves, each with its own flags and ring
     ring256 = 2 * 8 * 32 * 3 * 64 * 128 * 4
     assert ring256 <= w256 < ring256 + (1 << 17)
+    w32p = f(8, 4096, 32, 32, 1, 128, 256, 1)   # P = 32 is padded: the ring still holds 64 rows
+    assert w32p == f(8, 4096, 32, 64, 1, 128, 256, 1)
+    assert f(8, 4096, 32, 128, 1, 256, 256, 1) == 2 * w256   # four launches of 64 x 128 states
     w32 = f(4, 2048, 80, 64, 1, 128, 256, 0)    # CUDA-core path: every chunk state
     assert w32 >= 4 * nc * 80 * 64 * 128 * 4 + 4 * 80 * nc * 256 * 4
     assert f(0, 2048, 80, 64, 1, 128, 256, 1) == 0      # batch < 1
@@ -73,6 +76,12 @@ def test_launch_count(lib):
     assert lib.ssd_fwd_launch_count(4, 2048, 80, 64, 1, 128, 256, 1) == 1    # one fused launch
     assert lib.ssd_fwd_launch_count(8, 4096, 32, 64, 1, 256, 256, 1) == 2    # N = 256: two state halves
     assert lib.ssd_fwd_stage_name(8, 4096, 32, 64, 1, 256, 256, 1, 1) == b"ssd_fused_n128_255"
+    assert lib.ssd_fwd_launch_count(2, 4096, 32, 128, 1, 128, 256, 1) == 2   # P = 128: two column halves
+    assert lib.ssd_fwd_stage_name(2, 4096, 32, 128, 1, 128, 256, 1, 1) == b"ssd_fused_p64_127"
+    assert lib.ssd_fwd_launch_count(2, 4096, 32, 128, 1, 256, 256, 1) == 4   # both splits
+    assert lib.ssd_fwd_stage_name(2, 4096, 32, 128, 1, 256, 256, 1, 2) == b"ssd_fused_p0_63_n128_255"
+    assert lib.ssd_fwd_launch_count(2, 4096, 32, 32, 1, 128, 256, 1) == 1    # P = 32: padded, one launch
+    assert lib.ssd_fwd_launch_count(2, 4096, 32, 36, 1, 128, 256, 1) == 4    # P % 8 != 0: CUDA-core stages
     assert lib.ssd_fwd_launch_count(1, 0, 2, 16, 1, 16, 64, 0) == 0
     assert lib.ssd_fwd_launch_count(1, 10, 3, 16, 2, 16, 64, 0) == 0
 

@@ -46,6 +46,12 @@ SMALL = [
     (1, 700, 4, 64, 256, 2, 256, "bf16", True),   # N = 256 on the tensor cores: two half-state launches
     (2, 333, 2, 64, 256, 1, 128, "bf16", True),   # the same with one row block per chunk, ragged
     (1, 100, 2, 64, 256, 1, 256, "bf16", True),   # ... and a single short chunk
+    (1, 700, 4, 32, 128, 2, 256, "bf16", True),   # P = 32 on the tensor cores: zero-padded to 64 columns
+    (2, 333, 3, 8, 64, 1, 128, "bf16", True),     # the narrowest head, one row block per chunk
+    (1, 600, 2, 48, 16, 1, 256, "bf16", False),   # P = 48, small N
+    (1, 700, 4, 128, 128, 2, 256, "bf16", True),  # P = 128: two launches over head-column halves
+    (2, 300, 2, 128, 64, 1, 128, "bf16", True),   # the same with one row block per chunk
+    (1, 520, 2, 128, 256, 1, 256, "bf16", True),  # P = 128, N = 256: four launches
 ]
 
 
