@@ -17,9 +17,9 @@ cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D
                               const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
 bool fused_supported(const Shape &sh, int dtype);
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
-                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
-                             const Shape &full, int p_half, int n_half, const FusedDebug *dbg, cudaStream_t st);
+                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
+                             const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
+                             int n_half, const FusedDebug *dbg, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -113,11 +113,8 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
     const size_t stride = w.total / passes;  // one launch's counter, flags and ring
     for (int k = 0; k < passes; ++k) {
         char *pw = ws + k * stride;
-        if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, reinterpret_cast<float *>(pw + w.ring_off),
-                                  reinterpret_cast<int *>(pw + w.ready_off), reinterpret_cast<int *>(pw + w.cons_off),
-                                  reinterpret_cast<int *>(pw + w.counter_off),
-                                  reinterpret_cast<int *>(ws + w.status_off), y, sh, k % pp, k / pp, dbg,
-                                  st) != cudaSuccess ||
+        if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, pw, w, reinterpret_cast<int *>(ws + w.status_off), y,
+                                  sh, k % pp, k / pp, dbg, st) != cudaSuccess ||
             !mk.mark(2 + k, st))
             return SSD_ERR_CUDA;
     }

@@ -81,18 +81,35 @@ __device__ __forceinline__ void stage_rows(float *dst, int dld, const T *src, si
     }
 }
 
-// Slots per (batch, head) of the fused path's ring of chunk states.
-constexpr int kRingSlots = 3;
-
 // Problem shape as every kernel sees it.
 struct Shape {
     int batch, T, H, P, G, N, Q, nc;
     int heads_per_group;  // H / G
 };
 
+// The fused path's inter-chunk chain.  The owner of chunk c forms the outgoing state
+// S~_c = exp(sigma_c) S~_{c-1} + L_c from the one before.  With look-back depth D > 1 every owner
+// also publishes its local state L_c and total decay sigma_c as soon as its products are done, and
+// the owner of chunk c starts from the most recent published S~_j with j >= c - D, folding in
+// L_{j+1} .. L_{c-1} (the decoupled look-back of a single-pass scan), so that a long sequence is not
+// bound by one hand-off per chunk.  D > 1 is used where the chain would be long and the ring, twice
+// as large, stays small enough to live in L2.  `s` is one launch's shape (64 head columns, at most
+// 128 state columns).
+inline int fused_lookback(const Shape &s) {
+    const size_t bh = (size_t)s.batch * s.H;
+    const size_t slot_bytes = 2 * sizeof(float) * 64 * (size_t)s.N;  // S~ and L
+    return (s.nc >= 32 && bh * 8 * slot_bytes <= (size_t(48) << 20)) ? 4 : 1;
+}
+// Ring slots per (batch, head): chunk c's states go to slot c % R.  Three with D = 1; 2D with look-back,
+// so that the slot an owner overwrites was last read by owners at least D chunks back.
+inline int fused_ring_slots(int d) { return d == 1 ? 3 : 2 * d; }
+// floats per slot: S~ (64 x N), and L (64 x N) after it with look-back
+inline size_t fused_slot_floats(const Shape &s, int d) { return (size_t)64 * s.N * (d == 1 ? 1 : 2); }
+
 // The two launch sequences: stage-per-kernel on CUDA cores (any shape and
-// dtype within the limits) or the fused tensor-core kernel (bf16, P = 64,
-// N a multiple of 16 up to 128, Q in {128, 256}).
+// dtype within the limits) or the fused tensor-core kernel (bf16, P a multiple
+// of 8 up to 64 or P = 128, N a multiple of 16 up to 128 or N = 256, Q in
+// {128, 256}).
 enum Path { kPathSimt = 0, kPathFused = 1 };
 
 // Test hooks of the fused kernel's hand-off (ssd_fwd_withhold_publish):
@@ -111,12 +128,14 @@ struct FusedDebug {
 struct Workspace {
     size_t status_off;  // int status word
     size_t counter_off; // int unit counter (fused path)
-    size_t ready_off;   // int ready[batch * H] (fused path)
-    size_t cons_off;    // int cons[batch * H][kRingSlots] (fused path)
+    size_t inc_off;     // fused path: int inc[batch * H][R] (one count per sequence without look-back)
+    size_t agg_off;     // fused path: int agg[batch * H][R], c + 1 once L_c and sigma_c are in slot c % R
+    size_t cons_off;    // fused path: int cons[batch * H][R], reads of the slot so far (a count)
+    size_t sig_off;     // fused path: float sigma[batch * H][R], chunk c's total log2 decay in slot c % R
     size_t clear_bytes; // bytes from offset 0 cleared per call
     size_t s_off;       // CUDA-core path: float s[batch][H][nc][Q], inclusive log-decay prefix sums per chunk
     size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
-    size_t ring_off;    // fused path: float ring[batch][H][kRingSlots][P/4][N][4], outgoing states of recent chunks
+    size_t ring_off;    // fused path: float ring[batch][H][R][1 or 2][16][N][4], states of recent chunks
     size_t total;
 };
 
@@ -156,17 +175,23 @@ inline Workspace workspace_layout_one(const Shape &s, Path path) {
     w.status_off = 0;
     w.counter_off = 4;
     size_t off = 256;
-    w.ready_off = off;
-    off += sizeof(int) * bh;
+    const int d = (path == kPathFused) ? fused_lookback(s) : 1, R = fused_ring_slots(d);
+    const size_t per_slot = (d == 1) ? 0 : bh * R;  // agg and sigma: look-back only
+    w.inc_off = off;
+    off += sizeof(int) * (d == 1 ? bh : bh * R);
     w.cons_off = off;
-    off += sizeof(int) * bh * kRingSlots;
+    off += sizeof(int) * bh * R;
+    w.agg_off = off;
+    off += sizeof(int) * per_slot;
+    w.sig_off = off;
+    off += sizeof(float) * per_slot;
     off = align256(off);
     w.clear_bytes = (path == kPathFused) ? off : 256;
     w.s_off = off;
     if (path != kPathFused) off = align256(off + sizeof(float) * bh * s.nc * s.Q);
     w.state_off = w.ring_off = off;
     if (path == kPathFused)
-        off = align256(off + sizeof(float) * bh * kRingSlots * s.P * s.N);
+        off = align256(off + sizeof(float) * bh * R * fused_slot_floats(s, d));
     else
         off = align256(off + sizeof(float) * (size_t)s.batch * s.nc * s.H * s.P * s.N);
     w.total = off;

@@ -82,8 +82,6 @@ constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units)
 constexpr uint32_t kSmemBytes = kOffAux + 2 * kAuxFloats * 4 + 1024;
 
 constexpr uint32_t kDefaultFlagPolls = 1u << 22;
-// Ring slots per sequence: chunk c's state goes to slot c % kSlots (see the hand-out order in decode).
-constexpr int kSlots = kRingSlots;
 
 struct Params {
     Shape sh;
@@ -92,9 +90,14 @@ struct Params {
     const float *D;     // [H]
     const float *init;  // [b][H][P][N] or null
     float *fin;         // [b][H][P][N] or null
-    float *ring;        // [b][H][kSlots][P/4][N][4]: outgoing states of recent chunks (see ring_quad)
-    int *ready;         // [b*H]: chunks whose outgoing state is published
-    int *cons;          // [b*H][kSlots]: per ring slot, non-owner blocks that have read it (a count)
+    // The chain (see fused_lookback; the depth D is the kernel's template argument): chunk c's states
+    // live in slot c % R of its sequence, S~_c first, then (look-back only) L_c, each [P/4][N][4]
+    // (see ring_quad).
+    float *ring;        // [b*H][R][1 or 2][P/4][N][4]
+    int *inc;           // c + 1 once S~_c is published: [b*H] without look-back, [b*H][R] with (inc_flag)
+    int *agg;           // [b*H][R]: c + 1 once L_c and sigma_c are published (look-back only)
+    int *cons;          // [b*H][R]: reads of the slot so far, every use (a count)
+    float *sig;         // [b*H][R]: sigma_c, chunk c's total decay in log2 units (look-back only)
     int *counter;       // unit dispenser
     int *status;
     __nv_bfloat16 *y;   // y + p_off (row stride p_full); read back only by the second state half
@@ -151,10 +154,11 @@ struct Unit {
 // block owning chunk c's state (the last one) is handed out one step ahead of chunk c-1's other block:
 //   [owners of chunk 0] [owners of 1, others of 0] [owners of 2, others of 1] ... [others of nc-1]
 // so that the owners, which carry the inter-chunk chain, run ahead of the blocks that wait for it.
-// Every unit still waits only for units handed out before it: an owner waits for the owner of the
-// chunk before (one step earlier) and for the other block of chunk c-2 to have read the ring slot it
-// overwrites (one step earlier too, with three slots); another block waits for the owner of the chunk
-// before (two steps earlier).  So there is no deadlock however many CTAs are resident.
+// Every unit still waits only for units handed out before it: an owner waits for the owners of the
+// D chunks before (earlier steps) and for the readers of the ring slot it overwrites, chunk c-R's (the
+// owners up to chunk c-R+D and the other block of chunk c-R+1, handed out with the owners of c-R+2, at
+// least one step earlier as R >= 3); another block waits for the owner of the chunk before (two steps
+// earlier).  So there is no deadlock however many CTAs are resident.
 __device__ __forceinline__ Unit decode(int u, const Params &p) {
     Unit un;
     const int M = p.units_per_role;
@@ -254,6 +258,15 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // per 16-byte access.
 __device__ __forceinline__ size_t ring_quad(int N, int n, int quad) { return (size_t)quad * N + n; }
 
+// The flag that publishes S~_c of sequence bh.  Without look-back owners publish in chunk order, so
+// one count per sequence serves (it reads c + 1 once S~_0 .. S~_c are out; a count measured faster
+// here than a flag per slot); with look-back they may publish out of order: one flag per ring slot.
+template <int kD>
+__device__ __forceinline__ int *inc_flag(int *inc, int bh, int c) {
+    constexpr int R = kD == 1 ? 3 : 2 * kD;
+    return kD == 1 ? inc + bh : inc + bh * R + c % R;
+}
+
 // Eight bf16 scaled by w (fp32 products, one rounding to bf16).
 __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
     const float2 ww = make_float2(w, w);
@@ -275,7 +288,8 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
 using namespace fz;
 
 // kAccum: the second half of a 256-wide state, which adds its y to the first half's.
-template <bool kAccum>
+// kD: the chain's look-back depth D (1: every owner waits for the chunk before).
+template <bool kAccum, int kD>
 __global__ void __launch_bounds__(fz::kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                      const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY,
@@ -290,7 +304,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     __shared__ int s_abort, s_broken;
     // per pipeline, for its publisher: warps that finished an owner's ring stores, and warps that
     // finished reading another block's state from the ring (8 per head in either case)
-    __shared__ uint32_t s_owned[2], s_copied[2];
+    __shared__ uint32_t s_owned[2], s_copied[2], s_agg[2];
+    __shared__ int s_base[2];  // per pipeline: the chunk whose S~ the owner starts from (-1: initial state)
     volatile int *abort = &s_abort;
     volatile int *broken = &s_broken;
 
@@ -298,12 +313,13 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     const int warp = tid >> 5, lane = tid & 31;
     const Shape sh = p.sh;
     const int N = sh.N, NK = p.NK;
+    constexpr int R = kD == 1 ? 3 : 2 * kD;  // ring slots per sequence (see fused_ring_slots)
 
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     if (tid == 0) {
         s_abort = 0;
         s_broken = 0;
-        s_owned[0] = s_owned[1] = s_copied[0] = s_copied[1] = 0;
+        s_owned[0] = s_owned[1] = s_copied[0] = s_copied[1] = s_agg[0] = s_agg[1] = 0;
         uint64_t *all = reinterpret_cast<uint64_t *>(&bars);
         for (int i = 0; i < (int)(sizeof(Bars) / 8); ++i) mbar_init(&all[i], 1);
         mbar_init(&bars.unit_empty, kSimtWarps + 3);
@@ -325,15 +341,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // ------------------------------------------------------------------
         // Publisher warps: warp 18 + pl makes pipeline pl's hand-offs visible
         // to other CTAs, so that neither the CUDA-core warps nor the issuer
-        // wait for a GPU-scope release.  After an owner's ring stores it
-        // releases `ready` (S~_c readable); once another block's copy of
-        // S~_{c-1} has been read it adds one to that slot's `cons` (the
-        // slot may be rewritten).  The warps signal through CTA-scope release
-        // counts in shared memory, acquired here, which puts their stores
-        // before this thread's GPU-scope release (release is cumulative).
+        // wait for a GPU-scope release.  After an owner's stores of L_c it
+        // releases `agg` (look-back only); after its store of S~_c it adds
+        // one to `cons` of each slot it may have read and releases `inc`;
+        // once another block has read S~_{c-1} it adds one to that slot's
+        // `cons`.  The warps signal through CTA-scope release counts in
+        // shared memory, acquired here by every lane, which puts their stores
+        // before the lanes' GPU-scope releases (release is cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
-        uint32_t ucnt = 0, ocnt = 0, tcnt = 0;
+        uint32_t ucnt = 0, ocnt = 0, tcnt = 0, acnt = 0;
         // bounded wait for one of this pipeline's shared-memory counts to reach `target`
         auto wait_count = [&](const uint32_t *cnt, uint32_t target) {
             if (ld_acquire_cta_shared(cnt) >= target) return;
@@ -359,13 +376,23 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             for (int h = un.h0 + pl; h < un.h1; h += 2) {
                 const int bh = un.b * sh.H + h;
                 if (un.owner) {
+                    const bool publish =
+                        un.c < sh.nc - 1 && !(bh == p.withhold_bh && un.c == p.withhold_c);
+                    if (kD > 1 && un.c < sh.nc - 1) {
+                        // L_c and sigma_c stored
+                        wait_count(&s_agg[pl], kPipeWarps * ++acnt);
+                        if (lane == 0 && publish) st_release_gpu(p.agg + bh * R + un.c % R, un.c + 1);
+                    }
                     wait_count(&s_owned[pl], kPipeWarps * ++ocnt);
-                    const bool withheld = (bh == p.withhold_bh && un.c == p.withhold_c);
-                    if (lane == 0 && un.c < sh.nc - 1 && !withheld) st_release_gpu(p.ready + bh, un.c + 1);
+                    if (lane == 0 && publish) st_release_gpu(inc_flag<kD>(p.inc, bh, un.c), un.c + 1);
+                    // with look-back the owner has read (at most) the slots of the D chunks before it:
+                    // count them all (without, its read of S~_{c-1} precedes every later owner's
+                    // publication, so the owner of chunk c-1+R cannot overwrite it first)
+                    if (kD > 1 && lane < min(kD, un.c)) red_release_add_gpu(p.cons + bh * R + (un.c - 1 - lane) % R, 1);
                 } else if (un.c > 0) {
-                    // chunk c has read slot (c-1) & 1 (chunk 0 reads the initial state)
+                    // the other block of chunk c has read S~_{c-1} (chunk 0's reads the initial state)
                     wait_count(&s_copied[pl], kPipeWarps * ++tcnt);
-                    if (lane == 0) red_release_add_gpu(p.cons + kSlots * bh + (un.c - 1) % kSlots, 1);
+                    if (lane == 0) red_release_add_gpu(p.cons + bh * R + (un.c - 1) % R, 1);
                 }
                 __syncwarp();
             }
@@ -600,9 +627,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             const float *dtp = p.dt + ((size_t)un.b * sh.T + un.t0 + wtid) * sh.H;
             float dt_next = 0.f, a_next = 0.f, d_cur = p.D ? __ldg(p.D + h) : 0.f;
             scan((wtid < un.len) ? __ldg(dtp + h) : 0.f, __ldg(p.A + h));
-            // ctl reads `ready` of the pipeline's head early (acquire), so that the wait usually costs
-            // nothing by the time the state is needed (ctl's warp builds only zero mask slabs)
-            int ready_seen = (ctl && un.c > 0) ? ld_acquire_gpu(p.ready + un.b * sh.H + h) : 0;
+            // ctl reads `inc` of the chunk before for the pipeline's head early (acquire), so that the
+            // wait usually costs nothing by the time the state is needed (ctl's warp builds only zero
+            // mask slabs)
+            int ready_seen =
+                (ctl && un.c > 0) ? ld_acquire_gpu(inc_flag<kD>(p.inc, un.b * sh.H + h, un.c - 1)) : 0;
             bool first_head = true;
             for (; h < un.h1; h += 2, ++use) {
                 const int bh = un.b * sh.H + h;
@@ -664,8 +693,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 // it zeros.  Warpgroup 0 takes the diagonal slab, warpgroup 1 the other three.
                 // an owner's slot count, read (acquire) before the mask for the same reason
                 int cons_seen = 0;
-                if (own && ctl && writes_ring && p.halves == 2 && un.c >= 2)
-                    cons_seen = ld_acquire_gpu(p.cons + kSlots * bh + un.c % kSlots);
+                if (own && ctl && writes_ring && un.c >= R && (kD > 1 || p.halves == 2))
+                    cons_seen = ld_acquire_gpu(p.cons + bh * R + un.c % R);
                 if (first_head) wait_bar(&bars.g_done, par(gphase), p.status, broken);
                 fence_after_sync();
                 {
@@ -728,113 +757,323 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 // the pipeline publishes this)
                 if (ctl) bulk_wait_read();
 
-                // ---- stage 3: the state entering the block: S~_{c-1} from the ring (published by the
-                // owner of chunk c-1) or the initial state.  Chunk c's state goes to slot c % kSlots,
-                // which held chunk c - kSlots's, read by the other block of chunk c - kSlots + 1; the
-                // other blocks of chunks k >= 1 read slot (k - 1) % kSlots, so that slot has had
-                // c / kSlots reads once that one is in, and no later reader can add to the count before
-                // this owner publishes.
-                const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
-                const bool nv = n < N;
-                if (ctl) {
-                    if (un.c > 0 && ready_seen < un.c) wait_flag(p.ready + bh, un.c, p.flag_polls, abort, p.status);
-                    if (writes_ring && p.halves == 2 && un.c >= kSlots && cons_seen < un.c / kSlots)
-                        wait_flag(p.cons + kSlots * bh + un.c % kSlots, un.c / kSlots, p.flag_polls, abort,
-                                  p.status);
-                }
-                named_bar_sync(bar_id, kPipeThreads);
-                float old[32];
-                if (un.c == 0) {
-                    const size_t ld = p.state_ld;
-                    const int pv = p.p_full - p.p_off - half * 32;  // valid state rows among this thread's 32
-                    const float *src =
-                        p.init ? p.init + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n : nullptr;
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) old[q] = (src && nv && q < pv) ? __ldg(src + (size_t)q * ld) : 0.f;
-                } else {
-                    const float4 *src =
-                        reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * kSlots + (un.c - 1) % kSlots) * PN);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 t =
-                            nv ? __ldcg(src + ring_quad(N, n, half * 8 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        old[4 * q] = t.x;
-                        old[4 * q + 1] = t.y;
-                        old[4 * q + 2] = t.z;
-                        old[4 * q + 3] = t.w;
+                // ---- stage 3: the state entering the block
+                if constexpr (kD == 1) {
+                    // without look-back: S~_{c-1} from the ring (published by the owner of chunk c-1) or
+                    // the initial state.  Chunk c's state goes to slot c % 3, which held chunk c-3's, read
+                    // by the other block of chunk c-2 (and by the owner of chunk c-2, whose read precedes
+                    // the publication this owner waited for); the other blocks of chunks k >= 1 read slot
+                    // (k - 1) % 3, so that slot has had c / 3 counted reads once that one is in, and no
+                    // later reader can add to the count before this owner publishes.
+                    const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
+                    const bool nv = n < N;
+                    if (ctl) {
+                        if (un.c > 0 && ready_seen < un.c)
+                            wait_flag(inc_flag<kD>(p.inc, bh, un.c - 1), un.c, p.flag_polls, abort, p.status);
+                        if (writes_ring && p.halves == 2 && un.c >= R && cons_seen < un.c / R)
+                            wait_flag(p.cons + R * bh + un.c % R, un.c / R, p.flag_polls, abort,
+                                      p.status);
                     }
-                }
-                uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
-                if (own) {
-                    wait_bar(&pb.d_done, par(ocnt), p.status, broken);
-                    ++ocnt;
-                    fence_after_sync();
-                    if (un.r == 1) {
-                        // E = exp(s_127) S~_{c-1} + S_pre
-                        const float e_start = ex2(s_ref);
+                    named_bar_sync(bar_id, kPipeThreads);
+                    float old[32];
+                    if (un.c == 0) {
+                        const size_t ld = p.state_ld;
+                        const int pv = p.p_full - p.p_off - half * 32;  // valid state rows among this thread's 32
+                        const float *src =
+                            p.init ? p.init + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n : nullptr;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) old[q] = (src && nv && q < pv) ? __ldg(src + (size_t)q * ld) : 0.f;
+                    } else {
+                        const float4 *src =
+                            reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * R + (un.c - 1) % R) * PN);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 t =
+                                nv ? __ldcg(src + ring_quad(N, n, half * 8 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            old[4 * q] = t.x;
+                            old[4 * q + 1] = t.y;
+                            old[4 * q + 2] = t.z;
+                            old[4 * q + 3] = t.w;
+                        }
+                    }
+                    uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
+                    if (own) {
+                        wait_bar(&pb.d_done, par(ocnt), p.status, broken);
+                        ++ocnt;
+                        fence_after_sync();
+                        if (un.r == 1) {
+                            // E = exp(s_127) S~_{c-1} + S_pre
+                            const float e_start = ex2(s_ref);
+#pragma unroll
+                            for (int q0 = 0; q0 < 32; q0 += 16) {
+                                uint32_t t[16];
+                                tmem_ld16(tA + half * 32 + q0 + lane_base, t);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int q = 0; q < 16; ++q)
+                                    old[q0 + q] = fmaf(e_start, old[q0 + q], __uint_as_float(t[q]));
+                            }
+                        }
+                    }
+                    // E in bf16 into row n of the tile (128-byte swizzled)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint4 t;
+                        t.x = pack_bf16x2(old[8 * k + 0], old[8 * k + 1]);
+                        t.y = pack_bf16x2(old[8 * k + 2], old[8 * k + 3]);
+                        t.z = pack_bf16x2(old[8 * k + 4], old[8 * k + 5]);
+                        t.w = pack_bf16x2(old[8 * k + 6], old[8 * k + 7]);
+                        if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
+                        sts128(sE + swz(n, half * 4 + k), t);
+                    }
+                    fence_view_async_shared();
+                    if (!own) {
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive(&pb.s_full);
+                            // the ring entries are consumed: the publisher may count the slot as read
+                            if (un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
+                        }
+                    } else {
+                        // S~_c = exp(s_end - s_{r-1}) E + S_own.  S_own is read from TMEM before s_full,
+                        // after which the issuer overwrites that accumulator.
+                        const float e_rest = ex2(s_end - s_ref);
 #pragma unroll
                         for (int q0 = 0; q0 < 32; q0 += 16) {
                             uint32_t t[16];
-                            tmem_ld16(tA + half * 32 + q0 + lane_base, t);
+                            tmem_ld16(tB + half * 32 + q0 + lane_base, t);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int q = 0; q < 16; ++q)
-                                old[q0 + q] = fmaf(e_start, old[q0 + q], __uint_as_float(t[q]));
+                            for (int q = 0; q < 16; ++q) old[q0 + q] = fmaf(e_rest, old[q0 + q], __uint_as_float(t[q]));
                         }
-                    }
-                }
-                // E in bf16 into row n of the tile (128-byte swizzled)
+                        fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&pb.s_full);
+                        if (writes_ring) {
+                            float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * R + un.c % R) * PN);
+                            if (nv) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    uint4 t;
-                    t.x = pack_bf16x2(old[8 * k + 0], old[8 * k + 1]);
-                    t.y = pack_bf16x2(old[8 * k + 2], old[8 * k + 3]);
-                    t.z = pack_bf16x2(old[8 * k + 4], old[8 * k + 5]);
-                    t.w = pack_bf16x2(old[8 * k + 6], old[8 * k + 7]);
-                    if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
-                    sts128(sE + swz(n, half * 4 + k), t);
-                }
-                fence_view_async_shared();
-                if (!own) {
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(&pb.s_full);
-                        // the ring entries are consumed: the publisher may count the slot as read
-                        if (un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
+                                for (int q = 0; q < 8; ++q)
+                                    __stcg(dst + ring_quad(N, n, half * 8 + q),
+                                           make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                            }
+                        } else if (nv && p.fin) {
+                            const size_t ld = p.state_ld;
+                            const int pv = p.p_full - p.p_off - half * 32;
+                            float *fin = p.fin + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n;
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (q < pv) fin[(size_t)q * ld] = old[q];
+                        }
+                        __syncwarp();
+                        if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
                     }
                 } else {
-                    // S~_c = exp(s_end - s_{r-1}) E + S_own.  S_own is read from TMEM before s_full,
-                    // after which the issuer overwrites that accumulator.
-                    const float e_rest = ex2(s_end - s_ref);
-#pragma unroll
-                    for (int q0 = 0; q0 < 32; q0 += 16) {
-                        uint32_t t[16];
-                        tmem_ld16(tB + half * 32 + q0 + lane_base, t);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) old[q0 + q] = fmaf(e_rest, old[q0 + q], __uint_as_float(t[q]));
+                    // look-back: the owner may start from an earlier S~_j and fold in the local states
+                    // after it, S~_i = exp(sigma_i) S~_{i-1} + L_i.  Every owner forms its own S~_c by
+                    // that same fp32 expression, so the result does not depend on where the fold
+                    // started.  Chunk c's states go to slot c % R, which held chunk c - R's: the owner
+                    // overwrites it once that chunk's readers (the D owners after it and the next
+                    // chunk's other block) have all added themselves to `cons`.
+                    const int reads_per_use = kD + (p.halves == 2 ? 1 : 0);
+                    const size_t PN2 = 2 * PN;  // a slot: S~, then L
+                    const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
+                    const bool nv = n < N;
+                    const float *ring_bh = p.ring + (size_t)bh * R * PN2;
+                    const int quad0 = half * 8;
+                    if (own && writes_ring) {
+                        // publish L_c = exp(s_end - s_{r-1}) S_pre + S_own (S_own alone for r = 0) and
+                        // sigma_c as soon as the state products are done
+                        if (ctl && un.c >= R && cons_seen < (un.c / R) * reads_per_use)
+                            wait_flag(p.cons + bh * R + un.c % R, (un.c / R) * reads_per_use, p.flag_polls, abort,
+                                      p.status);
+                        named_bar_sync(bar_id, kPipeThreads);
                     }
-                    fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pb.s_full);
-                    if (writes_ring) {
-                        float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * kSlots + un.c % kSlots) * PN);
-                        if (nv) {
+                    if (own) {
+                        wait_bar(&pb.d_done, par(ocnt), p.status, broken);
+                        ++ocnt;
+                        fence_after_sync();
+                    }
+                    if (own && writes_ring) {
+                        const float e_rest = ex2(s_end - s_ref);
+                        float4 *dst = reinterpret_cast<float4 *>(const_cast<float *>(ring_bh) + (un.c % R) * PN2 + PN);
+#pragma unroll
+                        for (int q0 = 0; q0 < 32; q0 += 8) {
+                            uint32_t a[8], b[8];
+                            if (un.r == 1) tmem_ld8(tA + half * 32 + q0 + lane_base, a);
+                            tmem_ld8(tB + half * 32 + q0 + lane_base, b);
+                            tmem_wait_ld();
+                            float l[8];
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
-                                __stcg(dst + ring_quad(N, n, half * 8 + q),
-                                       make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                                l[q] = (un.r == 1) ? fmaf(e_rest, __uint_as_float(a[q]), __uint_as_float(b[q]))
+                                                   : __uint_as_float(b[q]);
+                            if (nv) {
+                                __stcg(dst + ring_quad(N, n, quad0 + q0 / 4), make_float4(l[0], l[1], l[2], l[3]));
+                                __stcg(dst + ring_quad(N, n, quad0 + q0 / 4 + 1), make_float4(l[4], l[5], l[6], l[7]));
+                            }
                         }
-                    } else if (nv && p.fin) {
-                        const size_t ld = p.state_ld;
-                        const int pv = p.p_full - p.p_off - half * 32;
-                        float *fin = p.fin + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n;
-#pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            if (q < pv) fin[(size_t)q * ld] = old[q];
+                        if (ctl) __stcg(p.sig + bh * R + un.c % R, s_end);
+                        __syncwarp();
+                        if (lane == 0) red_release_cta_shared_add(&s_agg[pl], 1);  // the publisher releases them
                     }
-                    __syncwarp();
-                    if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
+                    int base = un.c - 1;  // the chunk whose S~ the fold starts from (-1: the initial state)
+                    if (own) {
+                        // ctl's warp polls the flags of the D chunks before this one at once (lane l:
+                        // chunk c-1-l) and takes the most recent S~_j whose later chunks all have L out
+                        if ((wtid >> 5) == 4) {
+                            const unsigned full = 0xffffffffu;
+                            const int jl = un.c - 1 - lane;
+                            const bool seen = __shfl_sync(full, ready_seen, 0) >= un.c;  // S~_{c-1} seen early
+                            uint32_t polls = 0;
+                            int found = seen ? un.c - 1 : -2;
+                            while (found == -2) {
+                                bool inc_ok = false, agg_ok = false;
+                                if (lane < kD) {
+                                    if (jl >= 0) {
+                                        inc_ok = ld_acquire_gpu(inc_flag<kD>(p.inc, bh, jl)) >= jl + 1;
+                                        agg_ok = ld_acquire_gpu(p.agg + bh * R + jl % R) >= jl + 1;
+                                    } else {
+                                        inc_ok = (jl == -1);  // the initial state
+                                    }
+                                }
+                                const unsigned im = __ballot_sync(full, inc_ok), am = __ballot_sync(full, agg_ok);
+                                const int run = __ffs(~am) - 1;  // chunks c-1 .. c-run have L published
+                                const unsigned cand = im & ((2u << run) - 1u);
+                                if (cand) {
+                                    found = un.c - __ffs(cand);
+                                    break;
+                                }
+                                bool give_up = *abort != 0;
+                                if (!give_up && ++polls >= p.flag_polls) {
+                                    if (lane == 0) atomicExch(p.status, SSD_ERR_TIMEOUT);
+                                    give_up = true;
+                                }
+                                if (!give_up && ld_relaxed_gpu(p.status) != 0) give_up = true;
+                                if (__any_sync(full, give_up)) {
+                                    if (lane == 0) *abort = 1;
+                                    found = max(un.c - kD, -1);  // in bounds; the results are not valid
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
+                            __syncwarp();
+                            if (lane == 0) s_base[pl] = found;
+                        }
+                        named_bar_sync(bar_id, kPipeThreads);
+                        base = s_base[pl];
+                    } else {
+                        if (ctl && un.c > 0 && ready_seen < un.c)
+                            wait_flag(inc_flag<kD>(p.inc, bh, un.c - 1), un.c, p.flag_polls, abort, p.status);
+                        named_bar_sync(bar_id, kPipeThreads);
+                    }
+                    float old[32];
+                    if (base < 0) {
+                        const size_t ld = p.state_ld;
+                        const int pv = p.p_full - p.p_off - half * 32;  // valid state rows among this thread's 32
+                        const float *src =
+                            p.init ? p.init + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n : nullptr;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) old[q] = (src && nv && q < pv) ? __ldg(src + (size_t)q * ld) : 0.f;
+                    } else {
+                        const float4 *src = reinterpret_cast<const float4 *>(ring_bh + (base % R) * PN2);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 t = nv ? __ldcg(src + ring_quad(N, n, quad0 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            old[4 * q] = t.x;
+                            old[4 * q + 1] = t.y;
+                            old[4 * q + 2] = t.z;
+                            old[4 * q + 3] = t.w;
+                        }
+                    }
+#pragma unroll 1
+                    for (int i = base + 1; i < un.c; ++i) {
+                        const float e = ex2(__ldcg(p.sig + bh * R + i % R));
+                        const float4 *src = reinterpret_cast<const float4 *>(ring_bh + (i % R) * PN2 + PN);
+                        float4 t[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            t[q] = nv ? __ldcg(src + ring_quad(N, n, quad0 + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            old[4 * q] = fmaf(e, old[4 * q], t[q].x);
+                            old[4 * q + 1] = fmaf(e, old[4 * q + 1], t[q].y);
+                            old[4 * q + 2] = fmaf(e, old[4 * q + 2], t[q].z);
+                            old[4 * q + 3] = fmaf(e, old[4 * q + 3], t[q].w);
+                        }
+                    }
+                    uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
+                    if (own) {
+                        // E = exp(s_{r-1}) S~_{c-1} + S_pre (S~_{c-1} for r = 0) into the tile, and
+                        // S~_c = exp(sigma_c) S~_{c-1} + L_c in place, with L_c exactly as published.  S_pre
+                        // and S_own are read from TMEM before s_full, after which the issuer overwrites them.
+                        const float e_start = ex2(s_ref), e_rest = ex2(s_end - s_ref), e_c = ex2(s_end);
+#pragma unroll
+                        for (int q0 = 0; q0 < 32; q0 += 8) {
+                            uint32_t a[8], b[8];
+                            if (un.r == 1) tmem_ld8(tA + half * 32 + q0 + lane_base, a);
+                            tmem_ld8(tB + half * 32 + q0 + lane_base, b);
+                            tmem_wait_ld();
+                            uint32_t e[4];
+#pragma unroll
+                            for (int q = 0; q < 8; q += 2) {
+                                float ev[2];
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) {
+                                    const float o = old[q0 + q + k];
+                                    const float sp = (un.r == 1) ? __uint_as_float(a[q + k]) : 0.f;
+                                    const float so = __uint_as_float(b[q + k]);
+                                    ev[k] = (un.r == 1) ? fmaf(e_start, o, sp) : o;
+                                    const float l = (un.r == 1) ? fmaf(e_rest, sp, so) : so;
+                                    old[q0 + q + k] = fmaf(e_c, o, l);
+                                }
+                                e[q / 2] = pack_bf16x2(ev[0], ev[1]);
+                            }
+                            sts128(sE + swz(n, half * 4 + q0 / 8),
+                                   nv ? make_uint4(e[0], e[1], e[2], e[3]) : make_uint4(0u, 0u, 0u, 0u));
+                        }
+                        fence_view_async_shared();
+                        fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&pb.s_full);
+                        if (writes_ring) {
+                            float4 *dst = reinterpret_cast<float4 *>(const_cast<float *>(ring_bh) + (un.c % R) * PN2);
+                            if (nv) {
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    __stcg(dst + ring_quad(N, n, quad0 + q),
+                                           make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
+                            }
+                        } else if (nv && p.fin) {
+                            const size_t ld = p.state_ld;
+                            const int pv = p.p_full - p.p_off - half * 32;
+                            float *fin = p.fin + ((size_t)bh * p.p_full + p.p_off + half * 32) * ld + p.n_off + n;
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (q < pv) fin[(size_t)q * ld] = old[q];
+                        }
+                        __syncwarp();
+                        if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
+                    } else {
+                        // S~_{c-1} in bf16 into row n of the tile (128-byte swizzled)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            uint4 t;
+                            t.x = pack_bf16x2(old[8 * k + 0], old[8 * k + 1]);
+                            t.y = pack_bf16x2(old[8 * k + 2], old[8 * k + 3]);
+                            t.z = pack_bf16x2(old[8 * k + 4], old[8 * k + 5]);
+                            t.w = pack_bf16x2(old[8 * k + 6], old[8 * k + 7]);
+                            if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
+                            sts128(sE + swz(n, half * 4 + k), t);
+                        }
+                        fence_view_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive(&pb.s_full);
+                            // the ring entries are consumed: the publisher may count the slot as read
+                            if (un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
+                        }
+                    }
                 }
 
                 // the next head's prefix sums, while this head's products run
@@ -889,7 +1128,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (ctl) {
                         tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
-                        if (has_next && un.c > 0) ready_seen = ld_acquire_gpu(p.ready + bh + 2);
+                        if (has_next && un.c > 0)
+                            ready_seen = ld_acquire_gpu(inc_flag<kD>(p.inc, bh + 2, un.c - 1));
                     }
                 }
             }
@@ -929,10 +1169,11 @@ static int heads_per_unit(const Shape &sh) {
 // Launches the fused kernel for state columns [n_half * 128, ...) and head columns [p_half * 64, ...)
 // of the problem `full` (all of them when full.N <= 128 and full.P <= 64).  The second half of a
 // 256-wide state adds to the y of the first.
+// `pw` is this launch's part of the workspace, laid out as `w`; the status word is shared.
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, float *ring,
-                             int *ready, int *cons, int *counter, int *status, __nv_bfloat16 *y,
-                             const Shape &full, int p_half, int n_half, const FusedDebug *dbg, cudaStream_t st) {
+                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
+                             const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
+                             int n_half, const FusedDebug *dbg, cudaStream_t st) {
     Shape sh = full;
     const int n_off = n_half * 128, p_off = p_half * kP;
     if (full.N > 128) sh.N = 128;
@@ -964,14 +1205,17 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.p_off = p_off;
     p.init = init;
     p.fin = fin;
-    p.ring = ring;
-    p.ready = ready;
-    p.cons = cons;
-    p.counter = counter;
+    p.ring = reinterpret_cast<float *>(pw + w.ring_off);
+    p.inc = reinterpret_cast<int *>(pw + w.inc_off);
+    p.agg = reinterpret_cast<int *>(pw + w.agg_off);
+    p.cons = reinterpret_cast<int *>(pw + w.cons_off);
+    p.sig = reinterpret_cast<float *>(pw + w.sig_off);
+    p.counter = reinterpret_cast<int *>(pw + w.counter_off);
     p.status = status;
     p.y = y;
     p.NK = (sh.N + 63) / 64;
     p.halves = sh.Q / kRows;
+
     p.heads_per_unit = heads_per_unit(sh);
     p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
     p.units_per_role = sh.batch * sh.G * p.blocks_per_group;
@@ -979,7 +1223,10 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;
-    auto kernel = (n_half > 0) ? ssd_fused_kernel<true> : ssd_fused_kernel<false>;
+    // the look-back depth of the workspace's layout (the same shape: P = 64, N <= 128)
+    const bool lookback = fused_lookback(sh) == 4;
+    auto kernel = (n_half > 0) ? (lookback ? ssd_fused_kernel<true, 4> : ssd_fused_kernel<true, 1>)
+                               : (lookback ? ssd_fused_kernel<false, 4> : ssd_fused_kernel<false, 1>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = min(p.n_units, device_sm_count());

@@ -60,6 +60,9 @@ def test_workspace_bytes(lib):
     w256 = f(8, 4096, 32, 64, 1, 256, 256, 1)   # N = 256: two halves, each with its own flags and ring
     ring256 = 2 * 8 * 32 * 3 * 64 * 128 * 4
     assert ring256 <= w256 < ring256 + (1 << 17)
+    wlong = f(1, 131072, 48, 64, 8, 128, 256, 1)   # look-back over 4 chunks: 8 slots of S~ and L
+    ringlong = 48 * 8 * 2 * 64 * 128 * 4
+    assert ringlong <= wlong < ringlong + (1 << 17)
     w32p = f(8, 4096, 32, 32, 1, 128, 256, 1)   # P = 32 is padded: the ring still holds 64 rows
     assert w32p == f(8, 4096, 32, 64, 1, 128, 256, 1)
     assert f(8, 4096, 32, 128, 1, 256, 256, 1) == 2 * w256   # four launches of 64 x 128 states

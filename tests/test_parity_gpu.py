@@ -113,6 +113,31 @@ def test_chunk_size_does_not_change_the_function(Q, cuda_device):
     assert_close(fin, fin_ref, "bf16", f"final_state Q={Q}")
 
 
+@pytest.mark.parametrize("nc", [1, 2, 3, 5, 15, 16, 17, 31, 32, 33, 64, 129, 512])
+def test_chunk_count_sweep_with_initial_state(nc, cuda_device):
+    # 1 to 512 chunks of 128 tokens, the last one ragged: the inter-chunk chain with one hand-off per
+    # chunk (below 32 chunks) and with look-back over 4 chunks (32 and more)
+    T = nc * 128 - (37 if nc > 1 else 0)
+    inp = make_inputs(1, T, 3, 64, 64, 1, "bf16", seed=500 + nc, with_init=True)
+    y, fin = _gpu(inp, 128, cuda_device)
+    y_ref, fin_ref = _oracle(inp)
+    assert_close(y, y_ref, "bf16", f"y nc={nc}")
+    assert_close(fin, fin_ref, "bf16", f"final_state nc={nc}")
+
+
+@pytest.mark.parametrize("case", [(1, 9000, 4, 64, 128, 2, 256), (1, 8300, 2, 128, 256, 1, 256),
+                                  (2, 4500, 3, 32, 64, 3, 128)],
+                         ids=lambda c: "b{}_T{}_H{}_P{}_N{}_G{}_Q{}".format(*c))
+def test_look_back_shapes_match_oracle(case, cuda_device):
+    # long sequences with few heads: the chain uses look-back (with both column splits in the second)
+    batch, T, H, P, N, G, Q = case
+    inp = make_inputs(batch, T, H, P, N, G, "bf16", seed=77 + T, with_init=True)
+    y, fin = _gpu(inp, Q, cuda_device)
+    y_ref, fin_ref = _oracle(inp)
+    assert_close(y, y_ref, "bf16", "y")
+    assert_close(fin, fin_ref, "bf16", "final_state")
+
+
 def test_repeated_runs_are_bitwise_identical(cuda_device):
     w = WORKLOADS["mamba2_2p7b_layer"]
     inp = workload_inputs(w)

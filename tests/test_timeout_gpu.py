@@ -26,9 +26,13 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("withhold", [(0, 0, 0), (1, 3, 1)])
-def test_a_withheld_state_times_out_and_the_device_stays_usable(withhold, cuda_device):
-    batch, T, H, P, N, G, Q = 2, 768, 4, 64, 128, 1, 256
+@pytest.mark.parametrize("shape,withhold", [
+    ((2, 768, 4, 64, 128, 1, 256), (0, 0, 0)),
+    ((2, 768, 4, 64, 128, 1, 256), (1, 3, 1)),
+    ((1, 8448, 2, 64, 128, 1, 256), (0, 1, 5)),   # 33 chunks: look-back finds neither S~_5 nor L_5
+])
+def test_a_withheld_state_times_out_and_the_device_stays_usable(shape, withhold, cuda_device):
+    batch, T, H, P, N, G, Q = shape
     inp = make_inputs(batch, T, H, P, N, G, "bf16", seed=41, with_init=True)
     d = {k: v.to(cuda_device) for k, v in inp.items()}
     lib = S.load()
