@@ -1159,8 +1159,12 @@ static int device_sm_count() {
 
 // Heads per work unit: enough to amortise the unit's C, B and G over several
 // heads, few enough that every SM gets several units.
-static int heads_per_unit(const Shape &sh) {
+// Heads per unit: up to 8 (C, B and G are loaded and formed once per unit).  With look-back (long
+// sequences, few heads) units of 2 heads, one per pipeline: a unit's later heads would otherwise wait
+// behind its first head's chain step, and the chunks in flight would advance at that pace.
+static int heads_per_unit(const Shape &sh, bool lookback) {
     const int hpg = sh.heads_per_group;
+    if (lookback) return hpg < 2 ? hpg : 2;
     if (hpg <= 8) return hpg;
     const int blocks = (hpg + 7) / 8;
     return (hpg + blocks - 1) / blocks;
@@ -1216,15 +1220,14 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.NK = (sh.N + 63) / 64;
     p.halves = sh.Q / kRows;
 
-    p.heads_per_unit = heads_per_unit(sh);
+    const bool lookback = fused_lookback(sh) == 4;  // the workspace's layout has the same shape
+    p.heads_per_unit = heads_per_unit(sh, lookback);
     p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
     p.units_per_role = sh.batch * sh.G * p.blocks_per_group;
     p.n_units = sh.nc * p.units_per_role * p.halves;
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;
-    // the look-back depth of the workspace's layout (the same shape: P = 64, N <= 128)
-    const bool lookback = fused_lookback(sh) == 4;
     auto kernel = (n_half > 0) ? (lookback ? ssd_fused_kernel<true, 4> : ssd_fused_kernel<true, 1>)
                                : (lookback ? ssd_fused_kernel<false, 4> : ssd_fused_kernel<false, 1>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
