@@ -63,9 +63,13 @@ enum {
 
 /*
  * Bytes of device workspace ssd_fwd needs for this problem (256-byte
- * multiple).  Returns 0 for invalid dimensions.  The workspace holds the
- * per-chunk log-decay prefix sums (stage 0 / 1), the chunk states (stages 2-3)
- * and a status word.
+ * multiple).  Returns 0 for invalid dimensions.  The workspace holds a status
+ * word and, on the CUDA-core path, the per-chunk log-decay prefix sums and the
+ * chunk states (stages 0-3); on the fused tensor-core path (bf16 x, B, C;
+ * Q in {128, 256}; P a multiple of 8 up to 64, or 128; N a multiple of 16 up
+ * to 128, or 256), per launch, the unit counter, the inter-chunk hand-off
+ * flags and an L2-sized ring of the latest chunk states (with the local
+ * chunk states too where a long sequence uses look-back).
  */
 SSD_API size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
 
