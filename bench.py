@@ -399,6 +399,8 @@ def main():
             line["workloads"] = measure_workloads(w, dev, stream, flush, peaks)
         line["decode_step"] = measure_decode(w, host, dev, stream, flush, peaks)
         line["gate_norm"] = measure_gate_norm(w, y, dev, stream, flush, peaks)
+        line["gated_forward"] = measure_gated(w, d, dev, stream, flush, line["gate_norm"]["us_per_launch"],
+                                              ms_per_step)
         line["backward"] = measure_backward(w, d, dev, stream, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(host, w)
@@ -527,6 +529,42 @@ def measure_gate_norm(w, y, dev, stream, flush, peaks, steps=20):
     gbps = alg / (ms * 1e-3) / 1e9
     return {"rows": y.numel() // (w.H * w.P), "channels": w.H * w.P, "ngroups": w.H, "dtype": w.dtype,
             "alg_bytes": alg, "us_per_launch": ms * 1e3, "GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"]}
+
+
+def measure_gated(w, d, dev, stream, flush, gate_us, fwd_ms, steps=20):
+    """The forward with the gate and the per-head GroupNorm in the fused kernel's drain (ssd_fwd_gated) on
+    this workload, L2 flushed before each call, against the forward followed by the gate kernel (the
+    step line's ms_per_step plus the gate_norm object's time)."""
+    import torch
+    from structured_state_space_ssd_b200 import ssd as S
+    gen = torch.Generator().manual_seed(w.seed + 11)
+    z = torch.randn(tuple(d["x"].shape), generator=gen).to(d["x"].dtype).to(dev)
+    wt = (torch.rand(w.H * w.P, generator=gen) + 0.5).to(dev)
+    bs = torch.randn(w.H * w.P, generator=gen).to(dev)
+    out = torch.empty_like(d["x"])
+    fin = torch.empty((w.batch, w.H, w.P, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(S.ssd_fwd_workspace_bytes(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def one():
+        S.ssd_fwd_gated(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], w.Q, z, d["init_state"], wt, bs, 1e-5,
+                        out=out, final_state=fin, workspace=ws, stream=stream)
+
+    for _ in range(3):
+        flush.zero_()
+        one()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    launches = S.load().ssd_fwd_gated_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q,
+                                                   S._dtype_code(d["x"].dtype))
+    return {"ms_per_call": ms, "tokens_per_s": w.batch * w.T / (ms * 1e-3), "launches_per_call": launches,
+            "separate_ms": fwd_ms + gate_us * 1e-3, "with": "z, norm weight and bias; one group per head"}
 
 
 def backward_alg_flops(w):

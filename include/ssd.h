@@ -237,6 +237,37 @@ SSD_API int ssd_gate_norm(const void *y, const void *z, const float *weight, con
                   long long rows, int channels, int ngroups, float eps, int dtype, void *stream);
 
 /*
+ * The layer forward followed by the block's gate and GroupNorm with a group
+ * per head ("Transformers are SSMs", analysis page, section "The Mamba-2
+ * Architecture", paragraphs "Gating" and "Extra normalization"): per token
+ * and head, with y the ssd_fwd output and g = y * silu(z),
+ *
+ *     out = (g - mean(g)) / sqrt(var(g) + eps) * norm_weight + norm_bias
+ *
+ * over the head's P channels (population variance), i.e. ssd_gate_norm with
+ * ngroups = H on ssd_fwd's y.  Arguments as for ssd_fwd, plus
+ *
+ *   z            [batch][T][H][P]  dtype   the gate branch
+ *   norm_weight  [H * P]           fp32    NULL = 1 (16-byte aligned)
+ *   norm_bias    [H * P]           fp32    NULL = 0 (16-byte aligned)
+ *   eps          >= 0
+ *   out          [batch][T][H][P]  dtype   written in place of y; y itself is not returned
+ *
+ * On the fused tensor-core path with P = 64 and N <= 128 the gate and the norm
+ * run in the kernel's drain on the fp32 y (one launch, y never reaches
+ * memory); elsewhere ssd_fwd writes y into out and ssd_gate_norm runs over it
+ * in place (one more launch).  z must not overlap out.  Same workspace as
+ * ssd_fwd.  Returns as ssd_fwd.
+ */
+SSD_API int ssd_fwd_gated(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                  const float *D, int Q, const float *init_state, const void *z, const float *norm_weight,
+                  const float *norm_bias, float eps, void *out, float *final_state, int batch, int T, int H,
+                  int P, int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Kernel launches ssd_fwd_gated issues for these arguments (0 when they are invalid). */
+SSD_API int ssd_fwd_gated_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
+
+/*
  * Sequence split: contiguous shards of one sequence (on one GPU or one per
  * worker) run ssd_fwd from a zero state at the same time and exchange only
  * their states.  Workers process contiguous shards and pass recurrent states

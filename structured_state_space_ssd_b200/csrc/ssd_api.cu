@@ -19,7 +19,7 @@ bool fused_supported(const Shape &sh, int dtype);
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
                              const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
-                             int n_half, const FusedDebug *dbg, cudaStream_t st);
+                             int n_half, const FusedDebug *dbg, const FusedGate *gate, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -105,7 +105,8 @@ int run_simt(const Shape &sh, const T *x, const float *dt, const float *A, const
 
 int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
               const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
-              const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg) {
+              const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg,
+              const ssd::FusedGate *gate) {
     if (!mk.mark(1, st)) return SSD_ERR_CUDA;
     // launch k covers head-column half k % pp and state-column half k / pp: the second state half adds to
     // the y its first half wrote, so it comes after both head-column launches of that first half
@@ -114,7 +115,7 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
     for (int k = 0; k < passes; ++k) {
         char *pw = ws + k * stride;
         if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, pw, w, reinterpret_cast<int *>(ws + w.status_off), y,
-                                  sh, k % pp, k / pp, dbg, st) != cudaSuccess ||
+                                  sh, k % pp, k / pp, dbg, gate, st) != cudaSuccess ||
             !mk.mark(2 + k, st))
             return SSD_ERR_CUDA;
     }
@@ -124,7 +125,7 @@ int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const fl
 int fwd_impl(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D, int Q,
              const float *init_state, void *y, float *final_state, int batch, int T, int H, int P, int G, int N,
              int dtype, void *workspace, size_t workspace_bytes, void *stream, const Marks &mk,
-             const ssd::FusedDebug *dbg = nullptr) {
+             const ssd::FusedDebug *dbg = nullptr, const ssd::FusedGate *gate = nullptr) {
     Shape sh;
     int rc = check_dims(batch, T, H, P, G, N, Q, dtype, &sh);
     if (rc != SSD_OK) return rc;
@@ -144,6 +145,14 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     if (ybytes && (overlaps(y, ybytes, x, ybytes) || overlaps(y, ybytes, B, bcbytes) ||
                    overlaps(y, ybytes, C, bcbytes)))
         return SSD_ERR_INVALID_ARG;
+    // the gate in the fused kernel's drain: one launch with whole 64-column heads
+    const bool gate_fused = gate && path == ssd::kPathFused && ssd::fused_passes(sh) == 1 && P == 64;
+    if (gate) {
+        if ((T > 0 && !gate->z) || !(gate->eps >= 0.f) || !aligned(gate->z, gate_fused ? 16 : es) ||
+            !aligned(gate->weight, 16) || !aligned(gate->bias, 16) || (ybytes && overlaps(y, ybytes, gate->z, ybytes)))
+            return SSD_ERR_INVALID_ARG;
+        if (P > 4096) return SSD_ERR_UNSUPPORTED;
+    }
 
     if (dbg && path != ssd::kPathFused) return SSD_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -163,16 +172,22 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
         return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
     }
     if (path == ssd::kPathFused)
-        return run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
-                         static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
-                         final_state, ws, w, st, mk, dbg);
-    if (dtype == SSD_BF16)
-        return run_simt<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
-                                       static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C),
-                                       D, init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, w, st, mk);
-    return run_simt<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
-                           static_cast<const float *>(C), D, init_state, static_cast<float *>(y), final_state, ws,
-                           w, st, mk);
+        rc = run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+                       static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
+                       final_state, ws, w, st, mk, dbg, gate_fused ? gate : nullptr);
+    else if (dtype == SSD_BF16)
+        rc = run_simt<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
+                                     static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C), D,
+                                     init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, w, st, mk);
+    else
+        rc = run_simt<float>(sh, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
+                             static_cast<const float *>(C), D, init_state, static_cast<float *>(y), final_state, ws,
+                             w, st, mk);
+    // elsewhere the gate runs as its own kernel over the y just written (in place)
+    if (rc == SSD_OK && gate && !gate_fused)
+        rc = ssd_gate_norm(y, gate->z, gate->weight, gate->bias, y, (long long)batch * T, H * P, H, gate->eps, dtype,
+                           stream);
+    return rc;
 }
 
 }  // namespace
@@ -248,6 +263,24 @@ int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B,
             return SSD_ERR_CUDA;
     }
     return SSD_OK;
+}
+
+int ssd_fwd_gated(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
+                  int Q, const float *init_state, const void *z, const float *norm_weight, const float *norm_bias,
+                  float eps, void *out, float *final_state, int batch, int T, int H, int P, int G, int N, int dtype,
+                  void *workspace, size_t workspace_bytes, void *stream) {
+    ssd::FusedGate gate{z, norm_weight, norm_bias, eps};
+    return fwd_impl(x, dt, A, B, C, D, Q, init_state, out, final_state, batch, T, H, P, G, N, dtype, workspace,
+                    workspace_bytes, stream, Marks{}, nullptr, &gate);
+}
+
+int ssd_fwd_gated_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
+    Shape sh;
+    if (check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;
+    const ssd::Path path = choose_path(sh, dtype);
+    const int k = launch_count(sh, path);
+    if (k == 0) return 0;
+    return (path == ssd::kPathFused && ssd::fused_passes(sh) == 1 && P == 64) ? k : k + 1;
 }
 
 int ssd_fwd_withhold_publish(const void *x, const float *dt, const float *A, const void *B, const void *C,

@@ -112,6 +112,14 @@ inline size_t fused_slot_floats(const Shape &s, int d) { return (size_t)64 * s.N
 // {128, 256}).
 enum Path { kPathSimt = 0, kPathFused = 1 };
 
+// Gate and per-head GroupNorm applied in the fused kernel's drain (ssd_fwd_gated): z as x, bf16;
+// weight and bias [H * P] fp32 or null.
+struct FusedGate {
+    const void *z;
+    const float *weight, *bias;
+    float eps;
+};
+
 // Test hooks of the fused kernel's hand-off (ssd_fwd_withhold_publish):
 // each wait on another CTA's flag gives up after flag_polls polls (0: the
 // default bound), and the owner of chunk withhold_c of sequence withhold_bh

@@ -79,7 +79,8 @@ constexpr uint32_t kOffPipe = 98304;    // per pipeline: x rows 0..127 | W | x r
 constexpr uint32_t kPipeBytes = 49152;  // W: scaled x rows, then the entering-state tile [n][p]
 constexpr uint32_t kOffAux = kOffPipe + 2 * kPipeBytes;
 constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units), column factors, warp totals
-constexpr uint32_t kSmemBytes = kOffAux + 2 * kAuxFloats * 4 + 1024;
+constexpr uint32_t kOffStat = kOffAux + 2 * kAuxFloats * 4;  // gated drain: per pipeline, half, row (mean, M2)
+constexpr uint32_t kSmemBytes = kOffStat + 2 * 2 * kRows * 8 + 1024;
 
 constexpr uint32_t kDefaultFlagPolls = 1u << 22;
 
@@ -116,6 +117,11 @@ struct Params {
     // (D == null) and adds its result to the y the first one wrote (kernel template argument).
     int state_ld;
     int n_off;
+    // Gated output (kernel template argument kGated): out = GroupNorm(y * silu(z)) with a group per head
+    // (its 64 channels), written through the y tensor map in y's place; y itself is not written.
+    const __nv_bfloat16 *z;  // [b][T][H][64]
+    const float *gw, *gb;    // [H * 64] or null (1, 0)
+    float eps;
     // The tile is 64 columns of p wide: a head dimension below 64 is zero-padded (x loads past P read
     // zero, y stores past P are clipped, state rows past P are neither read nor written), and P = 128
     // runs as two launches over columns p_off = 0 and 64 (the rows of the state are independent).
@@ -289,7 +295,8 @@ using namespace fz;
 
 // kAccum: the second half of a 256-wide state, which adds its y to the first half's.
 // kD: the chain's look-back depth D (1: every owner waits for the chunk before).
-template <bool kAccum, int kD>
+// kGated: the drain applies the gate and the per-head GroupNorm (Params::z) and stores that instead of y.
+template <bool kAccum, int kD, bool kGated>
 __global__ void __launch_bounds__(fz::kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                      const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY,
@@ -643,6 +650,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
                 const float Dh = d_cur;
                 if (has_next) d_cur = p.D ? __ldg(p.D + h + 2) : 0.f;
+                // gated drain: this head's z rows on their way to L2 (one 128-byte line per row)
+                if (kGated && half == 0 && j < un.len)
+                    prefetch_l2(p.z + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP);
                 const float s_end = sJ[end];
                 const float s_ref = (un.r == 1) ? sJ[kRows - 1] : 0.f;  // s_{r-1}
                 const float sj = sJ[j];
@@ -1076,6 +1086,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     }
                 }
 
+                // gated drain: z of this row's 32 channels, loaded while the products run
+                uint4 zv[4];
+                if (kGated) {
+                    const bool jv = j < un.len;
+                    const uint4 *zp = reinterpret_cast<const uint4 *>(
+                        p.z + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP + half * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) zv[q] = jv ? __ldg(zp + q) : make_uint4(0u, 0u, 0u, 0u);
+                }
+
                 // the next head's prefix sums, while this head's products run
                 if (has_next) scan(dt_next, a_next);
 
@@ -1094,7 +1114,75 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
                 wait_bar(&pb.mx_done, par(use), p.status, broken);
                 fence_after_sync();
-                {
+                if constexpr (kGated) {
+                    // g = y * silu(z) in fp32 (y is never rounded), then the row's 64 channels normalised:
+                    // two passes over this thread's 32, merged with the other warpgroup's through shared
+                    // memory (mean and sum of squared deviations of two halves of 32)
+                    float g[32];
+#pragma unroll
+                    for (int q0 = 0; q0 < 32; q0 += 16) {
+                        uint32_t a[16], b[16];
+                        tmem_ld16(tA + half * 32 + q0 + lane_base, a);
+                        tmem_ld16(tB + half * 32 + q0 + lane_base, b);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float2 r =
+                                fma_f32x2(make_float2(ej, ej),
+                                          make_float2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1])),
+                                          make_float2(__uint_as_float(b[2 * q]), __uint_as_float(b[2 * q + 1])));
+                            const uint4 &v = zv[q0 / 8 + q / 4];
+                            const uint32_t zz = (q & 3) == 0 ? v.x : (q & 3) == 1 ? v.y : (q & 3) == 2 ? v.z : v.w;
+                            const float z0 = bf16lo(zz), z1 = bf16hi(zz);
+                            g[q0 + 2 * q] = r.x * silu_approx(z0);
+                            g[q0 + 2 * q + 1] = r.y * silu_approx(z1);
+                        }
+                    }
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pb.acc_free);
+                    float sa[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: shorter dependent chains
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sa[q & 3] += g[q];
+                    const float m = ((sa[0] + sa[1]) + (sa[2] + sa[3])) * (1.f / 32);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) sa[k] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) sa[q & 3] = fmaf(g[q] - m, g[q] - m, sa[q & 3]);
+                    const float m2 = (sa[0] + sa[1]) + (sa[2] + sa[3]);
+                    float2 *sStat = reinterpret_cast<float2 *>(smem + kOffStat) + pl * 2 * kRows;
+                    sStat[half * kRows + lrow] = make_float2(m, m2);
+                    named_bar_sync(bar_id, kPipeThreads);
+                    const float2 o = sStat[(1 - half) * kRows + lrow];
+                    const float dm = m - o.x;
+                    const float mean = 0.5f * (m + o.x);
+                    const float rstd = rsqrtf(fmaf(16.f * dm, dm, m2 + o.y) * (1.f / 64) + p.eps);
+                    const float4 *wp = p.gw ? reinterpret_cast<const float4 *>(p.gw + h * kP + half * 32) : nullptr;
+                    const float4 *bp = p.gb ? reinterpret_cast<const float4 *>(p.gb + h * kP + half * 32) : nullptr;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t o4[4];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int q = 8 * k + 4 * e;
+                            const float4 wv = wp ? __ldg(wp + q / 4) : make_float4(1.f, 1.f, 1.f, 1.f);
+                            const float4 bv = bp ? __ldg(bp + q / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            o4[2 * e] = pack_bf16x2(fmaf((g[q] - mean) * rstd, wv.x, bv.x),
+                                                    fmaf((g[q + 1] - mean) * rstd, wv.y, bv.y));
+                            o4[2 * e + 1] = pack_bf16x2(fmaf((g[q + 2] - mean) * rstd, wv.z, bv.z),
+                                                        fmaf((g[q + 3] - mean) * rstd, wv.w, bv.w));
+                        }
+                        sts128(sW + swz(lrow, half * 4 + k), make_uint4(o4[0], o4[1], o4[2], o4[3]));
+                    }
+                    fence_view_async_shared();
+                    named_bar_sync(bar_id, kPipeThreads);
+                    if (ctl) {
+                        tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
+                        bulk_commit();
+                        if (has_next && un.c > 0)
+                            ready_seen = ld_acquire_gpu(inc_flag<kD>(p.inc, bh + 2, un.c - 1));
+                    }
+                } else {
 #pragma unroll
                     for (int q0 = 0; q0 < 32; q0 += 16) {
                         uint32_t a[16], b[16];
@@ -1177,7 +1265,9 @@ static int heads_per_unit(const Shape &sh, bool lookback) {
 cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
                              const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
-                             int n_half, const FusedDebug *dbg, cudaStream_t st) {
+                             int n_half, const FusedDebug *dbg, const FusedGate *gate, cudaStream_t st) {
+    // the gate needs the whole row of a head in one launch
+    if (gate && (full.P != kP || full.N > 128)) return cudaErrorInvalidValue;
     Shape sh = full;
     const int n_off = n_half * 128, p_off = p_half * kP;
     if (full.N > 128) sh.N = 128;
@@ -1205,6 +1295,10 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.D = (n_half == 0) ? D : nullptr;
     p.state_ld = full.N;
     p.n_off = n_off;
+    p.z = gate ? static_cast<const __nv_bfloat16 *>(gate->z) : nullptr;
+    p.gw = gate ? gate->weight : nullptr;
+    p.gb = gate ? gate->bias : nullptr;
+    p.eps = gate ? gate->eps : 0.f;
     p.p_full = full.P;
     p.p_off = p_off;
     p.init = init;
@@ -1228,8 +1322,9 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;
-    auto kernel = (n_half > 0) ? (lookback ? ssd_fused_kernel<true, 4> : ssd_fused_kernel<true, 1>)
-                               : (lookback ? ssd_fused_kernel<false, 4> : ssd_fused_kernel<false, 1>);
+    auto kernel = gate ? (lookback ? ssd_fused_kernel<false, 4, true> : ssd_fused_kernel<false, 1, true>)
+                  : (n_half > 0) ? (lookback ? ssd_fused_kernel<true, 4, false> : ssd_fused_kernel<true, 1, false>)
+                                 : (lookback ? ssd_fused_kernel<false, 4, false> : ssd_fused_kernel<false, 1, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = min(p.n_units, device_sm_count());

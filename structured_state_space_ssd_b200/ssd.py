@@ -22,7 +22,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "S
           4: "SSD_ERR_TIMEOUT"}
 
 # Every symbol include/ssd.h declares.
-EXPORTS = ("ssd_fwd", "ssd_fwd_workspace_bytes", "ssd_fwd_launch_count", "ssd_fwd_timed",
+EXPORTS = ("ssd_fwd", "ssd_fwd_gated", "ssd_fwd_gated_launch_count", "ssd_fwd_workspace_bytes",
+           "ssd_fwd_launch_count", "ssd_fwd_timed",
            "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_fwd_withhold_publish", "ssd_status_string", "ssd_version",
            "ssd_fwd_no_alloc", "ssd_fwd_no_alloc_check", "ssd_step", "ssd_gate_norm", "ssd_split_logdecay",
            "ssd_split_combine", "ssd_split_correct", "ssd_bwd", "ssd_bwd_workspace_bytes")
@@ -52,6 +53,11 @@ def load():
     vp, fp, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.ssd_fwd.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.ssd_fwd.restype = i
+    lib.ssd_fwd_gated.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, fp, ctypes.c_float, vp, fp, i, i, i, i, i,
+                                  i, i, vp, sz, vp]
+    lib.ssd_fwd_gated.restype = i
+    lib.ssd_fwd_gated_launch_count.argtypes = [i] * 8
+    lib.ssd_fwd_gated_launch_count.restype = i
     lib.ssd_fwd_workspace_bytes.argtypes = [i] * 8
     lib.ssd_fwd_workspace_bytes.restype = sz
     lib.ssd_fwd_launch_count.argtypes = [i] * 8
@@ -141,9 +147,71 @@ def ssd_fwd(x, dt, A, B, C, D, Q: int, init_state=None, *, y=None, final_state=N
     it waits for the stream and appends each kernel's milliseconds, then the
     whole call's span, to the list.
     """
+    b, T, H, P, G, N, code, workspace, handle = _prepare_fwd(x, dt, A, B, C, D, Q, init_state, workspace, stream,
+                                                             "ssd_fwd")
+    dev = x.device
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    lib = load()
+    args = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(Q), _ptr(init_state),
+            _ptr(y), _ptr(final_state), b, T, H, P, G, N, code, _ptr(workspace),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size()), ctypes.c_void_p(handle))
+    if stage_ms is None:
+        rc = lib.ssd_fwd(*args)
+        if rc != 0:
+            raise SSDError(rc, "ssd_fwd")
+    else:
+        ms = (ctypes.c_float * 8)()
+        total = ctypes.c_float(0)
+        rc = lib.ssd_fwd_timed(*args, ctypes.cast(ms, ctypes.c_void_p), 8,
+                               ctypes.cast(ctypes.pointer(total), ctypes.c_void_p))
+        if rc != 0:
+            raise SSDError(rc, "ssd_fwd_timed")
+        k = int(lib.ssd_fwd_launch_count(b, T, H, P, G, N, int(Q), code))
+        stage_ms.extend(float(ms[i]) for i in range(min(k, 8)))
+        stage_ms.append(float(total.value))
+    return y, final_state
+
+
+def ssd_fwd_gated(x, dt, A, B, C, D, Q: int, z, init_state=None, norm_weight=None, norm_bias=None,
+                  eps: float = 1e-5, *, out=None, final_state=None, return_final_state: bool = True,
+                  workspace=None, stream=None):
+    """The layer forward followed by the gate and a GroupNorm with a group per head, on the GPU.
+
+    Arguments as for ``ssd_fwd``, plus z (x's shape and dtype) and the norm's fp32 [H*P] weight and bias
+    (None: 1 and 0).  Returns ``(out, final_state)`` with out = GroupNorm(y * silu(z)) over each head's P
+    channels (y itself is not returned).  One fused launch where the tensor-core path takes whole
+    64-column heads in one launch; otherwise ``ssd_fwd`` then ``ssd_gate_norm`` in place.
+    """
+    b, T, H, P, G, N, code, workspace, handle = _prepare_fwd(x, dt, A, B, C, D, Q, init_state, workspace, stream,
+                                                             "ssd_fwd_gated")
+    dev = x.device
+    if z.shape != x.shape or z.dtype != x.dtype or z.device != dev or not z.is_contiguous():
+        raise ValueError("z must be a contiguous tensor of x's shape, dtype and device")
+    for k, t in (("norm_weight", norm_weight), ("norm_bias", norm_bias)):
+        if t is not None and (t.dtype != torch.float32 or t.numel() != H * P or t.device != dev
+                              or not t.is_contiguous()):
+            raise ValueError(f"{k} must be a contiguous float32 [{H * P}] tensor on {dev}")
+    if out is None:
+        out = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    rc = load().ssd_fwd_gated(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(Q), _ptr(init_state),
+                              _ptr(z), _ptr(norm_weight), _ptr(norm_bias), float(eps), _ptr(out), _ptr(final_state),
+                              b, T, H, P, G, N, code, _ptr(workspace),
+                              ctypes.c_size_t(workspace.numel() * workspace.element_size()), ctypes.c_void_p(handle))
+    if rc != 0:
+        raise SSDError(rc, "ssd_fwd_gated")
+    return out, final_state
+
+
+def _prepare_fwd(x, dt, A, B, C, D, Q, init_state, workspace, stream, what):
+    """Argument checks shared by the forward entry points; returns the dims, dtype code, workspace, stream."""
     dev = x.device
     if dev.type != "cuda":
-        raise ValueError("ssd_fwd needs CUDA tensors (there is no CPU path)")
+        raise ValueError(f"{what} needs CUDA tensors (there is no CPU path)")
     b, T, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     code = _dtype_code(x.dtype)
@@ -166,12 +234,7 @@ def ssd_fwd(x, dt, A, B, C, D, Q: int, init_state=None, *, y=None, final_state=N
         raise ValueError("B and C must be [b,T,G,N]")
     if init_state is not None and tuple(init_state.shape) != (b, H, P, N):
         raise ValueError("init_state must be [b,H,P,N]")
-    if y is None:
-        y = torch.empty_like(x)
-    if final_state is None and return_final_state:
-        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
-    lib = load()
-    need = int(lib.ssd_fwd_workspace_bytes(b, T, H, P, G, N, int(Q), code))
+    need = int(load().ssd_fwd_workspace_bytes(b, T, H, P, G, N, int(Q), code))
     if need == 0:
         raise SSDError(1, "ssd_fwd_workspace_bytes")
     if workspace is None or workspace.numel() * workspace.element_size() < need:
@@ -179,24 +242,7 @@ def ssd_fwd(x, dt, A, B, C, D, Q: int, init_state=None, *, y=None, final_state=N
     if stream is None:
         stream = torch.cuda.current_stream(dev)
     handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-    args = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(Q), _ptr(init_state),
-            _ptr(y), _ptr(final_state), b, T, H, P, G, N, code, _ptr(workspace),
-            ctypes.c_size_t(workspace.numel() * workspace.element_size()), ctypes.c_void_p(handle))
-    if stage_ms is None:
-        rc = lib.ssd_fwd(*args)
-        if rc != 0:
-            raise SSDError(rc, "ssd_fwd")
-    else:
-        ms = (ctypes.c_float * 8)()
-        total = ctypes.c_float(0)
-        rc = lib.ssd_fwd_timed(*args, ctypes.cast(ms, ctypes.c_void_p), 8,
-                               ctypes.cast(ctypes.pointer(total), ctypes.c_void_p))
-        if rc != 0:
-            raise SSDError(rc, "ssd_fwd_timed")
-        k = int(lib.ssd_fwd_launch_count(b, T, H, P, G, N, int(Q), code))
-        stage_ms.extend(float(ms[i]) for i in range(min(k, 8)))
-        stage_ms.append(float(total.value))
-    return y, final_state
+    return b, T, H, P, G, N, code, workspace, handle
 
 
 def ssd_fwd_check(workspace, stream=None) -> int:
