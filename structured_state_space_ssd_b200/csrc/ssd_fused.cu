@@ -452,6 +452,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 next_u = -1;
                 continue;
             }
+            // this pipeline's first head of the unit: its x rows now, ahead of C, B and G (the pipeline's own
+            // products of the previous unit have completed, so its x buffers are free)
+            const int h_first = un.h0 + pl;
+            if (leader && h_first < un.h1) {
+                mbar_arrive_expect_tx(&pb.x_full, ((un.r == 1) ? 2u : 1u) * 16384u);
+                tma_load_4d(sXlo, &mX, &pb.x_full, 0, h_first, un.t0, un.b);
+                if (un.r == 1) tma_load_4d(sXhi, &mX, &pb.x_full, 0, h_first, un.t0 + kRows, un.b);
+            }
+            __syncwarp();
             if (pl == 0) {
                 // both pipelines are done with the previous unit's C, B and G
                 if (udone > 0) wait_bar(&bars.unit_done, par(udone - 1), p.status, broken);
@@ -477,6 +486,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             for (int hh = nx.h0; hh < min(nx.h0 + 2, nx.h1); ++hh)
                                 for (int q = 0; q <= nx.r; ++q)
                                     tma_prefetch_4d(&mX, 0, hh, nx.t0 + q * kRows, nx.b);
+                            // the chunk's dt (all heads: one contiguous block) for the first prefix sums
+                            const float *dtb = p.dt + ((size_t)nx.b * sh.T + nx.t0) * sh.H;
+                            const uint32_t dtbytes = ((uint32_t)nx.len * sh.H * 4u) & ~15u;
+                            if ((reinterpret_cast<uintptr_t>(dtb) & 15) == 0 && dtbytes > 0)
+                                bulk_prefetch_l2(dtb, dtbytes);
                         }
                     }
                 }
@@ -506,13 +520,16 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             bool any = false;
             for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
                 any = true;
-                // this head's x rows; warm L2 for the pipeline's next head
+                // this head's x rows (the unit's first head's are already on their way); warm L2 for the
+                // pipeline's next head
                 if (use > 0) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
                 if (leader) {
                     const uint32_t xboxes = (un.r == 1) ? 2u : 1u;
-                    mbar_arrive_expect_tx(&pb.x_full, xboxes * 16384u);
-                    tma_load_4d(sXlo, &mX, &pb.x_full, 0, h, un.t0, un.b);
-                    if (un.r == 1) tma_load_4d(sXhi, &mX, &pb.x_full, 0, h, un.t0 + kRows, un.b);
+                    if (h != h_first) {
+                        mbar_arrive_expect_tx(&pb.x_full, xboxes * 16384u);
+                        tma_load_4d(sXlo, &mX, &pb.x_full, 0, h, un.t0, un.b);
+                        if (un.r == 1) tma_load_4d(sXhi, &mX, &pb.x_full, 0, h, un.t0 + kRows, un.b);
+                    }
                     if (h + 2 < un.h1)
                         for (uint32_t q = 0; q < xboxes; ++q)
                             tma_prefetch_4d(&mX, 0, h + 2, un.t0 + (int)q * kRows, un.b);

@@ -383,6 +383,11 @@ __device__ __forceinline__ float silu_approx(float z) {
     return fmaf(h, tanh_approx(h), h);
 }
 
+// Bring `bytes` bytes from p on into L2 (p 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Bring the 128-byte line holding p into L2.
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
