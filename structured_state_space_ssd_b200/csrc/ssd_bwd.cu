@@ -35,12 +35,21 @@ cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S,
 cudaError_t launch_state_passing(float *S, const float *s, const float *init, float *fin, const Shape &sh,
                                  cudaStream_t st);
 
+// The masked scans on the tensor cores (ssd_bwd_tc.cu); which of the three run there: bit 0 dx, bit 1 the
+// per-head dB terms, bit 2 the per-head dC terms.
+bool scan_tc_supported(const Shape &sh, int dtype);
+cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int k_head, const void *V, int v_head,
+                                  int KD, int W, bool anti, const float *St, int st_kw, const float *D, void *out,
+                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st);
+constexpr int kScanTcRoles = 7;
+
 namespace {
 
 // ---------------------------------------------------------------------------
 // Workspace of one backward call (all offsets 256-byte aligned).
 // ---------------------------------------------------------------------------
 struct BwdWorkspace {
+    size_t status_off;  // int status word of the tensor-core scans' bounded waits (cleared per call)
     size_t s_off;     // float s[batch][H][nc][Q]
     size_t hin_off;   // float Hin[batch][nc][H][P][N]: chunk states, then the state entering each chunk
     size_t gout_off;  // float G[batch][nc][H][P][N]: chunk sums of dy C^T, then dHout of each chunk
@@ -59,6 +68,8 @@ BwdWorkspace bwd_layout(const Shape &s) {
     const size_t states = sizeof(float) * (size_t)s.batch * s.nc * s.H * PN;
     const size_t perhead = sizeof(float) * (size_t)s.batch * s.T * s.H * s.N;
     size_t off = 0;
+    w.status_off = off;
+    off = 256;
     w.s_off = off;
     off = align256(off + sizeof(float) * bh * s.nc * s.Q);
     w.hin_off = off;
@@ -629,6 +640,8 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     float *dsig = reinterpret_cast<float *>(ws + w.dsig_off);
     double *pa = reinterpret_cast<double *>(ws + w.pa_off);
     double *pd = reinterpret_cast<double *>(ws + w.pd_off);
+    int *status = reinterpret_cast<int *>(ws + w.status_off);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
     if (launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     // forward states: Hin_c, and the final state when a final-state gradient is given
     if (launch_chunk_state<T>(x, B, s, Hin, sh, st, false) != cudaSuccess) return SSD_ERR_CUDA;
@@ -643,15 +656,36 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     const bool al = is_aligned(x, 16) && is_aligned(dy, 16) && is_aligned(B, 16) && is_aligned(C, 16);
     const int vec = al && sh.P % VE == 0 && sh.N % VE == 0;
     const int st_vec = sh.P % 4 == 0 && sh.N % 4 == 0;
+    // The three masked scans: on the tensor cores (ssd_bwd_tc.cu) for bf16 inputs with P = 64, N in {64, 128},
+    // Q in {128, 256} and 16-byte aligned tensors, else on the CUDA cores.
+    const bool tc = scan_tc_supported(sh, sizeof(T) == 2 ? SSD_BF16 : SSD_F32) && al && kScanTcRoles != 0;
     // dx: rows of B against columns of C, values dy, state dHout as [P][N] = [W][KD], skip D dy
-    ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx, vec, st_vec};
-    if (launch_scan<T, T, true>(ax, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (tc && (kScanTcRoles & 1)) {
+        if (launch_masked_scan_tc(B, 0, C, 0, dy, 1, sh.N, sh.P, true, Gout, 0, D, dx, true, s, status, sh, st) !=
+            cudaSuccess)
+            return SSD_ERR_CUDA;
+    } else {
+        ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx, vec, st_vec};
+        if (launch_scan<T, T, true>(ax, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    }
     // dB^(h): rows of x against columns of dy, values C, state dHout as [P][N] = [KD][W]
-    ScanArgs ab{x, dy, C, 1, 1, 0, Gout, 1, sh.P, sh.N, nullptr, dBh, vec, st_vec};
-    if (launch_scan<T, float, true>(ab, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (tc && (kScanTcRoles & 2)) {
+        if (launch_masked_scan_tc(x, 1, dy, 1, C, 0, sh.P, sh.N, true, Gout, 1, nullptr, dBh, false, s, status, sh,
+                                  st) != cudaSuccess)
+            return SSD_ERR_CUDA;
+    } else {
+        ScanArgs ab{x, dy, C, 1, 1, 0, Gout, 1, sh.P, sh.N, nullptr, dBh, vec, st_vec};
+        if (launch_scan<T, float, true>(ab, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    }
     // dC^(h): rows of dy against columns of x, values B, state Hin as [P][N] = [KD][W]
-    ScanArgs ac{dy, x, B, 1, 1, 0, Hin, 1, sh.P, sh.N, nullptr, dCh, vec, st_vec};
-    if (launch_scan<T, float, false>(ac, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    if (tc && (kScanTcRoles & 4)) {
+        if (launch_masked_scan_tc(dy, 1, x, 1, B, 0, sh.P, sh.N, false, Hin, 1, nullptr, dCh, false, s, status, sh,
+                                  st) != cudaSuccess)
+            return SSD_ERR_CUDA;
+    } else {
+        ScanArgs ac{dy, x, B, 1, 1, 0, Hin, 1, sh.P, sh.N, nullptr, dCh, vec, st_vec};
+        if (launch_scan<T, float, false>(ac, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    }
     const long long units = (long long)sh.batch * sh.T * sh.G;
     group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;

@@ -1,0 +1,380 @@
+// ssd_bwd_tc.cu -- the backward's masked chunk scans on the tensor cores (tcgen05, TMEM, TMA).
+//
+// The same operation as masked_scan_kernel in ssd_bwd.cu, for one (chunk, 128-row block, head) per CTA:
+//
+//   out_r[w] = e_r * sum_k R_r[k] St[k][w]
+//            + sum_{i in chunk, i >= r (kAnti) or i <= r} exp(+-(s_i - s_r)) (R_r . K_i) V_i[w]
+//            + D_h V_r[w]                                          (when D is given)
+//
+// with e_r = exp(s_end - s_r) (kAnti) or exp(s_r).  It is the adjoint of the forward's block decomposition
+// ("Transformers are SSMs", analysis page, section "The Block-Decomposition SSD Algorithm"): the quadratic
+// (masked) form inside a chunk and the state term across chunks, here with given chunk states instead of
+// a chain.  The products run as bf16 x bf16 -> fp32 MMAs, over the chunk's columns on the mask's side of
+// the block (128 or 256 of them) in halves of 128:
+//
+//   G    = R_blk K_half^T        (M = 128 rows, N = 128, K = KD)
+//   M    = G o exp(+-(s_i - s_r)) on the triangle, bf16, in tensor memory (built by the CUDA-core warps)
+//   acc += M V_half              (A from tensor memory, N = W)
+//   acc2 = R_blk St^T            (the state tile [k][w] in bf16, built by the CUDA-core warps; N = W)
+//   out  = e_r acc2 + acc (+ D V_r), one row per thread, stored from registers.
+//
+// For the per-head dB and dC terms the mask and the state tile also enter as bf16 low parts (what the
+// rounding to bf16 left out), so those products are as accurate as fp32 accumulation allows.
+// Shapes: KD, W in {64, 128}; Q in {128, 256}; R, K, V bf16 rows of [batch][T][heads or groups][dim].
+// Tensor memory (512 columns): G at 0, the mask at 128 (its low part at 192), acc at 256, acc2 at 384.
+// One CTA per SM (it takes all of tensor memory); 9 warps: 0-7 CUDA-core work (two warpgroups over the
+// 128 lanes, each half of the columns), 8 TMA and MMA issue.  Every wait is bounded (about 2 s of
+// %globaltimer, 1 ms once any CTA has given up): on expiry the CTA records SSD_ERR_TIMEOUT in the status
+// word, and the issuer still waits (bounded) for its own MMAs before tensor memory is freed.
+#include "ssd_common.cuh"
+#include "tc_prims.cuh"
+#include "tma_host.h"
+
+namespace ssd {
+
+using namespace tc;
+
+namespace bt {
+
+constexpr int kRows = 128;
+constexpr int kCudaWarps = 8;
+constexpr int kThreads = 32 * kCudaWarps + 32;
+constexpr uint32_t kTmemCols = 512;
+// tensor memory: G of one 128-column half at 0; the half's mask at 128 (bf16; its low part at 192 when
+// split); acc at 256; acc2 at 384
+constexpr uint32_t kColG = 0, kColMhi = 128, kColMlo = 192, kColAcc = 256, kColAcc2 = 384;
+// shared memory (1 KiB aligned): R [KD/64 atoms][128 rows], K and V [atoms][256 rows], the state tile
+// [W/64 atoms][KD rows] and its low part, prefix sums [256]
+constexpr uint32_t kOffR = 0;           // 2 x 16 KiB
+constexpr uint32_t kOffK = 32768;       // 2 x 32 KiB
+constexpr uint32_t kOffV = 98304;       // 2 x 32 KiB
+constexpr uint32_t kOffSt = 163840;     // 2 x 16 KiB
+constexpr uint32_t kOffStLo = 196608;   // 2 x 8 KiB (split: KD = 64)
+constexpr uint32_t kOffS = 212992;      // 256 floats
+constexpr uint32_t kSmemBytes = kOffS + 1024 + 1024;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct Args {
+    const float *s;    // [batch][H][nc][Q] chunk prefix sums of dt * A (natural units)
+    const float *St;   // [batch][nc][H][P * N]: read as [KD][W] (st_kw) or [W][KD]
+    int st_kw;
+    const float *D;    // per head, or null
+    const __nv_bfloat16 *V;  // for the D term (row r of V), [batch][T][heads or groups][W]
+    int v_head;
+    void *out;         // [batch][T][H][W], bf16 (kOutBf16) or fp32
+    int *status;
+    Shape sh;
+};
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on one of the CTA's own barriers (its producers are its own TMA, MMAs and warps, so only a
+// defect of the kernel can make it expire).  Once any CTA has given up (the status word is set) the limit
+// drops to 1 ms, so that a defect common to every CTA still ends the grid in seconds.
+constexpr uint64_t kBrokenWaitNs = 1000000ull;
+__device__ __forceinline__ void wait_bar(uint64_t *bar, uint32_t parity, int *status) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_ns(), limit = ld_relaxed_gpu(status) ? kBrokenWaitNs : kWaitNs;
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit) {
+            atomicExch(status, SSD_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
+}
+
+// bf16 pair of (a, b) and, for the split operands, the pair of what rounding left out
+__device__ __forceinline__ uint32_t pack_lo(float a, float b, uint32_t hi) {
+    return pack_bf16x2(a - bf16lo(hi), b - bf16hi(hi));
+}
+
+}  // namespace bt
+
+using namespace bt;
+
+// kSplit: the mask and the state tile enter the products as a bf16 high part plus a bf16 low part (two
+// MMAs each); R, K and V are bf16 inputs and exact, so the products are then as accurate as fp32
+// accumulation allows.  Used for the per-head dB and dC terms, from which the dt, A and D gradients follow
+// through differences of large terms.
+template <int KD, int W, bool kAnti, bool kOutBf16, bool kSplit>
+__global__ void __launch_bounds__(bt::kThreads, 1)
+    masked_scan_tc_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mK,
+                          const __grid_constant__ CUtensorMap mV, const bt::Args a, int r_head, int k_head,
+                          int v_head) {
+    static_assert(!kSplit || KD == 64, "the low part of the state tile has room for KD = 64");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t ld_full, g_done, st_full, m_full, mx_done, fin_done;
+    __shared__ uint32_t tslot;
+    const Shape &sh = a.sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int blocks = sh.Q / kRows;
+    const int c = blockIdx.x / blocks, rb = blockIdx.x - c * blocks;
+    const int h = blockIdx.y, b = blockIdx.z, g = h / sh.heads_per_group;
+    const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), r0 = rb * kRows;
+    if (r0 >= len) return;  // whole CTA: a block past a ragged chunk's end
+    // the columns on the mask's side of the block, [r0, Q) or [0, r0 + 128), in halves of 128
+    const int cbeg = kAnti ? r0 : 0;
+    const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;  // 1 or 2
+
+    if (warp == 0) tmem_alloc(&tslot, kTmemCols);
+    if (tid == 0) {
+        mbar_init(&ld_full, 1);
+        mbar_init(&g_done, 1);
+        mbar_init(&mx_done, 1);
+        mbar_init(&fin_done, 1);
+        mbar_init(&st_full, kCudaWarps);
+        mbar_init(&m_full, kCudaWarps);
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    uint8_t *sR = smem + kOffR, *sK = smem + kOffK, *sV = smem + kOffV, *sSt = smem + kOffSt;
+    uint8_t *sStLo = smem + kOffStLo;
+    float *sq = reinterpret_cast<float *>(smem + kOffS);
+
+    if (warp == kCudaWarps) {
+        // ---------------- TMA and MMA issue (lane 0) ----------------
+        if (lane == 0) {
+            const int hr = r_head ? h : g, hk = k_head ? h : g, hv = v_head ? h : g;
+            const uint32_t bytes = (uint32_t)(KD / 64) * 16384u + (uint32_t)(KD / 64 + W / 64) * nh * 16384u;
+            mbar_arrive_expect_tx(&ld_full, bytes);
+            for (int k = 0; k < KD / 64; ++k) {
+                tma_load_4d(sR + k * 16384, &mR, &ld_full, k * 64, hr, t0 + r0, b);
+                for (int q = 0; q < nh; ++q)
+                    tma_load_4d(sK + k * 32768 + q * 16384, &mK, &ld_full, k * 64, hk, t0 + cbeg + q * kRows, b);
+            }
+            for (int k = 0; k < W / 64; ++k)
+                for (int q = 0; q < nh; ++q)
+                    tma_load_4d(sV + k * 32768 + q * 16384, &mV, &ld_full, k * 64, hv, t0 + cbeg + q * kRows, b);
+            wait_bar(&ld_full, 0, a.status);
+            fence_after_sync();
+            const uint32_t idG = idesc_bf16_f32(kRows, kRows, 0, 0);  // R (K-major) x K rows (K-major)
+            const uint32_t idW = idesc_bf16_f32(kRows, W, 0, 1);      // x V [i][w] or the state tile [k][w]
+            for (int ch = 0; ch < nh; ++ch) {
+                // G of this half into columns 0..127, once the warps have read the previous half's out
+                if (ch > 0) wait_bar(&m_full, (ch - 1) & 1, a.status);
+                fence_after_sync();
+                for (int kk = 0; kk < KD / 16; ++kk) {
+                    const int atom = kk >> 2, kin = kk & 3;
+                    mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024),
+                           smem_desc_sw128(smem_u32(sK) + atom * 32768 + ch * 16384 + kin * 32, 16, 1024), idG,
+                           kk > 0);
+                }
+                mma_commit(&g_done);
+                // acc += M V over the half's 128 rows of V (A from tensor memory)
+                wait_bar(&m_full, ch & 1, a.status);
+                fence_after_sync();
+                for (int kk = 0; kk < kRows / 16; ++kk) {
+                    const uint64_t vd =
+                        smem_desc_sw128(smem_u32(sV) + ch * 16384 + kk * 2048, 32768, 1024);
+                    mma_ts(tmem + kColAcc, tmem + kColMhi + kk * 8, vd, idW, ch > 0 || kk > 0);
+                    if (kSplit) mma_ts(tmem + kColAcc, tmem + kColMlo + kk * 8, vd, idW, 1);
+                }
+                mma_commit(&mx_done);
+            }
+            // acc2 = R St^T
+            wait_bar(&st_full, 0, a.status);
+            fence_after_sync();
+            for (int kk = 0; kk < KD / 16; ++kk) {
+                const int atom = kk >> 2, kin = kk & 3;
+                const uint64_t rd = smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024);
+                mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sSt) + kk * 2048, 16384, 1024), idW, kk > 0);
+                if (kSplit)
+                    mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sStLo) + kk * 2048, 8192, 1024), idW, 1);
+            }
+            mma_commit(&fin_done);
+            // nothing this CTA issued is in flight when it leaves
+            wait_bar(&fin_done, 0, a.status);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- CUDA-core warps ----------------
+        const int wq = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+        const int lrow = wq * 32 + lane;            // this thread's row of the block
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        const int j = r0 + lrow;                    // row within the chunk
+        const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+        for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) sq[i] = sch[i];
+        // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows
+        const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
+        for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
+            const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
+            float v[8];
+            if (a.st_kw) {
+                const float4 u0 = *reinterpret_cast<const float4 *>(Sp + (size_t)k * W + w0);
+                const float4 u1 = *reinterpret_cast<const float4 *>(Sp + (size_t)k * W + w0 + 4);
+                v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+                v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = Sp[(size_t)(w0 + e) * KD + k];
+            }
+            const uint4 t = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                       pack_bf16x2(v[6], v[7]));
+            *reinterpret_cast<uint4 *>(sSt + (w0 >> 6) * 16384 + swz(k, (w0 & 63) >> 3)) = t;
+            if (kSplit) {
+                const uint4 tl = make_uint4(pack_lo(v[0], v[1], t.x), pack_lo(v[2], v[3], t.y),
+                                            pack_lo(v[4], v[5], t.z), pack_lo(v[6], v[7], t.w));
+                *reinterpret_cast<uint4 *>(sStLo + (w0 >> 6) * 8192 + swz(k, (w0 & 63) >> 3)) = tl;
+            }
+        }
+        fence_view_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&st_full);
+        named_bar_sync(1, 32 * kCudaWarps);  // the prefix sums are in
+        const float sj = (j < len) ? sq[j] : 0.f;
+
+        // the mask, one 128-column half at a time: this thread's row, its 64 of the half's columns
+        for (int ch = 0; ch < nh; ++ch) {
+            wait_bar(&g_done, ch & 1, a.status);
+            if (ch > 0) wait_bar(&mx_done, (ch - 1) & 1, a.status);  // the previous half's mask was used
+            fence_after_sync();
+#pragma unroll 1
+            for (int q0 = half * 64; q0 < half * 64 + 64; q0 += 16) {
+                uint32_t gv[16];
+                tmem_ld16(tmem + kColG + q0 + lane_base, gv);
+                tmem_wait_ld();
+                uint32_t o[8], ol[8];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    float m[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int i = cbeg + ch * kRows + q0 + e + k;  // column within the chunk
+                        const bool ok = j < len && i < len && (kAnti ? i >= j : i <= j);
+                        m[k] = ok ? __uint_as_float(gv[e + k]) * ex2((kAnti ? sq[i] - sj : sj - sq[i]) * kLog2e)
+                                  : 0.f;
+                    }
+                    o[e / 2] = pack_bf16x2(m[0], m[1]);
+                    if (kSplit) ol[e / 2] = pack_lo(m[0], m[1], o[e / 2]);
+                }
+                tmem_st8(tmem + kColMhi + q0 / 2 + lane_base, o);
+                if (kSplit) tmem_st8(tmem + kColMlo + q0 / 2 + lane_base, ol);
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&m_full);
+        }
+
+        // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns
+        wait_bar(&fin_done, 0, a.status);
+        fence_after_sync();
+        const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
+        const float Dh = a.D ? a.D[h] : 0.f;
+        const size_t tok = (size_t)b * sh.T + t0 + j;
+        const __nv_bfloat16 *vrow =
+            a.V + (tok * (a.v_head ? sh.H : sh.G) + (a.v_head ? h : g)) * (size_t)W;
+        for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
+            uint32_t u[16], u2[16];
+            tmem_ld16(tmem + kColAcc + w0 + lane_base, u);
+            tmem_ld16(tmem + kColAcc2 + w0 + lane_base, u2);
+            tmem_wait_ld();
+            if (j >= len) continue;
+            float r[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = fmaf(e_r, __uint_as_float(u2[e]), __uint_as_float(u[e]));
+            if (a.D) {
+                const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + w0);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint4 vv = vp[q];
+                    const uint32_t ww[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        r[8 * q + 2 * e] = fmaf(Dh, bf16lo(ww[e]), r[8 * q + 2 * e]);
+                        r[8 * q + 2 * e + 1] = fmaf(Dh, bf16hi(ww[e]), r[8 * q + 2 * e + 1]);
+                    }
+                }
+            }
+            if (kOutBf16) {
+                uint4 *op = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + (tok * sh.H + h) * W + w0);
+                op[0] = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                                   pack_bf16x2(r[6], r[7]));
+                op[1] = make_uint4(pack_bf16x2(r[8], r[9]), pack_bf16x2(r[10], r[11]), pack_bf16x2(r[12], r[13]),
+                                   pack_bf16x2(r[14], r[15]));
+            } else {
+                float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + (tok * sh.H + h) * W + w0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) op[q] = make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+bool scan_tc_supported(const Shape &sh, int dtype) {
+    return dtype == SSD_BF16 && sh.P == 64 && (sh.N == 64 || sh.N == 128) && (sh.Q == 128 || sh.Q == 256) &&
+           sh.batch <= 65535 && sh.H <= 65535;
+}
+
+// One masked scan.  R, K, V: bf16 [batch][T][heads or groups][KD, KD, W]; *_head: 1 = per head, 0 = per
+// group.  St, st_kw, D, out as for the CUDA-core scan; out bf16 (dx) or fp32.
+cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int k_head, const void *V, int v_head,
+                                  int KD, int W, bool anti, const float *St, int st_kw, const float *D, void *out,
+                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st) {
+    auto dims = [&](int head, int d, uint64_t *dm, uint64_t *sb) {
+        const int n = head ? sh.H : sh.G;
+        dm[0] = (uint64_t)d;
+        dm[1] = (uint64_t)n;
+        dm[2] = (uint64_t)sh.T;
+        dm[3] = (uint64_t)sh.batch;
+        sb[0] = (uint64_t)d * 2;
+        sb[1] = (uint64_t)n * d * 2;
+        sb[2] = (uint64_t)sh.T * n * d * 2;
+    };
+    const uint32_t box[4] = {64, 1, kRows, 1};
+    CUtensorMap mR, mK, mV;
+    uint64_t dm[4], sb[3];
+    dims(r_head, KD, dm, sb);
+    if (!make_map_bf16(&mR, R, 4, dm, sb, box)) return cudaErrorInvalidValue;
+    dims(k_head, KD, dm, sb);
+    if (!make_map_bf16(&mK, K, 4, dm, sb, box)) return cudaErrorInvalidValue;
+    dims(v_head, W, dm, sb);
+    if (!make_map_bf16(&mV, V, 4, dm, sb, box)) return cudaErrorInvalidValue;
+    Args a;
+    a.s = s;
+    a.St = St;
+    a.st_kw = st_kw;
+    a.D = D;
+    a.V = static_cast<const __nv_bfloat16 *>(V);
+    a.v_head = v_head;
+    a.out = out;
+    a.status = status;
+    a.sh = sh;
+    void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Args, int, int, int) = nullptr;
+#define SSD_SCAN_TC_CASE(KDv, Wv, AN, OB, SP)                                                \
+    if (KD == KDv && W == Wv && anti == AN && out_bf16 == OB) k = masked_scan_tc_kernel<KDv, Wv, AN, OB, SP>;
+    SSD_SCAN_TC_CASE(128, 64, true, true, false)   // dx at N = 128
+    SSD_SCAN_TC_CASE(64, 64, true, true, false)    // dx at N = 64
+    SSD_SCAN_TC_CASE(64, 128, true, false, true)   // dB^(h) at N = 128
+    SSD_SCAN_TC_CASE(64, 64, true, false, true)    // dB^(h) at N = 64
+    SSD_SCAN_TC_CASE(64, 128, false, false, true)  // dC^(h) at N = 128
+    SSD_SCAN_TC_CASE(64, 64, false, false, true)   // dC^(h) at N = 64
+#undef SSD_SCAN_TC_CASE
+    if (!k) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(sh.nc * (sh.Q / kRows), sh.H, sh.batch);
+    k<<<grid, kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd
