@@ -42,6 +42,10 @@ cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int 
                                   int KD, int W, bool anti, const float *St, int st_kw, const float *D, void *out,
                                   bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st);
 constexpr int kScanTcRoles = 7;
+// chunk states on the tensor cores (ssd_bwd_tc.cu): bf16, P = 64, N = 128, Q in {128, 256}
+bool chunk_state_tc_supported(const Shape &sh, int dtype);
+cudaError_t launch_chunk_state_tc(const void *x, const void *B, const float *s, float *S, bool from_start,
+                                  int *status, const Shape &sh, cudaStream_t st);
 
 namespace {
 
@@ -643,17 +647,22 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     int *status = reinterpret_cast<int *>(ws + w.status_off);
     if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
     if (launch_chunk_cumsum(dt, A, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
-    // forward states: Hin_c, and the final state when a final-state gradient is given
-    if (launch_chunk_state<T>(x, B, s, Hin, sh, st, false) != cudaSuccess) return SSD_ERR_CUDA;
-    if (launch_state_passing(Hin, s, init, dfin ? fin : nullptr, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
-    // backward states: sum_i exp(s_i) dy_i C_i^T per chunk, then dHout_c and dinit
-    if (launch_chunk_state<T>(dy, C, s, Gout, sh, st, true) != cudaSuccess) return SSD_ERR_CUDA;
-    const int PN = sh.P * sh.N;
-    state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
-    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     // 16-byte operand loads need 16-byte aligned tensors whose rows are whole vectors
     constexpr int VE = 16 / (int)sizeof(T);
     const bool al = is_aligned(x, 16) && is_aligned(dy, 16) && is_aligned(B, 16) && is_aligned(C, 16);
+    const bool cs_tc = chunk_state_tc_supported(sh, sizeof(T) == 2 ? SSD_BF16 : SSD_F32) && al;
+    auto chunk_states = [&](const T *xx, const T *bb, float *out, bool from_start) {
+        return cs_tc ? launch_chunk_state_tc(xx, bb, s, out, from_start, status, sh, st)
+                     : launch_chunk_state<T>(xx, bb, s, out, sh, st, from_start);
+    };
+    // forward states: Hin_c, and the final state when a final-state gradient is given
+    if (chunk_states(x, B, Hin, false) != cudaSuccess) return SSD_ERR_CUDA;
+    if (launch_state_passing(Hin, s, init, dfin ? fin : nullptr, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
+    // backward states: sum_i exp(s_i) dy_i C_i^T per chunk, then dHout_c and dinit
+    if (chunk_states(dy, C, Gout, true) != cudaSuccess) return SSD_ERR_CUDA;
+    const int PN = sh.P * sh.N;
+    state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     const int vec = al && sh.P % VE == 0 && sh.N % VE == 0;
     const int st_vec = sh.P % 4 == 0 && sh.N % 4 == 0;
     // The three masked scans: on the tensor cores (ssd_bwd_tc.cu) for bf16 inputs with P = 64, N in {64, 128},

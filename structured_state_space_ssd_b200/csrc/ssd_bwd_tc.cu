@@ -318,6 +318,116 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Chunk states on the tensor cores: for one (chunk, head) per CTA,
+//
+//   S[p][n] = sum_{i in chunk} w_i x_i[p] B_i[n],   w_i = exp(s_end - s_i), or exp(s_i) (from_start)
+//
+// the forward's stage 2 ("Transformers are SSMs", analysis page, section "The Block-Decomposition SSD
+// Algorithm"), which the backward needs for the states entering every chunk, and (from the chunk's start,
+// with dy and C) for the gradients arriving at them.  S^T = B^T (w o x) runs as one MMA chain (M = 128
+// state columns n, N = 64 head columns p, K = the chunk's tokens, both operands MN-major); the weighted
+// rows w_i x_i enter as a bf16 high part plus a bf16 low part, so the states carry fp32 accuracy into the
+// gradients of dt, A and D.  Shapes: P = 64, N = 128, Q in {128, 256}; x [batch][T][H][64] and
+// B [batch][T][G][128] bf16; S [batch][nc][H][64][128] fp32.
+// ---------------------------------------------------------------------------
+namespace cs {
+constexpr uint32_t kOffB = 0;        // [2 n atoms][256 tokens] (32 KiB apart)
+constexpr uint32_t kOffX = 65536;    // [256 tokens][64 p], the weighted rows' high part after scaling
+constexpr uint32_t kOffXlo = 98304;  // their low part
+constexpr uint32_t kSmemBytes = 131072 + 1024;
+}  // namespace cs
+
+__global__ void __launch_bounds__(bt::kThreads, 1)
+    chunk_state_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
+                          const float *__restrict__ s, float *__restrict__ S, int *status, Shape sh,
+                          int from_start) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t ld_full, x_ready, done;
+    __shared__ uint32_t tslot;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / sh.heads_per_group;
+    const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), nq = sh.Q / kRows;
+    if (warp == 0) tmem_alloc(&tslot, 64);
+    if (tid == 0) {
+        mbar_init(&ld_full, 1);
+        mbar_init(&done, 1);
+        mbar_init(&x_ready, kCudaWarps);
+        mbar_fence_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    uint8_t *sB = smem + cs::kOffB, *sX = smem + cs::kOffX, *sXlo = smem + cs::kOffXlo;
+    if (warp == kCudaWarps) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&ld_full, (uint32_t)(3 * nq) * 16384u);
+            for (int q = 0; q < nq; ++q) {
+                tma_load_4d(sX + q * 16384, &mX, &ld_full, 0, h, t0 + q * kRows, b);
+                for (int k = 0; k < 2; ++k)
+                    tma_load_4d(sB + k * 32768 + q * 16384, &mB, &ld_full, k * 64, g, t0 + q * kRows, b);
+            }
+            wait_bar(&x_ready, 0, status);
+            fence_after_sync();
+            const uint32_t id = idesc_bf16_f32(kRows, 64, 1, 1);  // B^T (MN-major) x weighted rows (MN-major)
+            for (int part = 0; part < 2; ++part)
+                for (int kk = 0; kk < sh.Q / 16; ++kk)
+                    mma_ss(tmem, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
+                           smem_desc_sw128(smem_u32(part ? sXlo : sX) + kk * 2048, 16, 1024), id,
+                           part > 0 || kk > 0);
+            mma_commit(&done);
+            wait_bar(&done, 0, status);
+        }
+        __syncwarp();
+    } else {
+        // weight each token row in place (high part) and into the low part
+        wait_bar(&ld_full, 0, status);
+        const float *sc = s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+        const int i = tid;  // token row of the chunk
+        if (i < sh.Q) {
+            const float w = (i < len) ? ex2((from_start ? sc[i] : sc[sh.Q - 1] - sc[i]) * kLog2e) : 0.f;
+            uint8_t *row = sX + (i >> 7) * 16384, *rowlo = sXlo + (i >> 7) * 16384;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t off = swz(i & 127, k);
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + off);
+                const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a0 = bf16lo(vv[e]) * w, a1 = bf16hi(vv[e]) * w;
+                    hi[e] = pack_bf16x2(a0, a1);
+                    lo[e] = pack_lo(a0, a1, hi[e]);
+                }
+                *reinterpret_cast<uint4 *>(row + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(rowlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_view_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_ready);
+        // S^T in tensor memory: lane n, column p; warpgroup `half` writes p in [32 half, 32 half + 32)
+        wait_bar(&done, 0, status);
+        fence_after_sync();
+        const int wq = warp & 3, half = warp >> 2, n = wq * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+        float *Sp = S + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)(64 * 128);
+#pragma unroll
+        for (int q0 = 0; q0 < 32; q0 += 16) {
+            uint32_t u[16];
+            tmem_ld16(tmem + half * 32 + q0 + lane_base, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) Sp[(size_t)(half * 32 + q0 + e) * 128 + n] = __uint_as_float(u[e]);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 bool scan_tc_supported(const Shape &sh, int dtype) {
@@ -374,6 +484,31 @@ cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int 
     if (e != cudaSuccess) return e;
     const dim3 grid(sh.nc * (sh.Q / kRows), sh.H, sh.batch);
     k<<<grid, kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
+    return cudaGetLastError();
+}
+
+bool chunk_state_tc_supported(const Shape &sh, int dtype) {
+    return dtype == SSD_BF16 && sh.P == 64 && sh.N == 128 && (sh.Q == 128 || sh.Q == 256) && sh.batch <= 65535 &&
+           sh.H <= 65535;
+}
+
+// S [batch][nc][H][64][128] = the chunk states of x (per head) against B (per group), weighted from the
+// chunk's end, or from its start (from_start).
+cudaError_t launch_chunk_state_tc(const void *x, const void *B, const float *s, float *S, bool from_start,
+                                  int *status, const Shape &sh, cudaStream_t st) {
+    const uint32_t box[4] = {64, 1, kRows, 1};
+    CUtensorMap mX, mB;
+    const uint64_t dx[4] = {64, (uint64_t)sh.H, (uint64_t)sh.T, (uint64_t)sh.batch};
+    const uint64_t sx[3] = {128, (uint64_t)sh.H * 128, (uint64_t)sh.T * sh.H * 128};
+    const uint64_t db[4] = {128, (uint64_t)sh.G, (uint64_t)sh.T, (uint64_t)sh.batch};
+    const uint64_t sbb[3] = {256, (uint64_t)sh.G * 256, (uint64_t)sh.T * sh.G * 256};
+    if (!make_map_bf16(&mX, x, 4, dx, sx, box) || !make_map_bf16(&mB, B, 4, db, sbb, box))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)cs::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    chunk_state_tc_kernel<<<dim3(sh.nc, sh.H, sh.batch), kThreads, cs::kSmemBytes, st>>>(mX, mB, s, S, status, sh,
+                                                                                          from_start ? 1 : 0);
     return cudaGetLastError();
 }
 
