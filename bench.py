@@ -401,7 +401,7 @@ def main():
         line["gate_norm"] = measure_gate_norm(w, y, dev, stream, flush, peaks)
         line["gated_forward"] = measure_gated(w, d, dev, stream, flush, line["gate_norm"]["us_per_launch"],
                                               ms_per_step)
-        line["backward"] = measure_backward(w, d, dev, stream, flush)
+        line["backward"] = measure_backward(w, d, dev, stream, flush, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(host, w)
         print(json.dumps(line), flush=True)
@@ -576,10 +576,12 @@ def backward_alg_flops(w):
     return per_chunk * w.batch * w.nc
 
 
-def measure_backward(w, d, dev, stream, flush, steps=5):
+def measure_backward(w, d, dev, stream, flush, peaks, steps=5):
     """The layer's backward (ssd_bwd: every input gradient for given dy and dfinal) on this workload,
-    L2 flushed before each call.  It runs on the CUDA cores in fp32, so its bound is the FFMA rate:
-    148 SMs x 128 lanes x 2 flops per cycle at the clock's maximum (74.4 TFLOP/s at 1965 MHz)."""
+    L2 flushed before each call.  Its products (the three masked chunk scans and the chunk states) run on
+    the bf16 tensor cores, so the block count is set against the measured bf16 peak; the products of the
+    per-head dB, dC terms and of the chunk states are issued twice (high and low bf16 parts), which the
+    block count does not include."""
     import torch
     from structured_state_space_ssd_b200 import ssd as S
     from structured_state_space_ssd_b200.inputs import make_output_grads
@@ -605,10 +607,10 @@ def measure_backward(w, d, dev, stream, flush, steps=5):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
-    peak = 148 * 128 * 2 * 1.965e9
+    tflops = alg_flops / (ms * 1e-3) / 1e12
     return {"ms": ms, "tokens_per_s": w.tokens / (ms * 1e-3), "alg_flops": alg_flops,
-            "tflops": alg_flops / (ms * 1e-3) / 1e12, "bound": "alu",
-            "frac_of_fp32_ffma_peak": alg_flops / (ms * 1e-3) / peak, "launches_per_call": 11,
+            "tflops": tflops, "bound": "tensor", "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "launches_per_call": 11,
             "with": "dfinal_state and init_state" if w.with_init else "dfinal_state (the workload has no init_state)"}
 
 
