@@ -56,6 +56,7 @@ CASES = [
     (1, 129, 3, 32, 64, 3, 64, "bf16", True, False),        # one row past a chunk
     (3, 1, 2, 8, 8, 1, 16, "f32", True, True),              # a single token
     (1, 64, 6, 64, 128, 2, 256, "bf16", False, False),      # T < Q
+    (2, 600, 4, 64, 64, 2, 128, "bf16", True, True),        # tensor-core scans at N = 64, Q = 128
     (1, 200, 2, 5, 7, 1, 32, "f32", True, True),            # odd P and N
 ]
 
