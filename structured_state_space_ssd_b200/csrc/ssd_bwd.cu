@@ -469,6 +469,8 @@ __global__ void __launch_bounds__(256) group_reduce_kernel(const float *__restri
         sb[m] = 0.f;
         sc[m] = 0.f;
     }
+    // four heads' rows in flight at once; the sums still run in head order
+#pragma unroll 4
     for (int hh = 0; hh < sh.heads_per_group; ++hh) {
         const int h = g * sh.heads_per_group + hh;
         const size_t hrow = ((size_t)tok * sh.H + h) * sh.N;
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
                                                              const float *__restrict__ dfin,
                                                              const float *__restrict__ fin, float *__restrict__ ddt,
                                                              double *__restrict__ pa, double *__restrict__ pd,
-                                                             Shape sh) {
+                                                             Shape sh, int vec) {
     __shared__ double red[kDtThreads];
     __shared__ double suf[kDtThreads];
     const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -564,12 +566,32 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
     }
     const double dA_part = block_sum(da, red);
 
+    // dD's share: sum over the row's tokens of <dy_t, x_t> for this head.  With 16-byte rows, eight
+    // elements per load (their products summed in fp32, then in fp64), four loads in flight per thread.
     double dd = 0.0;
-    const long long TP = (long long)sh.T * sh.P;
-    for (long long idx = tid; idx < TP; idx += kDtThreads) {
-        const int t = (int)(idx / sh.P), p = (int)(idx - (long long)t * sh.P);
-        const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + p;
-        dd += (double)to_f32(dy[off]) * (double)to_f32(x[off]);
+    constexpr int VE = 16 / (int)sizeof(T);
+    if (vec) {
+        const int cpt = sh.P / VE;  // 16-byte pieces per token row
+        const long long total = (long long)sh.T * cpt;
+#pragma unroll 4
+        for (long long idx = tid; idx < total; idx += kDtThreads) {
+            const int t = (int)(idx / cpt), q = (int)(idx - (long long)t * cpt);
+            const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + (size_t)q * VE;
+            float fy[VE], fx[VE];
+            unpack16(*reinterpret_cast<const uint4 *>(dy + off), fy, T());
+            unpack16(*reinterpret_cast<const uint4 *>(x + off), fx, T());
+            float f = 0.f;
+#pragma unroll
+            for (int e = 0; e < VE; ++e) f = fmaf(fy[e], fx[e], f);
+            dd += (double)f;
+        }
+    } else {
+        const long long TP = (long long)sh.T * sh.P;
+        for (long long idx = tid; idx < TP; idx += kDtThreads) {
+            const int t = (int)(idx / sh.P), p = (int)(idx - (long long)t * sh.P);
+            const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + p;
+            dd += (double)to_f32(dy[off]) * (double)to_f32(x[off]);
+        }
     }
     const double dD_part = block_sum(dd, red);
     if (tid == 0) {
@@ -698,7 +720,8 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     const long long units = (long long)sh.batch * sh.T * sh.G;
     group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
-    dt_scan_kernel<T><<<dim3(sh.H, sh.batch), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh);
+    dt_scan_kernel<T><<<dim3(sh.H, sh.batch), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh,
+                                                                    vec);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     param_reduce_kernel<<<(sh.H + 255) / 256, 256, 0, st>>>(pa, pd, dA, dD, sh.batch, sh.H);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
