@@ -31,10 +31,17 @@
 //    S~_c into a three-slot fp32 ring (or final_state after the last chunk).
 //    Other blocks only read S~_{c-1} and count themselves as done with it;
 //    an owner overwrites a slot only after every reader of the chunk before
-//    has read it.  Every wait on another CTA is bounded: on expiry the
-//    status word is set to SSD_ERR_TIMEOUT and the waits that follow give up
-//    at once (the CTA's own barriers are still waited for, so nothing it
-//    issued is in flight when it exits).
+//    has read it.  On long sequences (template argument kD = 4) the owners
+//    also publish their local states L_c early and start from the most recent
+//    published S~_j of the 4 chunks before, folding in the L after it (a
+//    decoupled look-back; see fused_lookback).  Every wait on another CTA is
+//    bounded: on expiry the status word is set to SSD_ERR_TIMEOUT and the
+//    waits that follow give up at once (the CTA's own barriers are still
+//    waited for, so nothing it issued is in flight when it exits).
+//  * A launch covers 64 head columns and up to 128 state columns: P = 128 and
+//    N = 256 run as two launches each (the second state half adds to y;
+//    kAccum), a head below 64 columns is zero-padded.  With kGated the drain
+//    applies the block's gate and a per-head GroupNorm instead of storing y.
 //
 // Warp roles: two head pipelines per CTA, pipeline pl taking every other head
 // of a unit.  Its eight CUDA-core warps (two warpgroups over the 128 TMEM
