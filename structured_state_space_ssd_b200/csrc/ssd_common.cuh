@@ -92,7 +92,9 @@ struct Shape {
 // also publishes its local state L_c and total decay sigma_c as soon as its products are done, and
 // the owner of chunk c starts from the most recent published S~_j with j >= c - D, folding in
 // L_{j+1} .. L_{c-1} (the decoupled look-back of a single-pass scan), so that a long sequence is not
-// bound by one hand-off per chunk.  D > 1 is used where the chain would be long and the ring, twice
+// bound by one hand-off per chunk.  This is valid because the chunk recurrence is a 1-semiseparable
+// product, associative on (decay, state) pairs ("Transformers are SSMs", analysis page, section "The
+// 1-Semiseparable Matrix: Building Block for Everything": the associative-scan decomposition).  D > 1 is used where the chain would be long and the ring, twice
 // as large, stays small enough to live in L2.  `s` is one launch's shape (64 head columns, at most
 // 128 state columns).
 inline int fused_lookback(const Shape &s) {
