@@ -339,6 +339,15 @@ SSD_API int ssd_bwd(const void *x, const float *dt, const float *A, const void *
                     float *dA, void *dB, void *dC, float *dD, float *dinit_state, int batch, int T, int H, int P,
                     int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Waits for `stream` and returns the status word of the last ssd_bwd call on
+ * this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a bounded wait of the
+ * tensor-core kernels gave up (a defect of the kernel, not of the inputs; the
+ * gradients of that call are then not valid).  SSD_ERR_INVALID_ARG for a NULL
+ * workspace, SSD_ERR_CUDA if the stream or the copy fails.
+ */
+SSD_API int ssd_bwd_check(const void *workspace, void *stream);
+
 /* Static, NUL-terminated description of a status code. */
 SSD_API const char *ssd_status_string(int status);
 

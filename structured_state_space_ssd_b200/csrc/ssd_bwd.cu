@@ -730,6 +730,15 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
 }  // namespace
 }  // namespace ssd
 
+extern "C" int ssd_bwd_check(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+    int status = 0;  // the status word heads the backward's workspace
+    if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    return status;
+}
+
 extern "C" size_t ssd_bwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype) {
     ssd::Shape sh;
     if (ssd::check_dims(batch, T, H, P, G, N, Q, dtype, &sh) != SSD_OK) return 0;

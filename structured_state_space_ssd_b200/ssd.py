@@ -26,7 +26,7 @@ EXPORTS = ("ssd_fwd", "ssd_fwd_gated", "ssd_fwd_gated_launch_count", "ssd_fwd_wo
            "ssd_fwd_launch_count", "ssd_fwd_timed",
            "ssd_fwd_stage_name", "ssd_fwd_check", "ssd_fwd_withhold_publish", "ssd_status_string", "ssd_version",
            "ssd_fwd_no_alloc", "ssd_fwd_no_alloc_check", "ssd_step", "ssd_gate_norm", "ssd_split_logdecay",
-           "ssd_split_combine", "ssd_split_correct", "ssd_bwd", "ssd_bwd_workspace_bytes")
+           "ssd_split_combine", "ssd_split_correct", "ssd_bwd", "ssd_bwd_workspace_bytes", "ssd_bwd_check")
 
 
 class SSDError(RuntimeError):
@@ -68,6 +68,8 @@ def load():
     lib.ssd_fwd_stage_name.restype = ctypes.c_char_p
     lib.ssd_fwd_check.argtypes = [vp, vp]
     lib.ssd_fwd_check.restype = i
+    lib.ssd_bwd_check.argtypes = [vp, vp]
+    lib.ssd_bwd_check.restype = i
     lib.ssd_fwd_withhold_publish.argtypes = lib.ssd_fwd.argtypes + [i, i, i, ctypes.c_uint]
     lib.ssd_fwd_withhold_publish.restype = i
     lib.ssd_fwd_no_alloc.argtypes = [vp, fp, fp, vp, vp, fp, i, fp, vp, fp, i, i, i, i, i, i, i, vp]

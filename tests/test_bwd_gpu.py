@@ -183,3 +183,18 @@ def test_backward_of_a_split_sequence_matches_the_whole(split, cuda_device):
     for name in ("dA", "dD"):
         _check(name, (g1[name] + g2[name]).cpu().numpy(), full[name].double().cpu().numpy(), "f32")
     _check("dinit_state", g1["dinit_state"].cpu().numpy(), full["dinit_state"].double().cpu().numpy(), "f32")
+
+
+def test_status_word_is_clear_after_a_tensor_core_backward(cuda_device):
+    import ctypes
+    from structured_state_space_ssd_b200 import ssd as S
+    inp = make_inputs(1, 600, 4, 64, 128, 2, "bf16", seed=91, with_init=True)
+    grads = make_output_grads(1, 600, 4, 64, 128, "bf16", seed=91, with_dfinal=True)
+    d, g = _to(cuda_device, inp), _to(cuda_device, grads)
+    ws = torch.empty(S.ssd_bwd_workspace_bytes(1, 600, 4, 64, 2, 128, 256, torch.bfloat16), dtype=torch.uint8,
+                     device=cuda_device)
+    ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], g["dy"], 256, d["init_state"], g["dfinal_state"],
+            workspace=ws)
+    stream = torch.cuda.current_stream(cuda_device)
+    assert S.load().ssd_bwd_check(ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(stream.cuda_stream)) == 0
+    assert S.load().ssd_bwd_check(None, ctypes.c_void_p(stream.cuda_stream)) == 1
