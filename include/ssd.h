@@ -68,8 +68,9 @@ enum {
  * chunk states (stages 0-3); on the fused tensor-core path (bf16 x, B, C;
  * Q in {128, 256}; P a multiple of 8 up to 64, or 128; N a multiple of 16 up
  * to 128, or 256), per launch, the unit counter, the inter-chunk hand-off
- * flags and an L2-sized ring of the latest chunk states (with the local
- * chunk states too where a long sequence uses look-back).
+ * flags and L2-sized rings of the latest chunk states (fp32, and bf16 tiles
+ * of them for the other row block of each chunk; fp32 local chunk states
+ * instead of the tiles where a long sequence uses look-back).
  */
 SSD_API size_t ssd_fwd_workspace_bytes(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
 

@@ -103,10 +103,17 @@ inline int fused_lookback(const Shape &s) {
     return (s.nc >= 32 && bh * 8 * slot_bytes <= (size_t(48) << 20)) ? 4 : 1;
 }
 // Ring slots per (batch, head): chunk c's states go to slot c % R.  Three with D = 1; 2D with look-back,
-// so that the slot an owner overwrites was last read by owners at least D chunks back.
+// so that the slot an owner overwrites was last read by owners at least D chunks back.  With D = 1 only
+// the bf16 state tiles (read by the other blocks) use the R slots: the fp32 state is read by the next
+// owner alone, which reads S~_{c-1} and writes S~_c in place, so it has one slot.  (With look-back
+// the other blocks read S~ from the fp32 slots, which the owners read too: there are no tiles.)
 inline int fused_ring_slots(int d) { return d == 1 ? 3 : 2 * d; }
-// floats per slot: S~ (64 x N), and L (64 x N) after it with look-back
-inline size_t fused_slot_floats(const Shape &s, int d) { return (size_t)64 * s.N * (d == 1 ? 1 : 2); }
+// fp32 floats per (batch, head): one slot of S~ (64 x N) with D = 1; R slots of S~ and L with look-back
+inline size_t fused_ring_floats(const Shape &s, int d) {
+    return d == 1 ? (size_t)64 * s.N : (size_t)fused_ring_slots(d) * 2 * 64 * s.N;
+}
+// Rows of a bf16 state tile: the K extent of the inter-chunk product (N rounded up to 64; rows past N zero).
+inline int fused_tile_rows(const Shape &s) { return (s.N + 63) / 64 * 64; }
 
 // The two launch sequences: stage-per-kernel on CUDA cores (any shape and
 // dtype within the limits) or the fused tensor-core kernel (bf16, P a multiple
@@ -139,13 +146,15 @@ struct Workspace {
     size_t status_off;  // int status word
     size_t counter_off; // int unit counter (fused path)
     size_t inc_off;     // fused path: int inc[batch * H][R] (one count per sequence without look-back)
+    size_t tin_off;     // fused path, D = 1: int tin[batch * H][R], c + 1 once the bf16 tile of S~_c is in slot c % R
     size_t agg_off;     // fused path: int agg[batch * H][R], c + 1 once L_c and sigma_c are in slot c % R
     size_t cons_off;    // fused path: int cons[batch * H][R], reads of the slot so far (a count)
     size_t sig_off;     // fused path: float sigma[batch * H][R], chunk c's total log2 decay in slot c % R
     size_t clear_bytes; // bytes from offset 0 cleared per call
     size_t s_off;       // CUDA-core path: float s[batch][H][nc][Q], inclusive log-decay prefix sums per chunk
     size_t state_off;   // CUDA-core path: float S[batch][nc][H][P][N], chunk states then entering states
-    size_t ring_off;    // fused path: float ring[batch][H][R][1 or 2][16][N][4], states of recent chunks
+    size_t ring_off;    // fused path: float ring[batch][H][1, or R x 2][16][N][4], states of recent chunks
+    size_t tile_off;    // fused path, D = 1: bf16 tile[batch * H][R][rows][64], S~ in the MMA's 128-byte swizzle
     size_t total;
 };
 
@@ -189,6 +198,8 @@ inline Workspace workspace_layout_one(const Shape &s, Path path) {
     const size_t per_slot = (d == 1) ? 0 : bh * R;  // agg and sigma: look-back only
     w.inc_off = off;
     off += sizeof(int) * (d == 1 ? bh : bh * R);
+    w.tin_off = off;
+    off += sizeof(int) * (d == 1 ? bh * R : 0);
     w.cons_off = off;
     off += sizeof(int) * bh * R;
     w.agg_off = off;
@@ -200,9 +211,12 @@ inline Workspace workspace_layout_one(const Shape &s, Path path) {
     w.s_off = off;
     if (path != kPathFused) off = align256(off + sizeof(float) * bh * s.nc * s.Q);
     w.state_off = w.ring_off = off;
-    if (path == kPathFused)
-        off = align256(off + sizeof(float) * bh * R * fused_slot_floats(s, d));
-    else
+    w.tile_off = off;
+    if (path == kPathFused) {
+        off = align256(off + sizeof(float) * bh * fused_ring_floats(s, d));
+        w.tile_off = off;
+        if (d == 1) off = align256(off + sizeof(uint16_t) * bh * R * fused_tile_rows(s) * 64);
+    } else
         off = align256(off + sizeof(float) * (size_t)s.batch * s.nc * s.H * s.P * s.N);
     w.total = off;
     return w;

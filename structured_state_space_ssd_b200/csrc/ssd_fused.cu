@@ -28,13 +28,17 @@
 //    no deadlock however many CTAs are resident.
 //  * The last block of a chunk owns the chunk state: it waits for S~_{c-1}
 //    (published by the owner of chunk c-1), forms E and S~_c, and writes
-//    S~_c into a three-slot fp32 ring (or final_state after the last chunk).
-//    Other blocks only read S~_{c-1} and count themselves as done with it;
-//    an owner overwrites a slot only after every reader of the chunk before
-//    has read it.  On long sequences (template argument kD = 4) the owners
+//    S~_c over S~_{c-1} in its sequence's fp32 slot (or final_state after
+//    the last chunk).  The other block of the next chunk needs S~_c only as
+//    the bf16 operand of its inter-chunk product, so the owner also writes
+//    that tile in the operand's layout and its publisher stores it with TMA
+//    into a three-slot ring, from which the other block's issuer loads it
+//    with TMA (no CUDA-core work); a tile slot is overwritten only after its
+//    reader has counted itself done.  On long sequences (kD = 4) the owners
 //    also publish their local states L_c early and start from the most recent
 //    published S~_j of the 4 chunks before, folding in the L after it (a
-//    decoupled look-back; see fused_lookback).  Every wait on another CTA is
+//    decoupled look-back; see fused_lookback), and the other blocks read the
+//    fp32 S~ from those slots too.  Every wait on another CTA is
 //    bounded: on expiry the status word is set to SSD_ERR_TIMEOUT and the
 //    waits that follow give up at once (the CTA's own barriers are still
 //    waited for, so nothing it issued is in flight when it exits).
@@ -48,8 +52,10 @@
 // lanes) form the prefix sums, scale x, build the decay mask, move the states
 // and drain the accumulators; its issuer warp (16 + pl) loads x with TMA and
 // issues tcgen05.mma; its publisher warp (18 + pl) makes the state hand-offs
-// visible to other CTAs.  C, B and G = C B^T (the block's 128 x 128) are shared
-// by the unit's heads.
+// visible to other CTAs (and stores an owner's bf16 state tile).  C, B and
+// G = C B^T (the block's 128 x 128) are shared by the unit's heads; an owner's
+// units hold half as many heads as the other block's, whose heads take about
+// half as long.
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
@@ -98,11 +104,15 @@ struct Params {
     const float *D;     // [H]
     const float *init;  // [b][H][P][N] or null
     float *fin;         // [b][H][P][N] or null
-    // The chain (see fused_lookback; the depth D is the kernel's template argument): chunk c's states
-    // live in slot c % R of its sequence, S~_c first, then (look-back only) L_c, each [P/4][N][4]
-    // (see ring_quad).
-    float *ring;        // [b*H][R][1 or 2][P/4][N][4]
+    // The chain (see fused_lookback; the depth D is the kernel's template argument).  fp32 states, each
+    // [P/4][N][4] (see ring_quad): with D = 1 one slot per sequence holding the latest S~ (only owners
+    // read it, each in place before writing its own); with look-back chunk c's S~_c and L_c in slot c % R.
+    // The other blocks read S~_{c-1} as a bf16 tile (tensor map mR: [b*H*R][tile_rows][64], slot c % R,
+    // the 128-byte swizzle of the stage-4 operand), stored by the owner's publisher with TMA.
+    float *ring;        // [b*H][1 or R][1 or 2][P/4][N][4]
+    int tile_rows;      // rows of a bf16 state tile: N rounded up to 64 (the K extent of stage 4)
     int *inc;           // c + 1 once S~_c is published: [b*H] without look-back, [b*H][R] with (inc_flag)
+    int *tin;           // [b*H][R]: c + 1 once the bf16 tile of S~_c is in slot c % R (tiles may land out of order)
     int *agg;           // [b*H][R]: c + 1 once L_c and sigma_c are published (look-back only)
     int *cons;          // [b*H][R]: reads of the slot so far, every use (a count)
     float *sig;         // [b*H][R]: sigma_c, chunk c's total decay in log2 units (look-back only)
@@ -111,9 +121,12 @@ struct Params {
     __nv_bfloat16 *y;   // y + p_off (row stride p_full); read back only by the second state half
     int NK;             // 64-wide K-atoms along N
     int halves;         // Q / 128
-    int heads_per_unit;
-    int blocks_per_group;
-    int units_per_role;  // units of one row block of one chunk: batch * G * blocks_per_group
+    // Units of row block r hold up to hpu[r] heads of a group (blocks[r] units per group, units[r] =
+    // batch * G * blocks[r] per chunk): the owners' block (r = 1) does more per head, so its units
+    // are smaller, which keeps unit lengths alike.  With one block per chunk r = 0 only.
+    int hpu[2];
+    int blocks[2];
+    int units[2];
     int n_units;
     uint32_t flag_polls;  // bound of each wait on another CTA's flag
     int withhold_bh;      // test hook: the owner of (b*H + h, chunk) below never publishes (-1: none)
@@ -146,6 +159,8 @@ struct PipeBars {
     uint64_t s_full;     // entering-state tile written, state accumulators read (8 warp arrivals)
     uint64_t mx_done;    // every product of the head done
     uint64_t acc_free;   // accumulators drained (8 warp arrivals)
+    uint64_t e_full;     // another block's entering-state tile landed (TMA from the bf16 ring)
+    uint64_t t_free;     // owner: its bf16 state tile (in x rows 0..127) read by the publisher's TMA store
 };
 
 struct Bars {
@@ -174,34 +189,34 @@ struct Unit {
 // earlier).  So there is no deadlock however many CTAs are resident.
 __device__ __forceinline__ Unit decode(int u, const Params &p) {
     Unit un;
-    const int M = p.units_per_role;
+    const int Mo = p.units[0], Mw = p.units[1];
     int idx;
     if (p.halves == 1) {
         un.r = 0;
-        un.c = u / M;
-        idx = u % M;
-    } else if (u < M) {
+        un.c = u / Mo;
+        idx = u % Mo;
+    } else if (u < Mw) {
         un.r = 1;
         un.c = 0;
         idx = u;
     } else {
-        const int v = u - M, t = v / (2 * M), j = v % (2 * M);
-        if (t < p.sh.nc - 1 && j < M) {
+        const int v = u - Mw, t = v / (Mw + Mo), j = v % (Mw + Mo);
+        if (t < p.sh.nc - 1 && j < Mw) {
             un.r = 1;
             un.c = t + 1;
             idx = j;
         } else {
             un.r = 0;
             un.c = t;
-            idx = (t < p.sh.nc - 1) ? j - M : j;
+            idx = (t < p.sh.nc - 1) ? j - Mw : j;
         }
     }
-    const int hb = idx % p.blocks_per_group;
-    idx /= p.blocks_per_group;
+    const int hb = idx % p.blocks[un.r];
+    idx /= p.blocks[un.r];
     un.g = idx % p.sh.G;
     un.b = idx / p.sh.G;
-    un.h0 = un.g * p.sh.heads_per_group + hb * p.heads_per_unit;
-    un.h1 = min(un.h0 + p.heads_per_unit, (un.g + 1) * p.sh.heads_per_group);
+    un.h0 = un.g * p.sh.heads_per_group + hb * p.hpu[un.r];
+    un.h1 = min(un.h0 + p.hpu[un.r], (un.g + 1) * p.sh.heads_per_group);
     un.t0 = un.c * p.sh.Q;
     un.len = min(p.sh.Q, p.sh.T - un.t0);
     un.row0 = un.r * kRows;
@@ -307,7 +322,7 @@ template <bool kAccum, int kD, bool kGated>
 __global__ void __launch_bounds__(fz::kThreads, 1)
     ssd_fused_kernel(const __grid_constant__ CUtensorMap mC, const __grid_constant__ CUtensorMap mB,
                      const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mY,
-                     const fz::Params p) {
+                     const __grid_constant__ CUtensorMap mR, const fz::Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1k(smem_raw);
     uint8_t *sC = smem + kOffC;
@@ -356,14 +371,18 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // Publisher warps: warp 18 + pl makes pipeline pl's hand-offs visible
         // to other CTAs, so that neither the CUDA-core warps nor the issuer
         // wait for a GPU-scope release.  After an owner's stores of L_c it
-        // releases `agg` (look-back only); after its store of S~_c it adds
-        // one to `cons` of each slot it may have read and releases `inc`;
-        // once another block has read S~_{c-1} it adds one to that slot's
-        // `cons`.  The warps signal through CTA-scope release counts in
-        // shared memory, acquired here by every lane, which puts their stores
-        // before the lanes' GPU-scope releases (release is cumulative).
+        // releases `agg` (look-back only); after its store of S~_c it releases
+        // `inc` and adds one to `cons` of each slot it may have read, then
+        // stores the bf16 tile of S~_c with TMA (once the slot's earlier
+        // readers are done) and releases `tin`, so that the chain of owners
+        // never waits for the tile; once another block has read S~_{c-1} it
+        // adds one to that slot's `cons`.  The warps signal through CTA-scope release
+        // counts in shared memory, acquired here by every lane, which puts
+        // their stores before the lanes' GPU-scope releases (release is
+        // cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
+        const uint8_t *sTile = smem + kOffPipe + pl * kPipeBytes;  // the owner's x rows 0..127 buffer
         uint32_t ucnt = 0, ocnt = 0, tcnt = 0, acnt = 0;
         // bounded wait for one of this pipeline's shared-memory counts to reach `target`
         auto wait_count = [&](const uint32_t *cnt, uint32_t target) {
@@ -390,22 +409,43 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             for (int h = un.h0 + pl; h < un.h1; h += 2) {
                 const int bh = un.b * sh.H + h;
                 if (un.owner) {
-                    const bool publish =
-                        un.c < sh.nc - 1 && !(bh == p.withhold_bh && un.c == p.withhold_c);
-                    if (kD > 1 && un.c < sh.nc - 1) {
+                    const bool writes = un.c < sh.nc - 1;
+                    const bool publish = writes && !(bh == p.withhold_bh && un.c == p.withhold_c);
+                    if (kD > 1 && writes) {
                         // L_c and sigma_c stored
                         wait_count(&s_agg[pl], kPipeWarps * ++acnt);
                         if (lane == 0 && publish) st_release_gpu(p.agg + bh * R + un.c % R, un.c + 1);
                     }
                     wait_count(&s_owned[pl], kPipeWarps * ++ocnt);
+                    // the bf16 tile of S~_c (in the owner's x rows 0..127 buffer) for the next chunk's other
+                    // block goes to slot c % R once that slot's earlier readers are done (with look-back the
+                    // owner waited for them before storing L_c).  The store is issued first, so that it reads
+                    // shared memory while inc is released; the issuer reuses the buffer once it has, and
+                    // tin is released once the store is complete.
+                    const bool tile = kD == 1 && writes && p.halves == 2;
+                    if (tile && lane == 0) {
+                        if (kD == 1 && un.c >= R)
+                            wait_flag(p.cons + bh * R + un.c % R, un.c / R, p.flag_polls, abort, p.status);
+                        tma_store_3d(&mR, sTile, 0, 0, bh * R + un.c % R);
+                        bulk_commit();
+                    }
                     if (lane == 0 && publish) st_release_gpu(inc_flag<kD>(p.inc, bh, un.c), un.c + 1);
                     // with look-back the owner has read (at most) the slots of the D chunks before it:
-                    // count them all (without, its read of S~_{c-1} precedes every later owner's
-                    // publication, so the owner of chunk c-1+R cannot overwrite it first)
+                    // count them all (without, only owners read the fp32 state, each its one slot before
+                    // the publication the next owner waits for)
                     if (kD > 1 && lane < min(kD, un.c)) red_release_add_gpu(p.cons + bh * R + (un.c - 1 - lane) % R, 1);
+                    if (tile && lane == 0) {
+                        bulk_wait_read();
+                        mbar_arrive(&bars.pb[pl].t_free);
+                        bulk_wait_all();
+                        fence_proxy_async_global();
+                        if (publish) st_release_gpu(p.tin + bh * R + un.c % R, un.c + 1);
+                    }
                 } else if (un.c > 0) {
-                    // the other block of chunk c has read S~_{c-1} (chunk 0's reads the initial state)
-                    wait_count(&s_copied[pl], kPipeWarps * ++tcnt);
+                    // the other block of chunk c has read S~_{c-1} (without look-back its issuer counts the tile
+                    // once it landed, with look-back its eight warps their ring reads; chunk 0's block reads
+                    // the initial state)
+                    wait_count(&s_copied[pl], (kD == 1 ? 1 : kPipeWarps) * ++tcnt);
                     if (lane == 0) red_release_add_gpu(p.cons + bh * R + (un.c - 1) % R, 1);
                 }
                 __syncwarp();
@@ -435,6 +475,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         const uint32_t idInter = idesc_bf16_f32(kRows, kP, 0, 1);   // C (K-major) x state tile [n][p]
         const uint32_t idMX = idesc_bf16_f32(kRows, kP, 0, 1);      // mask (TMEM) x x rows [i][p]
         uint32_t use = 0, ocnt = 0, ucnt = 0, cbcnt = 0, udone = 0;
+        uint32_t scnt = 0, ecnt = 0;           // s_full and e_full phases (not every head has both)
+        uint32_t tiles = 0, tiles_freed = 0;   // an owner's bf16 state tiles stored from x rows 0..127
+        // x rows 0..127 hold an owner's state tile until its TMA store has read it: wait before reloading
+        auto free_x = [&]() {
+            if (tiles != tiles_freed) {
+                wait_bar(&pb.t_free, par(tiles - 1), p.status, broken);
+                tiles_freed = tiles;
+            }
+        };
         int next_u = -1;
         for (;;) {
             int u = 0;
@@ -462,6 +511,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             // this pipeline's first head of the unit: its x rows now, ahead of C, B and G (the pipeline's own
             // products of the previous unit have completed, so its x buffers are free)
             const int h_first = un.h0 + pl;
+            free_x();
             if (leader && h_first < un.h1) {
                 mbar_arrive_expect_tx(&pb.x_full, ((un.r == 1) ? 2u : 1u) * 16384u);
                 tma_load_4d(sXlo, &mX, &pb.x_full, 0, h_first, un.t0, un.b);
@@ -530,6 +580,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 // this head's x rows (the unit's first head's are already on their way); warm L2 for the
                 // pipeline's next head
                 if (use > 0) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
+                free_x();
                 if (leader) {
                     const uint32_t xboxes = (un.r == 1) ? 2u : 1u;
                     if (h != h_first) {
@@ -542,6 +593,24 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             tma_prefetch_4d(&mX, 0, h + 2, un.t0 + (int)q * kRows, un.b);
                 }
                 __syncwarp();
+                // without look-back another block past chunk 0 takes S~_{c-1} as the bf16 tile its owner
+                // stored: loaded here once published (while the CUDA-core warps build the mask), counted as
+                // read once it landed
+                const bool e_tma = kD == 1 && !un.owner && un.c > 0;
+                if (e_tma) {
+                    if (leader) {
+                        const int bh = un.b * sh.H + h;
+                        wait_flag(p.tin + bh * R + (un.c - 1) % R, un.c, p.flag_polls, abort, p.status);
+                        if (!*abort) {
+                            fence_proxy_async_global();
+                            mbar_arrive_expect_tx(&pb.e_full, (uint32_t)p.tile_rows * 128u);
+                            tma_load_3d(sXhi, &mR, &pb.e_full, 0, 0, bh * R + (un.c - 1) % R);
+                        } else {
+                            mbar_arrive(&pb.e_full);  // given up: no copy, the phase completes at once
+                        }
+                    }
+                    __syncwarp();
+                }
                 if (un.owner) {
                     // stages 2-3 products: S_pre = B_{<r}^T (scaled rows before the block) into A,
                     // S_own = B_r^T (scaled rows of the block) into B; M = n, N = p, K = tokens
@@ -563,7 +632,12 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     ++ocnt;
                 }
                 // stage 4 product: Y_inter = C_r E^T into A (E: the entering-state tile [n][p])
-                wait_bar(&pb.s_full, par(use), p.status, broken);
+                if (e_tma) {
+                    wait_bar(&pb.e_full, par(ecnt++), p.status, broken);
+                    if (leader && un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
+                } else {
+                    wait_bar(&pb.s_full, par(scnt++), p.status, broken);
+                }
                 if (!un.owner && use > 0) wait_bar(&pb.acc_free, par(use - 1), p.status, broken);
                 fence_after_sync();
                 if (leader) {
@@ -585,6 +659,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     mma_commit(&pb.mx_done);
                 }
                 __syncwarp();
+                if (kD == 1 && un.owner && un.c < sh.nc - 1 && p.halves == 2) ++tiles;  // this head's state tile
             }
             // this pipeline is done with the unit once its last products completed
             if (any) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
@@ -658,11 +733,12 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             const float *dtp = p.dt + ((size_t)un.b * sh.T + un.t0 + wtid) * sh.H;
             float dt_next = 0.f, a_next = 0.f, d_cur = p.D ? __ldg(p.D + h) : 0.f;
             scan((wtid < un.len) ? __ldg(dtp + h) : 0.f, __ldg(p.A + h));
-            // ctl reads `inc` of the chunk before for the pipeline's head early (acquire), so that the
-            // wait usually costs nothing by the time the state is needed (ctl's warp builds only zero
-            // mask slabs)
-            int ready_seen =
-                (ctl && un.c > 0) ? ld_acquire_gpu(inc_flag<kD>(p.inc, un.b * sh.H + h, un.c - 1)) : 0;
+            // an owner's ctl reads `inc` of the chunk before for the pipeline's head early (acquire), so
+            // that the wait usually costs nothing by the time the state is needed (ctl's warp builds only
+            // zero mask slabs); another block's issuer waits for it instead
+            int ready_seen = (ctl && (own || kD > 1) && un.c > 0)
+                                 ? ld_acquire_gpu(inc_flag<kD>(p.inc, un.b * sh.H + h, un.c - 1))
+                                 : 0;
             bool first_head = true;
             for (; h < un.h1; h += 2, ++use) {
                 const int bh = un.b * sh.H + h;
@@ -727,7 +803,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 // it zeros.  Warpgroup 0 takes the diagonal slab, warpgroup 1 the other three.
                 // an owner's slot count, read (acquire) before the mask for the same reason
                 int cons_seen = 0;
-                if (own && ctl && writes_ring && un.c >= R && (kD > 1 || p.halves == 2))
+                if (kD > 1 && own && ctl && writes_ring && un.c >= R)
                     cons_seen = ld_acquire_gpu(p.cons + bh * R + un.c % R);
                 if (first_head) wait_bar(&bars.g_done, par(gphase), p.status, broken);
                 fence_after_sync();
@@ -792,22 +868,41 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 if (ctl) bulk_wait_read();
 
                 // ---- stage 3: the state entering the block
-                if constexpr (kD == 1) {
-                    // without look-back: S~_{c-1} from the ring (published by the owner of chunk c-1) or
-                    // the initial state.  Chunk c's state goes to slot c % 3, which held chunk c-3's, read
-                    // by the other block of chunk c-2 (and by the owner of chunk c-2, whose read precedes
-                    // the publication this owner waited for); the other blocks of chunks k >= 1 read slot
-                    // (k - 1) % 3, so that slot has had c / 3 counted reads once that one is in, and no
-                    // later reader can add to the count before this owner publishes.
-                    const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
-                    const bool nv = n < N;
-                    if (ctl) {
-                        if (un.c > 0 && ready_seen < un.c)
-                            wait_flag(inc_flag<kD>(p.inc, bh, un.c - 1), un.c, p.flag_polls, abort, p.status);
-                        if (writes_ring && p.halves == 2 && un.c >= R && cons_seen < un.c / R)
-                            wait_flag(p.cons + R * bh + un.c % R, un.c / R, p.flag_polls, abort,
-                                      p.status);
+                // An owner's bf16 tile of S~_c, for the next chunk's other block: row n of the 128-byte-swizzled
+                // [n][p] tile in its x rows 0..127 buffer (free once the state products are done), rows past
+                // N zero; the publisher stores it with TMA.
+                const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
+                const bool nv = n < N;
+                auto store_tile = [&](const float (&v)[32]) {
+                    if (n < p.tile_rows) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            uint4 t;
+                            t.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+                            t.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+                            t.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+                            t.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+                            if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
+                            sts128(sXlo + swz(n, half * 4 + k), t);
+                        }
                     }
+                    fence_view_async_shared();
+                };
+                if (kD == 1 && !own && un.c > 0) {
+                    // another block past chunk 0: its issuer loads the entering state, the bf16 tile of
+                    // S~_{c-1}, by TMA.  Without the next head's prefix sums below, this barrier is the one
+                    // that orders ctl's wait for the previous y tile before the drain writes W.
+                    if (!has_next) named_bar_sync(bar_id, kPipeThreads);
+                } else if constexpr (kD == 1) {
+                    // without look-back: an owner takes S~_{c-1} (published by the owner of chunk c-1) from
+                    // the sequence's one fp32 slot and writes S~_c over it (the next owner, the slot's only
+                    // other reader, waits for this one's publication); chunk 0's blocks take the initial
+                    // state.  The bf16 tile of S~_c goes to slot c % 3 of the tile ring, which held chunk
+                    // c-3's, read by the other block of chunk c-2; the publisher waits for that read (the
+                    // other blocks of chunks k >= 1 read slot (k - 1) % 3, so the slot has had c / 3 counted
+                    // reads once that one is in).
+                    if (ctl && un.c > 0 && ready_seen < un.c)
+                        wait_flag(inc_flag<kD>(p.inc, bh, un.c - 1), un.c, p.flag_polls, abort, p.status);
                     named_bar_sync(bar_id, kPipeThreads);
                     float old[32];
                     if (un.c == 0) {
@@ -818,8 +913,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 32; ++q) old[q] = (src && nv && q < pv) ? __ldg(src + (size_t)q * ld) : 0.f;
                     } else {
-                        const float4 *src =
-                            reinterpret_cast<const float4 *>(p.ring + ((size_t)bh * R + (un.c - 1) % R) * PN);
+                        const float4 *src = reinterpret_cast<const float4 *>(p.ring + (size_t)bh * PN);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             const float4 t =
@@ -863,11 +957,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     fence_view_async_shared();
                     if (!own) {
                         __syncwarp();
-                        if (lane == 0) {
-                            mbar_arrive(&pb.s_full);
-                            // the ring entries are consumed: the publisher may count the slot as read
-                            if (un.c > 0) red_release_cta_shared_add(&s_copied[pl], 1);
-                        }
+                        if (lane == 0) mbar_arrive(&pb.s_full);  // chunk 0's other block: the initial state
                     } else {
                         // S~_c = exp(s_end - s_{r-1}) E + S_own.  S_own is read from TMEM before s_full,
                         // after which the issuer overwrites that accumulator.
@@ -884,13 +974,14 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&pb.s_full);
                         if (writes_ring) {
-                            float4 *dst = reinterpret_cast<float4 *>(p.ring + ((size_t)bh * R + un.c % R) * PN);
+                            float4 *dst = reinterpret_cast<float4 *>(p.ring + (size_t)bh * PN);
                             if (nv) {
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
                                     __stcg(dst + ring_quad(N, n, half * 8 + q),
                                            make_float4(old[4 * q], old[4 * q + 1], old[4 * q + 2], old[4 * q + 3]));
                             }
+                            if (p.halves == 2) store_tile(old);
                         } else if (nv && p.fin) {
                             const size_t ld = p.state_ld;
                             const int pv = p.p_full - p.p_off - half * 32;
@@ -911,8 +1002,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     // chunk's other block) have all added themselves to `cons`.
                     const int reads_per_use = kD + (p.halves == 2 ? 1 : 0);
                     const size_t PN2 = 2 * PN;  // a slot: S~, then L
-                    const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
-                    const bool nv = n < N;
                     const float *ring_bh = p.ring + (size_t)bh * R * PN2;
                     const int quad0 = half * 8;
                     if (own && writes_ring) {
@@ -997,6 +1086,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         named_bar_sync(bar_id, kPipeThreads);
                         base = s_base[pl];
                     } else {
+                        // another block reads S~_{c-1} from the ring (chunk 0's the initial state)
                         if (ctl && un.c > 0 && ready_seen < un.c)
                             wait_flag(inc_flag<kD>(p.inc, bh, un.c - 1), un.c, p.flag_polls, abort, p.status);
                         named_bar_sync(bar_id, kPipeThreads);
@@ -1089,7 +1179,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         __syncwarp();
                         if (lane == 0) red_release_cta_shared_add(&s_owned[pl], 1);  // the publisher releases the stores
                     } else {
-                        // S~_{c-1} in bf16 into row n of the tile (128-byte swizzled)
+                        // S~_{c-1} (or the initial state) in bf16 into row n of the tile
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             uint4 t;
@@ -1203,7 +1293,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (ctl) {
                         tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
-                        if (has_next && un.c > 0)
+                        if (has_next && (own || kD > 1) && un.c > 0)
                             ready_seen = ld_acquire_gpu(inc_flag<kD>(p.inc, bh + 2, un.c - 1));
                     }
                 } else {
@@ -1240,7 +1330,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     if (ctl) {
                         tma_store_4d(&mY, sW, 0, h, un.t0 + un.row0, un.b);
                         bulk_commit();
-                        if (has_next && un.c > 0)
+                        if (has_next && (own || kD > 1) && un.c > 0)
                             ready_seen = ld_acquire_gpu(inc_flag<kD>(p.inc, bh + 2, un.c - 1));
                     }
                 }
@@ -1269,16 +1359,15 @@ static int device_sm_count() {
     return n;
 }
 
-// Heads per work unit: enough to amortise the unit's C, B and G over several
-// heads, few enough that every SM gets several units.
-// Heads per unit: up to 8 (C, B and G are loaded and formed once per unit).  With look-back (long
+// Heads per work unit: enough to amortise the unit's C, B and G over several heads (they are loaded
+// and formed once per unit), few enough that every SM gets several units.  Up to 8 for the other
+// blocks and 4 for the owners' block, whose heads take about twice as long; with look-back (long
 // sequences, few heads) units of 2 heads, one per pipeline: a unit's later heads would otherwise wait
 // behind its first head's chain step, and the chunks in flight would advance at that pace.
-static int heads_per_unit(const Shape &sh, bool lookback) {
-    const int hpg = sh.heads_per_group;
-    if (lookback) return hpg < 2 ? hpg : 2;
-    if (hpg <= 8) return hpg;
-    const int blocks = (hpg + 7) / 8;
+static int heads_per_unit(const Shape &sh, bool lookback, bool owners) {
+    const int hpg = sh.heads_per_group, most = lookback ? 2 : owners ? 4 : 8;
+    if (hpg <= most) return hpg;
+    const int blocks = (hpg + most - 1) / most;
     return (hpg + blocks - 1) / blocks;
 }
 
@@ -1328,7 +1417,9 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.init = init;
     p.fin = fin;
     p.ring = reinterpret_cast<float *>(pw + w.ring_off);
+    p.tile_rows = fused_tile_rows(sh);
     p.inc = reinterpret_cast<int *>(pw + w.inc_off);
+    p.tin = reinterpret_cast<int *>(pw + w.tin_off);
     p.agg = reinterpret_cast<int *>(pw + w.agg_off);
     p.cons = reinterpret_cast<int *>(pw + w.cons_off);
     p.sig = reinterpret_cast<float *>(pw + w.sig_off);
@@ -1339,10 +1430,23 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     p.halves = sh.Q / kRows;
 
     const bool lookback = fused_lookback(sh) == 4;  // the workspace's layout has the same shape
-    p.heads_per_unit = heads_per_unit(sh, lookback);
-    p.blocks_per_group = (sh.heads_per_group + p.heads_per_unit - 1) / p.heads_per_unit;
-    p.units_per_role = sh.batch * sh.G * p.blocks_per_group;
-    p.n_units = sh.nc * p.units_per_role * p.halves;
+    // the bf16 state tiles without look-back: [b*H*3][tile_rows][64], one TMA box per tile (with
+    // look-back there are none and the map, over the fp32 ring, is never used)
+    CUtensorMap mR;
+    {
+        const uint64_t slots = lookback ? 1 : (uint64_t)sh.batch * sh.H * fused_ring_slots(1);
+        const uint64_t dr[3] = {(uint64_t)kP, (uint64_t)p.tile_rows, slots};
+        const uint64_t sr[2] = {(uint64_t)kP * 2, (uint64_t)p.tile_rows * kP * 2};
+        const uint32_t boxr[3] = {(uint32_t)kP, (uint32_t)p.tile_rows, 1};
+        if (!make_map_bf16(&mR, pw + (lookback ? w.ring_off : w.tile_off), 3, dr, sr, boxr))
+            return cudaErrorInvalidValue;
+    }
+    for (int r = 0; r < 2; ++r) {
+        p.hpu[r] = heads_per_unit(sh, lookback, r == 1 && p.halves == 2);
+        p.blocks[r] = (sh.heads_per_group + p.hpu[r] - 1) / p.hpu[r];
+        p.units[r] = sh.batch * sh.G * p.blocks[r];
+    }
+    p.n_units = sh.nc * (p.halves == 2 ? p.units[0] + p.units[1] : p.units[0]);
     p.flag_polls = (dbg && dbg->flag_polls) ? dbg->flag_polls : kDefaultFlagPolls;
     p.withhold_bh = dbg ? dbg->withhold_bh : -1;
     p.withhold_c = dbg ? dbg->withhold_c : -1;
@@ -1352,7 +1456,7 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     const int grid = min(p.n_units, device_sm_count());
-    kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, p);
+    kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, mR, p);
     return cudaGetLastError();
 }
 

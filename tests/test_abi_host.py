@@ -52,17 +52,21 @@ def test_version_and_status_strings(lib):
 
 def test_workspace_bytes(lib):
     f = lib.ssd_fwd_workspace_bytes
-    w = f(4, 2048, 80, 64, 1, 128, 256, 1)      # fused tensor-core path: flags + the two-slot state ring
+    w = f(4, 2048, 80, 64, 1, 128, 256, 1)      # fused tensor-core path: flags + the state rings
     assert w % 256 == 0
     nc = 8
-    ring = 4 * 80 * 3 * 64 * 128 * 4   # three slots per (batch, head)
+    tile = 128 * 64 * 2                # a bf16 state tile (N = 128 rows of 64)
+    ring = 4 * 80 * (64 * 128 * 4 + 3 * tile)   # per (batch, head): one fp32 state, three bf16 tiles
     assert ring <= w < ring + (1 << 16)
-    w256 = f(8, 4096, 32, 64, 1, 256, 256, 1)   # N = 256: two halves, each with its own flags and ring
-    ring256 = 2 * 8 * 32 * 3 * 64 * 128 * 4
+    w256 = f(8, 4096, 32, 64, 1, 256, 256, 1)   # N = 256: two halves, each with its own flags and rings
+    ring256 = 2 * 8 * 32 * (64 * 128 * 4 + 3 * tile)
     assert ring256 <= w256 < ring256 + (1 << 17)
     wlong = f(1, 131072, 48, 64, 8, 128, 256, 1)   # look-back over 4 chunks: 8 slots of S~ and L
     ringlong = 48 * 8 * 2 * 64 * 128 * 4
     assert ringlong <= wlong < ringlong + (1 << 17)
+    assert f(8, 4096, 32, 64, 1, 64, 256, 1) < (8 * 32 * (64 * 64 * 4 + 3 * 64 * 64 * 2)) + (1 << 16)  # 64-row tiles
+    # the shapes the allocation-free entry point serves fit its 32 MiB scratch
+    assert w <= (32 << 20) and wlong <= (32 << 20)
     w32p = f(8, 4096, 32, 32, 1, 128, 256, 1)   # P = 32 is padded: the ring still holds 64 rows
     assert w32p == f(8, 4096, 32, 64, 1, 128, 256, 1)
     assert f(8, 4096, 32, 128, 1, 256, 256, 1) == 2 * w256   # four launches of 64 x 128 states
