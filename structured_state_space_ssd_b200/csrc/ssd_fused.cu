@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         // cumulative).
         // ------------------------------------------------------------------
         const int pl = warp - kSimtWarps - 2;
-        const uint8_t *sTile = smem + kOffPipe + pl * kPipeBytes;  // the owner's x rows 0..127 buffer
+        const uint8_t *sTile = smem + kOffPipe + pl * kPipeBytes + 16384;  // the owner's tile, in W
         uint32_t ucnt = 0, ocnt = 0, tcnt = 0, acnt = 0;
         // bounded wait for one of this pipeline's shared-memory counts to reach `target`
         auto wait_count = [&](const uint32_t *cnt, uint32_t target) {
@@ -416,18 +416,20 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         wait_count(&s_agg[pl], kPipeWarps * ++acnt);
                         if (lane == 0 && publish) st_release_gpu(p.agg + bh * R + un.c % R, un.c + 1);
                     }
-                    wait_count(&s_owned[pl], kPipeWarps * ++ocnt);
-                    // the bf16 tile of S~_c (in the owner's x rows 0..127 buffer) for the next chunk's other
-                    // block goes to slot c % R once that slot's earlier readers are done (with look-back the
-                    // owner waited for them before storing L_c).  The store is issued first, so that it reads
-                    // shared memory while inc is released; the issuer reuses the buffer once it has, and
-                    // tin is released once the store is complete.
+                    // the bf16 tile of S~_c (in the owner's W buffer) for the next chunk's other block goes to
+                    // slot c % R once that slot's earlier readers are done (waited for while the owner's warps
+                    // still work).  W is handed back (the drain stages y there) as soon as the store has read
+                    // it, before inc is released (whose fence takes longer); tin is released once the store
+                    // is complete.
                     const bool tile = kD == 1 && writes && p.halves == 2;
+                    if (tile && lane == 0 && un.c >= R)
+                        wait_flag(p.cons + bh * R + un.c % R, un.c / R, p.flag_polls, abort, p.status);
+                    wait_count(&s_owned[pl], kPipeWarps * ++ocnt);
                     if (tile && lane == 0) {
-                        if (kD == 1 && un.c >= R)
-                            wait_flag(p.cons + bh * R + un.c % R, un.c / R, p.flag_polls, abort, p.status);
                         tma_store_3d(&mR, sTile, 0, 0, bh * R + un.c % R);
                         bulk_commit();
+                        bulk_wait_read();
+                        mbar_arrive(&bars.pb[pl].t_free);
                     }
                     if (lane == 0 && publish) st_release_gpu(inc_flag<kD>(p.inc, bh, un.c), un.c + 1);
                     // with look-back the owner has read (at most) the slots of the D chunks before it:
@@ -435,8 +437,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     // the publication the next owner waits for)
                     if (kD > 1 && lane < min(kD, un.c)) red_release_add_gpu(p.cons + bh * R + (un.c - 1 - lane) % R, 1);
                     if (tile && lane == 0) {
-                        bulk_wait_read();
-                        mbar_arrive(&bars.pb[pl].t_free);
                         bulk_wait_all();
                         fence_proxy_async_global();
                         if (publish) st_release_gpu(p.tin + bh * R + un.c % R, un.c + 1);
@@ -475,15 +475,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         const uint32_t idInter = idesc_bf16_f32(kRows, kP, 0, 1);   // C (K-major) x state tile [n][p]
         const uint32_t idMX = idesc_bf16_f32(kRows, kP, 0, 1);      // mask (TMEM) x x rows [i][p]
         uint32_t use = 0, ocnt = 0, ucnt = 0, cbcnt = 0, udone = 0;
-        uint32_t scnt = 0, ecnt = 0;           // s_full and e_full phases (not every head has both)
-        uint32_t tiles = 0, tiles_freed = 0;   // an owner's bf16 state tiles stored from x rows 0..127
-        // x rows 0..127 hold an owner's state tile until its TMA store has read it: wait before reloading
-        auto free_x = [&]() {
-            if (tiles != tiles_freed) {
-                wait_bar(&pb.t_free, par(tiles - 1), p.status, broken);
-                tiles_freed = tiles;
-            }
-        };
+        uint32_t scnt = 0, ecnt = 0;  // s_full and e_full phases (not every head has both)
         int next_u = -1;
         for (;;) {
             int u = 0;
@@ -511,7 +503,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
             // this pipeline's first head of the unit: its x rows now, ahead of C, B and G (the pipeline's own
             // products of the previous unit have completed, so its x buffers are free)
             const int h_first = un.h0 + pl;
-            free_x();
             if (leader && h_first < un.h1) {
                 mbar_arrive_expect_tx(&pb.x_full, ((un.r == 1) ? 2u : 1u) * 16384u);
                 tma_load_4d(sXlo, &mX, &pb.x_full, 0, h_first, un.t0, un.b);
@@ -570,17 +561,18 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
                 __syncwarp();
             }
-            // x rows of this block; the entering-state tile: W for an owner, the unused x buffer for
-            // another block (so that it need not wait for the previous head's y tile to leave W)
+            // x rows of this block; the entering-state tile: for an owner of the second block x rows
+            // 0..127 (free once its state products are done; W then holds its bf16 tile of S~_c), W for
+            // the only block, the unused x buffer for another block (so that it need not wait for the
+            // previous head's y tile to leave W)
             uint8_t *sXr = (un.r == 1) ? sXhi : sXlo;
-            uint8_t *sE = un.owner ? sW : sXhi;
+            uint8_t *sE = un.owner ? (un.r == 1 ? sXlo : sW) : sXhi;
             bool any = false;
             for (int h = un.h0 + pl; h < un.h1; h += 2, ++use) {
                 any = true;
                 // this head's x rows (the unit's first head's are already on their way); warm L2 for the
                 // pipeline's next head
                 if (use > 0) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
-                free_x();
                 if (leader) {
                     const uint32_t xboxes = (un.r == 1) ? 2u : 1u;
                     if (h != h_first) {
@@ -659,7 +651,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     mma_commit(&pb.mx_done);
                 }
                 __syncwarp();
-                if (kD == 1 && un.owner && un.c < sh.nc - 1 && p.halves == 2) ++tiles;  // this head's state tile
             }
             // this pipeline is done with the unit once its last products completed
             if (any) wait_bar(&pb.mx_done, par(use - 1), p.status, broken);
@@ -695,7 +686,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         float *sTot = sF + 256;                                                   // warp totals
         const uint32_t tA = tmem + col_acc_a(pl), tB = tmem + col_acc_b(pl), tM = tmem + col_mask(pl);
         const size_t PN = (size_t)kP * N;
-        uint32_t use = 0, ocnt = 0, ucnt = 0, gcnt = 0;
+        uint32_t use = 0, ocnt = 0, ucnt = 0, gcnt = 0, tcnt = 0;  // tcnt: this pipeline's stored state tiles
 
         // stage 0: inclusive prefix sums of dt*A over the chunk, in log2 units, into sJ (and the
         // mask's column factors exp(s_{i|31} - s_i) <= 1 into sF); every thread of the pipeline
@@ -869,8 +860,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
 
                 // ---- stage 3: the state entering the block
                 // An owner's bf16 tile of S~_c, for the next chunk's other block: row n of the 128-byte-swizzled
-                // [n][p] tile in its x rows 0..127 buffer (free once the state products are done), rows past
-                // N zero; the publisher stores it with TMA.
+                // [n][p] tile in W (free once the state products are done; the drain waits for the store
+                // before it stages y there), rows past N zero; the publisher stores it with TMA.
                 const int n = lrow;  // state row of this thread (TMEM lane); p in [32 half, 32 half + 32)
                 const bool nv = n < N;
                 auto store_tile = [&](const float (&v)[32]) {
@@ -883,7 +874,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             t.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
                             t.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
                             if (!nv) t = make_uint4(0u, 0u, 0u, 0u);
-                            sts128(sXlo + swz(n, half * 4 + k), t);
+                            sts128(sW + swz(n, half * 4 + k), t);
                         }
                     }
                     fence_view_async_shared();
@@ -924,7 +915,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             old[4 * q + 3] = t.w;
                         }
                     }
-                    uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
+                    // the entering-state tile [n][p], B operand of stage 4 (as the issuer's sE)
+                    uint8_t *sE = own ? (un.r == 1 ? sXlo : sW) : sXhi;
                     if (own) {
                         wait_bar(&pb.d_done, par(ocnt), p.status, broken);
                         ++ocnt;
@@ -1126,7 +1118,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                             old[4 * q + 3] = fmaf(e, old[4 * q + 3], t[q].w);
                         }
                     }
-                    uint8_t *sE = own ? sW : sXhi;  // the entering-state tile [n][p], B operand of stage 4
+                    // the entering-state tile [n][p], B operand of stage 4 (as the issuer's sE)
+                    uint8_t *sE = own ? (un.r == 1 ? sXlo : sW) : sXhi;
                     if (own) {
                         // E = exp(s_{r-1}) S~_{c-1} + S_pre (S~_{c-1} for r = 0) into the tile, and
                         // S~_c = exp(sigma_c) S~_{c-1} + L_c in place, with L_c exactly as published.  S_pre
@@ -1227,6 +1220,8 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                         yprev[q] = (jv && 8 * q < pv) ? __ldg(yp + q) : make_uint4(0u, 0u, 0u, 0u);
                 }
                 wait_bar(&pb.mx_done, par(use), p.status, broken);
+                // an owner's bf16 state tile is in W until the publisher's store has read it
+                if (kD == 1 && writes_ring && p.halves == 2) wait_bar(&pb.t_free, par(tcnt++), p.status, broken);
                 fence_after_sync();
                 if constexpr (kGated) {
                     // g = y * silu(z) in fp32 (y is never rounded), then the row's 64 channels normalised:
