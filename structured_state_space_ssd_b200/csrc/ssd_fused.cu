@@ -93,7 +93,8 @@ constexpr uint32_t kPipeBytes = 49152;  // W: scaled x rows, then the entering-s
 constexpr uint32_t kOffAux = kOffPipe + 2 * kPipeBytes;
 constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units), column factors, warp totals
 constexpr uint32_t kOffStat = kOffAux + 2 * kAuxFloats * 4;  // gated drain: per pipeline, half, row (mean, M2)
-constexpr uint32_t kSmemBytes = kOffStat + 2 * 2 * kRows * 8 + 1024;
+constexpr uint32_t kOffWB = kOffStat + 2 * 2 * kRows * 8;      // gated drain: per pipeline, the head's weight, bias
+constexpr uint32_t kSmemBytes = kOffWB + 2 * 2 * kP * 4 + 1024;
 
 constexpr uint32_t kDefaultFlagPolls = 1u << 22;
 
@@ -684,6 +685,7 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
         float *sJ = reinterpret_cast<float *>(smem + kOffAux) + pl * kAuxFloats;  // s in log2 units
         float *sF = sJ + 256;                                                     // column factors
         float *sTot = sF + 256;                                                   // warp totals
+        float *sWB = reinterpret_cast<float *>(smem + kOffWB) + pl * 2 * kP;      // gated: weight, bias
         const uint32_t tA = tmem + col_acc_a(pl), tB = tmem + col_acc_b(pl), tM = tmem + col_mask(pl);
         const size_t PN = (size_t)kP * N;
         uint32_t use = 0, ocnt = 0, ucnt = 0, gcnt = 0, tcnt = 0;  // tcnt: this pipeline's stored state tiles
@@ -741,9 +743,15 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                 }
                 const float Dh = d_cur;
                 if (has_next) d_cur = p.D ? __ldg(p.D + h + 2) : 0.f;
-                // gated drain: this head's z rows on their way to L2 (one 128-byte line per row)
-                if (kGated && half == 0 && j < un.len)
-                    prefetch_l2(p.z + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP);
+                // gated drain: this head's z rows on their way to L2 (one 128-byte line per row), and its norm
+                // weight and bias into shared memory (an async copy: no register, so no barrier waits for it)
+                if (kGated) {
+                    if (half == 0 && j < un.len) prefetch_l2(p.z + (((size_t)un.b * sh.T + un.t0 + j) * sh.H + h) * kP);
+                    if (wtid < 32) {
+                        const float *src = (wtid < 16) ? p.gw : p.gb;
+                        if (src) cp_async16(sWB + wtid * 4, src + h * kP + (wtid & 15) * 4);
+                    }
+                }
                 const float s_end = sJ[end];
                 const float s_ref = (un.r == 1) ? sJ[kRows - 1] : 0.f;  // s_{r-1}
                 const float sj = sJ[j];
@@ -1193,7 +1201,11 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     }
                 }
 
-                // gated drain: z of this row's 32 channels, loaded while the products run
+                // the next head's prefix sums, while this head's products run
+                if (has_next) scan(dt_next, a_next);
+
+                // gated drain: z of this row's 32 channels (in L2 since the head's start), loaded after the
+                // prefix sums, whose barriers would otherwise wait for these loads
                 uint4 zv[4];
                 if (kGated) {
                     const bool jv = j < un.len;
@@ -1203,8 +1215,6 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     for (int q = 0; q < 4; ++q) zv[q] = jv ? __ldg(zp + q) : make_uint4(0u, 0u, 0u, 0u);
                 }
 
-                // the next head's prefix sums, while this head's products run
-                if (has_next) scan(dt_next, a_next);
 
                 // ---- stages 4-5: y_j = exp(s_j - s_{r-1}) Y_inter + Y_intra (the D skip is in the mask),
                 // staged as bf16 in W (128-byte swizzled [j][p]) and written by one TMA store (rows
@@ -1261,21 +1271,22 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
                     const float m2 = (sa[0] + sa[1]) + (sa[2] + sa[3]);
                     float2 *sStat = reinterpret_cast<float2 *>(smem + kOffStat) + pl * 2 * kRows;
                     sStat[half * kRows + lrow] = make_float2(m, m2);
+                    if (wtid < 32) cp_async_wait_all();  // the weight and bias, published by the barrier
                     named_bar_sync(bar_id, kPipeThreads);
                     const float2 o = sStat[(1 - half) * kRows + lrow];
                     const float dm = m - o.x;
                     const float mean = 0.5f * (m + o.x);
                     const float rstd = rsqrtf(fmaf(16.f * dm, dm, m2 + o.y) * (1.f / 64) + p.eps);
-                    const float4 *wp = p.gw ? reinterpret_cast<const float4 *>(p.gw + h * kP + half * 32) : nullptr;
-                    const float4 *bp = p.gb ? reinterpret_cast<const float4 *>(p.gb + h * kP + half * 32) : nullptr;
+                    const float4 *wp = p.gw ? reinterpret_cast<const float4 *>(sWB + half * 32) : nullptr;
+                    const float4 *bp = p.gb ? reinterpret_cast<const float4 *>(sWB + kP + half * 32) : nullptr;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         uint32_t o4[4];
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int q = 8 * k + 4 * e;
-                            const float4 wv = wp ? __ldg(wp + q / 4) : make_float4(1.f, 1.f, 1.f, 1.f);
-                            const float4 bv = bp ? __ldg(bp + q / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            const float4 wv = wp ? wp[q / 4] : make_float4(1.f, 1.f, 1.f, 1.f);
+                            const float4 bv = bp ? bp[q / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
                             o4[2 * e] = pack_bf16x2(fmaf((g[q] - mean) * rstd, wv.x, bv.x),
                                                     fmaf((g[q + 1] - mean) * rstd, wv.y, bv.y));
                             o4[2 * e + 1] = pack_bf16x2(fmaf((g[q + 2] - mean) * rstd, wv.z, bv.z),
