@@ -500,6 +500,87 @@ __global__ void __launch_bounds__(256) group_reduce_kernel(const float *__restri
     }
 }
 
+// The same sums with each lane on 4 consecutive n (16-byte loads of the per-head terms, 8 or 16 bytes of
+// B, C, dB, dC), for N a multiple of 4 and aligned rows: a row of 128 is one load per lane, and eight
+// heads' rows (four for N above 128) are in flight at once; the sums over heads still run in head order.
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 r = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&r.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&r.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 r;
+    r.x = *reinterpret_cast<const uint32_t *>(&a);
+    r.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = r;
+}
+
+// kNV: 4-vectors per lane (1 for N up to 128, 2 up to 256)
+template <typename T, int kNV>
+__global__ void __launch_bounds__(256) group_reduce_vec_kernel(const float *__restrict__ dBh,
+                                                               const float *__restrict__ dCh,
+                                                               const T *__restrict__ Bm, const T *__restrict__ Cm,
+                                                               T *__restrict__ dB, T *__restrict__ dC,
+                                                               float *__restrict__ dsig, Shape sh) {
+    const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long units = (long long)sh.batch * sh.T * sh.G;
+    if (unit >= units) return;
+    const int lane = threadIdx.x & 31;
+    const int g = (int)(unit % sh.G);
+    const long long tok = unit / sh.G;  // b * T + t
+    const int b = (int)(tok / sh.T), t = (int)(tok - (long long)b * sh.T);
+    const size_t grow = (size_t)unit * sh.N;  // row (b, t, g) of B, C, dB, dC
+    const int V = sh.N / 4;                   // 4-vectors per row
+    float4 bv[kNV], cv[kNV], sb[kNV], sc[kNV];
+#pragma unroll
+    for (int m = 0; m < kNV; ++m) {
+        const int v = lane + 32 * m;
+        const bool ok = v < V;
+        bv[m] = ok ? load4(Bm + grow + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cv[m] = ok ? load4(Cm + grow + 4 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sb[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+        sc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll(8 / kNV)
+    for (int hh = 0; hh < sh.heads_per_group; ++hh) {
+        const int h = g * sh.heads_per_group + hh;
+        const size_t hrow = ((size_t)tok * sh.H + h) * sh.N;
+        float d = 0.f;
+#pragma unroll
+        for (int m = 0; m < kNV; ++m) {
+            const int v = lane + 32 * m;
+            if (v < V) {
+                const float4 db = load4(dBh + hrow + 4 * v), dc = load4(dCh + hrow + 4 * v);
+                sb[m].x += db.x; sb[m].y += db.y; sb[m].z += db.z; sb[m].w += db.w;
+                sc[m].x += dc.x; sc[m].y += dc.y; sc[m].z += dc.z; sc[m].w += dc.w;
+                d = fmaf(cv[m].x, dc.x, d);
+                d = fmaf(-bv[m].x, db.x, d);
+                d = fmaf(cv[m].y, dc.y, d);
+                d = fmaf(-bv[m].y, db.y, d);
+                d = fmaf(cv[m].z, dc.z, d);
+                d = fmaf(-bv[m].z, db.z, d);
+                d = fmaf(cv[m].w, dc.w, d);
+                d = fmaf(-bv[m].w, db.w, d);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (lane == 0) dsig[((size_t)b * sh.H + h) * sh.T + t] = d;
+    }
+#pragma unroll
+    for (int m = 0; m < kNV; ++m) {
+        const int v = lane + 32 * m;
+        if (v < V) {
+            store4(dB + grow + 4 * v, sb[m]);
+            store4(dC + grow + 4 * v, sc[m]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Per (head, batch): the suffix sums of dsigma over the whole sequence (fp64),
 // plus <dfinal, final> at the last token, give d(dt_u A_h); write
@@ -718,7 +799,17 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
         if (launch_scan<T, float, false>(ac, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     }
     const long long units = (long long)sh.batch * sh.T * sh.G;
-    group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
+    // the vector form wants rows of B, C, dB, dC aligned to their 4-vectors (N a multiple of 4)
+    const size_t a4 = 4 * sizeof(T);
+    const bool gvec = sh.N % 4 == 0 && reinterpret_cast<uintptr_t>(B) % a4 == 0 &&
+                      reinterpret_cast<uintptr_t>(C) % a4 == 0 && reinterpret_cast<uintptr_t>(dB) % a4 == 0 &&
+                      reinterpret_cast<uintptr_t>(dC) % a4 == 0;
+    if (gvec && sh.N <= 128)
+        group_reduce_vec_kernel<T, 1><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
+    else if (gvec)
+        group_reduce_vec_kernel<T, 2><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
+    else
+        group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     dt_scan_kernel<T><<<dim3(sh.H, sh.batch), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh,
                                                                     vec);
