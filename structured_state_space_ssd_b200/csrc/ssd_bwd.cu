@@ -134,6 +134,44 @@ __global__ void __launch_bounds__(256) state_passing_bwd_kernel(float *__restric
     if (dinit) dinit[((size_t)b * sh.H + h) * PN + e] = run;
 }
 
+// The same with four consecutive channels per thread (16-byte loads and stores), for P*N a multiple of 4
+// and 16-byte aligned dfin and dinit: grid (ceil(P*N/1024), H, batch).
+__global__ void __launch_bounds__(256) state_passing_bwd_vec_kernel(float *__restrict__ Gs,
+                                                                    const float *__restrict__ s,
+                                                                    const float *__restrict__ dfin,
+                                                                    float *__restrict__ dinit, Shape sh) {
+    const int PN = sh.P * sh.N;
+    const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
+    const int h = blockIdx.y, b = blockIdx.z;
+    if (e >= PN) return;
+    float4 run = dfin ? *reinterpret_cast<const float4 *>(dfin + ((size_t)b * sh.H + h) * PN + e)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *sb = s + ((size_t)b * sh.H + h) * sh.nc * sh.Q;
+    const size_t cstride = (size_t)sh.H * PN;
+    float *base = Gs + ((size_t)b * sh.nc * sh.H + h) * PN + e;
+    for (int cend = sh.nc; cend > 0; cend -= 8) {
+        const int cn = min(8, cend), c0 = cend - cn;
+        float4 loc[8];
+        float dec[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < cn) {
+                loc[k] = *reinterpret_cast<const float4 *>(base + (size_t)(c0 + k) * cstride);
+                dec[k] = expf(sb[(size_t)(c0 + k) * sh.Q + sh.Q - 1]);
+            }
+        }
+#pragma unroll
+        for (int k = 7; k >= 0; --k) {
+            if (k < cn) {
+                *reinterpret_cast<float4 *>(base + (size_t)(c0 + k) * cstride) = run;
+                run = make_float4(fmaf(dec[k], run.x, loc[k].x), fmaf(dec[k], run.y, loc[k].y),
+                                  fmaf(dec[k], run.z, loc[k].z), fmaf(dec[k], run.w, loc[k].w));
+            }
+        }
+    }
+    if (dinit) *reinterpret_cast<float4 *>(dinit + ((size_t)b * sh.H + h) * PN + e) = run;
+}
+
 // ---------------------------------------------------------------------------
 // Masked scan over one chunk, one head and a 64-row tile:
 //
@@ -764,7 +802,11 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     // backward states: sum_i exp(s_i) dy_i C_i^T per chunk, then dHout_c and dinit
     if (chunk_states(dy, C, Gout, true) != cudaSuccess) return SSD_ERR_CUDA;
     const int PN = sh.P * sh.N;
-    state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
+    if (PN % 4 == 0 && reinterpret_cast<uintptr_t>(dfin) % 16 == 0 && reinterpret_cast<uintptr_t>(dinit) % 16 == 0)
+        state_passing_bwd_vec_kernel<<<dim3((PN + 1023) / 1024, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit,
+                                                                                             sh);
+    else
+        state_passing_bwd_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(Gout, s, dfin, dinit, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     const int vec = al && sh.P % VE == 0 && sh.N % VE == 0;
     const int st_vec = sh.P % 4 == 0 && sh.N % 4 == 0;

@@ -202,6 +202,43 @@ __global__ void __launch_bounds__(256) state_passing_kernel(float *__restrict__ 
     if (fin) fin[((size_t)b * sh.H + h) * PN + e] = run;
 }
 
+// The same with four consecutive channels per thread (16-byte loads and stores), for P*N a multiple of 4
+// and 16-byte aligned initial and final states: grid (ceil(P*N/1024), H, batch).
+__global__ void __launch_bounds__(256) state_passing_vec_kernel(float *__restrict__ S, const float *__restrict__ s,
+                                                                const float *__restrict__ init,
+                                                                float *__restrict__ fin, Shape sh) {
+    const int PN = sh.P * sh.N;
+    const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
+    const int h = blockIdx.y, b = blockIdx.z;
+    if (e >= PN) return;
+    float4 run = init ? *reinterpret_cast<const float4 *>(init + ((size_t)b * sh.H + h) * PN + e)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *sb = s + ((size_t)b * sh.H + h) * sh.nc * sh.Q;
+    const size_t cstride = (size_t)sh.H * PN;
+    float *base = S + ((size_t)b * sh.nc * sh.H + h) * PN + e;
+    for (int c0 = 0; c0 < sh.nc; c0 += 8) {
+        const int cn = min(8, sh.nc - c0);
+        float4 loc[8];
+        float dec[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < cn) {
+                loc[k] = *reinterpret_cast<const float4 *>(base + (size_t)(c0 + k) * cstride);
+                dec[k] = expf(sb[(size_t)(c0 + k) * sh.Q + sh.Q - 1]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k < cn) {
+                *reinterpret_cast<float4 *>(base + (size_t)(c0 + k) * cstride) = run;
+                run = make_float4(fmaf(dec[k], run.x, loc[k].x), fmaf(dec[k], run.y, loc[k].y),
+                                  fmaf(dec[k], run.z, loc[k].z), fmaf(dec[k], run.w, loc[k].w));
+            }
+        }
+    }
+    if (fin) *reinterpret_cast<float4 *>(fin + ((size_t)b * sh.H + h) * PN + e) = run;
+}
+
 // ---------------------------------------------------------------------------
 // Stages 1, 4 and 5 fused, plus the D skip, for one 64-row tile of one chunk
 // and one head:
@@ -400,7 +437,10 @@ cudaError_t launch_chunk_state(const T *x, const T *B, const float *s, float *S,
 cudaError_t launch_state_passing(float *S, const float *s, const float *init, float *fin, const Shape &sh,
                                  cudaStream_t st) {
     const int PN = sh.P * sh.N;
-    state_passing_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(S, s, init, fin, sh);
+    if (PN % 4 == 0 && reinterpret_cast<uintptr_t>(init) % 16 == 0 && reinterpret_cast<uintptr_t>(fin) % 16 == 0)
+        state_passing_vec_kernel<<<dim3((PN + 1023) / 1024, sh.H, sh.batch), 256, 0, st>>>(S, s, init, fin, sh);
+    else
+        state_passing_kernel<<<dim3((PN + 255) / 256, sh.H, sh.batch), 256, 0, st>>>(S, s, init, fin, sh);
     return cudaGetLastError();
 }
 
