@@ -111,6 +111,10 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                           const __grid_constant__ CUtensorMap mV, const bt::Args a, int r_head, int k_head,
                           int v_head) {
     static_assert(!kSplit || KD == 64, "the low part of the state tile has room for KD = 64");
+    static_assert(KD == 64 || W == 64, "the fp32 state is staged in the unused second atom of K or V");
+    // the fp32 state [KD][W] (32 KB), copied in asynchronously at the start: the K region's second atom
+    // (KD = 64) or the V region's (W = 64), which this shape leaves unused
+    constexpr uint32_t kOffRaw = (KD == 64) ? kOffK + 32768 : kOffV + 32768;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t ld_full, g_done, st_full, m_full, mx_done, fin_done;
@@ -205,34 +209,13 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         const int lrow = wq * 32 + lane;            // this thread's row of the block
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         const int j = r0 + lrow;                    // row within the chunk
+        // the fp32 state on its way into shared memory (async copies: no barrier waits for them, so its
+        // DRAM latency passes while the masks are built)
+        const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
+        float *sRaw = reinterpret_cast<float *>(smem + kOffRaw);
+        for (int i = tid; i < KD * W / 4; i += 32 * kCudaWarps) cp_async16(sRaw + 4 * i, Sp + 4 * i);
         const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
         for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) sq[i] = sch[i];
-        // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows
-        const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
-        for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
-            const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
-            float v[8];
-            if (a.st_kw) {
-                const float4 u0 = *reinterpret_cast<const float4 *>(Sp + (size_t)k * W + w0);
-                const float4 u1 = *reinterpret_cast<const float4 *>(Sp + (size_t)k * W + w0 + 4);
-                v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
-                v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = Sp[(size_t)(w0 + e) * KD + k];
-            }
-            const uint4 t = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                       pack_bf16x2(v[6], v[7]));
-            *reinterpret_cast<uint4 *>(sSt + (w0 >> 6) * 16384 + swz(k, (w0 & 63) >> 3)) = t;
-            if (kSplit) {
-                const uint4 tl = make_uint4(pack_lo(v[0], v[1], t.x), pack_lo(v[2], v[3], t.y),
-                                            pack_lo(v[4], v[5], t.z), pack_lo(v[6], v[7], t.w));
-                *reinterpret_cast<uint4 *>(sStLo + (w0 >> 6) * 8192 + swz(k, (w0 & 63) >> 3)) = tl;
-            }
-        }
-        fence_view_async_shared();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_full);
         named_bar_sync(1, 32 * kCudaWarps);  // the prefix sums are in
         const float sj = (j < len) ? sq[j] : 0.f;
 
@@ -268,6 +251,35 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&m_full);
         }
+
+        // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows,
+        // from the staged fp32 state
+        cp_async_wait_all();
+        named_bar_sync(1, 32 * kCudaWarps);  // every thread's copies are in
+        for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
+            const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
+            float v[8];
+            if (a.st_kw) {
+                const float4 u0 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0);
+                const float4 u1 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0 + 4);
+                v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+                v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = sRaw[(w0 + e) * KD + k];
+            }
+            const uint4 t = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                       pack_bf16x2(v[6], v[7]));
+            *reinterpret_cast<uint4 *>(sSt + (w0 >> 6) * 16384 + swz(k, (w0 & 63) >> 3)) = t;
+            if (kSplit) {
+                const uint4 tl = make_uint4(pack_lo(v[0], v[1], t.x), pack_lo(v[2], v[3], t.y),
+                                            pack_lo(v[4], v[5], t.z), pack_lo(v[6], v[7], t.w));
+                *reinterpret_cast<uint4 *>(sStLo + (w0 >> 6) * 8192 + swz(k, (w0 & 63) >> 3)) = tl;
+            }
+        }
+        fence_view_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&st_full);
 
         // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns
         wait_bar(&fin_done, 0, a.status);
