@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     constexpr uint32_t kOffRaw = (KD == 64) ? kOffK + 32768 : kOffV + 32768;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t ld_full, g_done, st_full, m_full, mx_done, fin_done;
+    __shared__ uint64_t ld_full, ld_v, g_done, st_full, m_full, mx_done, fin_done;
     __shared__ uint32_t tslot;
     const Shape &sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     if (tid == 0) {
         mbar_init(&ld_full, 1);
+        mbar_init(&ld_v, 1);
         mbar_init(&g_done, 1);
         mbar_init(&mx_done, 1);
         mbar_init(&fin_done, 1);
@@ -152,16 +153,17 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         // ---------------- TMA and MMA issue (lane 0) ----------------
         if (lane == 0) {
             const int hr = r_head ? h : g, hk = k_head ? h : g, hv = v_head ? h : g;
-            const uint32_t bytes = (uint32_t)(KD / 64) * 16384u + (uint32_t)(KD / 64 + W / 64) * nh * 16384u;
-            mbar_arrive_expect_tx(&ld_full, bytes);
+            // R and K (for G) on one barrier, V (for the masked product, later) on another
+            mbar_arrive_expect_tx(&ld_full, (uint32_t)(KD / 64) * (1u + (uint32_t)nh) * 16384u);
             for (int k = 0; k < KD / 64; ++k) {
                 tma_load_4d(sR + k * 16384, &mR, &ld_full, k * 64, hr, t0 + r0, b);
                 for (int q = 0; q < nh; ++q)
                     tma_load_4d(sK + k * 32768 + q * 16384, &mK, &ld_full, k * 64, hk, t0 + cbeg + q * kRows, b);
             }
+            mbar_arrive_expect_tx(&ld_v, (uint32_t)(W / 64) * (uint32_t)nh * 16384u);
             for (int k = 0; k < W / 64; ++k)
                 for (int q = 0; q < nh; ++q)
-                    tma_load_4d(sV + k * 32768 + q * 16384, &mV, &ld_full, k * 64, hv, t0 + cbeg + q * kRows, b);
+                    tma_load_4d(sV + k * 32768 + q * 16384, &mV, &ld_v, k * 64, hv, t0 + cbeg + q * kRows, b);
             wait_bar(&ld_full, 0, a.status);
             fence_after_sync();
             const uint32_t idG = idesc_bf16_f32(kRows, kRows, 0, 0);  // R (K-major) x K rows (K-major)
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                 }
                 mma_commit(&g_done);
                 // acc += M V over the half's 128 rows of V (A from tensor memory)
+                if (ch == 0) wait_bar(&ld_v, 0, a.status);
                 wait_bar(&m_full, ch & 1, a.status);
                 fence_after_sync();
                 for (int kk = 0; kk < kRows / 16; ++kk) {
@@ -355,7 +358,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                           int from_start) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t ld_full, x_ready, done;
+    __shared__ uint64_t ld_full, ld_b, x_ready, done;
     __shared__ uint32_t tslot;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / sh.heads_per_group;
@@ -363,6 +366,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     if (warp == 0) tmem_alloc(&tslot, 64);
     if (tid == 0) {
         mbar_init(&ld_full, 1);
+        mbar_init(&ld_b, 1);
         mbar_init(&done, 1);
         mbar_init(&x_ready, kCudaWarps);
         mbar_fence_init();
@@ -374,12 +378,14 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     uint8_t *sB = smem + cs::kOffB, *sX = smem + cs::kOffX, *sXlo = smem + cs::kOffXlo;
     if (warp == kCudaWarps) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(&ld_full, (uint32_t)(3 * nq) * 16384u);
-            for (int q = 0; q < nq; ++q) {
-                tma_load_4d(sX + q * 16384, &mX, &ld_full, 0, h, t0 + q * kRows, b);
+            // x (weighted by the CUDA-core warps first) on one barrier, B (for the product) on another
+            mbar_arrive_expect_tx(&ld_full, (uint32_t)nq * 16384u);
+            for (int q = 0; q < nq; ++q) tma_load_4d(sX + q * 16384, &mX, &ld_full, 0, h, t0 + q * kRows, b);
+            mbar_arrive_expect_tx(&ld_b, (uint32_t)(2 * nq) * 16384u);
+            for (int q = 0; q < nq; ++q)
                 for (int k = 0; k < 2; ++k)
-                    tma_load_4d(sB + k * 32768 + q * 16384, &mB, &ld_full, k * 64, g, t0 + q * kRows, b);
-            }
+                    tma_load_4d(sB + k * 32768 + q * 16384, &mB, &ld_b, k * 64, g, t0 + q * kRows, b);
+            wait_bar(&ld_b, 0, status);
             wait_bar(&x_ready, 0, status);
             fence_after_sync();
             const uint32_t id = idesc_bf16_f32(kRows, 64, 1, 1);  // B^T (MN-major) x weighted rows (MN-major)
@@ -393,12 +399,14 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         }
         __syncwarp();
     } else {
-        // weight each token row in place (high part) and into the low part
-        wait_bar(&ld_full, 0, status);
+        // weight each token row in place (high part) and into the low part; the weight's prefix sums are
+        // loaded while x is on its way
         const float *sc = s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
         const int i = tid;  // token row of the chunk
+        const float si = (i < len) ? sc[i] : 0.f, send = sc[sh.Q - 1];
+        wait_bar(&ld_full, 0, status);
         if (i < sh.Q) {
-            const float w = (i < len) ? ex2((from_start ? sc[i] : sc[sh.Q - 1] - sc[i]) * kLog2e) : 0.f;
+            const float w = (i < len) ? ex2((from_start ? si : send - si) * kLog2e) : 0.f;
             uint8_t *row = sX + (i >> 7) * 16384, *rowlo = sXlo + (i >> 7) * 16384;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
