@@ -52,6 +52,10 @@ namespace {
 // ---------------------------------------------------------------------------
 // Workspace of one backward call (all offsets 256-byte aligned).
 // ---------------------------------------------------------------------------
+// The dD dot products over a sequence run in this many token slices (more blocks in flight), each with
+// its own fp64 partial; the parameter sum adds them in a fixed order.
+constexpr int kDdSlices = 4;
+
 struct BwdWorkspace {
     size_t status_off;  // int status word of the tensor-core scans' bounded waits (cleared per call)
     size_t s_off;     // float s[batch][H][nc][Q]
@@ -62,7 +66,7 @@ struct BwdWorkspace {
     size_t dch_off;   // float dC^(h)[batch][T][H][N]
     size_t dsig_off;  // float dsigma[batch][H][T]
     size_t pa_off;    // double dA partial[batch][H]
-    size_t pd_off;    // double dD partial[batch][H]
+    size_t pd_off;    // double dD partial[kDdSlices][batch][H] (one per quarter of the tokens)
     size_t total;
 };
 
@@ -91,7 +95,7 @@ BwdWorkspace bwd_layout(const Shape &s) {
     w.pa_off = off;
     off = align256(off + sizeof(double) * bh);
     w.pd_off = off;
-    off = align256(off + sizeof(double) * bh);
+    off = align256(off + sizeof(double) * kDdSlices * bh);
     w.total = off;
     return w;
 }
@@ -623,9 +627,10 @@ __global__ void __launch_bounds__(256) group_reduce_vec_kernel(const float *__re
 // Per (head, batch): the suffix sums of dsigma over the whole sequence (fp64),
 // plus <dfinal, final> at the last token, give d(dt_u A_h); write
 // ddt = A_h d(dt A), and the batch row's shares of dA = sum dt d(dt A) and
-// dD = sum <dy, x> (fp64).  grid (H, batch), 256 threads: each thread owns a
-// contiguous run of tokens, a block scan of the run totals gives each run the
-// sum of the runs after it.
+// dD = sum <dy, x> (fp64).  grid (H, batch, kDdSlices), 256 threads: slice 0
+// runs the suffix sums (each thread owns a contiguous run of tokens, a block
+// scan of the run totals gives each run the sum of the runs after it); every
+// slice sums dD over its quarter of the tokens.
 // ---------------------------------------------------------------------------
 constexpr int kDtThreads = 256;
 
@@ -652,27 +657,30 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
                                                              Shape sh, int vec) {
     __shared__ double red[kDtThreads];
     __shared__ double suf[kDtThreads];
-    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, z = blockIdx.z;
     const size_t bh = (size_t)b * sh.H + h;
     const size_t PN = (size_t)sh.P * sh.N;
-    double fd = 0.0;
-    if (dfin)
-        for (size_t e = tid; e < PN; e += kDtThreads) fd += (double)dfin[bh * PN + e] * (double)fin[bh * PN + e];
-    const double fdot = block_sum(fd, red);
+    // the tokens of this block's dD slice
+    const int tq = (sh.T + kDdSlices - 1) / kDdSlices, tlo = min(sh.T, z * tq), thi = min(sh.T, tlo + tq);
+    if (z == 0) {
+        double fd = 0.0;
+        if (dfin)
+            for (size_t e = tid; e < PN; e += kDtThreads) fd += (double)dfin[bh * PN + e] * (double)fin[bh * PN + e];
+        const double fdot = block_sum(fd, red);
 
-    const float *ds = dsig + bh * sh.T;
-    const int run = (sh.T + kDtThreads - 1) / kDtThreads;
-    const int t0 = min(sh.T, tid * run), t1 = min(sh.T, t0 + run);
-    double part = 0.0;
-    for (int t = t0; t < t1; ++t) part += (double)ds[t];
-    suf[tid] = part;
-    __syncthreads();
-    // inclusive suffix scan of the run totals
-    for (int o = 1; o < kDtThreads; o <<= 1) {
-        const double v = tid + o < kDtThreads ? suf[tid + o] : 0.0;
+        const float *ds = dsig + bh * sh.T;
+        const int run = (sh.T + kDtThreads - 1) / kDtThreads;
+        const int t0 = min(sh.T, tid * run), t1 = min(sh.T, t0 + run);
+        double part = 0.0;
+        for (int t = t0; t < t1; ++t) part += (double)ds[t];
+        suf[tid] = part;
         __syncthreads();
-        suf[tid] += v;
-        __syncthreads();
+        // inclusive suffix scan of the run totals
+        for (int o = 1; o < kDtThreads; o <<= 1) {
+            const double v = tid + o < kDtThreads ? suf[tid + o] : 0.0;
+            __syncthreads();
+            suf[tid] += v;
+            __syncthreads();
     }
     double acc = (tid + 1 < kDtThreads ? suf[tid + 1] : 0.0) + fdot;
     const double Ah = (double)A[h];
@@ -684,6 +692,8 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
         da += (double)dt[it] * acc;
     }
     const double dA_part = block_sum(da, red);
+    if (tid == 0) pa[bh] = dA_part;
+    }
 
     // dD's share: sum over the row's tokens of <dy_t, x_t> for this head.  With 16-byte rows, eight
     // elements per load (their products summed in fp32, then in fp64), four loads in flight per thread.
@@ -691,9 +701,9 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
     constexpr int VE = 16 / (int)sizeof(T);
     if (vec) {
         const int cpt = sh.P / VE;  // 16-byte pieces per token row
-        const long long total = (long long)sh.T * cpt;
+        const long long total = (long long)thi * cpt;
 #pragma unroll 4
-        for (long long idx = tid; idx < total; idx += kDtThreads) {
+        for (long long idx = (long long)tlo * cpt + tid; idx < total; idx += kDtThreads) {
             const int t = (int)(idx / cpt), q = (int)(idx - (long long)t * cpt);
             const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + (size_t)q * VE;
             float fy[VE], fx[VE];
@@ -705,21 +715,18 @@ __global__ void __launch_bounds__(kDtThreads) dt_scan_kernel(const float *__rest
             dd += (double)f;
         }
     } else {
-        const long long TP = (long long)sh.T * sh.P;
-        for (long long idx = tid; idx < TP; idx += kDtThreads) {
+        const long long TP = (long long)thi * sh.P;
+        for (long long idx = (long long)tlo * sh.P + tid; idx < TP; idx += kDtThreads) {
             const int t = (int)(idx / sh.P), p = (int)(idx - (long long)t * sh.P);
             const size_t off = (((size_t)b * sh.T + t) * sh.H + h) * sh.P + p;
             dd += (double)to_f32(dy[off]) * (double)to_f32(x[off]);
         }
     }
     const double dD_part = block_sum(dd, red);
-    if (tid == 0) {
-        pa[bh] = dA_part;
-        pd[bh] = dD_part;
-    }
+    if (tid == 0) pd[(size_t)z * sh.batch * sh.H + bh] = dD_part;
 }
 
-// dA[h] = sum_b pa[b][h], dD[h] = sum_b pd[b][h], in batch order.
+// dA[h] = sum_b pa[b][h], dD[h] = sum_b sum_z pd[z][b][h], in batch order (and slice order).
 __global__ void __launch_bounds__(256) param_reduce_kernel(const double *__restrict__ pa,
                                                            const double *__restrict__ pd, float *__restrict__ dA,
                                                            float *__restrict__ dD, int batch, int H) {
@@ -728,7 +735,7 @@ __global__ void __launch_bounds__(256) param_reduce_kernel(const double *__restr
     double sa = 0.0, sd = 0.0;
     for (int b = 0; b < batch; ++b) {
         sa += pa[(size_t)b * H + h];
-        sd += pd[(size_t)b * H + h];
+        for (int z = 0; z < kDdSlices; ++z) sd += pd[((size_t)z * batch + b) * H + h];
     }
     dA[h] = (float)sa;
     dD[h] = (float)sd;
@@ -853,7 +860,7 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     else
         group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
-    dt_scan_kernel<T><<<dim3(sh.H, sh.batch), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh,
+    dt_scan_kernel<T><<<dim3(sh.H, sh.batch, kDdSlices), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh,
                                                                     vec);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
     param_reduce_kernel<<<(sh.H + 255) / 256, 256, 0, st>>>(pa, pd, dA, dD, sh.batch, sh.H);
