@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Chunk states on the tensor cores: for one (chunk, head) per CTA,
+// Chunk states on the tensor cores: for every (chunk, head),
 //
 //   S[p][n] = sum_{i in chunk} w_i x_i[p] B_i[n],   w_i = exp(s_end - s_i), or exp(s_i) (from_start)
 //
@@ -346,105 +346,157 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
 // B [batch][T][G][128] bf16; S [batch][nc][H][64][128] fp32.
 // ---------------------------------------------------------------------------
 namespace cs {
-constexpr uint32_t kOffB = 0;        // [2 n atoms][256 tokens] (32 KiB apart)
-constexpr uint32_t kOffX = 65536;    // [256 tokens][64 p], the weighted rows' high part after scaling
-constexpr uint32_t kOffXlo = 98304;  // their low part
-constexpr uint32_t kSmemBytes = 131072 + 1024;
+constexpr uint32_t kOffB = 0;         // [2 n atoms][256 tokens] (32 KiB apart)
+constexpr uint32_t kOffX = 65536;     // two buffers of [256 tokens][64 p] (32 KiB apart): the weighted rows' high part
+constexpr uint32_t kOffXlo = 131072;  // two buffers of their low part
+constexpr uint32_t kSmemBytes = 196608 + 1024;
 }  // namespace cs
 
+// Persistent: each CTA takes a contiguous run of `per_cta` (chunk, head) tiles, head fastest, so that B
+// (shared by a group's heads) is loaded once per (batch, chunk, group) it meets.  x and its low part are
+// double-buffered in shared memory and the accumulator in tensor memory (two 64-column halves), so that
+// the CUDA-core warps drain tile k-1 while the tensor cores run tile k and the next x is on its way.
 __global__ void __launch_bounds__(bt::kThreads, 1)
     chunk_state_tc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
                           const float *__restrict__ s, float *__restrict__ S, int *status, Shape sh,
-                          int from_start) {
+                          int from_start, int per_cta) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t ld_full, ld_b, x_ready, done;
+    __shared__ uint64_t x_full[2], x_ready[2], done[2], acc_free[2], b_full;
     __shared__ uint32_t tslot;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / sh.heads_per_group;
-    const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), nq = sh.Q / kRows;
-    if (warp == 0) tmem_alloc(&tslot, 64);
+    const int tiles = sh.nc * sh.H * sh.batch;
+    const int t_beg = blockIdx.x * per_cta, t_end = min(tiles, t_beg + per_cta);
+    if (t_beg >= t_end) return;  // whole CTA
+    const int nq = sh.Q / kRows;
+    // tile t: head fastest, then chunk, then batch row
+    auto tile = [&](int t, int &b, int &c, int &h) {
+        h = t % sh.H;
+        c = (t / sh.H) % sh.nc;
+        b = t / (sh.H * sh.nc);
+    };
+    if (warp == 0) tmem_alloc(&tslot, 128);
     if (tid == 0) {
-        mbar_init(&ld_full, 1);
-        mbar_init(&ld_b, 1);
-        mbar_init(&done, 1);
-        mbar_init(&x_ready, kCudaWarps);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&x_full[q], 1);
+            mbar_init(&done[q], 1);
+            mbar_init(&x_ready[q], kCudaWarps);
+            mbar_init(&acc_free[q], kCudaWarps);
+        }
+        mbar_init(&b_full, 1);
         mbar_fence_init();
     }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
-    uint8_t *sB = smem + cs::kOffB, *sX = smem + cs::kOffX, *sXlo = smem + cs::kOffXlo;
+    uint8_t *sB = smem + cs::kOffB;
     if (warp == kCudaWarps) {
         if (lane == 0) {
-            // x (weighted by the CUDA-core warps first) on one barrier, B (for the product) on another
-            mbar_arrive_expect_tx(&ld_full, (uint32_t)nq * 16384u);
-            for (int q = 0; q < nq; ++q) tma_load_4d(sX + q * 16384, &mX, &ld_full, 0, h, t0 + q * kRows, b);
-            mbar_arrive_expect_tx(&ld_b, (uint32_t)(2 * nq) * 16384u);
-            for (int q = 0; q < nq; ++q)
-                for (int k = 0; k < 2; ++k)
-                    tma_load_4d(sB + k * 32768 + q * 16384, &mB, &ld_b, k * 64, g, t0 + q * kRows, b);
-            wait_bar(&ld_b, 0, status);
-            wait_bar(&x_ready, 0, status);
-            fence_after_sync();
+            int cur_b = -1, cur_c = -1, cur_g = -1;
+            uint32_t bcnt = 0;
             const uint32_t id = idesc_bf16_f32(kRows, 64, 1, 1);  // B^T (MN-major) x weighted rows (MN-major)
-            for (int part = 0; part < 2; ++part)
-                for (int kk = 0; kk < sh.Q / 16; ++kk)
-                    mma_ss(tmem, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
-                           smem_desc_sw128(smem_u32(part ? sXlo : sX) + kk * 2048, 16, 1024), id,
-                           part > 0 || kk > 0);
-            mma_commit(&done);
-            wait_bar(&done, 0, status);
+            for (int t = t_beg, k = 0; t < t_end; ++t, ++k) {
+                int b, c, h;
+                tile(t, b, c, h);
+                const int g = h / sh.heads_per_group, buf = k & 1, t0 = c * sh.Q;
+                uint8_t *sX = smem + cs::kOffX + buf * 32768, *sXlo = smem + cs::kOffXlo + buf * 32768;
+                // this x buffer was last read by the product of tile k-2
+                if (k >= 2) wait_bar(&done[buf], ((k - 2) >> 1) & 1, status);
+                mbar_arrive_expect_tx(&x_full[buf], (uint32_t)nq * 16384u);
+                for (int q = 0; q < nq; ++q) tma_load_4d(sX + q * 16384, &mX, &x_full[buf], 0, h, t0 + q * kRows, b);
+                if (b != cur_b || c != cur_c || g != cur_g) {
+                    // B was last read by the product of tile k-1
+                    if (k >= 1) wait_bar(&done[(k - 1) & 1], ((k - 1) >> 1) & 1, status);
+                    mbar_arrive_expect_tx(&b_full, (uint32_t)(2 * nq) * 16384u);
+                    for (int q = 0; q < nq; ++q)
+                        for (int kk = 0; kk < 2; ++kk)
+                            tma_load_4d(sB + kk * 32768 + q * 16384, &mB, &b_full, kk * 64, g, t0 + q * kRows, b);
+                    wait_bar(&b_full, bcnt++ & 1, status);
+                    cur_b = b;
+                    cur_c = c;
+                    cur_g = g;
+                }
+                wait_bar(&x_ready[buf], (k >> 1) & 1, status);
+                // this accumulator was last drained for tile k-2
+                if (k >= 2) wait_bar(&acc_free[buf], ((k - 2) >> 1) & 1, status);
+                fence_after_sync();
+                for (int part = 0; part < 2; ++part)
+                    for (int kk = 0; kk < sh.Q / 16; ++kk)
+                        mma_ss(tmem + buf * 64, smem_desc_sw128(smem_u32(sB) + kk * 2048, 32768, 1024),
+                               smem_desc_sw128(smem_u32(part ? sXlo : sX) + kk * 2048, 16, 1024), id,
+                               part > 0 || kk > 0);
+                mma_commit(&done[buf]);
+            }
+            // nothing this CTA issued is in flight when it leaves
+            const int n = t_end - t_beg;
+            for (int k = max(0, n - 2); k < n; ++k) wait_bar(&done[k & 1], (k >> 1) & 1, status);
         }
         __syncwarp();
     } else {
-        // weight each token row in place (high part) and into the low part; the weight's prefix sums are
-        // loaded while x is on its way
-        const float *sc = s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
-        const int i = tid;  // token row of the chunk
-        const float si = (i < len) ? sc[i] : 0.f, send = sc[sh.Q - 1];
-        wait_bar(&ld_full, 0, status);
-        if (i < sh.Q) {
-            const float w = (i < len) ? ex2((from_start ? si : send - si) * kLog2e) : 0.f;
-            uint8_t *row = sX + (i >> 7) * 16384, *rowlo = sXlo + (i >> 7) * 16384;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = swz(i & 127, k);
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + off);
-                const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a0 = bf16lo(vv[e]) * w, a1 = bf16hi(vv[e]) * w;
-                    hi[e] = pack_bf16x2(a0, a1);
-                    lo[e] = pack_lo(a0, a1, hi[e]);
-                }
-                *reinterpret_cast<uint4 *>(row + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(rowlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-        }
-        fence_view_async_shared();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&x_ready);
-        // S^T in tensor memory: lane n, column p; warpgroup `half` writes p in [32 half, 32 half + 32)
-        wait_bar(&done, 0, status);
-        fence_after_sync();
-        const int wq = warp & 3, half = warp >> 2, n = wq * 32 + lane;
+        const int wq = warp & 3, half = warp >> 2;
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        float *Sp = S + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)(64 * 128);
+        // S^T of tile k in tensor memory: lane n, column p; warpgroup `half` writes p in [32 half, 32 half + 32)
+        auto drain = [&](int t, int k) {
+            int b, c, h;
+            tile(t, b, c, h);
+            const int buf = k & 1, n = wq * 32 + lane;
+            wait_bar(&done[buf], (k >> 1) & 1, status);
+            fence_after_sync();
+            float *Sp = S + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)(64 * 128);
 #pragma unroll
-        for (int q0 = 0; q0 < 32; q0 += 16) {
-            uint32_t u[16];
-            tmem_ld16(tmem + half * 32 + q0 + lane_base, u);
-            tmem_wait_ld();
+            for (int q0 = 0; q0 < 32; q0 += 16) {
+                uint32_t u[16];
+                tmem_ld16(tmem + buf * 64 + half * 32 + q0 + lane_base, u);
+                tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) Sp[(size_t)(half * 32 + q0 + e) * 128 + n] = __uint_as_float(u[e]);
+                for (int e = 0; e < 16; ++e) Sp[(size_t)(half * 32 + q0 + e) * 128 + n] = __uint_as_float(u[e]);
+            }
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_free[buf]);
+        };
+        for (int t = t_beg, k = 0; t < t_end; ++t, ++k) {
+            int b, c, h;
+            tile(t, b, c, h);
+            const int buf = k & 1, len = min(sh.Q, sh.T - c * sh.Q);
+            uint8_t *sX = smem + cs::kOffX + buf * 32768, *sXlo = smem + cs::kOffXlo + buf * 32768;
+            // weight each token row in place (high part) and into the low part; the weight's prefix sums
+            // are loaded while x is on its way
+            const float *sc = s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+            const int i = tid;  // token row of the chunk
+            const float si = (i < len) ? sc[i] : 0.f, send = sc[sh.Q - 1];
+            wait_bar(&x_full[buf], (k >> 1) & 1, status);
+            if (i < sh.Q) {
+                const float w = (i < len) ? ex2((from_start ? si : send - si) * kLog2e) : 0.f;
+                uint8_t *row = sX + (i >> 7) * 16384, *rowlo = sXlo + (i >> 7) * 16384;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = swz(i & 127, kk);
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + off);
+                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a0 = bf16lo(vv[e]) * w, a1 = bf16hi(vv[e]) * w;
+                        hi[e] = pack_bf16x2(a0, a1);
+                        lo[e] = pack_lo(a0, a1, hi[e]);
+                    }
+                    *reinterpret_cast<uint4 *>(row + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(rowlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+            }
+            fence_view_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x_ready[buf]);
+            // the previous tile's state, while this one's product runs
+            if (k >= 1) drain(t - 1, k - 1);
         }
+        drain(t_end - 1, t_end - 1 - t_beg);
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ---------------------------------------------------------------------------
@@ -527,8 +579,14 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *B, const float *s, 
     cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cs::kSmemBytes);
     if (e != cudaSuccess) return e;
-    chunk_state_tc_kernel<<<dim3(sh.nc, sh.H, sh.batch), kThreads, cs::kSmemBytes, st>>>(mX, mB, s, S, status, sh,
-                                                                                          from_start ? 1 : 0);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || sms <= 0)
+        sms = 148;
+    const int tiles = sh.nc * sh.H * sh.batch;
+    const int grid = min(tiles, sms), per_cta = (tiles + grid - 1) / grid;
+    chunk_state_tc_kernel<<<grid, kThreads, cs::kSmemBytes, st>>>(mX, mB, s, S, status, sh, from_start ? 1 : 0,
+                                                                   per_cta);
     return cudaGetLastError();
 }
 
