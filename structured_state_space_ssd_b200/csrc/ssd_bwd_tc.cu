@@ -1,6 +1,6 @@
 // ssd_bwd_tc.cu -- the backward's masked chunk scans on the tensor cores (tcgen05, TMEM, TMA).
 //
-// The same operation as masked_scan_kernel in ssd_bwd.cu, for one (chunk, 128-row block, head) per CTA:
+// The same operation as masked_scan_kernel in ssd_bwd.cu, per (chunk, 128-row block, head) tile:
 //
 //   out_r[w] = e_r * sum_k R_r[k] St[k][w]
 //            + sum_{i in chunk, i >= r (kAnti) or i <= r} exp(+-(s_i - s_r)) (R_r . K_i) V_i[w]
@@ -22,8 +22,9 @@
 // rounding to bf16 left out), so those products are as accurate as fp32 accumulation allows.
 // Shapes: KD, W in {64, 128}; Q in {128, 256}; R, K, V bf16 rows of [batch][T][heads or groups][dim].
 // Tensor memory (512 columns): G at 0, the mask at 128 (its low part at 192), acc at 256, acc2 at 384.
-// One CTA per SM (it takes all of tensor memory); 9 warps: 0-7 CUDA-core work (two warpgroups over the
-// 128 lanes, each half of the columns), 8 TMA and MMA issue.  Every wait is bounded (about 2 s of
+// One persistent CTA per SM (it takes all of tensor memory) taking every grid-th tile; while its warps
+// drain one tile, the next tile's loads and G product run.  9 warps: 0-7 CUDA-core work (two warpgroups
+// over the 128 lanes, each half of the columns), 8 TMA and MMA issue.  Every wait is bounded (about 2 s of
 // %globaltimer, 1 ms once any CTA has given up): on expiry the CTA records SSD_ERR_TIMEOUT in the status
 // word, and the issuer still waits (bounded) for its own MMAs before tensor memory is freed.
 #include "ssd_common.cuh"
@@ -112,23 +113,29 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                           int v_head) {
     static_assert(!kSplit || KD == 64, "the low part of the state tile has room for KD = 64");
     static_assert(KD == 64 || W == 64, "the fp32 state is staged in the unused second atom of K or V");
-    // the fp32 state [KD][W] (32 KB), copied in asynchronously at the start: the K region's second atom
-    // (KD = 64) or the V region's (W = 64), which this shape leaves unused
+    // the fp32 state [KD][W] (32 KB), copied in asynchronously: the K region's second atom (KD = 64) or the
+    // V region's (W = 64), which this shape leaves unused
     constexpr uint32_t kOffRaw = (KD == 64) ? kOffK + 32768 : kOffV + 32768;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t ld_full, ld_v, g_done, st_full, m_full, mx_done, fin_done;
+    __shared__ uint64_t ld_full, ld_v, g_done, st_full, m_full, mx_done, fin_done, acc_free;
     __shared__ uint32_t tslot;
     const Shape &sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int blocks = sh.Q / kRows;
-    const int c = blockIdx.x / blocks, rb = blockIdx.x - c * blocks;
-    const int h = blockIdx.y, b = blockIdx.z, g = h / sh.heads_per_group;
-    const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), r0 = rb * kRows;
-    if (r0 >= len) return;  // whole CTA: a block past a ragged chunk's end
-    // the columns on the mask's side of the block, [r0, Q) or [0, r0 + 128), in halves of 128
-    const int cbeg = kAnti ? r0 : 0;
-    const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;  // 1 or 2
+    // this CTA's tiles (chunk, 128-row block, head): every gridDim.x-th, so that each CTA gets the same mix
+    // of one- and two-half blocks
+    const int tiles = sh.batch * sh.nc * blocks * sh.H;
+    const int t_beg = blockIdx.x, t_end = tiles, t_step = gridDim.x;
+    if (t_beg >= t_end) return;  // whole CTA
+    auto tile = [&](int t, int &b, int &c, int &rb, int &h) {
+        h = t % sh.H;
+        int r = t / sh.H;
+        rb = r % blocks;
+        r /= blocks;
+        c = r % sh.nc;
+        b = r / sh.nc;
+    };
 
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     if (tid == 0) {
@@ -139,6 +146,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         mbar_init(&fin_done, 1);
         mbar_init(&st_full, kCudaWarps);
         mbar_init(&m_full, kCudaWarps);
+        mbar_init(&acc_free, kCudaWarps);
         mbar_fence_init();
     }
     fence_before_sync();
@@ -151,59 +159,82 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
 
     if (warp == kCudaWarps) {
         // ---------------- TMA and MMA issue (lane 0) ----------------
+        // Every barrier phase is counted on both sides; one tile's last MMA (fin_done) completes before the
+        // next tile's loads, and its G and masked products may run while the warps drain the tile before.
         if (lane == 0) {
-            const int hr = r_head ? h : g, hk = k_head ? h : g, hv = v_head ? h : g;
-            // R and K (for G) on one barrier, V (for the masked product, later) on another
-            mbar_arrive_expect_tx(&ld_full, (uint32_t)(KD / 64) * (1u + (uint32_t)nh) * 16384u);
-            for (int k = 0; k < KD / 64; ++k) {
-                tma_load_4d(sR + k * 16384, &mR, &ld_full, k * 64, hr, t0 + r0, b);
-                for (int q = 0; q < nh; ++q)
-                    tma_load_4d(sK + k * 32768 + q * 16384, &mK, &ld_full, k * 64, hk, t0 + cbeg + q * kRows, b);
-            }
-            mbar_arrive_expect_tx(&ld_v, (uint32_t)(W / 64) * (uint32_t)nh * 16384u);
-            for (int k = 0; k < W / 64; ++k)
-                for (int q = 0; q < nh; ++q)
-                    tma_load_4d(sV + k * 32768 + q * 16384, &mV, &ld_v, k * 64, hv, t0 + cbeg + q * kRows, b);
-            wait_bar(&ld_full, 0, a.status);
-            fence_after_sync();
+            uint32_t n_ld = 0, n_v = 0, n_m = 0, n_st = 0, n_fin = 0, n_free = 0;
+            long long rk_key = -1, v_key = -1;  // the group-shared operands now in shared memory
             const uint32_t idG = idesc_bf16_f32(kRows, kRows, 0, 0);  // R (K-major) x K rows (K-major)
             const uint32_t idW = idesc_bf16_f32(kRows, W, 0, 1);      // x V [i][w] or the state tile [k][w]
-            for (int ch = 0; ch < nh; ++ch) {
-                // G of this half into columns 0..127, once the warps have read the previous half's out
-                if (ch > 0) wait_bar(&m_full, (ch - 1) & 1, a.status);
+            for (int t = t_beg; t < t_end; t += t_step) {
+                int b, c, rb, h;
+                tile(t, b, c, rb, h);
+                const int g = h / sh.heads_per_group;
+                const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), r0 = rb * kRows;
+                if (r0 >= len) continue;  // a block past a ragged chunk's end
+                const int cbeg = kAnti ? r0 : 0;
+                const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;  // 1 or 2
+                const int hr = r_head ? h : g, hk = k_head ? h : g, hv = v_head ? h : g;
+                const long long gkey = (((long long)b * sh.nc + c) * blocks + rb) * sh.G + g;
+                // R and K (for G), kept while they are the group's and the block is the same
+                const bool new_rk = r_head || k_head || gkey != rk_key;
+                if (new_rk) {
+                    mbar_arrive_expect_tx(&ld_full, (uint32_t)(KD / 64) * (1u + (uint32_t)nh) * 16384u);
+                    for (int k = 0; k < KD / 64; ++k) {
+                        tma_load_4d(sR + k * 16384, &mR, &ld_full, k * 64, hr, t0 + r0, b);
+                        for (int q = 0; q < nh; ++q)
+                            tma_load_4d(sK + k * 32768 + q * 16384, &mK, &ld_full, k * 64, hk, t0 + cbeg + q * kRows,
+                                        b);
+                    }
+                    rk_key = (r_head || k_head) ? -1 : gkey;
+                }
+                const bool new_v = v_head || gkey != v_key;
+                if (new_v) {
+                    mbar_arrive_expect_tx(&ld_v, (uint32_t)(W / 64) * (uint32_t)nh * 16384u);
+                    for (int k = 0; k < W / 64; ++k)
+                        for (int q = 0; q < nh; ++q)
+                            tma_load_4d(sV + k * 32768 + q * 16384, &mV, &ld_v, k * 64, hv, t0 + cbeg + q * kRows, b);
+                    v_key = v_head ? -1 : gkey;
+                }
+                if (new_rk) wait_bar(&ld_full, n_ld++ & 1, a.status);
+                fence_after_sync();
+                for (int ch = 0; ch < nh; ++ch) {
+                    // G of this half into columns 0..127 (the warps have read the previous half's: m_full)
+                    for (int kk = 0; kk < KD / 16; ++kk) {
+                        const int atom = kk >> 2, kin = kk & 3;
+                        mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024),
+                               smem_desc_sw128(smem_u32(sK) + atom * 32768 + ch * 16384 + kin * 32, 16, 1024), idG,
+                               kk > 0);
+                    }
+                    mma_commit(&g_done);
+                    if (ch == 0 && new_v) wait_bar(&ld_v, n_v++ & 1, a.status);
+                    // acc += M V over the half's 128 rows of V (A from tensor memory), once the mask is in and
+                    // (first half) the previous tile's drain has read both accumulators
+                    wait_bar(&m_full, n_m++ & 1, a.status);
+                    if (ch == 0 && n_fin > 0) wait_bar(&acc_free, n_free++ & 1, a.status);
+                    fence_after_sync();
+                    for (int kk = 0; kk < kRows / 16; ++kk) {
+                        const uint64_t vd = smem_desc_sw128(smem_u32(sV) + ch * 16384 + kk * 2048, 32768, 1024);
+                        mma_ts(tmem + kColAcc, tmem + kColMhi + kk * 8, vd, idW, ch > 0 || kk > 0);
+                        if (kSplit) mma_ts(tmem + kColAcc, tmem + kColMlo + kk * 8, vd, idW, 1);
+                    }
+                    mma_commit(&mx_done);
+                }
+                // acc2 = R St^T
+                wait_bar(&st_full, n_st++ & 1, a.status);
                 fence_after_sync();
                 for (int kk = 0; kk < KD / 16; ++kk) {
                     const int atom = kk >> 2, kin = kk & 3;
-                    mma_ss(tmem + kColG, smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024),
-                           smem_desc_sw128(smem_u32(sK) + atom * 32768 + ch * 16384 + kin * 32, 16, 1024), idG,
-                           kk > 0);
+                    const uint64_t rd = smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024);
+                    mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sSt) + kk * 2048, 16384, 1024), idW, kk > 0);
+                    if (kSplit)
+                        mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sStLo) + kk * 2048, 8192, 1024), idW, 1);
                 }
-                mma_commit(&g_done);
-                // acc += M V over the half's 128 rows of V (A from tensor memory)
-                if (ch == 0) wait_bar(&ld_v, 0, a.status);
-                wait_bar(&m_full, ch & 1, a.status);
-                fence_after_sync();
-                for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint64_t vd =
-                        smem_desc_sw128(smem_u32(sV) + ch * 16384 + kk * 2048, 32768, 1024);
-                    mma_ts(tmem + kColAcc, tmem + kColMhi + kk * 8, vd, idW, ch > 0 || kk > 0);
-                    if (kSplit) mma_ts(tmem + kColAcc, tmem + kColMlo + kk * 8, vd, idW, 1);
-                }
-                mma_commit(&mx_done);
+                mma_commit(&fin_done);
+                // the tile's products are done before its R, K or V are replaced (and nothing is in flight
+                // when the CTA leaves)
+                wait_bar(&fin_done, n_fin++ & 1, a.status);
             }
-            // acc2 = R St^T
-            wait_bar(&st_full, 0, a.status);
-            fence_after_sync();
-            for (int kk = 0; kk < KD / 16; ++kk) {
-                const int atom = kk >> 2, kin = kk & 3;
-                const uint64_t rd = smem_desc_sw128(smem_u32(sR) + atom * 16384 + kin * 32, 16, 1024);
-                mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sSt) + kk * 2048, 16384, 1024), idW, kk > 0);
-                if (kSplit)
-                    mma_ss(tmem + kColAcc2, rd, smem_desc_sw128(smem_u32(sStLo) + kk * 2048, 8192, 1024), idW, 1);
-            }
-            mma_commit(&fin_done);
-            // nothing this CTA issued is in flight when it leaves
-            wait_bar(&fin_done, 0, a.status);
         }
         __syncwarp();
     } else {
@@ -211,120 +242,140 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         const int wq = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
         const int lrow = wq * 32 + lane;            // this thread's row of the block
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-        const int j = r0 + lrow;                    // row within the chunk
-        // the fp32 state on its way into shared memory (async copies: no barrier waits for them, so its
-        // DRAM latency passes while the masks are built)
-        const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
         float *sRaw = reinterpret_cast<float *>(smem + kOffRaw);
-        for (int i = tid; i < KD * W / 4; i += 32 * kCudaWarps) cp_async16(sRaw + 4 * i, Sp + 4 * i);
-        const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
-        for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) sq[i] = sch[i];
-        named_bar_sync(1, 32 * kCudaWarps);  // the prefix sums are in
-        const float sj = (j < len) ? sq[j] : 0.f;
+        uint32_t n_g = 0, n_mx = 0, n_fin = 0;
+        for (int t = t_beg; t < t_end; t += t_step) {
+            int b, c, rb, h;
+            tile(t, b, c, rb, h);
+            const int g = h / sh.heads_per_group;
+            const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), r0 = rb * kRows;
+            if (r0 >= len) continue;
+            const int cbeg = kAnti ? r0 : 0;
+            const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;
+            const int j = r0 + lrow;  // row within the chunk
+            // every thread is done with the previous tile's prefix sums and staged state
+            named_bar_sync(1, 32 * kCudaWarps);
+            // the fp32 state on its way into shared memory (async copies: no barrier waits for them, so
+            // its DRAM latency passes while the masks are built)
+            const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
+            for (int i = tid; i < KD * W / 4; i += 32 * kCudaWarps) cp_async16(sRaw + 4 * i, Sp + 4 * i);
+            const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+            for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) sq[i] = sch[i];
+            named_bar_sync(1, 32 * kCudaWarps);  // the prefix sums are in
+            const float sj = (j < len) ? sq[j] : 0.f;
 
-        // the mask, one 128-column half at a time: this thread's row, its 64 of the half's columns
-        for (int ch = 0; ch < nh; ++ch) {
-            wait_bar(&g_done, ch & 1, a.status);
-            if (ch > 0) wait_bar(&mx_done, (ch - 1) & 1, a.status);  // the previous half's mask was used
-            fence_after_sync();
+            // the mask, one 128-column half at a time: this thread's row, its 64 of the half's columns
+            const uint32_t mx0 = n_mx;
+            for (int ch = 0; ch < nh; ++ch) {
+                wait_bar(&g_done, n_g++ & 1, a.status);
+                if (ch > 0) wait_bar(&mx_done, (mx0 + ch - 1) & 1, a.status);  // the previous half's mask was used
+                fence_after_sync();
 #pragma unroll 1
-            for (int q0 = half * 64; q0 < half * 64 + 64; q0 += 16) {
-                uint32_t gv[16];
-                tmem_ld16(tmem + kColG + q0 + lane_base, gv);
-                tmem_wait_ld();
-                uint32_t o[8], ol[8];
+                for (int q0 = half * 64; q0 < half * 64 + 64; q0 += 16) {
+                    uint32_t gv[16];
+                    tmem_ld16(tmem + kColG + q0 + lane_base, gv);
+                    tmem_wait_ld();
+                    uint32_t o[8], ol[8];
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float m[2];
+                    for (int e = 0; e < 16; e += 2) {
+                        float m[2];
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int i = cbeg + ch * kRows + q0 + e + k;  // column within the chunk
-                        const bool ok = j < len && i < len && (kAnti ? i >= j : i <= j);
-                        m[k] = ok ? __uint_as_float(gv[e + k]) * ex2((kAnti ? sq[i] - sj : sj - sq[i]) * kLog2e)
-                                  : 0.f;
+                        for (int k = 0; k < 2; ++k) {
+                            const int i = cbeg + ch * kRows + q0 + e + k;  // column within the chunk
+                            const bool ok = j < len && i < len && (kAnti ? i >= j : i <= j);
+                            m[k] = ok ? __uint_as_float(gv[e + k]) * ex2((kAnti ? sq[i] - sj : sj - sq[i]) * kLog2e)
+                                      : 0.f;
+                        }
+                        o[e / 2] = pack_bf16x2(m[0], m[1]);
+                        if (kSplit) ol[e / 2] = pack_lo(m[0], m[1], o[e / 2]);
                     }
-                    o[e / 2] = pack_bf16x2(m[0], m[1]);
-                    if (kSplit) ol[e / 2] = pack_lo(m[0], m[1], o[e / 2]);
+                    tmem_st8(tmem + kColMhi + q0 / 2 + lane_base, o);
+                    if (kSplit) tmem_st8(tmem + kColMlo + q0 / 2 + lane_base, ol);
                 }
-                tmem_st8(tmem + kColMhi + q0 / 2 + lane_base, o);
-                if (kSplit) tmem_st8(tmem + kColMlo + q0 / 2 + lane_base, ol);
+                tmem_wait_st();
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&m_full);
             }
-            tmem_wait_st();
+            n_mx = mx0 + nh;
+
+            // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows,
+            // from the staged fp32 state (the previous tile's products, acc2 among them, are done: its drain
+            // waited for them)
+            cp_async_wait_all();
+            named_bar_sync(1, 32 * kCudaWarps);  // every thread's copies are in
+            for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
+                const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
+                float v[8];
+                if (a.st_kw) {
+                    const float4 u0 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0 + 4);
+                    v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+                    v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = sRaw[(w0 + e) * KD + k];
+                }
+                const uint4 tt = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                *reinterpret_cast<uint4 *>(sSt + (w0 >> 6) * 16384 + swz(k, (w0 & 63) >> 3)) = tt;
+                if (kSplit) {
+                    const uint4 tl = make_uint4(pack_lo(v[0], v[1], tt.x), pack_lo(v[2], v[3], tt.y),
+                                                pack_lo(v[4], v[5], tt.z), pack_lo(v[6], v[7], tt.w));
+                    *reinterpret_cast<uint4 *>(sStLo + (w0 >> 6) * 8192 + swz(k, (w0 & 63) >> 3)) = tl;
+                }
+            }
+            fence_view_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st_full);
+
+            // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns
+            wait_bar(&fin_done, n_fin++ & 1, a.status);
+            fence_after_sync();
+            const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
+            const float Dh = a.D ? a.D[h] : 0.f;
+            const size_t tok = (size_t)b * sh.T + t0 + j;
+            const __nv_bfloat16 *vrow =
+                a.V + (tok * (a.v_head ? sh.H : sh.G) + (a.v_head ? h : g)) * (size_t)W;
+            for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
+                uint32_t u[16], u2[16];
+                tmem_ld16(tmem + kColAcc + w0 + lane_base, u);
+                tmem_ld16(tmem + kColAcc2 + w0 + lane_base, u2);
+                tmem_wait_ld();
+                if (j >= len) continue;
+                float r[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = fmaf(e_r, __uint_as_float(u2[e]), __uint_as_float(u[e]));
+                if (a.D) {
+                    const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + w0);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 vv = vp[q];
+                        const uint32_t ww[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            r[8 * q + 2 * e] = fmaf(Dh, bf16lo(ww[e]), r[8 * q + 2 * e]);
+                            r[8 * q + 2 * e + 1] = fmaf(Dh, bf16hi(ww[e]), r[8 * q + 2 * e + 1]);
+                        }
+                    }
+                }
+                if (kOutBf16) {
+                    uint4 *op =
+                        reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + (tok * sh.H + h) * W + w0);
+                    op[0] = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                                       pack_bf16x2(r[6], r[7]));
+                    op[1] = make_uint4(pack_bf16x2(r[8], r[9]), pack_bf16x2(r[10], r[11]), pack_bf16x2(r[12], r[13]),
+                                       pack_bf16x2(r[14], r[15]));
+                } else {
+                    float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + (tok * sh.H + h) * W + w0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) op[q] = make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                }
+            }
+            // both accumulators are read: the next tile's masked product may overwrite them
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&m_full);
-        }
-
-        // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows,
-        // from the staged fp32 state
-        cp_async_wait_all();
-        named_bar_sync(1, 32 * kCudaWarps);  // every thread's copies are in
-        for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
-            const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
-            float v[8];
-            if (a.st_kw) {
-                const float4 u0 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0);
-                const float4 u1 = *reinterpret_cast<const float4 *>(sRaw + k * W + w0 + 4);
-                v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
-                v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = sRaw[(w0 + e) * KD + k];
-            }
-            const uint4 t = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                       pack_bf16x2(v[6], v[7]));
-            *reinterpret_cast<uint4 *>(sSt + (w0 >> 6) * 16384 + swz(k, (w0 & 63) >> 3)) = t;
-            if (kSplit) {
-                const uint4 tl = make_uint4(pack_lo(v[0], v[1], t.x), pack_lo(v[2], v[3], t.y),
-                                            pack_lo(v[4], v[5], t.z), pack_lo(v[6], v[7], t.w));
-                *reinterpret_cast<uint4 *>(sStLo + (w0 >> 6) * 8192 + swz(k, (w0 & 63) >> 3)) = tl;
-            }
-        }
-        fence_view_async_shared();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_full);
-
-        // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns
-        wait_bar(&fin_done, 0, a.status);
-        fence_after_sync();
-        const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
-        const float Dh = a.D ? a.D[h] : 0.f;
-        const size_t tok = (size_t)b * sh.T + t0 + j;
-        const __nv_bfloat16 *vrow =
-            a.V + (tok * (a.v_head ? sh.H : sh.G) + (a.v_head ? h : g)) * (size_t)W;
-        for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
-            uint32_t u[16], u2[16];
-            tmem_ld16(tmem + kColAcc + w0 + lane_base, u);
-            tmem_ld16(tmem + kColAcc2 + w0 + lane_base, u2);
-            tmem_wait_ld();
-            if (j >= len) continue;
-            float r[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = fmaf(e_r, __uint_as_float(u2[e]), __uint_as_float(u[e]));
-            if (a.D) {
-                const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + w0);
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const uint4 vv = vp[q];
-                    const uint32_t ww[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        r[8 * q + 2 * e] = fmaf(Dh, bf16lo(ww[e]), r[8 * q + 2 * e]);
-                        r[8 * q + 2 * e + 1] = fmaf(Dh, bf16hi(ww[e]), r[8 * q + 2 * e + 1]);
-                    }
-                }
-            }
-            if (kOutBf16) {
-                uint4 *op = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + (tok * sh.H + h) * W + w0);
-                op[0] = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
-                                   pack_bf16x2(r[6], r[7]));
-                op[1] = make_uint4(pack_bf16x2(r[8], r[9]), pack_bf16x2(r[10], r[11]), pack_bf16x2(r[12], r[13]),
-                                   pack_bf16x2(r[14], r[15]));
-            } else {
-                float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + (tok * sh.H + h) * W + w0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) op[q] = make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-            }
+            if (lane == 0) mbar_arrive(&acc_free);
         }
     }
     fence_before_sync();
@@ -554,8 +605,13 @@ cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int 
     if (!k) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid(sh.nc * (sh.Q / kRows), sh.H, sh.batch);
-    k<<<grid, kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
+    // persistent: one CTA per SM, each taking every grid-th (chunk, block, head) tile
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || sms <= 0)
+        sms = 148;
+    const int tiles = sh.batch * sh.nc * (sh.Q / kRows) * sh.H;
+    k<<<min(tiles, sms), kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
     return cudaGetLastError();
 }
 
