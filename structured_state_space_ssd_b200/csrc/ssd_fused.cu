@@ -6,7 +6,8 @@
 // tokens (stage 1), chunk-final states (stage 2), the scalar recurrence of
 // those states across chunks (stage 3), the inter-chunk output (stage 4) and
 // the sum (stage 5).  This kernel runs every stage in one launch; nothing but
-// the chained fp32 states (an L2-resident ring) leaves the SM.
+// the chained states (L2-resident: fp32, and bf16 operand tiles of them)
+// leaves the SM.
 //
 // Blocks of 128 rows.  A chunk of Q = 256 tokens is two blocks, and the
 // second block reaches the first through the state at the chunk's midpoint
@@ -89,7 +90,7 @@ __device__ __forceinline__ uint32_t col_mask(int pl) { return 256u + 192u * pl; 
 constexpr uint32_t kOffC = 0;           // C rows of the block: NK atoms x 128 rows
 constexpr uint32_t kOffB = 32768;       // B rows 0..Q-1: 2 atoms of 256 rows (atom stride 32 KiB)
 constexpr uint32_t kOffPipe = 98304;    // per pipeline: x rows 0..127 | W | x rows 128..255, 16 KiB each
-constexpr uint32_t kPipeBytes = 49152;  // W: scaled x rows, then the entering-state tile [n][p]
+constexpr uint32_t kPipeBytes = 49152;  // W: scaled x rows, then an owner's bf16 state tile or the y tile
 constexpr uint32_t kOffAux = kOffPipe + 2 * kPipeBytes;
 constexpr uint32_t kAuxFloats = 256 + 256 + 16;  // per pipeline: s (log2 units), column factors, warp totals
 constexpr uint32_t kOffStat = kOffAux + 2 * kAuxFloats * 4;  // gated drain: per pipeline, half, row (mean, M2)
@@ -184,10 +185,11 @@ struct Unit {
 //   [owners of chunk 0] [owners of 1, others of 0] [owners of 2, others of 1] ... [others of nc-1]
 // so that the owners, which carry the inter-chunk chain, run ahead of the blocks that wait for it.
 // Every unit still waits only for units handed out before it: an owner waits for the owners of the
-// D chunks before (earlier steps) and for the readers of the ring slot it overwrites, chunk c-R's (the
+// D chunks before (earlier steps) and for the readers of the slot it overwrites, chunk c-R's (the
 // owners up to chunk c-R+D and the other block of chunk c-R+1, handed out with the owners of c-R+2, at
-// least one step earlier as R >= 3); another block waits for the owner of the chunk before (two steps
-// earlier).  So there is no deadlock however many CTAs are resident.
+// least one step earlier as R >= 3; without look-back only the tile slot is counted, by its publisher);
+// another block waits for the owner of the chunk before (two steps earlier).  So there is no deadlock
+// however many CTAs are resident.
 __device__ __forceinline__ Unit decode(int u, const Params &p) {
     Unit un;
     const int Mo = p.units[0], Mw = p.units[1];
@@ -332,8 +334,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     __shared__ uint32_t tslot;
     __shared__ int s_unit;
     __shared__ int s_abort, s_broken;
-    // per pipeline, for its publisher: warps that finished an owner's ring stores, and warps that
-    // finished reading another block's state from the ring (8 per head in either case)
+    // per pipeline, for its publisher: warps that finished an owner's state stores (8 per head), and the
+    // reads of another block's entering state (its issuer's tile load, 1 per head; with look-back its
+    // warps' reads of the fp32 slot, 8 per head)
     __shared__ uint32_t s_owned[2], s_copied[2], s_agg[2];
     __shared__ int s_base[2];  // per pipeline: the chunk whose S~ the owner starts from (-1: initial state)
     volatile int *abort = &s_abort;
