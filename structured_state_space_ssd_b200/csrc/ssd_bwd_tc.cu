@@ -51,8 +51,8 @@ constexpr uint32_t kOffK = 32768;       // 2 x 32 KiB
 constexpr uint32_t kOffV = 98304;       // 2 x 32 KiB
 constexpr uint32_t kOffSt = 163840;     // 2 x 16 KiB
 constexpr uint32_t kOffStLo = 196608;   // 2 x 8 KiB (split: KD = 64)
-constexpr uint32_t kOffS = 212992;      // 256 floats
-constexpr uint32_t kSmemBytes = kOffS + 1024 + 1024;
+constexpr uint32_t kOffS = 212992;      // two buffers of 256 floats (this tile's and the next one's)
+constexpr uint32_t kSmemBytes = kOffS + 2048 + 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -243,25 +243,45 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         const int lrow = wq * 32 + lane;            // this thread's row of the block
         const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
         float *sRaw = reinterpret_cast<float *>(smem + kOffRaw);
+        float *const sqb[2] = {sq, sq + 256};
         uint32_t n_g = 0, n_mx = 0, n_fin = 0;
-        for (int t = t_beg; t < t_end; t += t_step) {
+        auto valid = [&](int t) {
+            int b, c, rb, h;
+            tile(t, b, c, rb, h);
+            return rb * kRows < min(sh.Q, sh.T - c * sh.Q);
+        };
+        // the prefix sums of tile t into buffer d, one 4-byte async copy per token, as one commit group
+        auto request_sq = [&](int t, float *d) {
+            int b, c, rb, h;
+            tile(t, b, c, rb, h);
+            const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
+            for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) cp_async4(d + i, sch + i);
+            cp_async_commit();
+        };
+        int t = t_beg;
+        while (t < t_end && !valid(t)) t += t_step;
+        if (t < t_end) request_sq(t, sqb[0]);
+        for (int k = 0; t < t_end; ++k) {
+            int tn = t + t_step;
+            while (tn < t_end && !valid(tn)) tn += t_step;
             int b, c, rb, h;
             tile(t, b, c, rb, h);
             const int g = h / sh.heads_per_group;
             const int t0 = c * sh.Q, len = min(sh.Q, sh.T - t0), r0 = rb * kRows;
-            if (r0 >= len) continue;
             const int cbeg = kAnti ? r0 : 0;
             const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;
             const int j = r0 + lrow;  // row within the chunk
-            // every thread is done with the previous tile's prefix sums and staged state
+            const float *sq = sqb[k & 1];
+            // every thread is done with the previous tile's staged state (and the prefix-sum buffer the next
+            // tile's go to)
             named_bar_sync(1, 32 * kCudaWarps);
             // the fp32 state on its way into shared memory (async copies: no barrier waits for them, so
-            // its DRAM latency passes while the masks are built)
+            // its DRAM latency passes while the masks are built), one commit group
             const float *Sp = a.St + (((size_t)b * sh.nc + c) * sh.H + h) * (size_t)sh.P * sh.N;
             for (int i = tid; i < KD * W / 4; i += 32 * kCudaWarps) cp_async16(sRaw + 4 * i, Sp + 4 * i);
-            const float *sch = a.s + (((size_t)b * sh.H + h) * sh.nc + c) * sh.Q;
-            for (int i = tid; i < sh.Q; i += 32 * kCudaWarps) sq[i] = sch[i];
-            named_bar_sync(1, 32 * kCudaWarps);  // the prefix sums are in
+            cp_async_commit();
+            cp_async_wait_group<1>();           // this tile's prefix sums (requested during the tile before)
+            named_bar_sync(1, 32 * kCudaWarps);  // everyone's are in
             const float sj = (j < len) ? sq[j] : 0.f;
 
             // the mask, one 128-column half at a time: this thread's row, its 64 of the half's columns
@@ -298,11 +318,16 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                 if (lane == 0) mbar_arrive(&m_full);
             }
             n_mx = mx0 + nh;
+            // the next tile's prefix sums into the other buffer, while this tile's state tile and drain run
+            if (tn < t_end) request_sq(tn, sqb[(k + 1) & 1]);
 
             // the state tile [k][w] in bf16 (and its low part), 128-byte swizzled, 64-wide w atoms of KD rows,
             // from the staged fp32 state (the previous tile's products, acc2 among them, are done: its drain
             // waited for them)
-            cp_async_wait_all();
+            if (tn < t_end)
+                cp_async_wait_group<1>();  // the state (the newest group, the next prefix sums, may still fly)
+            else
+                cp_async_wait_group<0>();
             named_bar_sync(1, 32 * kCudaWarps);  // every thread's copies are in
             for (int idx = tid; idx < KD * (W / 8); idx += 32 * kCudaWarps) {
                 const int k = idx / (W / 8), w0 = (idx - k * (W / 8)) * 8;
@@ -329,14 +354,21 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&st_full);
 
-            // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns
-            wait_bar(&fin_done, n_fin++ & 1, a.status);
-            fence_after_sync();
-            const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
-            const float Dh = a.D ? a.D[h] : 0.f;
+            // the drain: out = e_r acc2 + acc (+ D V_r), this thread's row, its half of the W columns; the D
+            // term's row of V (dx only) is loaded before the wait for the products, which covers its latency
             const size_t tok = (size_t)b * sh.T + t0 + j;
             const __nv_bfloat16 *vrow =
                 a.V + (tok * (a.v_head ? sh.H : sh.G) + (a.v_head ? h : g)) * (size_t)W;
+            const float Dh = a.D ? a.D[h] : 0.f;
+            uint4 vr[kOutBf16 ? W / 16 : 1];
+            if (kOutBf16 && a.D && j < len) {
+                const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + half * (W / 2));
+#pragma unroll
+                for (int q = 0; q < (kOutBf16 ? W / 16 : 1); ++q) vr[q] = vp[q];
+            }
+            wait_bar(&fin_done, n_fin++ & 1, a.status);
+            fence_after_sync();
+            const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
             for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
                 uint32_t u[16], u2[16];
                 tmem_ld16(tmem + kColAcc + w0 + lane_base, u);
@@ -350,7 +382,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                     const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + w0);
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
-                        const uint4 vv = vp[q];
+                        const uint4 vv = kOutBf16 ? vr[(w0 - half * (W / 2)) / 8 + q] : vp[q];
                         const uint32_t ww[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -376,6 +408,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free);
+            t = tn;
         }
     }
     fence_before_sync();
