@@ -52,7 +52,8 @@ constexpr uint32_t kOffV = 98304;       // 2 x 32 KiB
 constexpr uint32_t kOffSt = 163840;     // 2 x 16 KiB
 constexpr uint32_t kOffStLo = 196608;   // 2 x 8 KiB (split: KD = 64)
 constexpr uint32_t kOffS = 212992;      // two buffers of 256 floats (this tile's and the next one's)
-constexpr uint32_t kSmemBytes = kOffS + 2048 + 1024;
+constexpr uint32_t kOffF = kOffS + 2048;  // 256 floats: the mask's column factors
+constexpr uint32_t kSmemBytes = kOffF + 1024 + 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -283,6 +284,12 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             cp_async_wait_group<1>();           // this tile's prefix sums (requested during the tile before)
             named_bar_sync(1, 32 * kCudaWarps);  // everyone's are in
             const float sj = (j < len) ? sq[j] : 0.f;
+            // the mask's column factors, relative to the column's 16-wide piece: exp(s_i - s_{piece start})
+            // (anti-causal) or exp(s_{piece end} - s_i) (causal), both <= 1 for decaying inputs
+            float *sFac = reinterpret_cast<float *>(smem + kOffF);
+            if (tid < sh.Q)
+                sFac[tid] = ex2((kAnti ? sq[tid] - sq[tid & ~15] : sq[tid | 15] - sq[tid]) * kLog2e);
+            named_bar_sync(1, 32 * kCudaWarps);
 
             // the mask, one 128-column half at a time: this thread's row, its 64 of the half's columns
             const uint32_t mx0 = n_mx;
@@ -296,18 +303,49 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                     tmem_ld16(tmem + kColG + q0 + lane_base, gv);
                     tmem_wait_ld();
                     uint32_t o[8], ol[8];
+                    // a piece of 16 columns wholly on the kept side of this row (and inside the chunk) takes a
+                    // row factor times the column factors, one exponential per piece; a piece wholly on the
+                    // other side is zero; a piece the diagonal or the chunk's end crosses takes one exponential
+                    // per element
+                    const int i0 = cbeg + ch * kRows + q0;  // the piece's first column within the chunk
+                    const bool jv = j < len, whole = i0 + 15 < len;
+                    const bool fac = jv && whole && (kAnti ? i0 >= j : i0 + 15 <= j);
+                    const bool zero = !jv || (kAnti ? i0 + 15 < j : i0 > j);
+                    if (fac) {
+                        const float rf = ex2((kAnti ? sq[i0] - sj : sj - sq[i0 + 15]) * kLog2e);
+                        const float4 *f4 = reinterpret_cast<const float4 *>(sFac + i0);
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        float m[2];
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-                            const int i = cbeg + ch * kRows + q0 + e + k;  // column within the chunk
-                            const bool ok = j < len && i < len && (kAnti ? i >= j : i <= j);
-                            m[k] = ok ? __uint_as_float(gv[e + k]) * ex2((kAnti ? sq[i] - sj : sj - sq[i]) * kLog2e)
-                                      : 0.f;
+                        for (int e = 0; e < 16; e += 4) {
+                            const float4 f = f4[e / 4];
+                            const float m0 = __uint_as_float(gv[e]) * (rf * f.x);
+                            const float m1 = __uint_as_float(gv[e + 1]) * (rf * f.y);
+                            const float m2 = __uint_as_float(gv[e + 2]) * (rf * f.z);
+                            const float m3 = __uint_as_float(gv[e + 3]) * (rf * f.w);
+                            o[e / 2] = pack_bf16x2(m0, m1);
+                            o[e / 2 + 1] = pack_bf16x2(m2, m3);
+                            if (kSplit) {
+                                ol[e / 2] = pack_lo(m0, m1, o[e / 2]);
+                                ol[e / 2 + 1] = pack_lo(m2, m3, o[e / 2 + 1]);
+                            }
                         }
-                        o[e / 2] = pack_bf16x2(m[0], m[1]);
-                        if (kSplit) ol[e / 2] = pack_lo(m[0], m[1], o[e / 2]);
+                    } else if (zero) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[e] = ol[e] = 0u;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 2) {
+                            float m[2];
+#pragma unroll
+                            for (int k = 0; k < 2; ++k) {
+                                const int i = i0 + e + k;  // column within the chunk
+                                const bool ok = i < len && (kAnti ? i >= j : i <= j);
+                                m[k] = ok ? __uint_as_float(gv[e + k]) *
+                                                ex2((kAnti ? sq[i] - sj : sj - sq[i]) * kLog2e)
+                                          : 0.f;
+                            }
+                            o[e / 2] = pack_bf16x2(m[0], m[1]);
+                            if (kSplit) ol[e / 2] = pack_lo(m[0], m[1], o[e / 2]);
+                        }
                     }
                     tmem_st8(tmem + kColMhi + q0 / 2 + lane_base, o);
                     if (kSplit) tmem_st8(tmem + kColMlo + q0 / 2 + lane_base, ol);
