@@ -25,6 +25,8 @@
 // chunk_scan shape with the roles of its operands exchanged); the chunk sums
 // and the forward states reuse the forward's CUDA-core kernels.  Every
 // reduction runs in a fixed order: results are bitwise reproducible.
+#include <algorithm>
+
 #include "ssd_common.cuh"
 
 namespace ssd {
@@ -38,9 +40,14 @@ cudaError_t launch_state_passing(float *S, const float *s, const float *init, fl
 // The masked scans on the tensor cores (ssd_bwd_tc.cu); which of the three run there: bit 0 dx, bit 1 the
 // per-head dB terms, bit 2 the per-head dC terms.
 bool scan_tc_supported(const Shape &sh, int dtype);
+// With `part` given, the dB or dC scan sums its terms over each group's heads instead of storing them;
+// launch_head_sum_reduce then forms dB, dC and dsigma from both scans' partial results.
 cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int k_head, const void *V, int v_head,
                                   int KD, int W, bool anti, const float *St, int st_kw, const float *D, void *out,
-                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st);
+                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st,
+                                  const void *dotv = nullptr, float *dotp = nullptr, float *part = nullptr);
+cudaError_t launch_head_sum_reduce(const float *partB, const float *dotB, const float *partC, const float *dotC,
+                                   void *dB, void *dC, float *dsig, const Shape &sh, cudaStream_t st);
 constexpr int kScanTcRoles = 7;
 // chunk states on the tensor cores (ssd_bwd_tc.cu): bf16, P = 64, N = 128, Q in {128, 256}
 bool chunk_state_tc_supported(const Shape &sh, int dtype);
@@ -62,8 +69,8 @@ struct BwdWorkspace {
     size_t hin_off;   // float Hin[batch][nc][H][P][N]: chunk states, then the state entering each chunk
     size_t gout_off;  // float G[batch][nc][H][P][N]: chunk sums of dy C^T, then dHout of each chunk
     size_t fin_off;   // float final[batch][H][P][N]
-    size_t dbh_off;   // float dB^(h)[batch][T][H][N]
-    size_t dch_off;   // float dC^(h)[batch][T][H][N]
+    size_t dbh_off;   // float dB^(h)[batch][T][H][N], or the dB scan's head sums (bwd_sum_bytes)
+    size_t dch_off;   // float dC^(h)[batch][T][H][N], or the dC scan's head sums
     size_t dsig_off;  // float dsigma[batch][H][T]
     size_t pa_off;    // double dA partial[batch][H]
     size_t pd_off;    // double dD partial[kDdSlices][batch][H] (one per quarter of the tokens)
@@ -74,7 +81,7 @@ BwdWorkspace bwd_layout(const Shape &s) {
     BwdWorkspace w;
     const size_t bh = (size_t)s.batch * s.H, PN = (size_t)s.P * s.N;
     const size_t states = sizeof(float) * (size_t)s.batch * s.nc * s.H * PN;
-    const size_t perhead = sizeof(float) * (size_t)s.batch * s.T * s.H * s.N;
+    const size_t perhead = std::max(sizeof(float) * (size_t)s.batch * s.T * s.H * s.N, bwd_sum_bytes(s));
     size_t off = 0;
     w.status_off = off;
     off = 256;
@@ -779,6 +786,18 @@ bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+// dt, A and D gradients from dsigma: the dt scan, then the parameter sums
+template <typename T>
+int run_dt_tail(const Shape &sh, const float *dsig, const float *dt, const float *A, const T *x, const T *dy,
+                const float *dfin, const float *fin, float *ddt, float *dA, float *dD, double *pa, double *pd, int vec,
+                cudaStream_t st) {
+    dt_scan_kernel<T><<<dim3(sh.H, sh.batch, kDdSlices), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa,
+                                                                           pd, sh, vec);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    param_reduce_kernel<<<(sh.H + 255) / 256, 256, 0, st>>>(pa, pd, dA, dD, sh.batch, sh.H);
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
 template <typename T>
 int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const T *B, const T *C, const float *D,
             const float *init, const T *dy, const float *dfin, T *dx, float *ddt, float *dA, T *dB, T *dC,
@@ -829,6 +848,20 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
         ScanArgs ax{B, C, dy, 0, 0, 1, Gout, 0, sh.N, sh.P, D, dx, vec, st_vec};
         if (launch_scan<T, T, true>(ax, s, sh, st) != cudaSuccess) return SSD_ERR_CUDA;
     }
+    // dB and dC summed over each group's heads inside the scans (their per-head terms never reach memory):
+    // the dot products with B and C rows that dsigma needs are taken there too
+    if (tc && (kScanTcRoles & 6) == 6 && sh.Q % 128 == 0) {
+        float *partB = dBh, *partC = dCh;
+        float *dotB = reinterpret_cast<float *>(ws + w.dbh_off + bwd_sum_dot_off(sh));
+        float *dotC = reinterpret_cast<float *>(ws + w.dch_off + bwd_sum_dot_off(sh));
+        if (launch_masked_scan_tc(x, 1, dy, 1, C, 0, sh.P, sh.N, true, Gout, 1, nullptr, nullptr, false, s, status, sh,
+                                  st, B, dotB, partB) != cudaSuccess ||
+            launch_masked_scan_tc(dy, 1, x, 1, B, 0, sh.P, sh.N, false, Hin, 1, nullptr, nullptr, false, s, status,
+                                  sh, st, C, dotC, partC) != cudaSuccess ||
+            launch_head_sum_reduce(partB, dotB, partC, dotC, dB, dC, dsig, sh, st) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        return run_dt_tail(sh, dsig, dt, A, x, dy, dfin, fin, ddt, dA, dD, pa, pd, vec, st);
+    }
     // dB^(h): rows of x against columns of dy, values C, state dHout as [P][N] = [KD][W]
     if (tc && (kScanTcRoles & 2)) {
         if (launch_masked_scan_tc(x, 1, dy, 1, C, 0, sh.P, sh.N, true, Gout, 1, nullptr, dBh, false, s, status, sh,
@@ -860,11 +893,7 @@ int run_bwd(const Shape &sh, const T *x, const float *dt, const float *A, const 
     else
         group_reduce_kernel<T><<<(unsigned)((units + 7) / 8), 256, 0, st>>>(dBh, dCh, B, C, dB, dC, dsig, sh);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
-    dt_scan_kernel<T><<<dim3(sh.H, sh.batch, kDdSlices), kDtThreads, 0, st>>>(dsig, dt, A, x, dy, dfin, fin, ddt, pa, pd, sh,
-                                                                    vec);
-    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
-    param_reduce_kernel<<<(sh.H + 255) / 256, 256, 0, st>>>(pa, pd, dA, dD, sh.batch, sh.H);
-    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    return run_dt_tail(sh, dsig, dt, A, x, dy, dfin, fin, ddt, dA, dD, pa, pd, vec, st);
 }
 
 }  // namespace

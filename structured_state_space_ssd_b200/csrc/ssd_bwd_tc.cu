@@ -19,7 +19,11 @@
 //   out  = e_r acc2 + acc (+ D V_r), one row per thread, stored from registers.
 //
 // For the per-head dB and dC terms the mask and the state tile also enter as bf16 low parts (what the
-// rounding to bf16 left out), so those products are as accurate as fp32 accumulation allows.
+// rounding to bf16 left out), so those products are as accurate as fp32 accumulation allows.  Those terms
+// are summed over each group's heads in registers (dB = sum_h dB^(h), dC likewise) rather than stored:
+// each CTA takes a contiguous, cost-balanced run of tiles, head innermost, stores one partial sum per
+// (chunk, block, group) it touched plus each head's rows dotted with B or C (which dsigma needs), and
+// head_sum_reduce_kernel adds the partial sums of the few CTAs that share a (chunk, block, group).
 // Shapes: KD, W in {64, 128}; Q in {128, 256}; R, K, V bf16 rows of [batch][T][heads or groups][dim].
 // Tensor memory (512 columns): G at 0, the mask at 128 (its low part at 192), acc at 256, acc2 at 384.
 // One persistent CTA per SM (it takes all of tensor memory) taking every grid-th tile; while its warps
@@ -27,6 +31,8 @@
 // over the 128 lanes, each half of the columns), 8 TMA and MMA issue.  Every wait is bounded (about 2 s of
 // %globaltimer, 1 ms once any CTA has given up): on expiry the CTA records SSD_ERR_TIMEOUT in the status
 // word, and the issuer still waits (bounded) for its own MMAs before tensor memory is freed.
+#include <algorithm>
+
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
@@ -57,6 +63,74 @@ constexpr uint32_t kSmemBytes = kOffF + 1024 + 1024;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Contiguous, cost-balanced ranges of (chunk, 128-row block, head) tiles, head innermost, for the scans
+// that sum their per-head terms over each group's heads: CTA i takes the tiles whose cost before them lies
+// in [i, i + 1) * total / ncta.  A tile costs its number of 128-column halves plus one (the state product
+// and the drain), nothing for a block past a ragged chunk's end.  The same arithmetic tells the sum over
+// the CTAs' partial results which CTAs took part of a (chunk, block, group).
+struct TilePart {
+    int H, Q, nc, blocks, len_last, ncta, anti;
+    long long cfull, perseq, tiles, ctot;
+    __host__ __device__ int cost_len(int len, int rb) const {
+        const int r0 = rb * kRows;
+        return r0 >= len ? 0 : 1 + (anti ? Q - r0 : r0 + kRows) / kRows;
+    }
+    __host__ __device__ int cost(int c, int rb) const { return cost_len(c == nc - 1 ? len_last : Q, rb); }
+    __host__ void init(const Shape &sh, bool is_anti, int n) {
+        H = sh.H;
+        Q = sh.Q;
+        nc = sh.nc;
+        blocks = sh.Q / kRows;
+        len_last = sh.T - (sh.nc - 1) * sh.Q;
+        ncta = n;
+        anti = is_anti ? 1 : 0;
+        cfull = 0;
+        long long clast = 0;
+        for (int rb = 0; rb < blocks; ++rb) {
+            cfull += cost_len(Q, rb);
+            clast += cost_len(len_last, rb);
+        }
+        perseq = (long long)(nc - 1) * cfull + clast;
+        tiles = (long long)sh.batch * nc * blocks * H;
+        ctot = (long long)sh.batch * perseq * H;
+    }
+    // cost of the tiles before tile t (t = tiles gives the total)
+    __host__ __device__ long long cum(long long t) const {
+        const long long blk = t / H;
+        const int h = (int)(t - blk * H), rb = (int)(blk % blocks);
+        const long long r = blk / blocks;
+        const int c = (int)(r % nc);
+        const long long b = r / nc;
+        long long before = b * perseq + (long long)c * cfull;
+        for (int q = 0; q < rb; ++q) before += cost(c, q);
+        return before * H + (long long)cost(c, rb) * h;
+    }
+    // first tile of CTA i (i = ncta gives the end)
+    __host__ __device__ long long beg(int i) const {
+        if (i <= 0) return 0;
+        if (i >= ncta) return tiles;
+        long long lo = 0, hi = tiles;
+        const long long want = (long long)i * ctot;
+        while (lo < hi) {
+            const long long mid = (lo + hi) / 2;
+            if (cum(mid) * ncta >= want) hi = mid;
+            else lo = mid + 1;
+        }
+        return lo;
+    }
+    __host__ __device__ int cta_of(long long t) const {
+        const long long i = cum(t) * ncta / ctot;
+        return (int)(i < ncta - 1 ? i : ncta - 1);
+    }
+    // within a run of n tiles of cost cb starting at cost `base`: how many come before CTA i's range
+    __host__ __device__ int first_in(int i, long long base, int cb, int n) const {
+        const long long num = (long long)i * ctot - base * ncta;
+        if (num <= 0) return 0;
+        const long long m = (num + (long long)cb * ncta - 1) / ((long long)cb * ncta);
+        return (int)(m < n ? m : n);
+    }
+};
+
 struct Args {
     const float *s;    // [batch][H][nc][Q] chunk prefix sums of dt * A (natural units)
     const float *St;   // [batch][nc][H][P * N]: read as [KD][W] (st_kw) or [W][KD]
@@ -67,6 +141,13 @@ struct Args {
     void *out;         // [batch][T][H][W], bf16 (kOutBf16) or fp32
     int *status;
     Shape sh;
+    // head sums (kSum): the row each term is dotted with ([batch][T][G][W], bf16), the two column halves'
+    // dot products [batch][T][H][2], the CTAs' partial sums [CTA + (chunk, block, group) key][128][W], and
+    // the tile ranges
+    const __nv_bfloat16 *dotv;
+    float *dotp;
+    float *part;
+    TilePart tp;
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -107,13 +188,17 @@ using namespace bt;
 // MMAs each); R, K and V are bf16 inputs and exact, so the products are then as accurate as fp32
 // accumulation allows.  Used for the per-head dB and dC terms, from which the dt, A and D gradients follow
 // through differences of large terms.
-template <int KD, int W, bool kAnti, bool kOutBf16, bool kSplit>
+// kSum: the per-head terms are not stored; each CTA takes a contiguous run of tiles (TilePart), adds each
+// head's rows into registers in head order and stores the sum once per (chunk, block, group) it touched,
+// plus each head's row dotted with the row of a.dotv (the two column halves apart).
+template <int KD, int W, bool kAnti, bool kOutBf16, bool kSplit, bool kSum>
 __global__ void __launch_bounds__(bt::kThreads, 1)
     masked_scan_tc_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mK,
                           const __grid_constant__ CUtensorMap mV, const bt::Args a, int r_head, int k_head,
                           int v_head) {
     static_assert(!kSplit || KD == 64, "the low part of the state tile has room for KD = 64");
     static_assert(KD == 64 || W == 64, "the fp32 state is staged in the unused second atom of K or V");
+    static_assert(!kSum || !kOutBf16, "head sums are fp32");
     // the fp32 state [KD][W] (32 KB), copied in asynchronously: the K region's second atom (KD = 64) or the
     // V region's (W = 64), which this shape leaves unused
     constexpr uint32_t kOffRaw = (KD == 64) ? kOffK + 32768 : kOffV + 32768;
@@ -125,9 +210,11 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int blocks = sh.Q / kRows;
     // this CTA's tiles (chunk, 128-row block, head): every gridDim.x-th, so that each CTA gets the same mix
-    // of one- and two-half blocks
+    // of one- and two-half blocks; for head sums a contiguous run of about equal cost
     const int tiles = sh.batch * sh.nc * blocks * sh.H;
-    const int t_beg = blockIdx.x, t_end = tiles, t_step = gridDim.x;
+    const int t_beg = kSum ? (int)a.tp.beg(blockIdx.x) : (int)blockIdx.x;
+    const int t_end = kSum ? (int)a.tp.beg(blockIdx.x + 1) : tiles;
+    const int t_step = kSum ? 1 : (int)gridDim.x;
     if (t_beg >= t_end) return;  // whole CTA
     auto tile = [&](int t, int &b, int &c, int &rb, int &h) {
         h = t % sh.H;
@@ -246,6 +333,8 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
         float *sRaw = reinterpret_cast<float *>(smem + kOffRaw);
         float *const sqb[2] = {sq, sq + 256};
         uint32_t n_g = 0, n_mx = 0, n_fin = 0;
+        float hs[kSum ? W / 2 : 1];  // head sums: this thread's row, its half of the columns
+        int seg = -1;                // the (chunk, block, group) key they belong to
         auto valid = [&](int t) {
             int b, c, rb, h;
             tile(t, b, c, rb, h);
@@ -273,6 +362,12 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             const int nh = (kAnti ? sh.Q - r0 : r0 + kRows) / kRows;
             const int j = r0 + lrow;  // row within the chunk
             const float *sq = sqb[k & 1];
+            const int key = t / sh.heads_per_group;
+            if (kSum && key != seg) {
+#pragma unroll
+                for (int e = 0; e < (kSum ? W / 2 : 1); ++e) hs[e] = 0.f;
+                seg = key;
+            }
             // every thread is done with the previous tile's staged state (and the prefix-sum buffer the next
             // tile's go to)
             named_bar_sync(1, 32 * kCudaWarps);
@@ -398,15 +493,44 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
             const __nv_bfloat16 *vrow =
                 a.V + (tok * (a.v_head ? sh.H : sh.G) + (a.v_head ? h : g)) * (size_t)W;
             const float Dh = a.D ? a.D[h] : 0.f;
-            uint4 vr[kOutBf16 ? W / 16 : 1];
+            uint4 vr[(kOutBf16 || kSum) ? W / 16 : 1];
             if (kOutBf16 && a.D && j < len) {
                 const uint4 *vp = reinterpret_cast<const uint4 *>(vrow + half * (W / 2));
 #pragma unroll
                 for (int q = 0; q < (kOutBf16 ? W / 16 : 1); ++q) vr[q] = vp[q];
             }
+            if (kSum && j < len) {  // the row the head's term is dotted with
+                const uint4 *vp =
+                    reinterpret_cast<const uint4 *>(a.dotv + (tok * sh.G + g) * (size_t)W + half * (W / 2));
+#pragma unroll
+                for (int q = 0; q < (kSum ? W / 16 : 1); ++q) vr[q] = vp[q];
+            }
             wait_bar(&fin_done, n_fin++ & 1, a.status);
             fence_after_sync();
             const float e_r = ex2((kAnti ? sq[sh.Q - 1] - sj : sj) * kLog2e);
+            if constexpr (kSum) {
+                float dot = 0.f;
+#pragma unroll
+                for (int q = 0; q < W / 32; ++q) {
+                    uint32_t u[16], u2[16];
+                    tmem_ld16(tmem + kColAcc + half * (W / 2) + q * 16 + lane_base, u);
+                    tmem_ld16(tmem + kColAcc2 + half * (W / 2) + q * 16 + lane_base, u2);
+                    tmem_wait_ld();
+                    if (j >= len) continue;
+                    const uint32_t ww[8] = {vr[2 * q].x, vr[2 * q].y, vr[2 * q].z, vr[2 * q].w,
+                                            vr[2 * q + 1].x, vr[2 * q + 1].y, vr[2 * q + 1].z, vr[2 * q + 1].w};
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        const float r0v = fmaf(e_r, __uint_as_float(u2[e]), __uint_as_float(u[e]));
+                        const float r1v = fmaf(e_r, __uint_as_float(u2[e + 1]), __uint_as_float(u[e + 1]));
+                        hs[q * 16 + e] += r0v;
+                        hs[q * 16 + e + 1] += r1v;
+                        dot = fmaf(r0v, bf16lo(ww[e / 2]), dot);
+                        dot = fmaf(r1v, bf16hi(ww[e / 2]), dot);
+                    }
+                }
+                if (j < len) a.dotp[(tok * sh.H + h) * 2 + half] = dot;
+            } else {
             for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
                 uint32_t u[16], u2[16];
                 tmem_ld16(tmem + kColAcc + w0 + lane_base, u);
@@ -442,10 +566,19 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                     for (int q = 0; q < 4; ++q) op[q] = make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
                 }
             }
+            }
             // both accumulators are read: the next tile's masked product may overwrite them
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free);
+            // the sums over the key's heads, once its last head in this CTA's run is in: slot CTA + key
+            if (kSum && (tn >= t_end || tn / sh.heads_per_group != key) && j < len) {
+                float4 *pp = reinterpret_cast<float4 *>(a.part + ((size_t)(blockIdx.x + key) * kRows + lrow) * W +
+                                                        half * (W / 2));
+#pragma unroll
+                for (int q = 0; q < (kSum ? W / 8 : 0); ++q)
+                    pp[q] = make_float4(hs[4 * q], hs[4 * q + 1], hs[4 * q + 2], hs[4 * q + 3]);
+            }
             t = tn;
         }
     }
@@ -629,11 +762,29 @@ bool scan_tc_supported(const Shape &sh, int dtype) {
            sh.batch <= 65535 && sh.H <= 65535;
 }
 
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || sms <= 0)
+        sms = 148;
+    return sms;
+}
+
+// CTAs of the head-summing scans (one per SM, at most kBwdSumMaxCtas, at most one per tile); the scans and the
+// sum over their partial results take the same number
+int head_sum_ctas(const Shape &sh) {
+    const long long tiles = (long long)sh.batch * sh.nc * (sh.Q / kRows) * sh.H;
+    return (int)std::min<long long>(tiles, std::min(sm_count(), kBwdSumMaxCtas));
+}
+
 // One masked scan.  R, K, V: bf16 [batch][T][heads or groups][KD, KD, W]; *_head: 1 = per head, 0 = per
-// group.  St, st_kw, D, out as for the CUDA-core scan; out bf16 (dx) or fp32.
+// group.  St, st_kw, D, out as for the CUDA-core scan; out bf16 (dx) or fp32.  With `part` given the
+// per-head terms are summed over each group's heads instead (out unused): part receives the CTAs'
+// partial sums, dotp each head's rows dotted with the rows of dotv (see masked_scan_tc_kernel, kSum).
 cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int k_head, const void *V, int v_head,
                                   int KD, int W, bool anti, const float *St, int st_kw, const float *D, void *out,
-                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st) {
+                                  bool out_bf16, const float *s, int *status, const Shape &sh, cudaStream_t st,
+                                  const void *dotv, float *dotp, float *part) {
     auto dims = [&](int head, int d, uint64_t *dm, uint64_t *sb) {
         const int n = head ? sh.H : sh.G;
         dm[0] = (uint64_t)d;
@@ -663,26 +814,127 @@ cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int 
     a.out = out;
     a.status = status;
     a.sh = sh;
+    a.dotv = static_cast<const __nv_bfloat16 *>(dotv);
+    a.dotp = dotp;
+    a.part = part;
+    const bool sum = part != nullptr;
+    if (sum && (out_bf16 || !dotv || !dotp)) return cudaErrorInvalidValue;
     void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const Args, int, int, int) = nullptr;
-#define SSD_SCAN_TC_CASE(KDv, Wv, AN, OB, SP)                                                \
-    if (KD == KDv && W == Wv && anti == AN && out_bf16 == OB) k = masked_scan_tc_kernel<KDv, Wv, AN, OB, SP>;
-    SSD_SCAN_TC_CASE(128, 64, true, true, false)   // dx at N = 128
-    SSD_SCAN_TC_CASE(64, 64, true, true, false)    // dx at N = 64
-    SSD_SCAN_TC_CASE(64, 128, true, false, true)   // dB^(h) at N = 128
-    SSD_SCAN_TC_CASE(64, 64, true, false, true)    // dB^(h) at N = 64
-    SSD_SCAN_TC_CASE(64, 128, false, false, true)  // dC^(h) at N = 128
-    SSD_SCAN_TC_CASE(64, 64, false, false, true)   // dC^(h) at N = 64
+#define SSD_SCAN_TC_CASE(KDv, Wv, AN, OB, SP, SU)                                                  \
+    if (KD == KDv && W == Wv && anti == AN && out_bf16 == OB && sum == SU) \
+        k = masked_scan_tc_kernel<KDv, Wv, AN, OB, SP, SU>;
+    SSD_SCAN_TC_CASE(128, 64, true, true, false, false)   // dx at N = 128
+    SSD_SCAN_TC_CASE(64, 64, true, true, false, false)    // dx at N = 64
+    SSD_SCAN_TC_CASE(64, 128, true, false, true, false)   // dB^(h) at N = 128
+    SSD_SCAN_TC_CASE(64, 64, true, false, true, false)    // dB^(h) at N = 64
+    SSD_SCAN_TC_CASE(64, 128, false, false, true, false)  // dC^(h) at N = 128
+    SSD_SCAN_TC_CASE(64, 64, false, false, true, false)   // dC^(h) at N = 64
+    SSD_SCAN_TC_CASE(64, 128, true, false, true, true)    // dB head sums at N = 128
+    SSD_SCAN_TC_CASE(64, 64, true, false, true, true)     // dB head sums at N = 64
+    SSD_SCAN_TC_CASE(64, 128, false, false, true, true)   // dC head sums at N = 128
+    SSD_SCAN_TC_CASE(64, 64, false, false, true, true)    // dC head sums at N = 64
 #undef SSD_SCAN_TC_CASE
     if (!k) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    // persistent: one CTA per SM, each taking every grid-th (chunk, block, head) tile
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                  cudaSuccess || sms <= 0)
-        sms = 148;
+    // persistent: one CTA per SM, each taking every grid-th (chunk, block, head) tile, or (head sums) a
+    // contiguous run of them
     const int tiles = sh.batch * sh.nc * (sh.Q / kRows) * sh.H;
-    k<<<min(tiles, sms), kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
+    const int grid = sum ? head_sum_ctas(sh) : min(tiles, sm_count());
+    if (sum) a.tp.init(sh, anti, grid);
+    k<<<grid, kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// The sums over each group's heads from the head-summing scans' partial results: one warp per (batch,
+// token, group) row adds the partial rows of the CTAs that took part of its (chunk, block, group), in CTA
+// order, for dB and for dC, and writes each of the group's heads' dsigma_t = C_t . dC^(h)_t - B_t . dB^(h)_t
+// from the scans' half-row dot products.  Each lane takes 4 consecutive n.  256 threads per block.
+// ---------------------------------------------------------------------------
+template <int kNV>
+__global__ void __launch_bounds__(256) head_sum_reduce_kernel(const float *__restrict__ partB,
+                                                              const float *__restrict__ dotB,
+                                                              const float *__restrict__ partC,
+                                                              const float *__restrict__ dotC, const TilePart pb,
+                                                              const TilePart pc, __nv_bfloat16 *__restrict__ dB,
+                                                              __nv_bfloat16 *__restrict__ dC, float *__restrict__ dsig,
+                                                              Shape sh) {
+    const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long units = (long long)sh.batch * sh.T * sh.G;
+    if (unit >= units) return;
+    const int lane = threadIdx.x & 31;
+    const int g = (int)(unit % sh.G);
+    const long long tok = unit / sh.G;  // b * T + t
+    const int b = (int)(tok / sh.T), t = (int)(tok - (long long)b * sh.T);
+    const int c = t / sh.Q, rr = t - c * sh.Q, rb = rr / kRows, lr = rr - rb * kRows;
+    const long long blk = ((long long)b * sh.nc + c) * (sh.Q / kRows) + rb;
+    const long long key = blk * sh.G + g, k0 = blk * sh.H + (long long)g * sh.heads_per_group;
+    const int hpg = sh.heads_per_group, V = sh.N / 4;
+    auto gather = [&](const TilePart &p, const float *part, float4 *acc) {
+#pragma unroll
+        for (int m = 0; m < kNV; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const long long base = p.cum(k0);
+        const int cb = p.cost(c, rb), i0 = p.cta_of(k0), i1 = p.cta_of(k0 + hpg - 1);
+        int f0 = p.first_in(i0, base, cb, hpg);
+        for (int i = i0; i <= i1; ++i) {
+            const int f1 = p.first_in(i + 1, base, cb, hpg);
+            if (f0 < f1) {  // CTA i took heads f0 .. f1 - 1 of the group
+                const float *row = part + ((size_t)(i + key) * kRows + lr) * sh.N;
+#pragma unroll
+                for (int m = 0; m < kNV; ++m) {
+                    const int v = lane + 32 * m;
+                    if (v < V) {
+                        const float4 x = *reinterpret_cast<const float4 *>(row + 4 * v);
+                        acc[m].x += x.x;
+                        acc[m].y += x.y;
+                        acc[m].z += x.z;
+                        acc[m].w += x.w;
+                    }
+                }
+            }
+            f0 = f1;
+        }
+    };
+    float4 sb[kNV], sc[kNV];
+    gather(pb, partB, sb);
+    gather(pc, partC, sc);
+    const size_t grow = (size_t)unit * sh.N;  // row (b, t, g) of dB, dC
+#pragma unroll
+    for (int m = 0; m < kNV; ++m) {
+        const int v = lane + 32 * m;
+        if (v < V) {
+            const __nv_bfloat162 b0 = __floats2bfloat162_rn(sb[m].x, sb[m].y), b1 = __floats2bfloat162_rn(sb[m].z, sb[m].w);
+            const __nv_bfloat162 c0 = __floats2bfloat162_rn(sc[m].x, sc[m].y), c1 = __floats2bfloat162_rn(sc[m].z, sc[m].w);
+            uint2 rb2, rc2;
+            rb2.x = *reinterpret_cast<const uint32_t *>(&b0);
+            rb2.y = *reinterpret_cast<const uint32_t *>(&b1);
+            rc2.x = *reinterpret_cast<const uint32_t *>(&c0);
+            rc2.y = *reinterpret_cast<const uint32_t *>(&c1);
+            *reinterpret_cast<uint2 *>(dB + grow + 4 * v) = rb2;
+            *reinterpret_cast<uint2 *>(dC + grow + 4 * v) = rc2;
+        }
+    }
+    for (int hh = lane; hh < hpg; hh += 32) {
+        const int h = g * hpg + hh;
+        const float2 db = *reinterpret_cast<const float2 *>(dotB + ((size_t)tok * sh.H + h) * 2);
+        const float2 dc = *reinterpret_cast<const float2 *>(dotC + ((size_t)tok * sh.H + h) * 2);
+        dsig[((size_t)b * sh.H + h) * sh.T + t] = (dc.x + dc.y) - (db.x + db.y);
+    }
+}
+
+cudaError_t launch_head_sum_reduce(const float *partB, const float *dotB, const float *partC, const float *dotC,
+                                   void *dB, void *dC, float *dsig, const Shape &sh, cudaStream_t st) {
+    if (sh.N % 4 != 0 || sh.N > 256) return cudaErrorInvalidValue;
+    const int n = head_sum_ctas(sh);
+    TilePart pb, pc;
+    pb.init(sh, true, n);
+    pc.init(sh, false, n);
+    const long long units = (long long)sh.batch * sh.T * sh.G;
+    auto k = sh.N <= 128 ? head_sum_reduce_kernel<1> : head_sum_reduce_kernel<2>;
+    k<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(partB, dotB, partC, dotC, pb, pc,
+                                                   static_cast<__nv_bfloat16 *>(dB), static_cast<__nv_bfloat16 *>(dC),
+                                                   dsig, sh);
     return cudaGetLastError();
 }
 
@@ -706,12 +958,8 @@ cudaError_t launch_chunk_state_tc(const void *x, const void *B, const float *s, 
     cudaError_t e = cudaFuncSetAttribute(chunk_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cs::kSmemBytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                  cudaSuccess || sms <= 0)
-        sms = 148;
     const int tiles = sh.nc * sh.H * sh.batch;
-    const int grid = min(tiles, sms), per_cta = (tiles + grid - 1) / grid;
+    const int grid = min(tiles, sm_count()), per_cta = (tiles + grid - 1) / grid;
     chunk_state_tc_kernel<<<grid, kThreads, cs::kSmemBytes, st>>>(mX, mB, s, S, status, sh, from_start ? 1 : 0,
                                                                    per_cta);
     return cudaGetLastError();

@@ -168,6 +168,21 @@ int check_dims(int batch, int T, int H, int P, int G, int N, int Q, int dtype, S
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// The backward's head-summing scans (bf16, Q a multiple of 128) keep, for dB and for dC, one partial sum
+// of 128 rows per (CTA, (chunk, 128-row block, group)) pair, in slot CTA + pair (at most kBwdSumMaxCtas
+// CTAs), and two half-row dot products per (batch, token, head).
+constexpr int kBwdSumMaxCtas = 256;
+inline size_t bwd_sum_bytes(const Shape &s) {
+    if (s.Q % 128 != 0) return 0;
+    const size_t keys = (size_t)s.batch * s.nc * (s.Q / 128) * s.G;
+    return align256(sizeof(float) * (kBwdSumMaxCtas + keys) * 128 * s.N) +
+           align256(sizeof(float) * 2 * (size_t)s.batch * s.T * s.H);
+}
+inline size_t bwd_sum_dot_off(const Shape &s) {
+    const size_t keys = (size_t)s.batch * s.nc * (s.Q / 128) * s.G;
+    return align256(sizeof(float) * (kBwdSumMaxCtas + keys) * 128 * s.N);
+}
+
 // The fused path works on 64 head columns and up to 128 state columns per launch: P = 128 runs as two
 // launches over column halves of x and y, N = 256 as two over halves of the state (the second adding to
 // y).  Each launch has its own counter, flags and ring (one after the other in the workspace); the
