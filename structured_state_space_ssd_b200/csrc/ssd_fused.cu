@@ -1371,10 +1371,11 @@ static int device_sm_count() {
 // Heads per work unit: enough to amortise the unit's C, B and G over several heads (they are loaded
 // and formed once per unit), few enough that every SM gets several units.  Up to 8 for the other
 // blocks and 4 for the owners' block, whose heads take about twice as long; with look-back (long
-// sequences, few heads) units of 2 heads, one per pipeline: a unit's later heads would otherwise wait
-// behind its first head's chain step, and the chunks in flight would advance at that pace.
+// sequences, few heads) owners' units of 2 heads, one per pipeline: a unit's later heads would otherwise
+// wait behind its first head's chain step, and the chunks in flight would advance at that pace.  The
+// other blocks read a state their chunk's predecessor published well before, so theirs stay large.
 static int heads_per_unit(const Shape &sh, bool lookback, bool owners) {
-    const int hpg = sh.heads_per_group, most = lookback ? 2 : owners ? 4 : 8;
+    const int hpg = sh.heads_per_group, most = owners ? (lookback ? 2 : 4) : 8;
     if (hpg <= most) return hpg;
     const int blocks = (hpg + most - 1) / most;
     return (hpg + blocks - 1) / blocks;

@@ -164,8 +164,8 @@ def _cases(n, seed0):
     rnd = random.Random(seed0)
     for seed in range(n):
         halves = rnd.choice([1, 2])
-        heads = rnd.choice([1, 2, 3, 4])
-        split = rnd.choice([1, 2]) if heads % 2 == 0 and halves == 2 else 1
+        heads = rnd.choice([1, 2, 3, 4, 6])
+        split = rnd.choice([d for d in (1, 2, 3) if heads % d == 0]) if halves == 2 else 1
         yield dict(nc=rnd.choice([1, 2, 3, 5, 9, 17, 33]), halves=halves, M=rnd.choice([1, 2, 3]),
                    heads=heads, split=split, D=rnd.choice([1, 4]), ctas=rnd.choice([1, 2, 3, 5, 8, 30]),
                    lastlen=rnd.choice([128 * halves, 1, 77] + ([129] if halves == 2 else [])), seed=seed)
