@@ -66,17 +66,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Contiguous, cost-balanced ranges of (chunk, 128-row block, head) tiles, head innermost, for the scans
 // that sum their per-head terms over each group's heads: CTA i takes the tiles whose cost before them lies
 // in [i, i + 1) * total / ncta.  A tile costs its number of 128-column halves plus one (the state product
-// and the drain), nothing for a block past a ragged chunk's end.  The same arithmetic tells the sum over
-// the CTAs' partial results which CTAs took part of a (chunk, block, group).
+// and the drain), nothing for a block past a ragged chunk's end.  The host works the ranges out
+// (TilePart) and hands the kernels their starts (TileRanges): a CTA reads its run from the table, and
+// the sum over the CTAs' partial results finds which CTAs took part of a (chunk, block, group) by
+// intersecting the runs with the group's tiles.
+struct TileRanges {
+    int ncta;
+    int beg[kBwdSumMaxCtas + 1];  // first tile of CTA i; beg[ncta] = the tile count
+};
+
 struct TilePart {
     int H, Q, nc, blocks, len_last, ncta, anti;
     long long cfull, perseq, tiles, ctot;
-    __host__ __device__ int cost_len(int len, int rb) const {
+    int cost_len(int len, int rb) const {
         const int r0 = rb * kRows;
         return r0 >= len ? 0 : 1 + (anti ? Q - r0 : r0 + kRows) / kRows;
     }
-    __host__ __device__ int cost(int c, int rb) const { return cost_len(c == nc - 1 ? len_last : Q, rb); }
-    __host__ void init(const Shape &sh, bool is_anti, int n) {
+    int cost(int c, int rb) const { return cost_len(c == nc - 1 ? len_last : Q, rb); }
+    void init(const Shape &sh, bool is_anti, int n) {
         H = sh.H;
         Q = sh.Q;
         nc = sh.nc;
@@ -95,7 +102,7 @@ struct TilePart {
         ctot = (long long)sh.batch * perseq * H;
     }
     // cost of the tiles before tile t (t = tiles gives the total)
-    __host__ __device__ long long cum(long long t) const {
+    long long cum(long long t) const {
         const long long blk = t / H;
         const int h = (int)(t - blk * H), rb = (int)(blk % blocks);
         const long long r = blk / blocks;
@@ -105,8 +112,9 @@ struct TilePart {
         for (int q = 0; q < rb; ++q) before += cost(c, q);
         return before * H + (long long)cost(c, rb) * h;
     }
-    // first tile of CTA i (i = ncta gives the end)
-    __host__ __device__ long long beg(int i) const {
+    // first tile of CTA i (i = ncta gives the end): the first tile whose cost before it reaches i / ncta
+    // of the total
+    long long beg(int i) const {
         if (i <= 0) return 0;
         if (i >= ncta) return tiles;
         long long lo = 0, hi = tiles;
@@ -118,16 +126,9 @@ struct TilePart {
         }
         return lo;
     }
-    __host__ __device__ int cta_of(long long t) const {
-        const long long i = cum(t) * ncta / ctot;
-        return (int)(i < ncta - 1 ? i : ncta - 1);
-    }
-    // within a run of n tiles of cost cb starting at cost `base`: how many come before CTA i's range
-    __host__ __device__ int first_in(int i, long long base, int cb, int n) const {
-        const long long num = (long long)i * ctot - base * ncta;
-        if (num <= 0) return 0;
-        const long long m = (num + (long long)cb * ncta - 1) / ((long long)cb * ncta);
-        return (int)(m < n ? m : n);
+    void ranges(TileRanges *r) const {
+        r->ncta = ncta;
+        for (int i = 0; i <= ncta; ++i) r->beg[i] = (int)beg(i);
     }
 };
 
@@ -142,12 +143,12 @@ struct Args {
     int *status;
     Shape sh;
     // head sums (kSum): the row each term is dotted with ([batch][T][G][W], bf16), the two column halves'
-    // dot products [batch][T][H][2], the CTAs' partial sums [CTA + (chunk, block, group) key][128][W], and
+    // dot products [batch][H][T][2], the CTAs' partial sums [CTA + (chunk, block, group) key][128][W], and
     // the tile ranges
     const __nv_bfloat16 *dotv;
     float *dotp;
     float *part;
-    TilePart tp;
+    TileRanges tr;
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -194,7 +195,8 @@ using namespace bt;
 template <int KD, int W, bool kAnti, bool kOutBf16, bool kSplit, bool kSum>
 __global__ void __launch_bounds__(bt::kThreads, 1)
     masked_scan_tc_kernel(const __grid_constant__ CUtensorMap mR, const __grid_constant__ CUtensorMap mK,
-                          const __grid_constant__ CUtensorMap mV, const bt::Args a, int r_head, int k_head,
+                          const __grid_constant__ CUtensorMap mV, const __grid_constant__ bt::Args a, int r_head,
+                          int k_head,
                           int v_head) {
     static_assert(!kSplit || KD == 64, "the low part of the state tile has room for KD = 64");
     static_assert(KD == 64 || W == 64, "the fp32 state is staged in the unused second atom of K or V");
@@ -212,8 +214,8 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
     // this CTA's tiles (chunk, 128-row block, head): every gridDim.x-th, so that each CTA gets the same mix
     // of one- and two-half blocks; for head sums a contiguous run of about equal cost
     const int tiles = sh.batch * sh.nc * blocks * sh.H;
-    const int t_beg = kSum ? (int)a.tp.beg(blockIdx.x) : (int)blockIdx.x;
-    const int t_end = kSum ? (int)a.tp.beg(blockIdx.x + 1) : tiles;
+    const int t_beg = kSum ? a.tr.beg[blockIdx.x] : (int)blockIdx.x;
+    const int t_end = kSum ? a.tr.beg[blockIdx.x + 1] : tiles;
     const int t_step = kSum ? 1 : (int)gridDim.x;
     if (t_beg >= t_end) return;  // whole CTA
     auto tile = [&](int t, int &b, int &c, int &rb, int &h) {
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(bt::kThreads, 1)
                         dot = fmaf(r1v, bf16hi(ww[e / 2]), dot);
                     }
                 }
-                if (j < len) a.dotp[(tok * sh.H + h) * 2 + half] = dot;
+                if (j < len) a.dotp[(((size_t)b * sh.H + h) * sh.T + t0 + j) * 2 + half] = dot;
             } else {
             for (int w0 = half * (W / 2); w0 < half * (W / 2) + W / 2; w0 += 16) {
                 uint32_t u[16], u2[16];
@@ -841,100 +843,131 @@ cudaError_t launch_masked_scan_tc(const void *R, int r_head, const void *K, int 
     // contiguous run of them
     const int tiles = sh.batch * sh.nc * (sh.Q / kRows) * sh.H;
     const int grid = sum ? head_sum_ctas(sh) : min(tiles, sm_count());
-    if (sum) a.tp.init(sh, anti, grid);
+    if (sum) {
+        TilePart tp;
+        tp.init(sh, anti, grid);
+        if (tp.tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+        tp.ranges(&a.tr);
+    }
     k<<<grid, kThreads, kSmemBytes, st>>>(mR, mK, mV, a, r_head, k_head, v_head);
     return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// The sums over each group's heads from the head-summing scans' partial results: one warp per (batch,
-// token, group) row adds the partial rows of the CTAs that took part of its (chunk, block, group), in CTA
-// order, for dB and for dC, and writes each of the group's heads' dsigma_t = C_t . dC^(h)_t - B_t . dB^(h)_t
-// from the scans' half-row dot products.  Each lane takes 4 consecutive n.  256 threads per block.
+// The sums over each group's heads from the head-summing scans' partial results.  One block per (32
+// tokens, group, batch) (32 tokens never straddle a 128-row block): it finds which CTAs took part of the
+// tokens' (chunk, block, group) for dB and for dC (one candidate CTA per thread, from the scans' run
+// table), adds their partial rows in CTA order, writes dB and dC, and each of the
+// group's heads' dsigma_t = C_t . dC^(h)_t - B_t . dB^(h)_t from the scans' half-row dot products.
+// 256 threads; each thread takes 4 consecutive n of a row.
 // ---------------------------------------------------------------------------
-template <int kNV>
+constexpr int kRedTok = 32;
+
 __global__ void __launch_bounds__(256) head_sum_reduce_kernel(const float *__restrict__ partB,
                                                               const float *__restrict__ dotB,
                                                               const float *__restrict__ partC,
-                                                              const float *__restrict__ dotC, const TilePart pb,
-                                                              const TilePart pc, __nv_bfloat16 *__restrict__ dB,
+                                                              const float *__restrict__ dotC,
+                                                              const __grid_constant__ TileRanges rB,
+                                                              const __grid_constant__ TileRanges rC,
+                                                              __nv_bfloat16 *__restrict__ dB,
                                                               __nv_bfloat16 *__restrict__ dC, float *__restrict__ dsig,
                                                               Shape sh) {
-    const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const long long units = (long long)sh.batch * sh.T * sh.G;
-    if (unit >= units) return;
-    const int lane = threadIdx.x & 31;
-    const int g = (int)(unit % sh.G);
-    const long long tok = unit / sh.G;  // b * T + t
-    const int b = (int)(tok / sh.T), t = (int)(tok - (long long)b * sh.T);
-    const int c = t / sh.Q, rr = t - c * sh.Q, rb = rr / kRows, lr = rr - rb * kRows;
+    static_assert(kBwdSumMaxCtas <= 256, "one candidate CTA per thread");
+    __shared__ int slots[2][kBwdSumMaxCtas];  // partial-sum slots of the contributing CTAs, in CTA order
+    __shared__ int nslot[2];
+    const int tid = threadIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tb = blockIdx.x * kRedTok;  // first token
+    const int c = tb / sh.Q, rb = (tb - c * sh.Q) / kRows, lr0 = tb - c * sh.Q - rb * kRows;
+    const int hpg = sh.heads_per_group;
     const long long blk = ((long long)b * sh.nc + c) * (sh.Q / kRows) + rb;
-    const long long key = blk * sh.G + g, k0 = blk * sh.H + (long long)g * sh.heads_per_group;
-    const int hpg = sh.heads_per_group, V = sh.N / 4;
-    auto gather = [&](const TilePart &p, const float *part, float4 *acc) {
+    const long long key = blk * sh.G + g, k0 = blk * sh.H + (long long)g * hpg;
+    // CTA tid contributes when its run holds a head of the key (tiles k0 .. k0 + hpg - 1)
+    for (int w = 0; w < 2; ++w) {
+        const TileRanges &rg = w ? rC : rB;
+        const int i = tid;
+        const bool take = i < rg.ncta && max((long long)rg.beg[i], k0) < min((long long)rg.beg[i + 1], k0 + hpg);
+        // compact in CTA order: a block-wide prefix count over the candidates
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        __shared__ int wcnt[8];
+        if ((tid & 31) == 0) wcnt[tid >> 5] = __popc(bal);
+        __syncthreads();
+        int before = __popc(bal & ((1u << (tid & 31)) - 1u));
+        for (int q = 0; q < (tid >> 5); ++q) before += wcnt[q];
+        if (take) slots[w][before] = i + (int)key;
+        if (tid == 0) {
+            int n = 0;
+            for (int q = 0; q < 8; ++q) n += wcnt[q];
+            nslot[w] = n;
+        }
+        __syncthreads();
+    }
+    const int V = sh.N / 4;  // 4-vectors per row
+    const int ntok = min(kRedTok, sh.T - tb);
+    // this thread's items (row, 4-vector) tid, tid + 256, ...: every slot's loads for all of them go out
+    // together
+    constexpr int kItems = kRedTok * 64 / 256;  // N <= 256
+    float4 sb[kItems], sc[kItems];
 #pragma unroll
-        for (int m = 0; m < kNV; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const long long base = p.cum(k0);
-        const int cb = p.cost(c, rb), i0 = p.cta_of(k0), i1 = p.cta_of(k0 + hpg - 1);
-        int f0 = p.first_in(i0, base, cb, hpg);
-        for (int i = i0; i <= i1; ++i) {
-            const int f1 = p.first_in(i + 1, base, cb, hpg);
-            if (f0 < f1) {  // CTA i took heads f0 .. f1 - 1 of the group
-                const float *row = part + ((size_t)(i + key) * kRows + lr) * sh.N;
+    for (int q = 0; q < kItems; ++q) sb[q] = sc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto gather = [&](const float *part, int w, float4 (&acc)[kItems]) {
+        for (int k = 0; k < nslot[w]; ++k) {
+            const float *base = part + ((size_t)slots[w][k] * kRows + lr0) * sh.N;
 #pragma unroll
-                for (int m = 0; m < kNV; ++m) {
-                    const int v = lane + 32 * m;
-                    if (v < V) {
-                        const float4 x = *reinterpret_cast<const float4 *>(row + 4 * v);
-                        acc[m].x += x.x;
-                        acc[m].y += x.y;
-                        acc[m].z += x.z;
-                        acc[m].w += x.w;
-                    }
+            for (int q = 0; q < kItems; ++q) {
+                const int item = tid + 256 * q, r = item / V, v = item - r * V;
+                if (r < ntok) {
+                    const float4 x = *reinterpret_cast<const float4 *>(base + (size_t)r * sh.N + 4 * v);
+                    acc[q].x += x.x;
+                    acc[q].y += x.y;
+                    acc[q].z += x.z;
+                    acc[q].w += x.w;
                 }
             }
-            f0 = f1;
         }
     };
-    float4 sb[kNV], sc[kNV];
-    gather(pb, partB, sb);
-    gather(pc, partC, sc);
-    const size_t grow = (size_t)unit * sh.N;  // row (b, t, g) of dB, dC
+    gather(partB, 0, sb);
+    gather(partC, 1, sc);
 #pragma unroll
-    for (int m = 0; m < kNV; ++m) {
-        const int v = lane + 32 * m;
-        if (v < V) {
-            const __nv_bfloat162 b0 = __floats2bfloat162_rn(sb[m].x, sb[m].y), b1 = __floats2bfloat162_rn(sb[m].z, sb[m].w);
-            const __nv_bfloat162 c0 = __floats2bfloat162_rn(sc[m].x, sc[m].y), c1 = __floats2bfloat162_rn(sc[m].z, sc[m].w);
-            uint2 rb2, rc2;
-            rb2.x = *reinterpret_cast<const uint32_t *>(&b0);
-            rb2.y = *reinterpret_cast<const uint32_t *>(&b1);
-            rc2.x = *reinterpret_cast<const uint32_t *>(&c0);
-            rc2.y = *reinterpret_cast<const uint32_t *>(&c1);
-            *reinterpret_cast<uint2 *>(dB + grow + 4 * v) = rb2;
-            *reinterpret_cast<uint2 *>(dC + grow + 4 * v) = rc2;
-        }
+    for (int q = 0; q < kItems; ++q) {
+        const int item = tid + 256 * q, r = item / V, v = item - r * V;
+        if (r >= ntok) continue;
+        const size_t grow = (((size_t)b * sh.T + tb + r) * sh.G + g) * sh.N + 4 * v;  // row (b, t, g)
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(sb[q].x, sb[q].y), b1 = __floats2bfloat162_rn(sb[q].z, sb[q].w);
+        const __nv_bfloat162 c0 = __floats2bfloat162_rn(sc[q].x, sc[q].y), c1 = __floats2bfloat162_rn(sc[q].z, sc[q].w);
+        uint2 ub, uc;
+        ub.x = *reinterpret_cast<const uint32_t *>(&b0);
+        ub.y = *reinterpret_cast<const uint32_t *>(&b1);
+        uc.x = *reinterpret_cast<const uint32_t *>(&c0);
+        uc.y = *reinterpret_cast<const uint32_t *>(&c1);
+        *reinterpret_cast<uint2 *>(dB + grow) = ub;
+        *reinterpret_cast<uint2 *>(dC + grow) = uc;
     }
-    for (int hh = lane; hh < hpg; hh += 32) {
-        const int h = g * hpg + hh;
-        const float2 db = *reinterpret_cast<const float2 *>(dotB + ((size_t)tok * sh.H + h) * 2);
-        const float2 dc = *reinterpret_cast<const float2 *>(dotC + ((size_t)tok * sh.H + h) * 2);
-        dsig[((size_t)b * sh.H + h) * sh.T + t] = (dc.x + dc.y) - (db.x + db.y);
+    // dsigma: a warp per head, a lane per token
+    const int lane = tid & 31;
+#pragma unroll 4
+    for (int hh = tid >> 5; hh < hpg; hh += 8) {
+        if (lane >= ntok) continue;
+        const size_t at = ((size_t)b * sh.H + g * hpg + hh) * sh.T + tb + lane;
+        const float2 db = *reinterpret_cast<const float2 *>(dotB + 2 * at);
+        const float2 dc = *reinterpret_cast<const float2 *>(dotC + 2 * at);
+        dsig[at] = (dc.x + dc.y) - (db.x + db.y);
     }
 }
 
 cudaError_t launch_head_sum_reduce(const float *partB, const float *dotB, const float *partC, const float *dotC,
                                    void *dB, void *dC, float *dsig, const Shape &sh, cudaStream_t st) {
-    if (sh.N % 4 != 0 || sh.N > 256) return cudaErrorInvalidValue;
+    if (sh.N % 4 != 0 || sh.N > 256 || sh.G > 65535 || sh.batch > 65535) return cudaErrorInvalidValue;
     const int n = head_sum_ctas(sh);
     TilePart pb, pc;
     pb.init(sh, true, n);
     pc.init(sh, false, n);
-    const long long units = (long long)sh.batch * sh.T * sh.G;
-    auto k = sh.N <= 128 ? head_sum_reduce_kernel<1> : head_sum_reduce_kernel<2>;
-    k<<<(unsigned)((units + 7) / 8), 256, 0, st>>>(partB, dotB, partC, dotC, pb, pc,
-                                                   static_cast<__nv_bfloat16 *>(dB), static_cast<__nv_bfloat16 *>(dC),
-                                                   dsig, sh);
+    if (pb.tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    TileRanges rB, rC;
+    pb.ranges(&rB);
+    pc.ranges(&rC);
+    const dim3 grid((unsigned)((sh.T + kRedTok - 1) / kRedTok), (unsigned)sh.G, (unsigned)sh.batch);
+    head_sum_reduce_kernel<<<grid, 256, 0, st>>>(partB, dotB, partC, dotC, rB, rC, static_cast<__nv_bfloat16 *>(dB),
+                                                 static_cast<__nv_bfloat16 *>(dC), dsig, sh);
     return cudaGetLastError();
 }
 

@@ -1,12 +1,13 @@
 """Host model of the backward's head-summing scans' tile partition (``TilePart`` in csrc/ssd_bwd_tc.cu).
 
 The dB and dC scans on the tensor cores sum their per-head terms over each group's heads: CTA i takes the
-contiguous run of (chunk, 128-row block, head) tiles whose cost before them lies in [i, i + 1) * total / n,
-and stores one partial sum per (chunk, block, group) key it touched, in slot i + key.  The reduce finds
-the CTAs that touched a key from the same arithmetic, without a table.  This model restates both views in
-integers and checks, over many shapes, that they agree: every key's heads are covered once, by exactly
-the CTAs the reduce visits, in CTA order, and no two (CTA, key) pairs share a slot.  The GPU parity tests
-check the kernels themselves against the oracle.
+contiguous run of (chunk, 128-row block, head) tiles whose cost before them lies in [i, i + 1) * total / n
+(the host works out each run's first tile), and stores one partial sum per (chunk, block, group) key it
+touched, in slot i + key.  The reduce takes, for each key, the CTAs whose runs intersect the key's tiles.
+This model restates the runs in integers and checks, over many shapes, that the two views agree: every
+key's heads are covered once, by exactly the CTAs the reduce visits, in CTA order, that the runs balance
+the cost, and that no two (CTA, key) pairs share a slot.  The GPU parity tests check the kernels
+themselves against the oracle.
 """
 import random
 
@@ -60,15 +61,6 @@ class Part:
                 lo = mid + 1
         return lo
 
-    def cta_of(self, t):
-        return min(self.n - 1, self.cum(t) * self.n // self.ctot)
-
-    def first_in(self, i, base, cb, n):
-        num = i * self.ctot - base * self.n
-        if num <= 0:
-            return 0
-        return min(n, -(-num // (cb * self.n)))
-
     def valid(self, t):
         blk = t // self.H
         r, rb = divmod(blk, self.blocks)
@@ -88,21 +80,16 @@ def kernel_view(p):
     return seen
 
 
-def reduce_view(p, key):
-    """CTAs the reduce adds for one valid key, with the heads it credits to each, in visiting order."""
+def reduce_view(p, table, key):
+    """CTAs the reduce adds for one valid key (those whose runs intersect the key's tiles), with the heads
+    the intersection holds, in visiting order."""
     blk, g = divmod(key, p.G)
-    r, rb = divmod(blk, p.blocks)
-    c = r % p.nc
     k0 = blk * p.H + g * p.hpg
-    base, cb = p.cum(k0), p.cost(c, rb)
-    i0, i1 = p.cta_of(k0), p.cta_of(k0 + p.hpg - 1)
     out = []
-    f0 = p.first_in(i0, base, cb, p.hpg)
-    for i in range(i0, i1 + 1):
-        f1 = p.first_in(i + 1, base, cb, p.hpg)
-        if f0 < f1:
-            out.append((i, list(range(f0, f1))))
-        f0 = f1
+    for i in range(p.n):
+        lo, hi = max(table[i], k0), min(table[i + 1], k0 + p.hpg)
+        if lo < hi:
+            out.append((i, list(range(lo - k0, hi - k0))))
     return out
 
 
@@ -125,9 +112,10 @@ def test_partition_and_reduce_agree(anti):
         tiles = batch * ((T + Q - 1) // Q) * (Q // ROWS) * H
         for n in {1, min(tiles, 148), min(tiles, rng.randint(1, MAX_CTAS))}:
             p = Part(batch, T, H, G, Q, anti, n)
+            table = [p.beg(i) for i in range(n + 1)]
             # the ranges cover every tile once, in order
-            assert p.beg(0) == 0 and p.beg(n) == p.tiles
-            assert all(p.beg(i) <= p.beg(i + 1) for i in range(n))
+            assert table[0] == 0 and table[n] == p.tiles
+            assert all(table[i] <= table[i + 1] for i in range(n))
             seen = kernel_view(p)
             nkeys = p.tiles // p.hpg
             # slots are unique and inside the workspace's region
@@ -139,7 +127,7 @@ def test_partition_and_reduce_agree(anti):
                 if not p.valid(key * p.hpg):
                     continue
                 want = sorted((i, sorted(hs)) for (i, k), hs in seen.items() if k == key)
-                got = reduce_view(p, key)
+                got = reduce_view(p, table, key)
                 assert got == want, (batch, T, H, G, Q, n, key)
                 assert sorted(h for _, hs in got for h in hs) == list(range(p.hpg))
 
