@@ -16,10 +16,12 @@ template <typename T>
 cudaError_t launch_chunk_scan(const T *x, const T *B, const T *C, const float *D, const float *s,
                               const float *Sprev, T *y, const Shape &sh, cudaStream_t st);
 bool fused_supported(const Shape &sh, int dtype);
-cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
-                             const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
-                             int n_half, const FusedDebug *dbg, const FusedGate *gate, cudaStream_t st);
+cudaError_t prepare_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
+                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
+                              const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
+                              int n_half, const FusedDebug *dbg, const FusedGate *gate, int slot);
+cudaError_t enqueue_fused_clear(char *ws, size_t stride, size_t bytes, int passes, cudaStream_t st);
+cudaError_t enqueue_ssd_fused(int slot, bool after_clear, cudaStream_t st);
 }  // namespace ssd
 
 using ssd::Shape;
@@ -80,10 +82,13 @@ int launch_count(const Shape &sh, ssd::Path path) {
 }
 
 // Optional event marks: ev[0] at the start of the call (before the workspace
-// clear), ev[1] before the first kernel, ev[k+2] after kernel k.
+// clear), ev[1] before the first kernel, ev[k+2] after kernel k.  A path whose
+// first kernel directly follows the start (the clear being part of its first
+// stage) records ev[0] alone and sets `stage0_at_start`.
 struct Marks {
     cudaEvent_t *ev = nullptr;
     int n = 0;
+    mutable bool stage0_at_start = false;
     bool mark(int i, cudaStream_t st) const { return !(ev && i < n) || cudaEventRecord(ev[i], st) == cudaSuccess; }
 };
 
@@ -103,22 +108,29 @@ int run_simt(const Shape &sh, const T *x, const float *dt, const float *A, const
     return SSD_OK;
 }
 
+// The fused path: every launch is worked out on the host first; then the call's marks, the clear of each
+// launch's counter and flags (a kernel the first launch may overlap: it waits for the clear before any
+// global access), and the launches go to the stream back to back.  The first stage's span covers the
+// clear and the first launch.
 int run_fused(const Shape &sh, const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
               const __nv_bfloat16 *C, const float *D, const float *init, __nv_bfloat16 *y, float *fin, char *ws,
               const ssd::Workspace &w, cudaStream_t st, const Marks &mk, const ssd::FusedDebug *dbg,
               const ssd::FusedGate *gate) {
-    if (!mk.mark(1, st)) return SSD_ERR_CUDA;
     // launch k covers head-column half k % pp and state-column half k / pp: the second state half adds to
     // the y its first half wrote, so it comes after both head-column launches of that first half
     const int passes = ssd::fused_passes(sh), pp = ssd::fused_p_passes(sh);
+    if (passes > ssd::kMaxFusedPasses) return SSD_ERR_UNSUPPORTED;
     const size_t stride = w.total / passes;  // one launch's counter, flags and ring
-    for (int k = 0; k < passes; ++k) {
-        char *pw = ws + k * stride;
-        if (ssd::launch_ssd_fused(x, dt, A, B, C, D, init, fin, pw, w, reinterpret_cast<int *>(ws + w.status_off), y,
-                                  sh, k % pp, k / pp, dbg, gate, st) != cudaSuccess ||
-            !mk.mark(2 + k, st))
+    for (int k = 0; k < passes; ++k)
+        if (ssd::prepare_ssd_fused(x, dt, A, B, C, D, init, fin, ws + k * stride, w,
+                                   reinterpret_cast<int *>(ws + w.status_off), y, sh, k % pp, k / pp, dbg, gate,
+                                   k) != cudaSuccess)
             return SSD_ERR_CUDA;
-    }
+    if (!mk.mark(0, st)) return SSD_ERR_CUDA;
+    mk.stage0_at_start = true;
+    if (ssd::enqueue_fused_clear(ws, stride, w.clear_bytes, passes, st) != cudaSuccess) return SSD_ERR_CUDA;
+    for (int k = 0; k < passes; ++k)
+        if (ssd::enqueue_ssd_fused(k, k == 0, st) != cudaSuccess || !mk.mark(2 + k, st)) return SSD_ERR_CUDA;
     return SSD_OK;
 }
 
@@ -157,6 +169,16 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
     if (dbg && path != ssd::kPathFused) return SSD_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
+    if (path == ssd::kPathFused && T > 0) {
+        rc = run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+                       static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
+                       final_state, ws, w, st, mk, dbg, gate_fused ? gate : nullptr);
+        // elsewhere the gate runs as its own kernel over the y just written (in place)
+        if (rc == SSD_OK && gate && !gate_fused)
+            rc = ssd_gate_norm(y, gate->z, gate->weight, gate->bias, y, (long long)batch * T, H * P, H, gate->eps,
+                               dtype, stream);
+        return rc;
+    }
     if (!mk.mark(0, st)) return SSD_ERR_CUDA;
     if (cudaMemsetAsync(ws, 0, w.clear_bytes, st) != cudaSuccess) return SSD_ERR_CUDA;
     if (path == ssd::kPathFused)
@@ -171,11 +193,7 @@ int fwd_impl(const void *x, const float *dt, const float *A, const void *B, cons
                                    : cudaMemsetAsync(final_state, 0, fb, st);
         return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
     }
-    if (path == ssd::kPathFused)
-        rc = run_fused(sh, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
-                       static_cast<const __nv_bfloat16 *>(C), D, init_state, static_cast<__nv_bfloat16 *>(y),
-                       final_state, ws, w, st, mk, dbg, gate_fused ? gate : nullptr);
-    else if (dtype == SSD_BF16)
+    if (dtype == SSD_BF16)
         rc = run_simt<__nv_bfloat16>(sh, static_cast<const __nv_bfloat16 *>(x), dt, A,
                                      static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C), D,
                                      init_state, static_cast<__nv_bfloat16 *>(y), final_state, ws, w, st, mk);
@@ -255,7 +273,8 @@ int ssd_fwd_timed(const void *x, const float *dt, const float *A, const void *B,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
     for (int i = 0; i < k && i < max_stages && stage_ms; ++i)
-        if (cudaEventElapsedTime(&stage_ms[i], events[dev][i + 1], events[dev][i + 2]) != cudaSuccess)
+        if (cudaEventElapsedTime(&stage_ms[i], events[dev][(i == 0 && mk.stage0_at_start) ? 0 : i + 1],
+                                 events[dev][i + 2]) != cudaSuccess)
             return SSD_ERR_CUDA;
     if (total_ms) {
         *total_ms = 0.f;

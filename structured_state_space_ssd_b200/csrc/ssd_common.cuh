@@ -190,6 +190,7 @@ inline size_t bwd_sum_dot_off(const Shape &s) {
 inline int fused_p_passes(const Shape &s) { return s.P > 64 ? 2 : 1; }
 inline int fused_n_passes(const Shape &s) { return s.N > 128 ? 2 : 1; }
 inline int fused_passes(const Shape &s) { return fused_p_passes(s) * fused_n_passes(s); }
+constexpr int kMaxFusedPasses = 4;
 
 inline Workspace workspace_layout_one(const Shape &s, Path path);
 

@@ -57,6 +57,8 @@
 // G = C B^T (the block's 128 x 128) are shared by the unit's heads; an owner's
 // units hold half as many heads as the other block's, whose heads take about
 // half as long.
+#include <algorithm>
+
 #include "ssd_common.cuh"
 #include "tc_prims.cuh"
 #include "tma_host.h"
@@ -369,6 +371,9 @@ __global__ void __launch_bounds__(fz::kThreads, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
+    // launched as a programmatic dependent of the workspace clear: everything above overlapped it; no
+    // thread touches global memory before the clear has completed and its stores are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp >= kSimtWarps + 2) {
         // ------------------------------------------------------------------
@@ -1381,21 +1386,37 @@ static int heads_per_unit(const Shape &sh, bool lookback, bool owners) {
     return (hpg + blocks - 1) / blocks;
 }
 
-// Launches the fused kernel for state columns [n_half * 128, ...) and head columns [p_half * 64, ...)
-// of the problem `full` (all of them when full.N <= 128 and full.P <= 64).  The second half of a
-// 256-wide state adds to the y of the first.
+// One launch of the fused kernel, worked out on the host ahead of the call's first enqueued operation
+// (so that the GPU does not wait on tensor-map encoding between the workspace clear and the launch).
+// Held per host thread: a call prepares its launches and enqueues them before it returns.
+namespace {
+using FusedKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, Params);
+struct FusedLaunch {
+    CUtensorMap mC, mB, mX, mY, mR;
+    Params p;
+    FusedKernel kernel;
+    int grid;
+};
+thread_local FusedLaunch g_launch[kMaxFusedPasses];
+}  // namespace
+
+// Prepares launch `slot` of the fused kernel for state columns [n_half * 128, ...) and head columns
+// [p_half * 64, ...) of the problem `full` (all of them when full.N <= 128 and full.P <= 64).  The second
+// half of a 256-wide state adds to the y of the first.
 // `pw` is this launch's part of the workspace, laid out as `w`; the status word is shared.
-cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                             const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
-                             const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
-                             int n_half, const FusedDebug *dbg, const FusedGate *gate, cudaStream_t st) {
+cudaError_t prepare_ssd_fused(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
+                              const __nv_bfloat16 *C, const float *D, const float *init, float *fin, char *pw,
+                              const Workspace &w, int *status, __nv_bfloat16 *y, const Shape &full, int p_half,
+                              int n_half, const FusedDebug *dbg, const FusedGate *gate, int slot) {
+    if (slot < 0 || slot >= kMaxFusedPasses) return cudaErrorInvalidValue;
+    FusedLaunch &L = g_launch[slot];
     // the gate needs the whole row of a head in one launch
     if (gate && (full.P != kP || full.N > 128)) return cudaErrorInvalidValue;
     Shape sh = full;
     const int n_off = n_half * 128, p_off = p_half * kP;
     if (full.N > 128) sh.N = 128;
     sh.P = kP;
-    CUtensorMap mC, mB, mX;
+    CUtensorMap &mC = L.mC, &mB = L.mB, &mX = L.mX, &mY = L.mY, &mR = L.mR;
     const uint64_t dbc[4] = {(uint64_t)sh.N, (uint64_t)sh.G, (uint64_t)sh.T, (uint64_t)sh.batch};
     const uint64_t sbc[3] = {(uint64_t)full.N * 2, (uint64_t)sh.G * full.N * 2,
                              (uint64_t)sh.T * sh.G * full.N * 2};
@@ -1407,11 +1428,11 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     const uint64_t sx[3] = {(uint64_t)full.P * 2, (uint64_t)sh.H * full.P * 2, (uint64_t)sh.T * sh.H * full.P * 2};
     x += p_off;
     y += p_off;
-    CUtensorMap mY;
     if (!make_map_bf16(&mC, C, 4, dbc, sbc, box) || !make_map_bf16(&mB, B, 4, dbc, sbc, box) ||
         !make_map_bf16(&mX, x, 4, dx, sx, box) || !make_map_bf16(&mY, y, 4, dx, sx, box))
         return cudaErrorInvalidValue;
-    Params p;
+    Params &p = L.p;
+    p = Params{};
     p.sh = sh;
     p.dt = dt;
     p.A = A;
@@ -1442,7 +1463,6 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
     const bool lookback = fused_lookback(sh) == 4;  // the workspace's layout has the same shape
     // the bf16 state tiles without look-back: [b*H*3][tile_rows][64], one TMA box per tile (with
     // look-back there are none and the map, over the fp32 ring, is never used)
-    CUtensorMap mR;
     {
         const uint64_t slots = lookback ? 1 : (uint64_t)sh.batch * sh.H * fused_ring_slots(1);
         const uint64_t dr[3] = {(uint64_t)kP, (uint64_t)p.tile_rows, slots};
@@ -1465,9 +1485,45 @@ cudaError_t launch_ssd_fused(const __nv_bfloat16 *x, const float *dt, const floa
                                  : (lookback ? ssd_fused_kernel<false, 4, false> : ssd_fused_kernel<false, 1, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int grid = min(p.n_units, device_sm_count());
-    kernel<<<grid, kThreads, kSmemBytes, st>>>(mC, mB, mX, mY, mR, p);
+    L.kernel = kernel;
+    L.grid = min(p.n_units, device_sm_count());
+    return cudaSuccess;
+}
+
+// The clear of each launch's counter, flags and status before a call (`passes` regions `stride` bytes
+// apart, `bytes` each, 16-byte multiples): it lets its dependent launch start at once, so that the fused
+// kernel's start-up overlaps it (the fused kernel waits for it to complete before any global access).
+__global__ void __launch_bounds__(256) fused_clear_kernel(char *ws, size_t stride, size_t bytes) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    uint4 *q = reinterpret_cast<uint4 *>(ws + blockIdx.y * stride);
+    const size_t n = bytes / 16;
+    for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (size_t)gridDim.x * 256)
+        q[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+cudaError_t enqueue_fused_clear(char *ws, size_t stride, size_t bytes, int passes, cudaStream_t st) {
+    if (bytes % 16 != 0 || passes < 1 || passes > kMaxFusedPasses) return cudaErrorInvalidValue;
+    const size_t blocks = std::min<size_t>(std::max<size_t>((bytes / 16 + 1023) / 1024, 1), 64);
+    fused_clear_kernel<<<dim3((unsigned)blocks, (unsigned)passes), 256, 0, st>>>(ws, stride, bytes);
     return cudaGetLastError();
+}
+
+// Enqueues launch `slot` as prepared by this host thread's last prepare_ssd_fused for it; `after_clear`:
+// it directly follows enqueue_fused_clear in the stream and may start while the clear runs.
+cudaError_t enqueue_ssd_fused(int slot, bool after_clear, cudaStream_t st) {
+    if (slot < 0 || slot >= kMaxFusedPasses) return cudaErrorInvalidValue;
+    const FusedLaunch &L = g_launch[slot];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)L.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_clear ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, L.kernel, L.mC, L.mB, L.mX, L.mY, L.mR, L.p);
 }
 
 }  // namespace ssd
