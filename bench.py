@@ -416,8 +416,9 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps,
                     "pipelined": "two device buffer sets; inputs in, compute and outputs out of neighbouring "
                                  "steps overlap on three streams"},
-            "gpu_launches": S.ssd_fwd_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
-            * args.steps,
+            # the main launches, plus the fused path's workspace-clear kernel (timed within its first stage)
+            "gpu_launches": (S.ssd_fwd_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)
+                             + (1 if names[0].startswith("ssd_fused") else 0)) * args.steps,
         }
         if world == 1 and not args.no_workloads:
             line["workloads"] = measure_workloads(w, dev, stream, flush, peaks)
@@ -587,6 +588,9 @@ def measure_gated(w, d, dev, stream, flush, gate_us, fwd_ms, steps=20):
     ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
     launches = S.load().ssd_fwd_gated_launch_count(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q,
                                                    S._dtype_code(d["x"].dtype))
+    # plus the fused path's workspace-clear kernel
+    if S.ssd_fwd_stage_names(w.batch, w.T, w.H, w.P, w.G, w.N, w.Q, d["x"].dtype)[0].startswith("ssd_fused"):
+        launches += 1
     return {"ms_per_call": ms, "tokens_per_s": w.batch * w.T / (ms * 1e-3), "launches_per_call": launches,
             "separate_ms": fwd_ms + gate_us * 1e-3, "with": "z, norm weight and bias; one group per head"}
 

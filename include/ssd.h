@@ -103,9 +103,13 @@ SSD_API int ssd_fwd(const void *x, const float *dt, const float *A, const void *
             size_t workspace_bytes, void *stream);
 
 /*
- * Number of kernel launches ssd_fwd issues for these arguments (0 when the
- * arguments are invalid).  Lets callers account for launches without a
- * profiler.
+ * Number of main kernel launches ssd_fwd issues for these arguments, which is
+ * also the number of stages ssd_fwd_timed reports (0 when the arguments are
+ * invalid).  The fused path also runs one small kernel that clears the
+ * workspace's counter and flags in front of its first launch (it overlaps
+ * that launch's start and is timed within the first stage); the CUDA-core
+ * path clears them with a memset.  Lets callers account for launches without
+ * a profiler.
  */
 SSD_API int ssd_fwd_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
 
@@ -265,7 +269,8 @@ SSD_API int ssd_fwd_gated(const void *x, const float *dt, const float *A, const 
                   const float *norm_bias, float eps, void *out, float *final_state, int batch, int T, int H,
                   int P, int G, int N, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
-/* Kernel launches ssd_fwd_gated issues for these arguments (0 when they are invalid). */
+/* Main kernel launches ssd_fwd_gated issues for these arguments (0 when they are invalid), counted as
+ * for ssd_fwd_launch_count (the fused path's workspace-clear kernel not included). */
 SSD_API int ssd_fwd_gated_launch_count(int batch, int T, int H, int P, int G, int N, int Q, int dtype);
 
 /*
