@@ -141,3 +141,55 @@ def test_partition_balances_cost():
                          for t in range(p.beg(i), p.beg(i + 1))))
     assert sum(costs) == p.ctot
     assert max(costs) - min(costs) <= 2 * 3  # within two tiles' cost of each other
+
+
+def _check(p, slot_of, reduce):
+    """The agreement checks of test_partition_and_reduce_agree for one partition, with the slot rule and the
+    reduce's view passed in (so that a planted mistake in either can be shown to fail)."""
+    table = [p.beg(i) for i in range(p.n + 1)]
+    seen = kernel_view(p)
+    nkeys = p.tiles // p.hpg
+    slots = [slot_of(i, key) for (i, key) in seen]
+    if len(set(slots)) != len(slots) or not all(0 <= s < MAX_CTAS + nkeys for s in slots):
+        return False
+    for key in range(nkeys):
+        if not p.valid(key * p.hpg):
+            continue
+        want = sorted((i, sorted(hs)) for (i, k), hs in seen.items() if k == key)
+        if reduce(p, table, key) != want:
+            return False
+    return True
+
+
+def _first_cta_only(p, table, key):
+    # a mistake: the reduce takes only the CTA whose run holds the key's first head
+    got = reduce_view(p, table, key)
+    return got[:1]
+
+
+def _off_by_one_end(p, table, key):
+    # a mistake: a run's end taken as inclusive
+    blk, g = divmod(key, p.G)
+    k0 = blk * p.H + g * p.hpg
+    out = []
+    for i in range(p.n):
+        lo, hi = max(table[i], k0), min(table[i + 1] + 1, k0 + p.hpg)
+        if lo < hi:
+            out.append((i, list(range(lo - k0, hi - k0))))
+    return out
+
+
+@pytest.mark.parametrize("mistake", ["slot_is_key", "first_cta_only", "inclusive_end"])
+def test_a_planted_mistake_in_the_partition_is_caught(mistake):
+    slot_of = (lambda i, key: key) if mistake == "slot_is_key" else (lambda i, key: i + key)
+    reduce = {"first_cta_only": _first_cta_only, "inclusive_end": _off_by_one_end}.get(mistake, reduce_view)
+    # the right rules pass on every shape; the planted one fails on at least one
+    caught = False
+    for batch, T, H, G, Q in list(shapes())[:20]:
+        tiles = batch * ((T + Q - 1) // Q) * (Q // ROWS) * H
+        for anti in (True, False):
+            p = Part(batch, T, H, G, Q, anti, min(tiles, 148))
+            assert _check(p, lambda i, key: i + key, reduce_view)
+            if not _check(p, slot_of, reduce):
+                caught = True
+    assert caught, mistake
