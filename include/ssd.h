@@ -116,9 +116,11 @@ SSD_API int ssd_fwd_launch_count(int batch, int T, int H, int P, int G, int N, i
 /*
  * ssd_fwd, instrumented for measurement: records a CUDA event on `stream`
  * before the first kernel and after each kernel, waits for the stream, and
- * writes each kernel's duration in milliseconds to stage_ms[0 .. k-1]
- * (k = min(ssd_fwd_launch_count(...), max_stages)) and the span of the whole
- * call to *total_ms (either pointer may be NULL).  The events are created on
+ * writes each stage's duration in milliseconds to stage_ms[0 .. k-1]
+ * (k = min(ssd_fwd_launch_count(...), max_stages); a stage is one main
+ * launch, on the fused path the first one together with the workspace clear
+ * in front of it) and the span of the whole call to *total_ms (either pointer
+ * may be NULL).  The events are created on
  * the first call in each host thread and kept until the process exits.  Same
  * arguments and results as ssd_fwd otherwise.
  */
