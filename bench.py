@@ -643,13 +643,25 @@ def measure_backward(w, d, dev, stream, flush, peaks, steps=5):
 
 
 def _traffic_from_profiles(kernel, w):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one matches."""
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if one matches this workload and was
+    taken on the kernel's current source (the entry records the SHA-256 of the source file it was captured
+    from; a changed kernel reports None until it is captured again)."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
-    return t.get(w.name, {}).get(kernel)
+    e = t.get(w.name, {}).get(kernel)
+    if not isinstance(e, dict):
+        return None
+    src = os.path.join(ROOT, "structured_state_space_ssd_b200", e.get("source", ""))
+    if not os.path.isfile(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != e.get("sha256"):
+            return None
+    return e.get("bytes")
 
 
 if __name__ == "__main__":

@@ -28,3 +28,27 @@ def test_backward_block_count():
     Q, N, P, H = 256, 128, 64, 80
     per = 2 * Q * Q * N + 2 * 2 * Q * Q * P * H + 2 * 2 * Q * Q * N * H + 5 * 2 * Q * N * P * H
     assert bench.backward_alg_flops(w) == 32 * per == 183_072_980_992
+
+
+def test_traffic_is_reported_only_for_the_captured_kernel_source(tmp_path, monkeypatch):
+    # profiles/traffic.json ties each DRAM figure to the SHA-256 of the kernel source it was captured from;
+    # any other source (a changed kernel) reads None until it is captured again
+    import hashlib
+    import json
+    src_dir = tmp_path / "structured_state_space_ssd_b200" / "csrc"
+    src_dir.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    kernel = src_dir / "k.cu"
+    kernel.write_text("// captured version\n")
+    digest = hashlib.sha256(kernel.read_bytes()).hexdigest()
+    entry = {"bytes": 123456, "source": "csrc/k.cu", "sha256": digest}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"wl": {"kern": entry}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+
+    class W:
+        name = "wl"
+
+    assert bench._traffic_from_profiles("kern", W) == 123456
+    assert bench._traffic_from_profiles("other", W) is None
+    kernel.write_text("// changed since the capture\n")
+    assert bench._traffic_from_profiles("kern", W) is None
