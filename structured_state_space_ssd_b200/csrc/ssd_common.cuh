@@ -141,7 +141,9 @@ struct FusedDebug {
 
 // Workspace carve-up, computed identically by ssd_fwd_workspace_bytes and ssd_fwd.
 // The front 256-byte block holds the status word and the unit counter; it and
-// the per-(batch, head) flags after it are cleared by one memset per call.
+// the per-(batch, head) flags after it are cleared at the start of every call
+// (on the fused path by a small kernel the first launch depends on, elsewhere
+// by a memset).
 struct Workspace {
     size_t status_off;  // int status word
     size_t counter_off; // int unit counter (fused path)
