@@ -192,6 +192,19 @@ def test_bwd_workspace_bytes(lib):
     assert f(1, 0, 2, 16, 1, 16, 64, 0) > 0             # empty sequence is valid
 
 
+def test_bwd_workspace_holds_the_head_sums(lib):
+    # the tensor-core dB and dC scans keep, in the per-head terms' regions, one 128-row partial sum per
+    # (CTA, (chunk, 128-row block, group)) slot (up to 256 CTAs) plus two half-row dot products per
+    # (batch, token, head); with one head per group and a ragged last chunk that exceeds the per-head terms
+    f = lib.ssd_bwd_workspace_bytes
+    for batch, T, H, G, N, Q in [(1, 130, 2, 2, 128, 256), (4, 2048, 80, 1, 128, 256), (2, 600, 8, 2, 64, 128)]:
+        nc = -(-T // Q)
+        keys = batch * nc * (Q // 128) * G
+        sums = (256 + keys) * 128 * N * 4 + 2 * batch * T * H * 4
+        perhead = batch * T * H * N * 4
+        assert f(batch, T, H, 64, G, N, Q, 1) >= 2 * max(sums, perhead)
+
+
 def _bwd(lib, **over):
     """ssd_bwd with fake (never dereferenced) pointers; only validation runs."""
     args = dict(x=0x10000, dt=0x20000, A=0x30000, B=0x40000, C=0x50000, D=0x60000, Q=64, init=None, dy=0x70000,
